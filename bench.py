@@ -1,0 +1,358 @@
+"""Benchmark: decode and prefill throughput of a Llama-3-8B-shaped decoder stack on B200.
+
+Default workload (one GPU): random-init bf16 weights of the Llama-3-8B shape (hidden 4096,
+32 layers, 32/8 heads of 128, SwiGLU 14336, vocab 128256, RoPE base 5e5); a 4096-token
+synthetic prompt is prefilled in chunks of 128 (timed: prefill tok/s), then batch-1 greedy
+decode steps run at context 4096+ (timed: the headline decode tok/s). Every decode step
+streams 15 GB of weights, far above the 126 MB L2, so no L2 flush is needed between steps.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU: one process per GPU under torchrun; each rank runs an independent replica
+(the path has no exchange step), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth import configs  # noqa: E402
+
+METRIC = "decode tok/s + % HBM roofline (8B-shape, b=1); prefill tok/s + % bf16 TC peak"
+PROMPT = 4096
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=j["hbm_gbs"], tc=j["bf16_tflops"], tc_sus=j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sus=1400.0, src="fallback")
+
+
+def layer_bytes(cfg):
+    h, d, nq, nkv, I = cfg["hidden"], cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ffn_inter"]
+    qkv = (nq * d + 2 * nkv * d) * h
+    return 2 * (qkv + h * nq * d + 3 * I * h)
+
+
+def step_bytes(cfg, B, ctx_list):
+    """Algorithmic bytes of one decode step: every weight once + each sequence's KV once."""
+    L, h, V = cfg["layers"], cfg["hidden"], cfg["vocab"]
+    kv_row = 2 * cfg["n_kv_heads"] * cfg["head_dim"] * 2  # k + v, bf16
+    weights = L * layer_bytes(cfg) + V * h * 2 + L * 2 * h * 4 + h * 4
+    kv = sum(L * c * kv_row for c in ctx_list)
+    return weights, kv
+
+
+def gemm_flops_per_token(cfg):
+    return 2 * (layer_bytes(cfg) // 2 * cfg["layers"])
+
+
+def attn_flops_prefill(cfg, T):
+    # causal: query t attends t+1 keys; QK and PV each 2*d flops per (head, key)
+    return 4 * cfg["head_dim"] * cfg["n_q_heads"] * cfg["layers"] * (T * (T + 1) / 2)
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+
+    def __init__(self, index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = subprocess.Popen(
+            ["nvidia-smi", f"--id={index}",
+             "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+             "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+
+    def stop(self):
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def make_device_weights(cfg, torch, seed=0):
+    """Weights of the synthetic recipe generated directly in device memory (same streams as
+    synth.make_weights, by the device twin of the generator)."""
+    dl = synth.dev_lib()
+    st = torch.cuda.current_stream().cuda_stream
+    keep = []
+
+    def mat(shape, tid, mean=0.0, std=synth.WEIGHT_STD):
+        t = torch.empty(shape, dtype=torch.int16, device="cuda")
+        assert dl.syn_dev_fill_bf16(t.data_ptr(), t.numel(), seed, tid, mean, std, st) == 0
+        keep.append(t)
+        return t
+
+    def vec(n, tid, mean, std):
+        t = torch.empty(n, dtype=torch.float32, device="cuda")
+        assert dl.syn_dev_fill_bf16_as_f32(t.data_ptr(), n, seed, tid, mean, std, st) == 0
+        keep.append(t)
+        return t
+
+    h, V = cfg["hidden"], cfg["vocab"]
+    w = dict(embed=mat((V, h), 1), lm_head=None if cfg.get("tied") else mat((V, h), 2),
+             final_norm=vec(h, 3, 1.0, synth.GAIN_STD), layers=[])
+    for l in range(cfg["layers"]):
+        lw = {}
+        for name, shape in synth.tensor_shapes(cfg).items():
+            if shape is None:
+                lw[name] = None
+            elif name in synth.GAINS:
+                lw[name] = vec(shape[0], synth.layer_tid(l, name), 1.0, synth.GAIN_STD)
+            elif name in synth.VECTORS:
+                lw[name] = vec(shape[0], synth.layer_tid(l, name), 0.0, synth.WEIGHT_STD)
+            elif name in ("e_gate", "e_up", "e_down"):
+                part = ("e_gate", "e_up", "e_down").index(name)
+                t = torch.empty(shape, dtype=torch.int16, device="cuda")
+                for e in range(shape[0]):
+                    assert dl.syn_dev_fill_bf16(t[e].data_ptr(), t[e].numel(), seed, synth.expert_tid(l, e, part),
+                                                0.0, synth.WEIGHT_STD, st) == 0
+                keep.append(t)
+                lw[name] = t
+            else:
+                lw[name] = mat(shape, synth.layer_tid(l, name))
+        w["layers"].append(lw)
+    torch.cuda.synchronize()
+    return w
+
+
+def time_gemv(dec, torch, N, K, reps=20):
+    """Average device time of the weight-streaming GEMV on one [N][K] matrix at B=1 (CUDA events
+    on the launching stream); the inputs rotate over buffers larger than L2."""
+    nbuf = max(2, int(math.ceil(300e6 / (N * K * 2))))
+    Ws = [torch.empty((N, K), dtype=torch.bfloat16, device="cuda").normal_(0, 0.02) for _ in range(nbuf)]
+    x = torch.randn((1, K), device="cuda").to(torch.bfloat16)
+    y = torch.empty((1, N), device="cuda")
+    for i in range(3):
+        dec.weight_gemv(Ws[i % nbuf], x, y)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for i in range(reps):
+        dec.weight_gemv(Ws[i % nbuf], x, y)
+    e1.record(s)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del Ws
+    return ms, N * K * 2 + K * 2 + N * 4
+
+
+def cpu_oracle_sample(cfg, ctx):
+    """Time the oracle (as it stands) on a bounded sample of the decode workload: layer 0 and
+    the LM head of the same model, one token at position ctx over a synthetic cache; the full
+    32-layer step time is extrapolated as L * t(layer) + t(head)."""
+    import oracle
+    c1 = configs.with_layers(cfg, 1, max_context=ctx + 1, max_batch=1)
+    w = synth.make_weights(c1)
+    m = oracle.Model(c1, w)
+    kvd = cfg["n_kv_heads"] * cfg["head_dim"]
+    k, v = synth.kv_fill(ctx, kvd, 2000, 0)
+    m.kv_write(0, 0, 0, k, v)
+    t0 = time.perf_counter()
+    m.forward(0, 1, ctx, want_logits=False)
+    t_layer = time.perf_counter() - t0
+    m.kv_write(0, 0, 0, k, v)
+    t0 = time.perf_counter()
+    m.forward(0, 1, ctx, want_logits=True)
+    t_head = max(0.0, time.perf_counter() - t0 - t_layer)
+    step = cfg["layers"] * t_layer + t_head
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return dict(value=1.0 / step, unit="tok/s", cores=threads, kind="oracle",
+                sample=f"1 of {cfg['layers']} layers + LM head, one decode token at context {ctx}, fp64 oracle; "
+                       f"step extrapolated as {cfg['layers']}*t_layer + t_head "
+                       f"(t_layer={t_layer:.3f}s, t_head={t_head:.3f}s)")
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on this host on a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = dict(configs.LLAMA3_8B)
+    steps = []
+    for _ in range(max(1, args.steps)):
+        cb = cpu_oracle_sample(cfg, PROMPT)
+        steps.append(1.0 / cb["value"])
+    val = 1.0 / statistics.median(steps)
+    cb["value"] = val
+    line = dict(metric=METRIC, value=val, unit="tok/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                ms_per_step=1000.0 / val, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                data="synthetic", impl="reference",
+                config=dict(workload="llama3-8b-shape decode b=1 ctx 4096 (oracle, bounded sample)",
+                            global_batch=1, seq_len=PROMPT),
+                cpu_baseline=cb, e2e=dict(value=val, unit="tok/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling only; not a bench number)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import decoder_only_transformer_layer_b200 as dec
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    W = max(3, args.warmup)
+    K = max(1, args.steps)
+    e2e_steps = min(K, 16)
+    cfg = dict(configs.LLAMA3_8B, max_context=PROMPT + W + K + e2e_steps + 8, max_batch=1, prefill_chunk=128)
+    if args.layers:
+        cfg = configs.with_layers(cfg, args.layers)
+    weights = make_device_weights(cfg, torch)
+    d = dec.Decoder(cfg, weights)
+    del weights
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+    prompt = synth.tokens(PROMPT, cfg["vocab"], 1000)
+
+    # ---- prefill (timed once, after a warm-up prefill of one chunk on a scratch sequence)
+    d.prefill(0, prompt[:128], 0)
+    d.reset(0)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    d.prefill(0, prompt, 0)
+    e1.record(stream)
+    e1.synchronize()
+    prefill_ms = e0.elapsed_time(e1)
+    tok = int(d.last_argmax(1)[0])
+
+    # ---- decode: W warm-up steps, then K timed steps (greedy, device-resident inputs)
+    pos = PROMPT
+    for _ in range(W):
+        d.step([tok], [pos])
+        tok = int(d.last_argmax(1)[0])
+        pos += 1
+    torch.cuda.synchronize()
+    barrier()
+    clk = Clocks(local)
+    time.sleep(0.3)
+    ctx_list = []
+    e0.record(stream)
+    for _ in range(K):
+        d.step([tok], [pos])
+        ctx_list.append(pos + 1)
+        pos += 1
+    e1.record(stream)
+    e1.synchronize()
+    clocks = clk.stop()
+    decode_ms = e0.elapsed_time(e1)
+    ms_step = decode_ms / K
+    if world > 1:
+        t = torch.tensor([ms_step, prefill_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, prefill_ms = t.tolist()
+
+    # ---- end to end through the C ABI with host buffers (tokens in, logits out per step)
+    host_logits = torch.empty((1, cfg["vocab"]), dtype=torch.float32).pin_memory().numpy()
+    torch.cuda.synchronize()
+    barrier()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        d.step([tok], [pos], host_logits)
+        tok = int(np.argmax(host_logits[0]))
+        pos += 1
+    e2e_s = (time.perf_counter() - t0) / e2e_steps
+
+    # ---- dominant kernel alone: weight-streaming GEMV on the fused gate/up matrix
+    P = peaks()
+    gemv_ms, gemv_bytes = time_gemv(dec, torch, 2 * cfg["ffn_inter"], cfg["hidden"])
+    gemv_gbs = gemv_bytes / (gemv_ms * 1e-3) / 1e9
+
+    wbytes, kvbytes = step_bytes(cfg, 1, ctx_list)
+    step_gbs = (wbytes + kvbytes / K) / (ms_step * 1e-3) / 1e9
+    value = world * 1.0 / (ms_step * 1e-3)
+    pf_tok_s = world * PROMPT / (prefill_ms * 1e-3)
+    pf_flops = gemm_flops_per_token(cfg) * PROMPT + attn_flops_prefill(cfg, PROMPT)
+    pf_tflops = pf_flops / (prefill_ms * 1e-3) / 1e12
+    chunk_hbm_floor_ms = (PROMPT / 128) * (cfg["layers"] * layer_bytes(cfg)) / (P["hbm"] * 1e9) * 1e3
+    launches_per_step = 1 + 5 * cfg["layers"] + 2
+
+    cpu_b = None
+    if rank == 0 and not args.no_cpu_baseline and not args.layers:
+        cpu_b = cpu_oracle_sample(dict(configs.LLAMA3_8B), PROMPT)
+    if rank == 0:
+        line = dict(
+            metric=METRIC, value=value, unit="tok/s", n_gpus=world, steps=K, warmup=W, ms_per_step=ms_step,
+            higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+            config=dict(workload="llama3-8b-shape decode b=1 at context 4096 after a 4096-token prefill (chunk 128)",
+                        global_batch=world, seq_len=PROMPT, model_shape="llama3-8b", layers=cfg["layers"],
+                        parallelism=f"replicas x{world}", l2="inputs larger than L2 (15 GB of weights per step)"),
+            roofline=dict(bound="hbm", achieved=round(gemv_gbs, 1), peak=P["hbm"], unit="GB/s",
+                          frac=round(gemv_gbs / P["hbm"], 4), traffic=None,
+                          kernel=f"gemv_kernel<1,SWIGLU-shaped> on [{2 * cfg['ffn_inter']}][{cfg['hidden']}] bf16",
+                          peak_source=P["src"]),
+            step_roofline=dict(bytes_per_step=wbytes + kvbytes / K, achieved_gbs=round(step_gbs, 1),
+                               frac=round(step_gbs / P["hbm"], 4), peak=P["hbm"], unit="GB/s"),
+            prefill=dict(tokens=PROMPT, chunk=128, ms=round(prefill_ms, 2), tok_s=round(pf_tok_s, 1),
+                         tflops=round(pf_tflops, 1), tc_frac=round(pf_tflops / P["tc_sus"], 4),
+                         hbm_floor_ms=round(chunk_hbm_floor_ms, 2),
+                         attainable_frac=round(chunk_hbm_floor_ms / prefill_ms, 4)),
+            cpu_baseline=cpu_b,
+            e2e=dict(value=world / e2e_s, unit="tok/s", h2d_bytes_per_step=8, d2h_bytes_per_step=4 * cfg["vocab"]),
+            gpu_launches=launches_per_step * K, clocks=clocks)
+        print(json.dumps(line))
+    d.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

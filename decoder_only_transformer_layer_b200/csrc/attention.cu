@@ -1,0 +1,671 @@
+// Causal GQA attention over a paged bf16 KV cache, decode and chunked prefill.
+//
+// What it computes (ANEDVD src/engine.zig: ropeAndCache, cpu.attentionDecode,
+// cpu.attentionPrefill; frink_models decoder.rs: gqa_attention / the CUDA
+// gqa_decode kernel; cortiq_engine pipeline.rs: attn_scale = 1/sqrt(head_dim)):
+//   q head h reads kv head g = h / (nq / nkv); the query at position p attends
+//   cache rows 0..p; o = sum_j softmax_j(q . k_j * scale) v_j.
+// Before attention q and the new k get an optional per-head RMSNorm (QK-norm)
+// and RoPE (half-split pairs (i, i + d/2), angle p * base^(-2i/d), evaluated in
+// fp64), and are rounded to bf16; k and v enter the cache once, at row p.
+//
+// B200 design:
+//  * decode: one CTA per (sequence, kv head, context split); the G = nq/nkv
+//    query heads of the group share one pass over the K/V pages (GQA packing
+//    into the 16 rows of an m16n8k16 tensor-core tile); 4 warps take pages in
+//    turn, each with a double-buffered cp.async page ring; online softmax in
+//    fp32 with quad shuffles; splits merged deterministically by the last CTA
+//    of each (sequence, kv head);
+//  * the softmax weights P enter the PV product as two bf16 terms (P_hi + P_lo)
+//    so that the weighted sum keeps fp32-level accuracy; Q.K is exact in fp32
+//    (both operands are the rounded bf16 values);
+//  * QK-norm, RoPE and the cache append of the new token are fused into the
+//    decode kernel: the CTA whose split holds row p writes it before reading.
+//  * prefill: the chunk's q/k/v are rotated and appended by rope_append_kernel;
+//    the attention kernel then gives each warp 16 (token, head) rows, shares
+//    64-key blocks of the cache among its 4 warps and skips fully masked pages.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dec {
+
+namespace {
+
+constexpr int kPage = 16;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// A warp transforms one head vector of D fp32 values: optional RMSNorm with weight
+// nw, optional RoPE at position pos, rounding to bf16. Lane l holds elements
+// l + 32 m; element l + 32 m (m < D/64) pairs with element l + 32 (m + D/64).
+template <int D>
+DEC_DEVINL void head_transform(const float* vals_in, bool in_bf16, const uint16_t* in_b, const float* nw,
+                               float eps, bool rope, int pos, float base, uint16_t* dst) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+    float v[E];
+#pragma unroll
+    for (int m = 0; m < E; ++m) v[m] = in_bf16 ? bf2f(in_b[lane + 32 * m]) : vals_in[lane + 32 * m];
+    if (nw) {
+        float ss = 0.f;
+#pragma unroll
+        for (int m = 0; m < E; ++m) ss = fmaf(v[m], v[m], ss);
+        ss = warp_sum(ss);
+        const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+#pragma unroll
+        for (int m = 0; m < E; ++m) v[m] = v[m] * inv * nw[lane + 32 * m];
+    }
+    if (rope) {
+#pragma unroll
+        for (int m = 0; m < E / 2; ++m) {
+            float c, s;
+            rope_cs(pos, lane + 32 * m, D, base, &c, &s);
+            const float x0 = v[m], x1 = v[m + E / 2];
+            v[m] = x0 * c - x1 * s;
+            v[m + E / 2] = x0 * s + x1 * c;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < E; ++m) dst[lane + 32 * m] = f2bf(v[m]);
+}
+
+// Online-softmax state update for one 16-key page held as two m16n8 score tiles.
+// sc[nt][0..1]: row g, keys nt*8 + 2t + {0,1}; sc[nt][2..3]: row g + 8.
+// Scores are already in log2 units; masked entries are -inf. Returns P in sc.
+DEC_DEVINL void softmax_page(float (&sc)[2][4], float (&m)[2], float (&l)[2], float (&corr)[2]) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        float mx = fmaxf(fmaxf(sc[0][2 * r], sc[0][2 * r + 1]), fmaxf(sc[1][2 * r], sc[1][2 * r + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m[r], mx);
+        if (mn == -INFINITY) {  // every key so far masked for this row
+            corr[r] = 1.f;
+            sc[0][2 * r] = sc[0][2 * r + 1] = sc[1][2 * r] = sc[1][2 * r + 1] = 0.f;
+            continue;
+        }
+        corr[r] = exp2f(m[r] - mn);
+        m[r] = mn;
+        float sum = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float p = exp2f(sc[nt][2 * r + c] - mn);
+                sc[nt][2 * r + c] = p;
+                sum += p;
+            }
+        l[r] = l[r] * corr[r] + sum;
+    }
+}
+
+// O += P V for one 16-key page: P (rows g, g+8) from sc, V page rows in shared memory
+// with row stride LD. P enters as bf16 hi + lo parts.
+template <int D, int LD>
+DEC_DEVINL void pv_page(const float (&sc)[2][4], const uint16_t* vd, float (&o)[D / 8][4]) {
+    const int lane = threadIdx.x & 31;
+    uint32_t ph[4], pl[4];
+    const float* p0 = sc[0];
+    const float* p1 = sc[1];
+    float v[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float a = v[2 * i], b = v[2 * i + 1];
+        const float ah = round_bf(a), bh = round_bf(b);
+        ph[i] = pack_bf2(ah, bh);
+        pl[i] = pack_bf2(a - ah, b - bh);
+    }
+    const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int dt2 = 0; dt2 < D / 16; ++dt2) {
+        uint32_t vb[4];
+        ldsm_x4_trans(vb, vd + key * LD + dt2 * 16 + (lane >> 4) * 8);
+        const uint32_t b0[2] = {vb[0], vb[1]}, b1[2] = {vb[2], vb[3]};
+        mma_bf16_16816(o[2 * dt2], ph, b0);
+        mma_bf16_16816(o[2 * dt2], pl, b0);
+        mma_bf16_16816(o[2 * dt2 + 1], ph, b1);
+        mma_bf16_16816(o[2 * dt2 + 1], pl, b1);
+    }
+}
+
+// S = Q K^T for one 16-key page: Q fragments qf (rows 0..15), K page rows in shared memory.
+template <int D, int LD>
+DEC_DEVINL void qk_page(const uint32_t (&qf)[D / 16][4], const uint16_t* kd, float (&sc)[2][4]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
+    const int key = (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t kb[4];
+        ldsm_x4(kb, kd + key * LD + ks * 16 + ((lane >> 3) & 1) * 8);
+        const uint32_t b0[2] = {kb[0], kb[1]}, b1[2] = {kb[2], kb[3]};
+        mma_bf16_16816(sc[0], qf[ks], b0);
+        mma_bf16_16816(sc[1], qf[ks], b1);
+    }
+}
+
+template <int D, int LD>
+DEC_DEVINL void load_q_frags(const uint16_t* qs, uint32_t (&qf)[D / 16][4]) {
+    const int lane = threadIdx.x & 31;
+    const int row = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) ldsm_x4(qf[ks], qs + row * LD + ks * 16 + (lane >> 4) * 8);
+}
+
+// Copy one page (16 rows x D) of K and V of kv head g into padded shared rows (one warp).
+template <int D, int LD>
+DEC_DEVINL void load_page_warp(const uint16_t* kpool, const uint16_t* vpool, int phys, int nkv, int g,
+                               uint16_t* kd, uint16_t* vd) {
+    const int lane = threadIdx.x & 31;
+    const size_t base = ((size_t)phys * nkv + g) * kPage * D;
+    constexpr int CH = kPage * D / 8;  // 16-byte chunks per page
+#pragma unroll
+    for (int c = lane; c < CH; c += 32) {
+        const int row = c / (D / 8), col = (c % (D / 8)) * 8;
+        cp_async16(kd + row * LD + col, kpool + base + row * D + col);
+        cp_async16(vd + row * LD + col, vpool + base + row * D + col);
+    }
+    cp_async_commit();
+}
+
+// ================================================================== decode
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
+    constexpr int LD = D + 8;
+    constexpr int PAGE = kPage * LD;
+    __shared__ __align__(16) uint16_t qs[16 * LD];
+    __shared__ float wm[4][16], wl[4][16];
+    __shared__ int ticket_s;
+    extern __shared__ __align__(16) uint8_t dyn[];
+    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [4 warps][2 bufs][K,V][16][LD]
+
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int G = a.nq / a.nkv;
+    pdl_trigger();
+    pdl_wait();
+
+    const int p = a.pos[b];
+    const int n = p + 1;
+    const int np = (n + kPage - 1) / kPage;
+    const int pps = (np + a.splits - 1) / a.splits;
+    const int pg0 = s * pps, pg1 = min(np, pg0 + pps);
+    const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
+    const bool has_last = pg0 < pg1 && pg1 == np;
+    const float sl2 = a.scale * kLog2e;
+
+    if (pg0 < pg1) {
+        // ---- q tile of the group (rows >= G are zero); the split holding row p appends it
+        for (int r = warp; r < 16; r += 4) {
+            uint16_t* dst = qs + r * LD;
+            if (r < G) {
+                const int h = g * G + r;
+                if (a.qkv)
+                    head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)h * D, false, nullptr, a.q_norm, a.eps,
+                                      a.rope, p, a.rope_base, dst);
+                else
+                    head_transform<D>(nullptr, true, a.q_bf + ((size_t)b * a.nq + h) * D, nullptr, a.eps, a.rope, p,
+                                      a.rope_base, dst);
+            } else {
+                for (int i = lane; i < D; i += 32) dst[i] = 0;
+            }
+        }
+        const bool have_new = a.qkv != nullptr || a.k_new != nullptr;
+        if (has_last && have_new && warp < 2) {
+            const int phys = bt[p / kPage];
+            const size_t off = (((size_t)phys * a.nkv + g) * kPage + (p % kPage)) * D;
+            if (warp == 0) {  // k: QK-norm, RoPE, bf16
+                if (a.qkv)
+                    head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + g) * D, false, nullptr, a.k_norm,
+                                      a.eps, a.rope, p, a.rope_base, a.k_pool + off);
+                else
+                    head_transform<D>(nullptr, true, a.k_new + ((size_t)b * a.nkv + g) * D, nullptr, a.eps, a.rope, p,
+                                      a.rope_base, a.k_pool + off);
+            } else {  // v: bf16 only
+                if (a.qkv)
+                    head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + a.nkv + g) * D, false, nullptr,
+                                      nullptr, a.eps, false, p, a.rope_base, a.v_pool + off);
+                else
+                    head_transform<D>(nullptr, true, a.v_new + ((size_t)b * a.nkv + g) * D, nullptr, a.eps, false, p,
+                                      a.rope_base, a.v_pool + off);
+            }
+        }
+        __syncthreads();  // q tile ready; the appended row is visible to the block's cp.async reads
+
+        uint32_t qf[D / 16][4];
+        load_q_frags<D, LD>(qs, qf);
+
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+        float o[D / 8][4];
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+        uint16_t* wbuf = kvbuf + (size_t)warp * 4 * PAGE;
+        int pg = pg0 + warp, buf = 0;
+        if (pg < pg1) load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg], a.nkv, g, wbuf, wbuf + PAGE);
+        const int t4 = lane & 3;
+        for (; pg < pg1; pg += 4) {
+            const int nxt = pg + 4;
+            if (nxt < pg1) {
+                uint16_t* nb = wbuf + (buf ^ 1) * 2 * PAGE;
+                load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[nxt], a.nkv, g, nb, nb + PAGE);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncwarp();
+            const uint16_t* kd = wbuf + buf * 2 * PAGE;
+            float sc[2][4];
+            qk_page<D, LD>(qf, kd, sc);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int key = pg * kPage + nt * 8 + 2 * t4 + (c & 1);
+                    sc[nt][c] = key < n ? sc[nt][c] * sl2 : -INFINITY;
+                }
+            float corr[2];
+            softmax_page(sc, m, l, corr);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                o[i][0] *= corr[0];
+                o[i][1] *= corr[0];
+                o[i][2] *= corr[1];
+                o[i][3] *= corr[1];
+            }
+            pv_page<D, LD>(sc, kd + PAGE, o);
+            __syncwarp();
+            buf ^= 1;
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+            l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+        }
+
+        // ---- merge the 4 warps of the CTA through shared memory
+        __syncthreads();  // page buffers are free
+        float* wo = reinterpret_cast<float*>(kvbuf);  // [4][16][D]
+        const int gr = lane >> 2;
+        if (t4 == 0) {
+            wm[warp][gr] = m[0];
+            wm[warp][gr + 8] = m[1];
+            wl[warp][gr] = l[0];
+            wl[warp][gr + 8] = l[1];
+        }
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            float* r0 = wo + ((size_t)warp * 16 + gr) * D + i * 8 + 2 * t4;
+            float* r1 = wo + ((size_t)warp * 16 + gr + 8) * D + i * 8 + 2 * t4;
+            r0[0] = o[i][0];
+            r0[1] = o[i][1];
+            r1[0] = o[i][2];
+            r1[1] = o[i][3];
+        }
+        __syncthreads();
+        for (int idx = tid; idx < G * D; idx += 128) {
+            const int r = idx / D, c = idx % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][r]);
+            float L = 0.f, O = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                if (wm[w][r] == -INFINITY) continue;
+                const float f = exp2f(wm[w][r] - M);
+                L += f * wl[w][r];
+                O += f * wo[((size_t)w * 16 + r) * D + c];
+            }
+            const int h = g * G + r;
+            if (a.splits == 1) {
+                a.out[(size_t)b * a.nq * D + (size_t)h * D + c] = f2bf(O / L);
+            } else {
+                float* pp = a.part + (((size_t)b * a.nq + h) * a.splits + s) * (D + 2);
+                pp[c] = O;
+                if (c == 0) {
+                    pp[D] = M;
+                    pp[D + 1] = L;
+                }
+            }
+        }
+    } else if (a.splits > 1) {
+        for (int idx = tid; idx < G; idx += 128) {
+            float* pp = a.part + (((size_t)b * a.nq + g * G + idx) * a.splits + s) * (D + 2);
+            pp[D] = -INFINITY;
+            pp[D + 1] = 0.f;
+        }
+    }
+    if (a.splits == 1) return;
+
+    // ---- the last CTA of (b, g) merges the splits in split order
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) ticket_s = atomicAdd(&a.counters[b * a.nkv + g], 1);
+    __syncthreads();
+    if (ticket_s != a.splits - 1) return;
+    __threadfence();
+    for (int idx = tid; idx < G * D; idx += 128) {
+        const int r = idx / D, c = idx % D;
+        const int h = g * G + r;
+        const float* pp = a.part + ((size_t)b * a.nq + h) * a.splits * (D + 2);
+        float M = -INFINITY;
+        for (int z = 0; z < a.splits; ++z) M = fmaxf(M, __ldcg(pp + (size_t)z * (D + 2) + D));
+        float L = 0.f, O = 0.f;
+        for (int z = 0; z < a.splits; ++z) {
+            const float mz = __ldcg(pp + (size_t)z * (D + 2) + D);
+            if (mz == -INFINITY) continue;
+            const float f = exp2f(mz - M);
+            L += f * __ldcg(pp + (size_t)z * (D + 2) + D + 1);
+            O += f * __ldcg(pp + (size_t)z * (D + 2) + c);
+        }
+        a.out[(size_t)b * a.nq * D + (size_t)h * D + c] = f2bf(O / L);
+    }
+    if (tid == 0) a.counters[b * a.nkv + g] = 0;
+}
+
+// ================================================================== prefill: rotate + append
+
+template <int D>
+__global__ void __launch_bounds__(128) rope_append_kernel(RopeAppendArgs a) {
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    pdl_trigger();
+    pdl_wait();
+    const int p = a.pos0 + t;
+    const float* row = a.qkv + (size_t)t * a.ld_qkv;
+    const int phys = a.block_row[p / kPage];
+    const int slot = p % kPage;
+    const int nh = a.nq + 2 * a.nkv;
+    for (int hh = warp; hh < nh; hh += 4) {
+        if (hh < a.nq) {
+            head_transform<D>(row + (size_t)hh * D, false, nullptr, a.q_norm, a.eps, true, p, a.rope_base,
+                              a.q_out + ((size_t)t * a.nq + hh) * D);
+        } else if (hh < a.nq + a.nkv) {
+            const int j = hh - a.nq;
+            head_transform<D>(row + (size_t)hh * D, false, nullptr, a.k_norm, a.eps, true, p, a.rope_base,
+                              a.k_pool + (((size_t)phys * a.nkv + j) * kPage + slot) * D);
+        } else {
+            const int j = hh - a.nq - a.nkv;
+            head_transform<D>(row + (size_t)hh * D, false, nullptr, nullptr, a.eps, false, p, a.rope_base,
+                              a.v_pool + (((size_t)phys * a.nkv + j) * kPage + slot) * D);
+        }
+    }
+}
+
+// ================================================================== prefill attention
+
+constexpr int kPrefRows = 64;   // (token, head) rows per CTA: 4 warps x 16
+constexpr int kPrefKeys = 64;   // keys per shared block (4 pages)
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_prefill_kernel(AttnPrefillArgs a) {
+    constexpr int LD = D + 8;
+    extern __shared__ __align__(16) uint8_t dyn[];
+    uint16_t* qsm = reinterpret_cast<uint16_t*>(dyn);   // [4][16][LD]
+    uint16_t* kb = qsm + 4 * 16 * LD;                   // [2][64][LD]
+    uint16_t* vb = kb + 2 * kPrefKeys * LD;             // [2][64][LD]
+    __shared__ int ticket_s;
+
+    const int qb = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+    const int G = a.nq / a.nkv;
+    const int R = a.T * G;
+    pdl_trigger();
+    pdl_wait();
+
+    const int rbase = qb * kPrefRows;
+    const int t_last = min(a.T - 1, (rbase + kPrefRows - 1) / G);
+    const int n_cta = a.pos0 + t_last + 1;  // keys any row of this CTA may see
+    const int np = (n_cta + kPage - 1) / kPage;
+    const int pps = (np + a.splits - 1) / a.splits;
+    const int pg0 = s * pps, pg1 = min(np, pg0 + pps);
+
+    // this warp's rows
+    const int r0 = rbase + warp * 16;
+    const int gr = lane >> 2, t4 = lane & 3;
+    const int ra = r0 + gr, rb2 = r0 + gr + 8;  // rows held by this thread
+    const int lim_a = ra < R ? a.pos0 + ra / G : -1;
+    const int lim_b = rb2 < R ? a.pos0 + rb2 / G : -1;
+    const int warp_max_row = min(R - 1, r0 + 15);
+    const int warp_lim = r0 < R ? a.pos0 + warp_max_row / G : -1;
+
+    // q rows -> shared -> fragments
+    uint16_t* qw = qsm + warp * 16 * LD;
+    for (int i = lane; i < 16 * (D / 8); i += 32) {
+        const int rr = i / (D / 8), col = (i % (D / 8)) * 8;
+        const int r = r0 + rr;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < R) {
+            const int t = r / G, h = g * G + r % G;
+            v = *reinterpret_cast<const uint4*>(a.q + ((size_t)t * a.nq + h) * D + col);
+        }
+        *reinterpret_cast<uint4*>(qw + rr * LD + col) = v;
+    }
+    __syncwarp();
+    uint32_t qf[D / 16][4];
+    load_q_frags<D, LD>(qw, qf);
+
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    const float sl2 = a.scale * kLog2e;
+
+    auto load_block = [&](int blk_pg, int buf) {
+        uint16_t* kd = kb + buf * kPrefKeys * LD;
+        uint16_t* vd = vb + buf * kPrefKeys * LD;
+        constexpr int CH = kPrefKeys * D / 8;
+        for (int c = tid; c < CH; c += 128) {
+            const int key = c / (D / 8), col = (c % (D / 8)) * 8;
+            const int pg = blk_pg + key / kPage;
+            if (pg < pg1) {
+                const int phys = a.block_row[pg];
+                const size_t off = (((size_t)phys * a.nkv + g) * kPage + key % kPage) * D + col;
+                cp_async16(kd + key * LD + col, a.k_pool + off);
+                cp_async16(vd + key * LD + col, a.v_pool + off);
+            }
+        }
+        cp_async_commit();
+    };
+
+    const int kpp = kPrefKeys / kPage;
+    int buf = 0;
+    if (pg0 < pg1) load_block(pg0, 0);
+    for (int bp = pg0; bp < pg1; bp += kpp) {
+        if (bp + kpp < pg1) {
+            load_block(bp + kpp, buf ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const uint16_t* kd = kb + buf * kPrefKeys * LD;
+        const uint16_t* vd = vb + buf * kPrefKeys * LD;
+        for (int pi = 0; pi < kpp; ++pi) {
+            const int pg = bp + pi;
+            if (pg >= pg1 || pg * kPage > warp_lim) break;  // fully masked for this warp
+            float sc[2][4];
+            qk_page<D, LD>(qf, kd + pi * kPage * LD, sc);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int key = pg * kPage + nt * 8 + 2 * t4 + (c & 1);
+                    const int lim = c < 2 ? lim_a : lim_b;
+                    sc[nt][c] = key <= lim ? sc[nt][c] * sl2 : -INFINITY;
+                }
+            float corr[2];
+            softmax_page(sc, m, l, corr);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                o[i][0] *= corr[0];
+                o[i][1] *= corr[0];
+                o[i][2] *= corr[1];
+                o[i][3] *= corr[1];
+            }
+            pv_page<D, LD>(sc, vd + pi * kPage * LD, o);
+        }
+        __syncthreads();  // buffer reuse
+        buf ^= 1;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+    }
+
+    // ---- write rows (or split partials)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int r = hr == 0 ? ra : rb2;
+        if (r >= R) continue;
+        const int t = r / G, h = g * G + r % G;
+        if (a.splits == 1) {
+            const float inv = 1.0f / l[hr];
+            uint16_t* dst = a.out + (size_t)t * a.nq * D + (size_t)h * D;
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                dst[i * 8 + 2 * t4] = f2bf(o[i][2 * hr] * inv);
+                dst[i * 8 + 2 * t4 + 1] = f2bf(o[i][2 * hr + 1] * inv);
+            }
+        } else {
+            float* pp = a.part + ((size_t)s * a.T * a.nq + (size_t)t * a.nq + h) * (D + 2);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                pp[i * 8 + 2 * t4] = o[i][2 * hr];
+                pp[i * 8 + 2 * t4 + 1] = o[i][2 * hr + 1];
+            }
+            if (t4 == 0) {
+                pp[D] = m[hr];
+                pp[D + 1] = l[hr];
+            }
+        }
+    }
+    if (a.splits == 1) return;
+
+    __threadfence();
+    __syncthreads();
+    const int cidx = qb * a.nkv + g;
+    if (tid == 0) ticket_s = atomicAdd(&a.counters[cidx], 1);
+    __syncthreads();
+    if (ticket_s != a.splits - 1) return;
+    __threadfence();
+    const int nrows = min(kPrefRows, R - rbase);
+    for (int idx = tid; idx < nrows * D; idx += 128) {
+        const int r = rbase + idx / D, c = idx % D;
+        const int t = r / G, h = g * G + r % G;
+        const size_t row = (size_t)t * a.nq + h;
+        float M = -INFINITY;
+        for (int z = 0; z < a.splits; ++z)
+            M = fmaxf(M, __ldcg(a.part + ((size_t)z * a.T * a.nq + row) * (D + 2) + D));
+        float L = 0.f, O = 0.f;
+        for (int z = 0; z < a.splits; ++z) {
+            const float* pp = a.part + ((size_t)z * a.T * a.nq + row) * (D + 2);
+            const float mz = __ldcg(pp + D);
+            if (mz == -INFINITY) continue;
+            const float f = exp2f(mz - M);
+            L += f * __ldcg(pp + D + 1);
+            O += f * __ldcg(pp + c);
+        }
+        a.out[(size_t)t * a.nq * D + (size_t)h * D + c] = f2bf(O / L);
+    }
+    if (tid == 0) a.counters[cidx] = 0;
+}
+
+template <typename K, typename Args>
+cudaError_t launch_ex(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, const Args& args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, args);
+}
+
+}  // namespace
+
+int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms) {
+    const int ctas = B * nkv;
+    int s = (2 * num_sms + ctas - 1) / ctas;
+    const int pages = (max_ctx + kPage - 1) / kPage;
+    const int max_s = (pages + 3) / 4;  // keep >= 4 pages per split
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    return s;
+}
+
+cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
+    const dim3 grid(a.splits, a.nkv, a.B);
+    if (a.d == 128) {
+        const size_t smem = (size_t)4 * 4 * kPage * (128 + 8) * 2;
+        cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_ex(attn_decode_kernel<128>, grid, dim3(128), smem, st, pdl, a);
+    }
+    if (a.d == 64) {
+        const size_t smem = (size_t)4 * 4 * kPage * (64 + 8) * 2 > (size_t)4 * 16 * 64 * 4
+                                ? (size_t)4 * 4 * kPage * (64 + 8) * 2
+                                : (size_t)4 * 16 * 64 * 4;
+        cudaError_t e =
+            cudaFuncSetAttribute(attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_ex(attn_decode_kernel<64>, grid, dim3(128), smem, st, pdl, a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t rope_append_launch(const RopeAppendArgs& a, cudaStream_t st, bool pdl) {
+    if (a.T <= 0) return cudaSuccess;
+    if (a.d == 128) return launch_ex(rope_append_kernel<128>, dim3(a.T), dim3(128), 0, st, pdl, a);
+    if (a.d == 64) return launch_ex(rope_append_kernel<64>, dim3(a.T), dim3(128), 0, st, pdl, a);
+    return cudaErrorInvalidValue;
+}
+
+int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms) {
+    const int G = nq / nkv;
+    const int qblocks = (T * G + kPrefRows - 1) / kPrefRows;
+    const int ctas = qblocks * nkv;
+    int s = (2 * num_sms + ctas - 1) / ctas;
+    const int blocks = (ctx + kPrefKeys - 1) / kPrefKeys;
+    if (s > blocks) s = blocks;
+    if (s < 1) s = 1;
+    return s;
+}
+
+size_t attn_prefill_part_floats(int T, int nq, int d, int splits) {
+    return splits > 1 ? (size_t)splits * T * nq * (d + 2) : 0;
+}
+
+cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl) {
+    const int G = a.nq / a.nkv;
+    const int qblocks = (a.T * G + kPrefRows - 1) / kPrefRows;
+    const dim3 grid(qblocks, a.nkv, a.splits);
+    if (a.d == 128) {
+        const size_t smem = ((size_t)4 * 16 + 4 * kPrefKeys) * (128 + 8) * 2;
+        cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_ex(attn_prefill_kernel<128>, grid, dim3(128), smem, st, pdl, a);
+    }
+    if (a.d == 64) {
+        const size_t smem = ((size_t)4 * 16 + 4 * kPrefKeys) * (64 + 8) * 2;
+        cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_ex(attn_prefill_kernel<64>, grid, dim3(128), smem, st, pdl, a);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dec

@@ -1,0 +1,920 @@
+// C ABI of the decoder-layer library: context, weights, paged KV cache, and the
+// two orchestrated paths (chunked prefill, batched decode) plus the standalone
+// hot-path entry points. Every step of the math runs in the kernels of this
+// library; the host side only validates, allocates pages and launches.
+//
+// Interface follows ANEDVD src/engine.zig (Engine.init / forward / prefill /
+// reset / deinit, ContextOverflow), frink_models decoder.rs (gqa_attention,
+// MultiSeqKv) and cortiq_engine pipeline.rs (each token forwarded once and
+// entered into the KV cache once; empty input refused).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/dec_api.h"
+#include "kernels.h"
+
+using namespace dec;
+
+namespace {
+
+thread_local std::string g_err;
+
+dec_status fail(dec_status s, const std::string& msg) {
+    g_err = msg;
+    return s;
+}
+
+#define CUDA_TRY(expr)                                                                          \
+    do {                                                                                        \
+        cudaError_t e_ = (expr);                                                                \
+        if (e_ != cudaSuccess)                                                                  \
+            return fail(DEC_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_));      \
+    } while (0)
+
+template <typename T>
+cudaError_t dmalloc(T** p, size_t count) {
+    if (count == 0) count = 1;
+    return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
+}
+
+bool is_host_ptr(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return true;
+    }
+    return at.type == cudaMemoryTypeHost || at.type == cudaMemoryTypeUnregistered;
+}
+
+struct LayerDev {
+    float *attn_norm = nullptr, *ffn_norm = nullptr, *bqkv = nullptr, *q_norm = nullptr, *k_norm = nullptr;
+    uint16_t *wqkv = nullptr, *wo = nullptr, *wgu = nullptr, *wdown = nullptr;
+    uint16_t *wrouter = nullptr, *egu = nullptr, *edown = nullptr, *sgu = nullptr, *sdown = nullptr;
+    float* sgate_vec = nullptr;
+    uint16_t *k_pool = nullptr, *v_pool = nullptr;
+};
+
+}  // namespace
+
+struct dec_ctx {
+    dec_config c{};
+    int device = 0, num_sms = 148, smem_cap = 0;
+    cudaStream_t stream = nullptr;  // stream all work is enqueued on
+    cudaStream_t user = nullptr;    // the caller's stream
+    bool bridge = false;            // caller gave the legacy default stream: own stream + events
+    cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+    int qd = 0, kvd = 0, qkv_rows = 0, max_pages = 0, n_pages = 0;
+    int max_tok = 0;  // rows of the per-step buffers: max(max_batch, prefill_chunk)
+    std::vector<LayerDev> L;
+    uint16_t *embed = nullptr, *head = nullptr;
+    float* final_norm = nullptr;
+    // paging
+    std::vector<int> free_pages;
+    std::vector<std::vector<int>> seq_pages;
+    std::vector<int> seq_len;
+    std::vector<int32_t> h_bt;
+    int32_t* d_bt = nullptr;
+    // step buffers
+    int32_t *d_tok = nullptr, *d_pos = nullptr, *d_argmax = nullptr;
+    float *x = nullptr, *qkv = nullptr, *logits = nullptr;
+    uint16_t *xn = nullptr, *qrot = nullptr, *attn = nullptr, *act = nullptr;
+    float* attn_part = nullptr;
+    int* attn_cnt = nullptr;
+    size_t attn_part_floats = 0;
+    int attn_cnt_n = 0;
+    float* gemm_ws = nullptr;
+    size_t gemm_ws_n = 0;
+    int* gemm_cnt = nullptr;
+    int gemm_cnt_n = 0;
+    int* d_err = nullptr;
+    int32_t* h_stage = nullptr;  // pinned: tokens, positions, block rows
+    int* h_err = nullptr;
+    int act_cols = 0;
+    int decode_splits = 1;
+    std::map<int, cudaGraphExec_t> graphs;
+    int last_rows = 0;
+    bool last_was_step = false;
+};
+
+namespace {
+
+// ----------------------------------------------------------------- validation
+
+dec_status check_config(const dec_config* c) {
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "config is NULL");
+    if (c->hidden <= 0 || c->layers <= 0 || c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->vocab <= 0)
+        return fail(DEC_ERR_INVALID_ARG, "hidden, layers, heads and vocab must be positive");
+    if (c->n_q_heads % c->n_kv_heads != 0) return fail(DEC_ERR_INVALID_ARG, "n_q_heads % n_kv_heads != 0");
+    if (c->n_q_heads / c->n_kv_heads > 16) return fail(DEC_ERR_UNSUPPORTED, "more than 16 q heads per kv head");
+    if (c->head_dim != 64 && c->head_dim != 128) return fail(DEC_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (c->hidden % 8 != 0) return fail(DEC_ERR_UNSUPPORTED, "hidden must be a multiple of 8");
+    if (c->page_size != 16) return fail(DEC_ERR_UNSUPPORTED, "page_size must be 16");
+    if (c->max_batch <= 0 || c->max_context <= 0 || c->prefill_chunk <= 0)
+        return fail(DEC_ERR_INVALID_ARG, "max_batch, max_context and prefill_chunk must be positive");
+    if (c->n_experts > 0) return fail(DEC_ERR_UNSUPPORTED, "MoE layers are not enabled in this build");
+    if (c->ffn_inter <= 0 || c->ffn_inter % 8 != 0)
+        return fail(DEC_ERR_UNSUPPORTED, "ffn_inter must be a positive multiple of 8");
+    if (!(c->rms_eps > 0.f)) return fail(DEC_ERR_INVALID_ARG, "rms_eps must be positive");
+    return DEC_OK;
+}
+
+cudaError_t copy_in(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+    if (!src) return cudaErrorInvalidValue;
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, st);
+}
+
+// Interleave rows of gate [rows][h] and up [rows][h] into dst [2*rows][h]: row 2j = gate j, 2j+1 = up j.
+cudaError_t interleave_in(uint16_t* dst, const void* gate, const void* up, size_t rows, int h, cudaStream_t st) {
+    if (!gate || !up) return cudaErrorInvalidValue;
+    const size_t rb = (size_t)h * 2;
+    cudaError_t e = cudaMemcpy2DAsync(dst, 2 * rb, gate, rb, rb, rows, cudaMemcpyDefault, st);
+    if (e != cudaSuccess) return e;
+    return cudaMemcpy2DAsync(reinterpret_cast<uint8_t*>(dst) + rb, 2 * rb, up, rb, rb, rows, cudaMemcpyDefault, st);
+}
+
+// ----------------------------------------------------------------- projections
+
+// y = W x for `n` token rows: GEMV when n is small, tcgen05 GEMM otherwise.
+struct Proj {
+    const uint16_t* W;
+    int M, K;
+};
+
+dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, const float* xr, const float* g,
+                    const uint16_t* xb, float* y, int ldy, const float* bias, uint16_t* act, int ldact,
+                    cudaStream_t st) {
+    if (n <= 8 && gemv_fits(n, p.K, c->smem_cap)) {
+        GemvArgs a{};
+        a.W = p.W;
+        a.N = p.M;
+        a.K = p.K;
+        a.B = n;
+        a.xb = fused_norm ? nullptr : xb;
+        a.xr = fused_norm ? xr : nullptr;
+        a.g = g;
+        a.eps = c->c.rms_eps;
+        a.ldx = p.K;
+        a.y = y;
+        a.ldy = ldy;
+        a.bias = bias;
+        a.act = act;
+        a.ldact = ldact;
+        a.err = c->d_err;
+        a.smem_cap = c->smem_cap;
+        const int ge = epi == GEMM_STORE ? GEMV_STORE : epi == GEMM_RESID ? GEMV_RESID : GEMV_SWIGLU;
+        CUDA_TRY(gemv_launch(a, ge, st, c->num_sms, true));
+        return DEC_OK;
+    }
+    const uint16_t* in = xb;
+    if (fused_norm) {
+        CUDA_TRY(rmsnorm_launch(xr, g, n, p.K, c->c.rms_eps, c->xn, st, true));
+        in = c->xn;
+    }
+    GemmPlan plan;
+    CUDA_TRY(gemm_plan(&plan, p.W, p.M, p.K, in, n, c->num_sms));
+    if (gemm_ws_floats(plan) > c->gemm_ws_n || gemm_tiles(plan) > c->gemm_cnt_n)
+        return fail(DEC_ERR_UNSUPPORTED, "GEMM workspace too small for this shape");
+    GemmArgs a{};
+    a.epi = epi;
+    a.y = y;
+    a.ldy = ldy;
+    a.bias = bias;
+    a.act = act;
+    a.ldact = ldact;
+    a.ws = c->gemm_ws;
+    a.counters = c->gemm_cnt;
+    a.err = c->d_err;
+    CUDA_TRY(gemm_launch(plan, a, st, true));
+    return DEC_OK;
+}
+
+// ----------------------------------------------------------------- one forward over n token rows
+
+// Decode: n = B sequences, one token each, positions in d_pos; attention reads the
+// per-sequence block table. Prefill: n tokens of one sequence at pos0..pos0+n-1.
+dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cudaStream_t st) {
+    const dec_config& k = c->c;
+    const int h = k.hidden, d = k.head_dim;
+    const float scale = 1.0f / sqrtf((float)d);
+    for (int li = 0; li < k.layers; ++li) {
+        LayerDev& L = c->L[li];
+        // attention input norm + fused QKV (+bias)
+        dec_status s = run_proj(c, {L.wqkv, c->qkv_rows, h}, n, GEMM_STORE, true, c->x, L.attn_norm, nullptr, c->qkv,
+                                c->qkv_rows, L.bqkv, nullptr, 0, st);
+        if (s != DEC_OK) return s;
+        if (decode) {
+            AttnDecodeArgs a{};
+            a.qkv = c->qkv;
+            a.ld_qkv = c->qkv_rows;
+            a.q_norm = L.q_norm;
+            a.k_norm = L.k_norm;
+            a.eps = k.rms_eps;
+            a.rope = 1;
+            a.rope_base = k.rope_base;
+            a.k_pool = L.k_pool;
+            a.v_pool = L.v_pool;
+            a.block_table = c->d_bt;
+            a.max_pages = c->max_pages;
+            a.pos = c->d_pos;
+            a.B = n;
+            a.nq = k.n_q_heads;
+            a.nkv = k.n_kv_heads;
+            a.d = d;
+            a.scale = scale;
+            a.splits = c->decode_splits;
+            a.part = c->attn_part;
+            a.counters = c->attn_cnt;
+            a.out = c->attn;
+            a.err = c->d_err;
+            CUDA_TRY(attn_decode_launch(a, st, true));
+        } else {
+            RopeAppendArgs r{};
+            r.qkv = c->qkv;
+            r.ld_qkv = c->qkv_rows;
+            r.q_norm = L.q_norm;
+            r.k_norm = L.k_norm;
+            r.eps = k.rms_eps;
+            r.rope_base = k.rope_base;
+            r.T = n;
+            r.pos0 = pos0;
+            r.nq = k.n_q_heads;
+            r.nkv = k.n_kv_heads;
+            r.d = d;
+            r.q_out = c->qrot;
+            r.k_pool = L.k_pool;
+            r.v_pool = L.v_pool;
+            r.block_row = c->d_bt + (size_t)seq * c->max_pages;
+            CUDA_TRY(rope_append_launch(r, st, true));
+            AttnPrefillArgs a{};
+            a.q = c->qrot;
+            a.k_pool = L.k_pool;
+            a.v_pool = L.v_pool;
+            a.block_row = r.block_row;
+            a.T = n;
+            a.pos0 = pos0;
+            a.nq = k.n_q_heads;
+            a.nkv = k.n_kv_heads;
+            a.d = d;
+            a.scale = scale;
+            a.splits = attn_prefill_splits(n, k.n_q_heads, k.n_kv_heads, pos0 + n, c->num_sms);
+            while (a.splits > 1 && attn_prefill_part_floats(n, k.n_q_heads, d, a.splits) > c->attn_part_floats)
+                --a.splits;
+            a.part = c->attn_part;
+            a.counters = c->attn_cnt;
+            a.out = c->attn;
+            a.err = c->d_err;
+            CUDA_TRY(attn_prefill_launch(a, st, true));
+        }
+        // o_proj + residual
+        s = run_proj(c, {L.wo, h, c->qd}, n, GEMM_RESID, false, nullptr, nullptr, c->attn, c->x, h, nullptr, nullptr,
+                     0, st);
+        if (s != DEC_OK) return s;
+        // FFN: norm + fused gate/up + SiLU, then down + residual
+        s = run_proj(c, {L.wgu, 2 * k.ffn_inter, h}, n, GEMM_SWIGLU, true, c->x, L.ffn_norm, nullptr, nullptr, 0,
+                     nullptr, c->act, c->act_cols, st);
+        if (s != DEC_OK) return s;
+        s = run_proj(c, {L.wdown, h, k.ffn_inter}, n, GEMM_RESID, false, nullptr, nullptr, c->act, c->x, h, nullptr,
+                     nullptr, 0, st);
+        if (s != DEC_OK) return s;
+    }
+    return DEC_OK;
+}
+
+// Final norm + LM head for `n` rows starting at residual row `row0` -> c->logits [n][V].
+dec_status head(dec_ctx* c, int row0, int n, cudaStream_t st) {
+    const dec_config& k = c->c;
+    dec_status s = run_proj(c, {c->head, k.vocab, k.hidden}, n, GEMM_STORE, true, c->x + (size_t)row0 * k.hidden,
+                            c->final_norm, nullptr, c->logits, k.vocab, nullptr, nullptr, 0, st);
+    if (s != DEC_OK) return s;
+    CUDA_TRY(argmax_launch(c->logits, n, k.vocab, c->d_argmax, st, true));
+    return DEC_OK;
+}
+
+dec_status ensure_pages(dec_ctx* c, int seq, int upto) {
+    // allocate pages so positions [0, upto) of seq are backed
+    std::vector<int>& pg = c->seq_pages[seq];
+    const int need = (upto + 15) / 16;
+    while ((int)pg.size() < need) {
+        if (c->free_pages.empty()) return fail(DEC_ERR_PAGES_EXHAUSTED, "KV page pool exhausted");
+        const int p = c->free_pages.back();
+        c->free_pages.pop_back();
+        c->h_bt[(size_t)seq * c->max_pages + pg.size()] = p;
+        pg.push_back(p);
+    }
+    return DEC_OK;
+}
+
+dec_status upload_bt_row(dec_ctx* c, int seq, cudaStream_t st) {
+    int32_t* stg = c->h_stage + 2 * c->max_tok;
+    memcpy(stg, &c->h_bt[(size_t)seq * c->max_pages], sizeof(int32_t) * c->max_pages);
+    CUDA_TRY(cudaMemcpyAsync(c->d_bt + (size_t)seq * c->max_pages, stg, sizeof(int32_t) * c->max_pages,
+                             cudaMemcpyHostToDevice, st));
+    // the staging area is reused by the next call: make the copy complete first
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return DEC_OK;
+}
+
+dec_status deliver_logits(dec_ctx* c, float* out, int rows, cudaStream_t st) {
+    if (!out) return DEC_OK;
+    const size_t bytes = (size_t)rows * c->c.vocab * sizeof(float);
+    if (is_host_ptr(out)) {
+        CUDA_TRY(cudaMemcpyAsync(out, c->logits, bytes, cudaMemcpyDeviceToHost, st));
+        CUDA_TRY(cudaStreamSynchronize(st));
+        if (*c->h_err) return fail(DEC_ERR_TIMEOUT, "a device wait ran out of time");
+    } else {
+        CUDA_TRY(cudaMemcpyAsync(out, c->logits, bytes, cudaMemcpyDeviceToDevice, st));
+    }
+    return DEC_OK;
+}
+
+// Order the context's stream after the caller's legacy-stream work, and back.
+void enter(dec_ctx* c) {
+    if (!c->bridge) return;
+    cudaEventRecord(c->ev_in, nullptr);
+    cudaStreamWaitEvent(c->stream, c->ev_in, 0);
+}
+void leave(dec_ctx* c) {
+    if (!c->bridge) return;
+    cudaEventRecord(c->ev_out, c->stream);
+    cudaStreamWaitEvent(nullptr, c->ev_out, 0);
+}
+
+struct Scope {
+    dec_ctx* c;
+    explicit Scope(dec_ctx* c_) : c(c_) { enter(c); }
+    ~Scope() { leave(c); }
+};
+
+// ----------------------------------------------------------------- standalone scratch (per device)
+
+struct Scratch {
+    float* attn_part = nullptr;
+    size_t attn_part_n = 0;
+    int* attn_cnt = nullptr;
+    size_t attn_cnt_n = 0;
+    float* ws = nullptr;
+    size_t ws_n = 0;
+    int* cnt = nullptr;
+    size_t cnt_n = 0;
+    int* err = nullptr;
+};
+std::mutex g_scratch_mu;
+std::map<int, Scratch> g_scratch;
+
+template <typename T>
+cudaError_t grow(T** p, size_t* have, size_t need, bool zero) {
+    if (need <= *have) return cudaSuccess;
+    if (*p) cudaFree(*p);
+    *p = nullptr;
+    *have = 0;
+    cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), need * sizeof(T));
+    if (e != cudaSuccess) return e;
+    if (zero) {
+        e = cudaMemset(*p, 0, need * sizeof(T));
+        if (e != cudaSuccess) return e;
+    }
+    *have = need;
+    return cudaSuccess;
+}
+
+int device_sms() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+int device_smem_cap() {
+    int dev = 0, cap = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&cap, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    return cap - 1024;
+}
+
+}  // namespace
+
+// =================================================================== ABI
+
+extern "C" {
+
+const char* dec_last_error(void) { return g_err.c_str(); }
+
+dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t stream, dec_ctx** out) {
+    g_err.clear();
+    if (!out) return fail(DEC_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    dec_status s = check_config(cfg);
+    if (s != DEC_OK) return s;
+    if (!w || !w->embed || !w->final_norm || !w->layers) return fail(DEC_ERR_INVALID_ARG, "weights missing");
+    if (!cfg->tied_embeddings && !w->lm_head) return fail(DEC_ERR_INVALID_ARG, "lm_head missing (untied)");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    dec_ctx* c = new dec_ctx();
+    c->c = *cfg;
+    c->user = st;
+    if (st == nullptr) {
+        // CUDA graphs cannot be captured on the legacy default stream: work runs on an own
+        // stream, ordered after and before the caller's default-stream work by events.
+        c->bridge = true;
+        if (cudaStreamCreateWithFlags(&c->stream, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&c->ev_in, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&c->ev_out, cudaEventDisableTiming) != cudaSuccess) {
+            fail(DEC_ERR_CUDA, "stream/event creation failed");
+            dec_free(c);
+            return DEC_ERR_CUDA;
+        }
+        st = c->stream;
+    } else {
+        c->stream = st;
+    }
+    cudaGetDevice(&c->device);
+    c->num_sms = device_sms();
+    c->smem_cap = device_smem_cap();
+    const dec_config& k = c->c;
+    const int h = k.hidden, d = k.head_dim;
+    c->qd = k.n_q_heads * d;
+    c->kvd = k.n_kv_heads * d;
+    c->qkv_rows = c->qd + 2 * c->kvd;
+    c->max_pages = (k.max_context + 15) / 16;
+    c->n_pages = k.n_pages > 0 ? k.n_pages : k.max_batch * c->max_pages;
+    c->max_tok = std::max(k.max_batch, k.prefill_chunk);
+    c->act_cols = k.ffn_inter;
+    auto cleanup = [&](dec_status st_) {
+        dec_free(c);
+        return st_;
+    };
+#define INIT_TRY(expr)                                                                         \
+    do {                                                                                       \
+        cudaError_t e_ = (expr);                                                               \
+        if (e_ != cudaSuccess) {                                                               \
+            dec_status code_ = e_ == cudaErrorMemoryAllocation ? DEC_ERR_OOM : DEC_ERR_CUDA;   \
+            fail(code_, std::string(#expr) + ": " + cudaGetErrorString(e_));                   \
+            cudaGetLastError();                                                                \
+            return cleanup(code_);                                                             \
+        }                                                                                      \
+    } while (0)
+
+    // ---- weights
+    const size_t V = (size_t)k.vocab;
+    INIT_TRY(dmalloc(&c->embed, V * h));
+    INIT_TRY(copy_in(c->embed, w->embed, V * h * 2, st));
+    if (k.tied_embeddings) {
+        c->head = c->embed;
+    } else {
+        INIT_TRY(dmalloc(&c->head, V * h));
+        INIT_TRY(copy_in(c->head, w->lm_head, V * h * 2, st));
+    }
+    INIT_TRY(dmalloc(&c->final_norm, h));
+    INIT_TRY(copy_in(c->final_norm, w->final_norm, (size_t)h * 4, st));
+    c->L.resize(k.layers);
+    const size_t page_elems = (size_t)c->n_pages * k.n_kv_heads * 16 * d;
+    for (int li = 0; li < k.layers; ++li) {
+        const dec_layer_weights& s_ = w->layers[li];
+        LayerDev& L = c->L[li];
+        INIT_TRY(dmalloc(&L.attn_norm, h));
+        INIT_TRY(copy_in(L.attn_norm, s_.attn_norm, (size_t)h * 4, st));
+        INIT_TRY(dmalloc(&L.ffn_norm, h));
+        INIT_TRY(copy_in(L.ffn_norm, s_.ffn_norm, (size_t)h * 4, st));
+        INIT_TRY(dmalloc(&L.wqkv, (size_t)c->qkv_rows * h));
+        INIT_TRY(copy_in(L.wqkv, s_.wqkv, (size_t)c->qkv_rows * h * 2, st));
+        if (k.qkv_bias) {
+            INIT_TRY(dmalloc(&L.bqkv, c->qkv_rows));
+            INIT_TRY(copy_in(L.bqkv, s_.bqkv, (size_t)c->qkv_rows * 4, st));
+        }
+        if (k.qk_norm) {
+            INIT_TRY(dmalloc(&L.q_norm, d));
+            INIT_TRY(copy_in(L.q_norm, s_.q_norm, (size_t)d * 4, st));
+            INIT_TRY(dmalloc(&L.k_norm, d));
+            INIT_TRY(copy_in(L.k_norm, s_.k_norm, (size_t)d * 4, st));
+        }
+        INIT_TRY(dmalloc(&L.wo, (size_t)h * c->qd));
+        INIT_TRY(copy_in(L.wo, s_.wo, (size_t)h * c->qd * 2, st));
+        INIT_TRY(dmalloc(&L.wgu, (size_t)2 * k.ffn_inter * h));
+        INIT_TRY(interleave_in(L.wgu, s_.w_gate, s_.w_up, (size_t)k.ffn_inter, h, st));
+        INIT_TRY(dmalloc(&L.wdown, (size_t)h * k.ffn_inter));
+        INIT_TRY(copy_in(L.wdown, s_.w_down, (size_t)h * k.ffn_inter * 2, st));
+        INIT_TRY(dmalloc(&L.k_pool, page_elems));
+        INIT_TRY(dmalloc(&L.v_pool, page_elems));
+        INIT_TRY(cudaMemsetAsync(L.k_pool, 0, page_elems * 2, st));
+        INIT_TRY(cudaMemsetAsync(L.v_pool, 0, page_elems * 2, st));
+    }
+
+    // ---- paging
+    c->free_pages.resize(c->n_pages);
+    for (int i = 0; i < c->n_pages; ++i) c->free_pages[i] = c->n_pages - 1 - i;  // pop_back gives 0, 1, ...
+    c->seq_pages.assign(k.max_batch, {});
+    c->seq_len.assign(k.max_batch, 0);
+    c->h_bt.assign((size_t)k.max_batch * c->max_pages, 0);
+    INIT_TRY(dmalloc(&c->d_bt, (size_t)k.max_batch * c->max_pages));
+    INIT_TRY(cudaMemsetAsync(c->d_bt, 0, (size_t)k.max_batch * c->max_pages * 4, st));
+
+    // ---- step buffers
+    const int T = c->max_tok;
+    INIT_TRY(dmalloc(&c->d_tok, T));
+    INIT_TRY(dmalloc(&c->d_pos, T));
+    INIT_TRY(dmalloc(&c->d_argmax, T));
+    INIT_TRY(dmalloc(&c->x, (size_t)T * h));
+    INIT_TRY(dmalloc(&c->qkv, (size_t)T * c->qkv_rows));
+    INIT_TRY(dmalloc(&c->logits, (size_t)k.max_batch * V));
+    INIT_TRY(dmalloc(&c->xn, (size_t)T * std::max(h, c->qd)));
+    INIT_TRY(dmalloc(&c->qrot, (size_t)T * c->qd));
+    INIT_TRY(dmalloc(&c->attn, (size_t)T * c->qd));
+    INIT_TRY(dmalloc(&c->act, (size_t)T * c->act_cols));
+    INIT_TRY(dmalloc(&c->d_err, 1));
+    INIT_TRY(cudaMemsetAsync(c->d_err, 0, 4, st));
+    INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_stage), sizeof(int32_t) * (2 * T + c->max_pages + 16)));
+    INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_err), sizeof(int)));
+    *c->h_err = 0;
+
+    // attention scratch: decode splits over max_context for max_batch; prefill splits over a chunk
+    c->decode_splits = attn_decode_splits(k.max_batch, k.n_kv_heads, k.max_context, c->num_sms);
+    size_t dec_part = c->decode_splits > 1 ? (size_t)k.max_batch * k.n_q_heads * c->decode_splits * (d + 2) : 0;
+    const int pre_T = std::min(k.prefill_chunk, k.max_context);
+    const int pre_s = attn_prefill_splits(pre_T, k.n_q_heads, k.n_kv_heads, k.max_context, c->num_sms);
+    size_t pre_part = attn_prefill_part_floats(pre_T, k.n_q_heads, d, pre_s);
+    c->attn_part_floats = std::max(dec_part, pre_part);
+    INIT_TRY(dmalloc(&c->attn_part, c->attn_part_floats));
+    const int G = k.n_q_heads / k.n_kv_heads;
+    const int qblocks = (pre_T * G + 63) / 64;
+    c->attn_cnt_n = std::max(k.max_batch * k.n_kv_heads, qblocks * k.n_kv_heads);
+    INIT_TRY(dmalloc(&c->attn_cnt, c->attn_cnt_n));
+    INIT_TRY(cudaMemsetAsync(c->attn_cnt, 0, (size_t)c->attn_cnt_n * 4, st));
+
+    // GEMM split workspace: the largest projection at the largest token count that uses the GEMM
+    {
+        size_t ws = 0;
+        int cnt = 0;
+        const int Ms[5] = {c->qkv_rows, h, 2 * k.ffn_inter, h, k.vocab};
+        const int Ks[5] = {h, c->qd, h, k.ffn_inter, h};
+        // every token count a prefill chunk (tail included) or a decode batch can have
+        for (int n = 1; n <= std::max(pre_T, k.max_batch); ++n)
+            for (int j = 0; j < 5; ++j) {
+                int bn = 0;
+                const int sp = gemm_choose_splits(Ms[j], n, Ks[j], c->num_sms, &bn);
+                if (sp > 1) ws = std::max(ws, (size_t)sp * n * Ms[j]);
+                cnt = std::max(cnt, ((Ms[j] + 127) / 128) * ((n + bn - 1) / bn));
+            }
+        c->gemm_ws_n = ws;
+        c->gemm_cnt_n = cnt;
+        INIT_TRY(dmalloc(&c->gemm_ws, ws));
+        INIT_TRY(dmalloc(&c->gemm_cnt, cnt));
+        INIT_TRY(cudaMemsetAsync(c->gemm_cnt, 0, (size_t)cnt * 4, st));
+    }
+    INIT_TRY(cudaStreamSynchronize(st));
+#undef INIT_TRY
+    *out = c;
+    return DEC_OK;
+}
+
+dec_status dec_free(dec_ctx* c) {
+    if (!c) return DEC_OK;
+    for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second);
+    for (auto& L : c->L) {
+        cudaFree(L.attn_norm);
+        cudaFree(L.ffn_norm);
+        cudaFree(L.bqkv);
+        cudaFree(L.q_norm);
+        cudaFree(L.k_norm);
+        cudaFree(L.wqkv);
+        cudaFree(L.wo);
+        cudaFree(L.wgu);
+        cudaFree(L.wdown);
+        cudaFree(L.wrouter);
+        cudaFree(L.egu);
+        cudaFree(L.edown);
+        cudaFree(L.sgu);
+        cudaFree(L.sdown);
+        cudaFree(L.sgate_vec);
+        cudaFree(L.k_pool);
+        cudaFree(L.v_pool);
+    }
+    if (c->head != c->embed) cudaFree(c->head);
+    cudaFree(c->embed);
+    cudaFree(c->final_norm);
+    cudaFree(c->d_bt);
+    cudaFree(c->d_tok);
+    cudaFree(c->d_pos);
+    cudaFree(c->d_argmax);
+    cudaFree(c->x);
+    cudaFree(c->qkv);
+    cudaFree(c->logits);
+    cudaFree(c->xn);
+    cudaFree(c->qrot);
+    cudaFree(c->attn);
+    cudaFree(c->act);
+    cudaFree(c->attn_part);
+    cudaFree(c->attn_cnt);
+    cudaFree(c->gemm_ws);
+    cudaFree(c->gemm_cnt);
+    cudaFree(c->d_err);
+    if (c->h_stage) cudaFreeHost(c->h_stage);
+    if (c->h_err) cudaFreeHost(c->h_err);
+    if (c->bridge) {
+        if (c->stream) cudaStreamDestroy(c->stream);
+        if (c->ev_in) cudaEventDestroy(c->ev_in);
+        if (c->ev_out) cudaEventDestroy(c->ev_out);
+    }
+    delete c;
+    return DEC_OK;
+}
+
+dec_status dec_reset(dec_ctx* c, int32_t seq) {
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    if (seq < -1 || seq >= c->c.max_batch) return fail(DEC_ERR_INVALID_ARG, "seq out of range");
+    for (int s = 0; s < c->c.max_batch; ++s) {
+        if (seq != -1 && s != seq) continue;
+        for (int p : c->seq_pages[s]) c->free_pages.push_back(p);
+        c->seq_pages[s].clear();
+        c->seq_len[s] = 0;
+    }
+    return DEC_OK;
+}
+
+dec_status dec_seq_len(dec_ctx* c, int32_t seq, int32_t* len_out) {
+    if (!c || !len_out) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
+    if (seq < 0 || seq >= c->c.max_batch) return fail(DEC_ERR_INVALID_ARG, "seq out of range");
+    *len_out = c->seq_len[seq];
+    return DEC_OK;
+}
+
+dec_status dec_prefill(dec_ctx* c, int32_t seq, const int32_t* tokens, int32_t T, int32_t pos0, float* logits_out) {
+    g_err.clear();
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    const dec_config& k = c->c;
+    if (seq < 0 || seq >= k.max_batch) return fail(DEC_ERR_INVALID_ARG, "seq out of range");
+    if (T <= 0 || !tokens) return fail(DEC_ERR_INVALID_ARG, "empty prompt");
+    if (pos0 < 0 || (int64_t)pos0 + T > k.max_context) return fail(DEC_ERR_CONTEXT_OVERFLOW, "pos0 + T > max_context");
+    if (pos0 != c->seq_len[seq]) return fail(DEC_ERR_INVALID_ARG, "pos0 must equal the sequence length");
+    for (int i = 0; i < T; ++i)
+        if (tokens[i] < 0 || tokens[i] >= k.vocab) return fail(DEC_ERR_INVALID_ARG, "token id out of range");
+    dec_status s = ensure_pages(c, seq, pos0 + T);
+    if (s != DEC_OK) return s;
+    cudaStream_t st = c->stream;
+    Scope scope(c);
+    s = upload_bt_row(c, seq, st);
+    if (s != DEC_OK) return s;
+    const int C = k.prefill_chunk;
+    int last_rows = 0;
+    for (int done = 0; done < T; done += C) {
+        const int n = std::min(C, T - done);
+        memcpy(c->h_stage, tokens + done, sizeof(int32_t) * n);
+        CUDA_TRY(cudaMemcpyAsync(c->d_tok, c->h_stage, sizeof(int32_t) * n, cudaMemcpyHostToDevice, st));
+        CUDA_TRY(embed_launch(c->embed, c->d_tok, n, k.hidden, c->x, st, false));
+        s = forward_layers(c, n, false, seq, pos0 + done, st);
+        if (s != DEC_OK) return s;
+        last_rows = n;
+        // the staging buffer is rewritten by the next chunk
+        CUDA_TRY(cudaStreamSynchronize(st));
+    }
+    s = head(c, last_rows - 1, 1, st);
+    if (s != DEC_OK) return s;
+    c->seq_len[seq] = pos0 + T;
+    c->last_rows = 1;
+    CUDA_TRY(cudaMemcpyAsync(c->h_err, c->d_err, 4, cudaMemcpyDeviceToHost, st));
+    return deliver_logits(c, logits_out, 1, st);
+}
+
+dec_status dec_step(dec_ctx* c, const int32_t* tokens, const int32_t* pos, int32_t B, float* logits_out) {
+    g_err.clear();
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    const dec_config& k = c->c;
+    if (B <= 0 || B > k.max_batch) return fail(DEC_ERR_INVALID_ARG, "B out of range");
+    if (!tokens || !pos) return fail(DEC_ERR_INVALID_ARG, "tokens/pos NULL");
+    for (int b = 0; b < B; ++b) {
+        if (tokens[b] < 0 || tokens[b] >= k.vocab) return fail(DEC_ERR_INVALID_ARG, "token id out of range");
+        if (pos[b] < 0 || pos[b] >= k.max_context) return fail(DEC_ERR_CONTEXT_OVERFLOW, "pos >= max_context");
+        if (pos[b] != c->seq_len[b]) return fail(DEC_ERR_INVALID_ARG, "pos must equal the sequence length");
+    }
+    cudaStream_t st = c->stream;
+    Scope scope(c);
+    bool bt_dirty = false;
+    for (int b = 0; b < B; ++b) {
+        const size_t before = c->seq_pages[b].size();
+        dec_status s = ensure_pages(c, b, pos[b] + 1);
+        if (s != DEC_OK) return s;
+        if (c->seq_pages[b].size() != before) bt_dirty = true;
+    }
+    int32_t* stg = c->h_stage;
+    memcpy(stg, tokens, sizeof(int32_t) * B);
+    memcpy(stg + c->max_tok, pos, sizeof(int32_t) * B);
+    CUDA_TRY(cudaMemcpyAsync(c->d_tok, stg, sizeof(int32_t) * B, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(c->d_pos, stg + c->max_tok, sizeof(int32_t) * B, cudaMemcpyHostToDevice, st));
+    if (bt_dirty)
+        CUDA_TRY(cudaMemcpyAsync(c->d_bt, c->h_bt.data(), sizeof(int32_t) * (size_t)B * c->max_pages,
+                                 cudaMemcpyHostToDevice, st));
+
+    auto it = c->graphs.find(B);
+    if (it == c->graphs.end()) {
+        cudaGraph_t g = nullptr;
+        CUDA_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+        dec_status s = DEC_OK;
+        if (embed_launch(c->embed, c->d_tok, B, k.hidden, c->x, st, false) != cudaSuccess)
+            s = fail(DEC_ERR_CUDA, "embed launch failed");
+        if (s == DEC_OK) s = forward_layers(c, B, true, 0, 0, st);
+        if (s == DEC_OK) s = head(c, 0, B, st);
+        cudaError_t e = cudaStreamEndCapture(st, &g);
+        if (s != DEC_OK) {
+            if (g) cudaGraphDestroy(g);
+            return s;
+        }
+        if (e != cudaSuccess) return fail(DEC_ERR_CUDA, std::string("graph capture: ") + cudaGetErrorString(e));
+        cudaGraphExec_t ex = nullptr;
+        e = cudaGraphInstantiate(&ex, g, 0);
+        cudaGraphDestroy(g);
+        if (e != cudaSuccess) return fail(DEC_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
+        it = c->graphs.emplace(B, ex).first;
+    }
+    CUDA_TRY(cudaGraphLaunch(it->second, st));
+    for (int b = 0; b < B; ++b) c->seq_len[b] = pos[b] + 1;
+    c->last_rows = B;
+    CUDA_TRY(cudaMemcpyAsync(c->h_err, c->d_err, 4, cudaMemcpyDeviceToHost, st));
+    dec_status s = deliver_logits(c, logits_out, B, st);
+    if (s != DEC_OK) return s;
+    // the pinned staging area is reused by the next call
+    if (!logits_out || !is_host_ptr(logits_out)) CUDA_TRY(cudaStreamSynchronize(st));
+    return DEC_OK;
+}
+
+dec_status dec_last_argmax(dec_ctx* c, int32_t* out, int32_t B) {
+    if (!c || !out) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
+    if (B != c->last_rows) return fail(DEC_ERR_INVALID_ARG, "B differs from the last call's rows");
+    CUDA_TRY(cudaMemcpyAsync(out, c->d_argmax, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, c->stream));
+    CUDA_TRY(cudaStreamSynchronize(c->stream));
+    return DEC_OK;
+}
+
+dec_status dec_kv_write(dec_ctx* c, int32_t seq, int32_t layer, int32_t pos0, int32_t n, const void* k_,
+                        const void* v_) {
+    if (!c || !k_ || !v_) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
+    if (seq < 0 || seq >= c->c.max_batch || layer < 0 || layer >= c->c.layers || n <= 0 || pos0 < 0)
+        return fail(DEC_ERR_INVALID_ARG, "bad seq/layer/range");
+    if ((int64_t)pos0 + n > c->c.max_context) return fail(DEC_ERR_CONTEXT_OVERFLOW, "range beyond max_context");
+    dec_status s = ensure_pages(c, seq, pos0 + n);
+    if (s != DEC_OK) return s;
+    cudaStream_t st = c->stream;
+    s = upload_bt_row(c, seq, st);
+    if (s != DEC_OK) return s;
+    const size_t bytes = (size_t)n * c->kvd * 2;
+    uint16_t *dk = nullptr, *dv = nullptr;
+    CUDA_TRY(cudaMalloc(&dk, bytes));
+    CUDA_TRY(cudaMalloc(&dv, bytes));
+    cudaMemcpyAsync(dk, k_, bytes, cudaMemcpyDefault, st);
+    cudaMemcpyAsync(dv, v_, bytes, cudaMemcpyDefault, st);
+    cudaError_t e = kv_move_launch(c->L[layer].k_pool, c->L[layer].v_pool, c->d_bt + (size_t)seq * c->max_pages, pos0,
+                                   n, c->c.n_kv_heads, c->c.head_dim, dk, dv, 1, st);
+    cudaError_t e2 = cudaStreamSynchronize(st);
+    cudaFree(dk);
+    cudaFree(dv);
+    if (e != cudaSuccess || e2 != cudaSuccess) return fail(DEC_ERR_CUDA, "kv write failed");
+    c->seq_len[seq] = std::max(c->seq_len[seq], pos0 + n);
+    return DEC_OK;
+}
+
+dec_status dec_kv_read(dec_ctx* c, int32_t seq, int32_t layer, int32_t pos0, int32_t n, void* k_, void* v_) {
+    if (!c || !k_ || !v_) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
+    if (seq < 0 || seq >= c->c.max_batch || layer < 0 || layer >= c->c.layers || n <= 0 || pos0 < 0)
+        return fail(DEC_ERR_INVALID_ARG, "bad seq/layer/range");
+    if ((int64_t)pos0 + n > c->seq_len[seq]) return fail(DEC_ERR_INVALID_ARG, "range beyond the sequence length");
+    cudaStream_t st = c->stream;
+    const size_t bytes = (size_t)n * c->kvd * 2;
+    uint16_t *dk = nullptr, *dv = nullptr;
+    CUDA_TRY(cudaMalloc(&dk, bytes));
+    CUDA_TRY(cudaMalloc(&dv, bytes));
+    cudaError_t e = kv_move_launch(c->L[layer].k_pool, c->L[layer].v_pool, c->d_bt + (size_t)seq * c->max_pages, pos0,
+                                   n, c->c.n_kv_heads, c->c.head_dim, dk, dv, 0, st);
+    cudaMemcpyAsync(k_, dk, bytes, cudaMemcpyDefault, st);
+    cudaMemcpyAsync(v_, dv, bytes, cudaMemcpyDefault, st);
+    cudaError_t e2 = cudaStreamSynchronize(st);
+    cudaFree(dk);
+    cudaFree(dv);
+    if (e != cudaSuccess || e2 != cudaSuccess) return fail(DEC_ERR_CUDA, "kv read failed");
+    return DEC_OK;
+}
+
+dec_status dec_last_routes(dec_ctx* c, int32_t* idx, int32_t B) {
+    (void)idx;
+    (void)B;
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    return fail(DEC_ERR_UNSUPPORTED, "the model has no MoE layers");
+}
+
+dec_status dec_last_hidden(dec_ctx* c, float* out, int32_t B) {
+    if (!c || !out) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
+    if (B != c->last_rows && !(B == 1)) return fail(DEC_ERR_INVALID_ARG, "B differs from the last call's rows");
+    CUDA_TRY(cudaMemcpyAsync(out, c->x, sizeof(float) * (size_t)B * c->c.hidden, cudaMemcpyDeviceToHost, c->stream));
+    CUDA_TRY(cudaStreamSynchronize(c->stream));
+    return DEC_OK;
+}
+
+// ------------------------------------------------------------------ standalone
+
+dec_status gqa_decode_attn(const void* q, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                           const int32_t* block_table, int32_t max_pages, const int32_t* pos, int32_t B, int32_t nq,
+                           int32_t nkv, int32_t d, int32_t page_size, float scale, int32_t fused_rope,
+                           float rope_base, void* out, dec_stream_t stream) {
+    g_err.clear();
+    if (!q || !k_pool || !v_pool || !block_table || !pos || !out) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
+    if ((k_new == nullptr) != (v_new == nullptr)) return fail(DEC_ERR_INVALID_ARG, "k_new and v_new: both or neither");
+    if (B <= 0 || nq <= 0 || nkv <= 0 || nq % nkv != 0 || max_pages <= 0)
+        return fail(DEC_ERR_INVALID_ARG, "bad B / heads / max_pages");
+    if (nq / nkv > 16) return fail(DEC_ERR_UNSUPPORTED, "more than 16 q heads per kv head");
+    if (d != 64 && d != 128) return fail(DEC_ERR_UNSUPPORTED, "d must be 64 or 128");
+    if (page_size != 16) return fail(DEC_ERR_UNSUPPORTED, "page_size must be 16");
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    Scratch& S = g_scratch[dev];
+    const int sms = device_sms();
+    const int splits = attn_decode_splits(B, nkv, max_pages * 16, sms);
+    CUDA_TRY(grow(&S.attn_part, &S.attn_part_n, (size_t)B * nq * splits * (d + 2), false));
+    CUDA_TRY(grow(&S.attn_cnt, &S.attn_cnt_n, (size_t)B * nkv, true));
+    size_t one = 0;
+    if (!S.err) CUDA_TRY(grow(&S.err, &one, 1, true));
+    AttnDecodeArgs a{};
+    a.q_bf = static_cast<const uint16_t*>(q);
+    a.k_new = static_cast<const uint16_t*>(k_new);
+    a.v_new = static_cast<const uint16_t*>(v_new);
+    a.eps = 1e-6f;
+    a.rope = fused_rope;
+    a.rope_base = rope_base;
+    a.k_pool = static_cast<uint16_t*>(k_pool);
+    a.v_pool = static_cast<uint16_t*>(v_pool);
+    a.block_table = block_table;
+    a.max_pages = max_pages;
+    a.pos = pos;
+    a.B = B;
+    a.nq = nq;
+    a.nkv = nkv;
+    a.d = d;
+    a.scale = scale;
+    a.splits = splits;
+    a.part = S.attn_part;
+    a.counters = S.attn_cnt;
+    a.out = static_cast<uint16_t*>(out);
+    a.err = S.err;
+    CUDA_TRY(attn_decode_launch(a, reinterpret_cast<cudaStream_t>(stream), false));
+    return DEC_OK;
+}
+
+dec_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k, int32_t renorm, int32_t* idx_out,
+                          float* w_out, dec_stream_t stream) {
+    g_err.clear();
+    if (!logits || !idx_out || !w_out) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
+    if (T <= 0 || E <= 0 || k <= 0 || k > E) return fail(DEC_ERR_INVALID_ARG, "bad T / E / k");
+    if (E > 256 || k > 16) return fail(DEC_ERR_UNSUPPORTED, "E <= 256 and k <= 16");
+    CUDA_TRY(topk_launch(logits, T, E, k, renorm, idx_out, w_out, reinterpret_cast<cudaStream_t>(stream), false));
+    return DEC_OK;
+}
+
+dec_status weight_gemv(const void* W, const void* x, int32_t B, int32_t N, int32_t K, float* y, dec_stream_t stream) {
+    g_err.clear();
+    if (!W || !x || !y) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
+    if (B <= 0 || N <= 0 || K <= 0) return fail(DEC_ERR_INVALID_ARG, "B, N, K must be positive");
+    if (K % 8 != 0) return fail(DEC_ERR_UNSUPPORTED, "K must be a multiple of 8");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    Scratch& S = g_scratch[dev];
+    size_t one = 0;
+    if (!S.err) CUDA_TRY(grow(&S.err, &one, 1, true));
+    const int sms = device_sms();
+    const int cap = device_smem_cap();
+    if (B <= 8 && gemv_fits(B, K, cap)) {
+        GemvArgs a{};
+        a.W = static_cast<const uint16_t*>(W);
+        a.N = N;
+        a.K = K;
+        a.B = B;
+        a.xb = static_cast<const uint16_t*>(x);
+        a.ldx = K;
+        a.y = y;
+        a.ldy = N;
+        a.err = S.err;
+        a.smem_cap = cap;
+        CUDA_TRY(gemv_launch(a, GEMV_STORE, st, sms, false));
+        return DEC_OK;
+    }
+    GemmPlan plan;
+    CUDA_TRY(gemm_plan(&plan, static_cast<const uint16_t*>(W), N, K, static_cast<const uint16_t*>(x), B, sms));
+    CUDA_TRY(grow(&S.ws, &S.ws_n, std::max<size_t>(1, gemm_ws_floats(plan)), false));
+    CUDA_TRY(grow(&S.cnt, &S.cnt_n, (size_t)gemm_tiles(plan), true));
+    GemmArgs a{};
+    a.epi = GEMM_STORE;
+    a.y = y;
+    a.ldy = N;
+    a.ws = S.ws;
+    a.counters = S.cnt;
+    a.err = S.err;
+    CUDA_TRY(gemm_launch(plan, a, st, false));
+    return DEC_OK;
+}
+
+}  // extern "C"

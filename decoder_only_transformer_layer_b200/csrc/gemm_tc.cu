@@ -1,0 +1,352 @@
+// Tensor-core projection for prefill chunks and large decode batches:
+//   D[m][n] = sum_k A[m][k] * B[n][k],  A = weights bf16 [M][K], B = activations
+//   bf16 [N][K] (N = tokens), both K-major; stored transposed as y[n][m].
+//
+// These are the same projections as the decode GEMV (ANEDVD src/engine.zig:
+// the chunk-wide 1x1 convs of Engine.prefill; cortiq_engine pipeline.rs: the
+// chunk GEMMs of prefill_batch), used where the token count makes them a real
+// dense contraction.
+//
+// B200 design (sm_100a, tcgen05):
+//  * one 128 x BN output tile per CTA (BN = 32/64/128 tokens), split over K when
+//    the tile count would leave SMs idle; split partials are summed in split order
+//    by the last CTA of the tile (deterministic, no atomics on data);
+//  * warp 0 / lane 0 drives TMA: 128B-swizzled 64-wide K slices of A and B into a
+//    6-8 stage shared-memory ring (mbarrier complete_tx); the weight slices of
+//    the first stages are issued before griddepcontrol.wait (they do not depend
+//    on the previous kernel), the activation slices after it;
+//  * warp 1 / lane 0 issues tcgen05.mma.cta_group::1.kind::f16 (M=128, N=BN,
+//    K=16 per instruction, fp32 accumulator in TMEM) and frees each stage with
+//    tcgen05.commit;
+//  * all 4 warps read the accumulator with tcgen05.ld (warp w owns TMEM lanes
+//    32w..32w+31 = weight rows) and apply the epilogue: store (+bias), residual
+//    add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dec {
+
+namespace {
+
+constexpr int BM = 128, BK = 64;
+
+template <int BN>
+struct Cfg {
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES = BN <= 64 ? 8 : 6;
+    static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
+    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+};
+
+DEC_DEVINL uint64_t sdesc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+    d |= (uint64_t)1 << 16;                    // leading byte offset (16 B; unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                    // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+
+template <int BN>
+__host__ __device__ constexpr uint32_t idesc_bf16() {
+    return (1u << 4)                      // accumulator F32
+           | (1u << 7)                    // A BF16
+           | (1u << 10)                   // B BF16
+           | ((uint32_t)(BN >> 3) << 17)  // N
+           | ((uint32_t)(BM >> 4) << 24); // M
+}
+
+DEC_DEVINL void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+DEC_DEVINL void tma_load_2d_hint(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+        "{%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+
+DEC_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+DEC_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+DEC_DEVINL void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
+DEC_DEVINL void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+DEC_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Apply the epilogue to value v of (row, t). All lanes of the warp must call it
+// together (the SwiGLU pairing uses a shuffle).
+DEC_DEVINL void epilogue(const GemmArgs& a, int row, int t, float v) {
+    const bool ok = row < a.M && t < a.N;
+    if (a.epi == GEMM_SWIGLU) {
+        const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
+        if (ok && (row & 1) == 0) {
+            const float sg = v * (1.0f / (1.0f + expf(-v)));
+            a.act[(size_t)t * a.ldact + (row >> 1)] = f2bf(sg * partner);
+        }
+    } else if (ok) {
+        float* dst = a.y + (size_t)t * a.ldy + row;
+        if (a.epi == GEMM_RESID)
+            *dst += v;
+        else
+            *dst = v + (a.bias ? a.bias[row] : 0.f);
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(128, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+    using C = Cfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* accb = empty + C::STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+    int* ticket = reinterpret_cast<int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN, z = blockIdx.z;
+    const int nkb = (a.K + BK - 1) / BK;
+    const int kb0 = (int)((int64_t)z * nkb / a.splits), kb1 = (int)((int64_t)(z + 1) * nkb / a.splits);
+    const int nk = kb1 - kb0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accb, 1);
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
+
+    bool ok = true;
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        const uint64_t pol = policy_evict_first();
+        const int pre = nk < C::STAGES ? nk : C::STAGES;
+        for (int i = 0; i < pre; ++i) {
+            mbar_arrive_expect_tx(&full[i], C::STAGE);
+            tma_load_2d_hint(smem + i * C::STAGE, &tmA, (kb0 + i) * BK, m0, &full[i], pol);
+        }
+        pdl_wait();
+        for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, (kb0 + i) * BK, n0, &full[i]);
+        for (int i = pre; i < nk; ++i) {
+            const int s = i % C::STAGES;
+            const uint32_t u = (uint32_t)(i / C::STAGES);
+            if (!mbar_wait_bounded(&empty[s], (u & 1u) ^ 1u, a.err)) break;
+            mbar_arrive_expect_tx(&full[s], C::STAGE);
+            tma_load_2d_hint(smem + s * C::STAGE, &tmA, (kb0 + i) * BK, m0, &full[s], pol);
+            tma_load_2d(smem + s * C::STAGE + C::A_BYTES, &tmB, (kb0 + i) * BK, n0, &full[s]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_bf16<BN>();
+        const uint32_t sbase = smem_u32(smem);
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % C::STAGES;
+            const uint32_t u = (uint32_t)(i / C::STAGES);
+            if (!mbar_wait_bounded(&full[s], u & 1u, a.err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t abase = sbase + s * C::STAGE, bbase = abase + C::A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+                tc_mma(tmem, sdesc_sw128(abase + kk * 32), sdesc_sw128(bbase + kk * 32), idesc,
+                       (i > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&empty[s]);
+        }
+        tc_commit(accb);
+    }
+    if (warp != 0) pdl_wait();  // every thread passes the grid dependency before finishing
+
+    // ---------------------------------------------------- epilogue
+    __syncwarp();
+    const bool acc_ready = mbar_wait_bounded(accb, 0, a.err);
+    tc_fence_after();
+    const int row = m0 + warp * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + (uint32_t)c0, r);
+        if (!acc_ready) continue;
+        if (a.splits == 1) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) epilogue(a, row, n0 + c0 + j, __uint_as_float(r[j]));
+        } else if (row < a.M) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int t = n0 + c0 + j;
+                if (t < a.N) a.ws[((size_t)z * a.N + t) * a.M + row] = __uint_as_float(r[j]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+    (void)ok;
+    if (a.splits == 1 || !acc_ready) return;
+
+    // ---------------------------------------------------- split-K: last CTA of the tile reduces
+    __threadfence();
+    __syncthreads();
+    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+    if (threadIdx.x == 0) *ticket = atomicAdd(&a.counters[tile], 1);
+    __syncthreads();
+    if (*ticket != a.splits - 1) return;
+    __threadfence();
+    const int ncols = min(BN, a.N - n0);
+    for (int c = 0; c < ncols; ++c) {
+        const int t = n0 + c;
+        float v = 0.f;
+        if (row < a.M)
+            for (int s = 0; s < a.splits; ++s) v += __ldcg(a.ws + ((size_t)s * a.N + t) * a.M + row);
+        epilogue(a, row, t, v);
+    }
+    if (threadIdx.x == 0) a.counters[tile] = 0;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+cudaError_t encode_2d(CUtensorMap* tm, const uint16_t* base, int rows, int K, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, bool pdl) {
+    using C = Cfg<BN>;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((p.M + BM - 1) / BM, (p.N + BN - 1) / BN, p.splits);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, a);
+}
+
+}  // namespace
+
+int gemm_tiles(const GemmPlan& p) { return ((p.M + BM - 1) / BM) * ((p.N + p.bn - 1) / p.bn); }
+
+size_t gemm_ws_floats(const GemmPlan& p) { return p.splits > 1 ? (size_t)p.splits * p.N * p.M : 0; }
+
+int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn_out) {
+    const int bn = N <= 32 ? 32 : N <= 64 ? 64 : 128;
+    if (bn_out) *bn_out = bn;
+    const int tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
+    const int nkb = (K + BK - 1) / BK;
+    int best = 1;
+    double best_eff = 0.0;
+    for (int s = 1; s <= 8 && s <= nkb / 4 + 1; ++s) {
+        const int ctas = tiles * s;
+        const int waves = (ctas + num_sms - 1) / num_sms;
+        const double eff = (double)ctas / ((double)waves * num_sms);
+        if (eff > best_eff + 0.05) {
+            best_eff = eff;
+            best = s;
+        }
+        if (eff >= 0.85) break;
+    }
+    if (best > nkb) best = nkb;
+    return best;
+}
+
+cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0) return cudaErrorInvalidValue;
+    p->M = M;
+    p->N = N;
+    p->K = K;
+    p->splits = gemm_choose_splits(M, N, K, num_sms, &p->bn);
+    cudaError_t e = encode_2d(&p->tmA, A, M, K, BM);
+    if (e != cudaSuccess) return e;
+    return encode_2d(&p->tmB, B, N, K, p->bn);
+}
+
+cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl) {
+    a.M = p.M;
+    a.N = p.N;
+    a.K = p.K;
+    a.splits = p.splits;
+    switch (p.bn) {
+        case 32: return launch_bn<32>(p, a, st, pdl);
+        case 64: return launch_bn<64>(p, a, st, pdl);
+        case 128: return launch_bn<128>(p, a, st, pdl);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dec

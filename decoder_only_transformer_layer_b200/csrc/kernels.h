@@ -1,0 +1,143 @@
+// Internal launcher interface between the C ABI (dec_api.cu) and the kernels.
+// All pointers are device pointers; bf16 tensors are uint16_t bit patterns.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dec {
+
+// ----------------------------------------------------------------- GEMV (decode projections)
+
+enum GemvEpi { GEMV_STORE = 0, GEMV_RESID = 1, GEMV_SWIGLU = 2 };
+
+struct GemvArgs {
+    const uint16_t* W;  // [N][K]
+    int N, K;
+    int B, nb;          // active columns; nb = compiled column count (set by the launcher)
+    const uint16_t* xb; // bf16 input [B][ldx], or
+    const float* xr;    // fp32 residual [B][ldx] normalised in the prologue with gain g
+    const float* g;
+    float eps;
+    int ldx;
+    float* y;           // STORE: y[b*ldy+n] = acc (+bias); RESID: y[b*ldy+n] += acc
+    int ldy;
+    const float* bias;
+    uint16_t* act;      // SWIGLU: act[b*ldact + n/2] = bf16(silu(acc[even]) * acc[odd])
+    int ldact;
+    int* err;
+    int smem_cap;
+};
+
+int gemv_nb_for(int B);
+bool gemv_fits(int B, int K, int smem_cap);
+cudaError_t gemv_launch(GemvArgs a, int epi, cudaStream_t st, int num_sms, bool pdl);
+
+// ----------------------------------------------------------------- tcgen05 GEMM (prefill, large batch)
+
+enum GemmEpi { GEMM_STORE = 0, GEMM_RESID = 1, GEMM_SWIGLU = 2 };
+
+struct GemmPlan {
+    CUtensorMap tmA;  // weights [M][K], box 64 x 128
+    CUtensorMap tmB;  // activations [N][K], box 64 x BN
+    int M, N, K, bn, splits;
+};
+
+struct GemmArgs {
+    int M, N, K;      // D[M][N] = A[M][K] . B[N][K]^T, stored transposed: y[n][m]
+    int epi;
+    float* y;
+    int ldy;
+    const float* bias;
+    uint16_t* act;
+    int ldact;
+    int splits;
+    float* ws;        // split partials [splits][N][M] fp32
+    int* counters;    // [tiles], zero on entry, left zero on exit
+    int* err;
+};
+
+// Build the tensor maps for one GEMM shape (host; encodes A and B addresses).
+cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms);
+size_t gemm_ws_floats(const GemmPlan& p);
+int gemm_tiles(const GemmPlan& p);
+cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl);
+
+// ----------------------------------------------------------------- attention
+
+struct AttnDecodeArgs {
+    // query and new row: fp32 qkv rows (model path) or bf16 tensors (standalone call)
+    const float* qkv;
+    int ld_qkv;
+    const uint16_t* q_bf;   // [B][nq][d]
+    const uint16_t* k_new;  // [B][nkv][d] or null
+    const uint16_t* v_new;
+    const float* q_norm;    // [d] or null (model path only)
+    const float* k_norm;
+    float eps;
+    int rope;               // rotate q and the new k to pos
+    float rope_base;
+    uint16_t* k_pool;       // [n_pages][nkv][16][d]
+    uint16_t* v_pool;
+    const int32_t* block_table;
+    int max_pages;
+    const int32_t* pos;     // [B]
+    int B, nq, nkv, d;
+    float scale;
+    int splits;
+    float* part;            // [B][nq][splits][d+2]
+    int* counters;          // [B][nkv]
+    uint16_t* out;          // [B][nq*d]
+    int* err;
+};
+cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl);
+int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms);
+
+struct RopeAppendArgs {
+    const float* qkv;  // [T][ld]
+    int ld_qkv;
+    const float* q_norm;
+    const float* k_norm;
+    float eps;
+    float rope_base;
+    int T, pos0, nq, nkv, d;
+    uint16_t* q_out;   // [T][nq][d]
+    uint16_t* k_pool;
+    uint16_t* v_pool;
+    const int32_t* block_row;  // block table row of the sequence
+};
+cudaError_t rope_append_launch(const RopeAppendArgs& a, cudaStream_t st, bool pdl);
+
+struct AttnPrefillArgs {
+    const uint16_t* q;  // [T][nq][d] (rotated, bf16)
+    const uint16_t* k_pool;
+    const uint16_t* v_pool;
+    const int32_t* block_row;
+    int T, pos0, nq, nkv, d;
+    float scale;
+    int splits;
+    float* part;        // [splits][T*nq][d+2]
+    int* counters;      // [qblocks*nkv]
+    uint16_t* out;      // [T][nq*d]
+    int* err;
+};
+cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl);
+int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms);
+size_t attn_prefill_part_floats(int T, int nq, int d, int splits);
+
+// ----------------------------------------------------------------- elementwise / small
+
+cudaError_t embed_launch(const uint16_t* E, const int32_t* tok, int B, int h, float* x, cudaStream_t st, bool pdl);
+cudaError_t rmsnorm_launch(const float* x, const float* g, int T, int h, float eps, uint16_t* out, cudaStream_t st,
+                           bool pdl);
+cudaError_t argmax_launch(const float* logits, int B, int V, int32_t* out, cudaStream_t st, bool pdl);
+cudaError_t topk_launch(const float* logits, int T, int E, int k, int renorm, int32_t* idx, float* w,
+                        cudaStream_t st, bool pdl);
+
+}  // namespace dec
+
+namespace dec {
+cudaError_t kv_move_launch(uint16_t* pool_k, uint16_t* pool_v, const int32_t* block_row, int pos0, int n, int nkv,
+                           int d, uint16_t* dense_k, uint16_t* dense_v, int to_pool, cudaStream_t st);
+int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn);
+}  // namespace dec

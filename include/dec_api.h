@@ -1,0 +1,210 @@
+/*
+ * dec_api.h — C ABI of the B200 decoder-layer library (libdec.so).
+ *
+ * The library runs the per-token forward of a decoder-only transformer layer
+ * stack over a paged bf16 KV cache, as chunked prefill and as batched
+ * single-token decode, entirely in CUDA kernels written for sm_100a.
+ *
+ * Sources (the pages this interface follows):
+ *   ANEDVD src/engine.zig — Engine.init / forward / prefill / reset / deinit,
+ *     the ContextOverflow error and its test "an over-long prompt is refused".
+ *   frink_models decoder.rs — gqa_attention (CUDA gqa_decode), MultiSeqKv
+ *     (per-sequence caches for batched decode), route_top_k.
+ *   cortiq_engine pipeline.rs — the prefill/decode contract (every token is
+ *     forwarded once and enters the KV cache once; logits come from the last
+ *     forwarded token), empty input refused.
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major [out][in] bf16 (passed as void*, 2 bytes per
+ *     element, IEEE bfloat16 bits). 1-D parameters (norm gains, biases, the
+ *     shared-expert gate vector) are fp32 arrays.
+ *   - Every call returns a dec_status. On failure nothing has been launched
+ *     unless the status is DEC_ERR_CUDA; dec_last_error() gives a message
+ *     (thread-local, valid until the next call on the same thread).
+ *   - Work is enqueued on the caller's stream and is not synchronised unless
+ *     a host output buffer is given (documented per call).
+ *   - A stream argument of 0 means the legacy default stream.
+ */
+#ifndef DEC_API_H
+#define DEC_API_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dec_stream_t; /* same type as cudaStream_t */
+
+typedef enum dec_status {
+    DEC_OK = 0,
+    DEC_ERR_INVALID_ARG = 1,      /* bad pointer, shape, token id or position */
+    DEC_ERR_CONTEXT_OVERFLOW = 2, /* pos0 + T > max_context (ANEDVD ContextOverflow) */
+    DEC_ERR_PAGES_EXHAUSTED = 3,  /* the KV page pool has no free page */
+    DEC_ERR_OOM = 4,              /* device allocation failed */
+    DEC_ERR_CUDA = 5,             /* a CUDA call failed; see dec_last_error() */
+    DEC_ERR_TIMEOUT = 6,          /* a bounded wait ran out */
+    DEC_ERR_UNSUPPORTED = 7       /* shape outside what the kernels handle */
+} dec_status;
+
+/* Model shape. Zero disables an optional feature. */
+typedef struct dec_config {
+    int32_t hidden;          /* h */
+    int32_t layers;          /* L */
+    int32_t n_q_heads;       /* nq */
+    int32_t n_kv_heads;      /* nkv; nq % nkv == 0; q head i reads kv head i / (nq / nkv) */
+    int32_t head_dim;        /* d: 64 or 128 */
+    int32_t ffn_inter;       /* I of the dense SwiGLU FFN (0 for MoE models) */
+    int32_t vocab;           /* V */
+    int32_t tied_embeddings; /* 1: the LM head is the embedding matrix */
+    int32_t qkv_bias;        /* 1: an fp32 bias is added to q, k, v before QK-norm and RoPE */
+    int32_t qk_norm;         /* 1: per-head RMSNorm of q and k (weights [d]) before RoPE */
+    int32_t n_experts;       /* E routed experts (0 = dense FFN) */
+    int32_t top_k;           /* experts per token */
+    int32_t expert_inter;    /* routed expert inter size */
+    int32_t shared_inter;    /* shared expert inter size (0 = none) */
+    int32_t shared_gate;     /* 1: the shared expert is scaled by sigmoid(gate_vec . xn) */
+    int32_t norm_topk_prob;  /* 1: the k routing weights are renormalised to sum to 1 */
+    float rms_eps;           /* RMSNorm epsilon */
+    float rope_base;         /* RoPE base (theta) */
+    int32_t max_batch;       /* sequences decoded together (dec_step's B <= max_batch) */
+    int32_t max_context;     /* positions per sequence */
+    int32_t page_size;       /* KV page size in tokens: 16 */
+    int32_t prefill_chunk;   /* tokens per prefill chunk (layer-major within a chunk) */
+    int32_t n_pages;         /* KV pages in the pool; 0 = max_batch * ceil(max_context / page_size) */
+} dec_config;
+
+/* One layer's weights. Pointers may be host or device memory; they are read
+ * during dec_init only (the library keeps its own repacked copies). */
+typedef struct dec_layer_weights {
+    const float* attn_norm;  /* [h] */
+    const float* ffn_norm;   /* [h] */
+    const void* wqkv;        /* bf16 [nq*d + 2*nkv*d][h]: rows q, then k, then v */
+    const float* bqkv;       /* [nq*d + 2*nkv*d] or NULL */
+    const float* q_norm;     /* [d] or NULL */
+    const float* k_norm;     /* [d] or NULL */
+    const void* wo;          /* bf16 [h][nq*d] */
+    const void* w_gate;      /* dense: bf16 [I][h] */
+    const void* w_up;        /* dense: bf16 [I][h] */
+    const void* w_down;      /* dense: bf16 [h][I] */
+    const void* w_router;    /* MoE: bf16 [E][h] */
+    const void* e_gate;      /* MoE: bf16 [E][Ie][h] */
+    const void* e_up;        /* MoE: bf16 [E][Ie][h] */
+    const void* e_down;      /* MoE: bf16 [E][h][Ie] */
+    const void* s_gate;      /* shared expert: bf16 [Is][h] or NULL */
+    const void* s_up;        /* bf16 [Is][h] */
+    const void* s_down;      /* bf16 [h][Is] */
+    const float* s_gate_vec; /* [h] or NULL */
+} dec_layer_weights;
+
+typedef struct dec_weights {
+    const void* embed;                /* bf16 [V][h] */
+    const void* lm_head;              /* bf16 [V][h]; ignored when tied_embeddings */
+    const float* final_norm;          /* [h] */
+    const dec_layer_weights* layers;  /* host array of L entries */
+} dec_weights;
+
+typedef struct dec_ctx dec_ctx;
+
+/* Build a context on the current device: validate the shape, copy and repack the
+ * weights into library-owned device memory (fused gate/up), allocate the paged
+ * KV pool, the block table and the workspace. Like ANEDVD Engine.init, but the
+ * caller's weight buffers may be freed as soon as this returns (the copies are
+ * complete: the call synchronises `stream`). */
+dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t stream, dec_ctx** out);
+
+/* Release everything dec_init allocated (ANEDVD Engine.deinit). NULL is a no-op. */
+dec_status dec_free(dec_ctx* ctx);
+
+/* Forget sequence `seq` (or all sequences when seq == -1): its pages return to the
+ * pool and its length becomes 0 (ANEDVD Engine.reset; cortiq kv_cache.clear). */
+dec_status dec_reset(dec_ctx* ctx, int32_t seq);
+
+/* Prefill T prompt tokens of sequence `seq` at positions pos0 .. pos0+T-1
+ * (ANEDVD Engine.prefill; cortiq prefill_batch). Runs layer-major over chunks of
+ * cfg.prefill_chunk tokens; every token's k and v enter the cache once.
+ *   tokens     host int32 [T], each in [0, V)
+ *   pos0       must equal the sequence's current length (each token enters once)
+ *   logits_out fp32 [V]: logits of the last token; device pointer (stream-ordered) or
+ *              host pointer (the call synchronises before returning); may be NULL.
+ * Errors: T <= 0 or a bad token -> INVALID_ARG; pos0 + T > max_context ->
+ * CONTEXT_OVERFLOW (exact fit allowed); no free page -> PAGES_EXHAUSTED. */
+dec_status dec_prefill(dec_ctx* ctx, int32_t seq, const int32_t* tokens, int32_t T, int32_t pos0,
+                       float* logits_out);
+
+/* One decode step for sequences 0..B-1 (ANEDVD Engine.forward, batched as frink
+ * MultiSeqKv): token tokens[b] at position pos[b] of sequence b.
+ *   tokens, pos host int32 [B]; pos[b] must equal sequence b's current length and be
+ *               < max_context (else CONTEXT_OVERFLOW).
+ *   logits_out  fp32 [B][V], device or host pointer as in dec_prefill; may be NULL.
+ * The whole step is replayed from a CUDA graph captured on the first call for each B. */
+dec_status dec_step(dec_ctx* ctx, const int32_t* tokens, const int32_t* pos, int32_t B, float* logits_out);
+
+/* Greedy tokens of the last dec_step / dec_prefill: argmax over each logits row,
+ * lowest index on ties. out: host int32 [B] (B = rows of the last call). Synchronises. */
+dec_status dec_last_argmax(dec_ctx* ctx, int32_t* out, int32_t B);
+
+/* ---------------------------------------------------------------- standalone hot-path calls */
+
+/* Causal GQA decode attention over a paged bf16 KV cache (frink gqa_attention /
+ * launch_gqa_decode; ANEDVD cpu.attentionDecode). For each sequence b the query
+ * sits at position p = pos[b] and attends cache rows 0..p:
+ *   out[b][h] = sum_j softmax_j(q[b][h] . K[b][j] * scale) V[b][j],  kv head h / (nq/nkv).
+ *   q          device bf16 [B][nq][d]
+ *   k_new/v_new device bf16 [B][nkv][d], or both NULL: the row p already holds them
+ *   k_pool/v_pool device bf16 [n_pages][nkv][page_size][d]; row j of sequence b is slot
+ *              j % page_size of page block_table[b][j / page_size]
+ *   block_table device int32 [B][max_pages]
+ *   pos        device int32 [B], 0 <= pos[b] < max_pages * page_size
+ *   fused_rope 1: q and k_new are rotated to position p (half-split pairs, angle
+ *              p * rope_base^(-2i/d)) and rounded to bf16 before use; k_new/v_new are
+ *              written to row p first (the cache append). 0: used as given.
+ *   out        device bf16 [B][nq][d]
+ * Scratch for the split-context partial results is allocated by the library on
+ * first use and kept for later calls on the same device. d must be 64 or 128,
+ * page_size 16. */
+dec_status gqa_decode_attn(const void* q, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                           const int32_t* block_table, int32_t max_pages, const int32_t* pos, int32_t B,
+                           int32_t nq, int32_t nkv, int32_t d, int32_t page_size, float scale,
+                           int32_t fused_rope, float rope_base, void* out, dec_stream_t stream);
+
+/* MoE routing (ANEDVD cpu.moeRoute; frink route_top_k; cortiq MoeFfn): for each of
+ * T rows of router logits, P = softmax over all E, then the k most probable experts
+ * in descending order (lower index first on equal probability); weights P, or P /
+ * sum_topk P when renorm. logits device fp32 [T][E]; idx_out device int32 [T][k];
+ * w_out device fp32 [T][k]. E <= 256, k <= E. */
+dec_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k, int32_t renorm, int32_t* idx_out,
+                          float* w_out, dec_stream_t stream);
+
+/* Weight-streaming projection y[b][n] = sum_k W[n][k] x[b][k] (ANEDVD 1x1 conv
+ * kernels; every projection of the layer). W device bf16 [N][K]; x device bf16
+ * [B][K]; y device fp32 [B][N]. K % 8 == 0. B <= 8 streams W once through the
+ * CUDA-core GEMV; larger B runs the tcgen05 tensor-core GEMM. */
+dec_status weight_gemv(const void* W, const void* x, int32_t B, int32_t N, int32_t K, float* y,
+                       dec_stream_t stream);
+
+/* ---------------------------------------------------------------- test hooks */
+
+/* Copy cache rows [pos0, pos0+n) of layer `layer` of sequence `seq` to / from host
+ * buffers bf16 [n][nkv*d] (k and v). dec_kv_write also extends the sequence's length
+ * to pos0+n when that is longer (allocating pages). Both synchronise. */
+dec_status dec_kv_read(dec_ctx* ctx, int32_t seq, int32_t layer, int32_t pos0, int32_t n, void* k, void* v);
+dec_status dec_kv_write(dec_ctx* ctx, int32_t seq, int32_t layer, int32_t pos0, int32_t n, const void* k,
+                        const void* v);
+
+/* Routing decisions of the last dec_step: host int32 [L][B][top_k]. Synchronises. */
+dec_status dec_last_routes(dec_ctx* ctx, int32_t* idx, int32_t B);
+
+/* Residual stream after the last layer of the last dec_step: host fp32 [B][h]. Synchronises. */
+dec_status dec_last_hidden(dec_ctx* ctx, float* out, int32_t B);
+
+/* Current length of sequence `seq`. */
+dec_status dec_seq_len(dec_ctx* ctx, int32_t seq, int32_t* len_out);
+
+/* Message for the last failure on this thread ("" if none). */
+const char* dec_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DEC_API_H */
