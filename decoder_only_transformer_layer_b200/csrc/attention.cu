@@ -34,14 +34,19 @@ namespace dec {
 namespace {
 
 constexpr int kPage = 16;
+constexpr int kRing = 3;  // pages in flight per warp in the decode kernel
 constexpr float kLog2e = 1.4426950408889634f;
 
 // A warp transforms one head vector of D fp32 values: optional RMSNorm with weight
 // nw, optional RoPE at position pos, rounding to bf16. Lane l holds elements
 // l + 32 m; element l + 32 m (m < D/64) pairs with element l + 32 (m + D/64).
+// With `tab` (the row of a host-built table for this position: (cos, sin) per pair,
+// evaluated in fp64 and rounded to fp32) the angles are read; without it they are
+// evaluated here in fp64.
 template <int D>
 DEC_DEVINL void head_transform(const float* vals_in, bool in_bf16, const uint16_t* in_b, const float* nw,
-                               float eps, bool rope, int pos, float base, uint16_t* dst) {
+                               float eps, bool rope, int pos, float base, uint16_t* dst,
+                               const float2* tab = nullptr) {
     constexpr int E = D / 32;
     const int lane = threadIdx.x & 31;
     float v[E];
@@ -60,7 +65,13 @@ DEC_DEVINL void head_transform(const float* vals_in, bool in_bf16, const uint16_
 #pragma unroll
         for (int m = 0; m < E / 2; ++m) {
             float c, s;
-            rope_cs(pos, lane + 32 * m, D, base, &c, &s);
+            if (tab) {
+                const float2 cs = tab[lane + 32 * m];
+                c = cs.x;
+                s = cs.y;
+            } else {
+                rope_cs(pos, lane + 32 * m, D, base, &c, &s);
+            }
             const float x0 = v[m], x1 = v[m + E / 2];
             v[m] = x0 * c - x1 * s;
             v[m + E / 2] = x0 * s + x1 * c;
@@ -198,6 +209,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
     const bool has_last = pg0 < pg1 && pg1 == np;
     const float sl2 = a.scale * kLog2e;
+    const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
 
     if (pg0 < pg1) {
         // ---- q tile of the group (rows >= G are zero); the split holding row p appends it
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
                 const int h = g * G + r;
                 if (a.qkv)
                     head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)h * D, false, nullptr, a.q_norm, a.eps,
-                                      a.rope, p, a.rope_base, dst);
+                                      a.rope, p, a.rope_base, dst, tab);
                 else
                     head_transform<D>(nullptr, true, a.q_bf + ((size_t)b * a.nq + h) * D, nullptr, a.eps, a.rope, p,
                                       a.rope_base, dst);
@@ -222,7 +234,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             if (warp == 0) {  // k: QK-norm, RoPE, bf16
                 if (a.qkv)
                     head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + g) * D, false, nullptr, a.k_norm,
-                                      a.eps, a.rope, p, a.rope_base, a.k_pool + off);
+                                      a.eps, a.rope, p, a.rope_base, a.k_pool + off, tab);
                 else
                     head_transform<D>(nullptr, true, a.k_new + ((size_t)b * a.nkv + g) * D, nullptr, a.eps, a.rope, p,
                                       a.rope_base, a.k_pool + off);
@@ -245,15 +257,19 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
-        uint16_t* wbuf = kvbuf + (size_t)warp * 4 * PAGE;
+        // each warp streams its pages (pg0 + warp, +4, ...) through a 3-page cp.async ring
+        uint16_t* wbuf = kvbuf + (size_t)warp * kRing * 2 * PAGE;
         int pg = pg0 + warp, buf = 0;
         if (pg < pg1) load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg], a.nkv, g, wbuf, wbuf + PAGE);
+        if (pg + 4 < pg1)
+            load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg + 4], a.nkv, g, wbuf + 2 * PAGE, wbuf + 3 * PAGE);
         const int t4 = lane & 3;
         for (; pg < pg1; pg += 4) {
-            const int nxt = pg + 4;
-            if (nxt < pg1) {
-                uint16_t* nb = wbuf + (buf ^ 1) * 2 * PAGE;
-                load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[nxt], a.nkv, g, nb, nb + PAGE);
+            if (pg + 8 < pg1) {
+                uint16_t* nb = wbuf + ((buf + 2) % kRing) * 2 * PAGE;
+                load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg + 8], a.nkv, g, nb, nb + PAGE);
+                cp_async_wait<2>();
+            } else if (pg + 4 < pg1) {
                 cp_async_wait<1>();
             } else {
                 cp_async_wait<0>();
@@ -280,7 +296,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             }
             pv_page<D, LD>(sc, kd + PAGE, o);
             __syncwarp();
-            buf ^= 1;
+            buf = (buf + 1) % kRing;
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
@@ -349,21 +365,43 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     __syncthreads();
     if (ticket_s != a.splits - 1) return;
     __threadfence();
+    // weights of each split: f_z = exp2(m_z - M) / sum_z exp2(m_z - M) l_z (one warp per head)
+    float* fz = reinterpret_cast<float*>(kvbuf);  // [G][splits]
+    for (int r = warp; r < G; r += 4) {
+        const float* pp = a.part + ((size_t)b * a.nq + g * G + r) * a.splits * (D + 2);
+        float M = -INFINITY;
+        for (int z = lane; z < a.splits; z += 32) M = fmaxf(M, __ldcg(pp + (size_t)z * (D + 2) + D));
+        M = warp_max(M);
+        float L = 0.f;
+        for (int z = lane; z < a.splits; z += 32) {
+            const float mz = __ldcg(pp + (size_t)z * (D + 2) + D);
+            const float f = mz == -INFINITY ? 0.f : exp2f(mz - M);
+            fz[r * a.splits + z] = f;
+            L += f * __ldcg(pp + (size_t)z * (D + 2) + D + 1);
+        }
+        L = warp_sum(L);
+        __syncwarp();
+        for (int z = lane; z < a.splits; z += 32) fz[r * a.splits + z] /= L;
+    }
+    __syncthreads();
+    // weighted sum over splits in split order; loads of one split are coalesced across threads
     for (int idx = tid; idx < G * D; idx += 128) {
         const int r = idx / D, c = idx % D;
         const int h = g * G + r;
-        const float* pp = a.part + ((size_t)b * a.nq + h) * a.splits * (D + 2);
-        float M = -INFINITY;
-        for (int z = 0; z < a.splits; ++z) M = fmaxf(M, __ldcg(pp + (size_t)z * (D + 2) + D));
-        float L = 0.f, O = 0.f;
-        for (int z = 0; z < a.splits; ++z) {
-            const float mz = __ldcg(pp + (size_t)z * (D + 2) + D);
-            if (mz == -INFINITY) continue;
-            const float f = exp2f(mz - M);
-            L += f * __ldcg(pp + (size_t)z * (D + 2) + D + 1);
-            O += f * __ldcg(pp + (size_t)z * (D + 2) + c);
+        const float* pp = a.part + ((size_t)b * a.nq + h) * a.splits * (D + 2) + c;
+        const float* f = fz + r * a.splits;
+        float O = 0.f;
+        int z = 0;
+        for (; z + 4 <= a.splits; z += 4) {
+            const float p0 = __ldcg(pp + (size_t)z * (D + 2)), p1 = __ldcg(pp + (size_t)(z + 1) * (D + 2));
+            const float p2 = __ldcg(pp + (size_t)(z + 2) * (D + 2)), p3 = __ldcg(pp + (size_t)(z + 3) * (D + 2));
+            O += f[z] * p0;
+            O += f[z + 1] * p1;
+            O += f[z + 2] * p2;
+            O += f[z + 3] * p3;
         }
-        a.out[(size_t)b * a.nq * D + (size_t)h * D + c] = f2bf(O / L);
+        for (; z < a.splits; ++z) O += f[z] * __ldcg(pp + (size_t)z * (D + 2));
+        a.out[(size_t)b * a.nq * D + (size_t)h * D + c] = f2bf(O);
     }
     if (tid == 0) a.counters[b * a.nkv + g] = 0;
 }
@@ -381,14 +419,15 @@ __global__ void __launch_bounds__(128) rope_append_kernel(RopeAppendArgs a) {
     const int phys = a.block_row[p / kPage];
     const int slot = p % kPage;
     const int nh = a.nq + 2 * a.nkv;
+    const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
     for (int hh = warp; hh < nh; hh += 4) {
         if (hh < a.nq) {
             head_transform<D>(row + (size_t)hh * D, false, nullptr, a.q_norm, a.eps, true, p, a.rope_base,
-                              a.q_out + ((size_t)t * a.nq + hh) * D);
+                              a.q_out + ((size_t)t * a.nq + hh) * D, tab);
         } else if (hh < a.nq + a.nkv) {
             const int j = hh - a.nq;
             head_transform<D>(row + (size_t)hh * D, false, nullptr, a.k_norm, a.eps, true, p, a.rope_base,
-                              a.k_pool + (((size_t)phys * a.nkv + j) * kPage + slot) * D);
+                              a.k_pool + (((size_t)phys * a.nkv + j) * kPage + slot) * D, tab);
         } else {
             const int j = hh - a.nq - a.nkv;
             head_transform<D>(row + (size_t)hh * D, false, nullptr, nullptr, a.eps, false, p, a.rope_base,
@@ -594,29 +633,36 @@ cudaError_t launch_ex(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s
 
 }  // namespace
 
+// One wave of (sequence, kv head, split) CTAs, each split at least 8 pages long.
 int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms) {
     const int ctas = B * nkv;
-    int s = (2 * num_sms + ctas - 1) / ctas;
+    int s = (num_sms + ctas - 1) / ctas;
     const int pages = (max_ctx + kPage - 1) / kPage;
-    const int max_s = (pages + 3) / 4;  // keep >= 4 pages per split
+    const int max_s = (pages + 7) / 8;
     if (s > max_s) s = max_s;
     if (s < 1) s = 1;
     return s;
 }
 
+template <int D>
+size_t decode_smem() {
+    const size_t ring = (size_t)4 * kRing * 2 * kPage * (D + 8) * 2;  // page rings of 4 warps
+    const size_t merge = (size_t)4 * 16 * D * 4;                     // per-warp partial outputs
+    return ring > merge ? ring : merge;
+}
+
 cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
     const dim3 grid(a.splits, a.nkv, a.B);
+    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64>()) return cudaErrorInvalidValue;
     if (a.d == 128) {
-        const size_t smem = (size_t)4 * 4 * kPage * (128 + 8) * 2;
+        const size_t smem = decode_smem<128>();
         cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         return launch_ex(attn_decode_kernel<128>, grid, dim3(128), smem, st, pdl, a);
     }
     if (a.d == 64) {
-        const size_t smem = (size_t)4 * 4 * kPage * (64 + 8) * 2 > (size_t)4 * 16 * 64 * 4
-                                ? (size_t)4 * 4 * kPage * (64 + 8) * 2
-                                : (size_t)4 * 16 * 64 * 4;
+        const size_t smem = decode_smem<64>();
         cudaError_t e =
             cudaFuncSetAttribute(attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

@@ -62,21 +62,27 @@ DEC_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
 
-// Bounded wait: gives up after `limit` polls (each poll may block up to ~1 ms in
-// hardware) and sets *err; the caller then skips its remaining work and exits.
-DEC_DEVINL bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err, uint32_t limit = 4000u) {
-    for (uint32_t i = 0; i < limit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    if (err) atomicExch(err, 1);
-    return false;
+// Bounded wait: polls until the phase completes or ~2^32 SM cycles (about 2 s at
+// 1.9 GHz) have passed; on time-out it sets *err and returns false so the caller can
+// skip its remaining work and exit instead of hanging.
+DEC_DEVINL bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > (1ll << 32)) {
+            if (err) atomicExch(err, 1);
+            return false;
+        }
+    }
+    return true;
 }
 
 // ----------------------------------------------------------------- bulk copy global -> shared (TMA engine)

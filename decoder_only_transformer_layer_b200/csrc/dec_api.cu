@@ -9,6 +9,7 @@
 // entered into the KV cache once; empty input refused).
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -83,7 +84,9 @@ struct dec_ctx {
     std::vector<int32_t> h_bt;
     int32_t* d_bt = nullptr;
     // step buffers
-    int32_t *d_tok = nullptr, *d_pos = nullptr, *d_argmax = nullptr;
+    int32_t *d_tok = nullptr, *d_pos = nullptr;
+    unsigned long long* d_amax = nullptr;  // packed greedy argmax, 32 words per row
+    float2* rope_tab = nullptr;            // [max_context][d/2] (cos, sin): fp64 on the host, stored fp32
     float *x = nullptr, *qkv = nullptr, *logits = nullptr;
     uint16_t *xn = nullptr, *qrot = nullptr, *attn = nullptr, *act = nullptr;
     float* attn_part = nullptr;
@@ -150,7 +153,7 @@ struct Proj {
 
 dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, const float* xr, const float* g,
                     const uint16_t* xb, float* y, int ldy, const float* bias, uint16_t* act, int ldact,
-                    cudaStream_t st) {
+                    cudaStream_t st, unsigned long long* amax = nullptr) {
     if (n <= 8 && gemv_fits(n, p.K, c->smem_cap)) {
         GemvArgs a{};
         a.W = p.W;
@@ -167,6 +170,7 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
         a.bias = bias;
         a.act = act;
         a.ldact = ldact;
+        a.amax = amax;
         a.err = c->d_err;
         a.smem_cap = c->smem_cap;
         const int ge = epi == GEMM_STORE ? GEMV_STORE : epi == GEMM_RESID ? GEMV_RESID : GEMV_SWIGLU;
@@ -191,6 +195,7 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
     a.ldact = ldact;
     a.ws = c->gemm_ws;
     a.counters = c->gemm_cnt;
+    a.amax = amax;
     a.err = c->d_err;
     CUDA_TRY(gemm_launch(plan, a, st, true));
     return DEC_OK;
@@ -219,6 +224,7 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
             a.eps = k.rms_eps;
             a.rope = 1;
             a.rope_base = k.rope_base;
+            a.rope_tab = c->rope_tab;
             a.k_pool = L.k_pool;
             a.v_pool = L.v_pool;
             a.block_table = c->d_bt;
@@ -243,6 +249,7 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
             r.k_norm = L.k_norm;
             r.eps = k.rms_eps;
             r.rope_base = k.rope_base;
+            r.rope_tab = c->rope_tab;
             r.T = n;
             r.pos0 = pos0;
             r.nq = k.n_q_heads;
@@ -288,14 +295,13 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
     return DEC_OK;
 }
 
-// Final norm + LM head for `n` rows starting at residual row `row0` -> c->logits [n][V].
+// Final norm + LM head for `n` rows starting at residual row `row0` -> c->logits [n][V];
+// the greedy token of each row is folded into the head's epilogue (packed argmax words).
 dec_status head(dec_ctx* c, int row0, int n, cudaStream_t st) {
     const dec_config& k = c->c;
-    dec_status s = run_proj(c, {c->head, k.vocab, k.hidden}, n, GEMM_STORE, true, c->x + (size_t)row0 * k.hidden,
-                            c->final_norm, nullptr, c->logits, k.vocab, nullptr, nullptr, 0, st);
-    if (s != DEC_OK) return s;
-    CUDA_TRY(argmax_launch(c->logits, n, k.vocab, c->d_argmax, st, true));
-    return DEC_OK;
+    CUDA_TRY(cudaMemsetAsync(c->d_amax, 0, sizeof(unsigned long long) * 32 * (size_t)n, st));
+    return run_proj(c, {c->head, k.vocab, k.hidden}, n, GEMM_STORE, true, c->x + (size_t)row0 * k.hidden,
+                    c->final_norm, nullptr, c->logits, k.vocab, nullptr, nullptr, 0, st, c->d_amax);
 }
 
 dec_status ensure_pages(dec_ctx* c, int seq, int upto) {
@@ -519,7 +525,19 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     const int T = c->max_tok;
     INIT_TRY(dmalloc(&c->d_tok, T));
     INIT_TRY(dmalloc(&c->d_pos, T));
-    INIT_TRY(dmalloc(&c->d_argmax, T));
+    INIT_TRY(dmalloc(&c->d_amax, (size_t)32 * k.max_batch));
+    {
+        // RoPE angles pos * base^(-2i/d), cos and sin evaluated in fp64, stored as fp32
+        std::vector<float2> tab((size_t)k.max_context * (d / 2));
+        for (int p = 0; p < k.max_context; ++p)
+            for (int i = 0; i < d / 2; ++i) {
+                const double theta = pow((double)k.rope_base, -2.0 * i / (double)d);
+                const double ang = (double)p * theta;
+                tab[(size_t)p * (d / 2) + i] = make_float2((float)cos(ang), (float)sin(ang));
+            }
+        INIT_TRY(dmalloc(&c->rope_tab, tab.size()));
+        INIT_TRY(cudaMemcpy(c->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice));
+    }
     INIT_TRY(dmalloc(&c->x, (size_t)T * h));
     INIT_TRY(dmalloc(&c->qkv, (size_t)T * c->qkv_rows));
     INIT_TRY(dmalloc(&c->logits, (size_t)k.max_batch * V));
@@ -601,7 +619,8 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->d_bt);
     cudaFree(c->d_tok);
     cudaFree(c->d_pos);
-    cudaFree(c->d_argmax);
+    cudaFree(c->d_amax);
+    cudaFree(c->rope_tab);
     cudaFree(c->x);
     cudaFree(c->qkv);
     cudaFree(c->logits);
@@ -745,8 +764,11 @@ dec_status dec_step(dec_ctx* c, const int32_t* tokens, const int32_t* pos, int32
 dec_status dec_last_argmax(dec_ctx* c, int32_t* out, int32_t B) {
     if (!c || !out) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
     if (B != c->last_rows) return fail(DEC_ERR_INVALID_ARG, "B differs from the last call's rows");
-    CUDA_TRY(cudaMemcpyAsync(out, c->d_argmax, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, c->stream));
+    std::vector<unsigned long long> w((size_t)32 * B);
+    CUDA_TRY(cudaMemcpyAsync(w.data(), c->d_amax, sizeof(unsigned long long) * 32 * B, cudaMemcpyDeviceToHost,
+                             c->stream));
     CUDA_TRY(cudaStreamSynchronize(c->stream));
+    for (int b = 0; b < B; ++b) out[b] = argmax_unpack(w[(size_t)32 * b]);
     return DEC_OK;
 }
 

@@ -102,22 +102,52 @@ DEC_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Apply the epilogue to value v of (row, t). All lanes of the warp must call it
-// together (the SwiGLU pairing uses a shuffle).
-DEC_DEVINL void epilogue(const GemmArgs& a, int row, int t, float v) {
-    const bool ok = row < a.M && t < a.N;
+// Apply the epilogue to the 16 values v[j] of (row, t0 + j). All lanes of the warp call
+// it together (the SwiGLU pairing uses a shuffle). Every global load of a chunk is issued
+// before any store, so the 16 accesses overlap instead of waiting on one another.
+DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v)[16]) {
+    const bool row_ok = row < a.M;
     if (a.epi == GEMM_SWIGLU) {
-        const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
-        if (ok && (row & 1) == 0) {
-            const float sg = v * (1.0f / (1.0f + expf(-v)));
-            a.act[(size_t)t * a.ldact + (row >> 1)] = f2bf(sg * partner);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const float partner = __shfl_xor_sync(0xffffffffu, v[j], 1);
+            if (row_ok && (row & 1) == 0 && t0 + j < a.N) {
+                const float sg = v[j] * (1.0f / (1.0f + expf(-v[j])));
+                a.act[(size_t)(t0 + j) * a.ldact + (row >> 1)] = f2bf(sg * partner);
+            }
         }
-    } else if (ok) {
-        float* dst = a.y + (size_t)t * a.ldy + row;
-        if (a.epi == GEMM_RESID)
-            *dst += v;
-        else
-            *dst = v + (a.bias ? a.bias[row] : 0.f);
+        return;
+    }
+    if (!row_ok) return;
+    if (a.epi == GEMM_RESID) {
+        float old[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) old[j] = t0 + j < a.N ? a.y[(size_t)(t0 + j) * a.ldy + row] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (t0 + j < a.N) a.y[(size_t)(t0 + j) * a.ldy + row] = old[j] + v[j];
+    } else {
+        const float bias = a.bias ? a.bias[row] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (t0 + j < a.N) a.y[(size_t)(t0 + j) * a.ldy + row] = v[j] + bias;
+    }
+}
+
+// Greedy argmax of the STORE epilogue: warp maximum of the packed (value, row) words of
+// each token, one atomicMax per warp and token (token words 256 bytes apart).
+DEC_DEVINL void argmax16(const GemmArgs& a, int row, int t0, const float (&v)[16]) {
+    const int lane = threadIdx.x & 31;
+    const float bias = (a.bias && row < a.M) ? a.bias[row] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        unsigned long long w = (row < a.M && t0 + j < a.N) ? argmax_pack(v[j] + bias, row) : 0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long u = __shfl_xor_sync(0xffffffffu, w, o);
+            w = u > w ? u : w;
+        }
+        if (lane == 0 && w) atomicMax(&a.amax[(size_t)(t0 + j) * 32], w);
     }
 }
 
@@ -211,14 +241,17 @@ __global__ void __launch_bounds__(128, 1)
         uint32_t r[16];
         tmem_ld16(lane_base + (uint32_t)c0, r);
         if (!acc_ready) continue;
-        if (a.splits == 1) {
+        float v[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) epilogue(a, row, n0 + c0 + j, __uint_as_float(r[j]));
+        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+        if (a.splits == 1) {
+            epilogue16(a, row, n0 + c0, v);
+            if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0, v);
         } else if (row < a.M) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int t = n0 + c0 + j;
-                if (t < a.N) a.ws[((size_t)z * a.N + t) * a.M + row] = __uint_as_float(r[j]);
+                if (t < a.N) a.ws[((size_t)z * a.N + t) * a.M + row] = v[j];
             }
         }
     }
@@ -241,12 +274,23 @@ __global__ void __launch_bounds__(128, 1)
     if (*ticket != a.splits - 1) return;
     __threadfence();
     const int ncols = min(BN, a.N - n0);
-    for (int c = 0; c < ncols; ++c) {
-        const int t = n0 + c;
-        float v = 0.f;
-        if (row < a.M)
-            for (int s = 0; s < a.splits; ++s) v += __ldcg(a.ws + ((size_t)s * a.N + t) * a.M + row);
-        epilogue(a, row, t, v);
+    for (int c0 = 0; c0 < ncols; c0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+        if (row < a.M) {
+            // splits summed in split order; all loads of a split are independent
+            for (int s = 0; s < a.splits; ++s) {
+                float p[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    p[j] = c0 + j < ncols ? __ldcg(a.ws + ((size_t)s * a.N + n0 + c0 + j) * a.M + row) : 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] += p[j];
+            }
+        }
+        epilogue16(a, row, n0 + c0, v);
+        if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0, v);
     }
     if (threadIdx.x == 0) a.counters[tile] = 0;
 }

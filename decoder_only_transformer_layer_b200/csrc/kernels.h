@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace dec {
 
@@ -25,6 +26,7 @@ struct GemvArgs {
     const float* bias;
     uint16_t* act;      // SWIGLU: act[b*ldact + n/2] = bf16(silu(acc[even]) * acc[odd])
     int ldact;
+    unsigned long long* amax;  // STORE: per column, packed greedy argmax of y (null = off)
     int* err;
     int smem_cap;
 };
@@ -54,6 +56,7 @@ struct GemmArgs {
     int splits;
     float* ws;        // split partials [splits][N][M] fp32
     int* counters;    // [tiles], zero on entry, left zero on exit
+    unsigned long long* amax;  // STORE: per token, packed greedy argmax of y (null = off)
     int* err;
 };
 
@@ -77,6 +80,7 @@ struct AttnDecodeArgs {
     float eps;
     int rope;               // rotate q and the new k to pos
     float rope_base;
+    const float2* rope_tab; // [max_ctx][d/2] (cos, sin), or null: evaluated in the kernel
     uint16_t* k_pool;       // [n_pages][nkv][16][d]
     uint16_t* v_pool;
     const int32_t* block_table;
@@ -100,6 +104,7 @@ struct RopeAppendArgs {
     const float* k_norm;
     float eps;
     float rope_base;
+    const float2* rope_tab;  // [max_ctx][d/2] (cos, sin), or null
     int T, pos0, nq, nkv, d;
     uint16_t* q_out;   // [T][nq][d]
     uint16_t* k_pool;
@@ -124,6 +129,17 @@ struct AttnPrefillArgs {
 cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl);
 int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms);
 size_t attn_prefill_part_floats(int T, int nq, int d, int splits);
+
+// Greedy argmax as one 64-bit word per row: high half an order-preserving key of the
+// fp32 value, low half ~index (so on equal values the lowest index is the largest word).
+// The zero word is below every real value. atomicMax of these words is order-free.
+__host__ __device__ inline unsigned long long argmax_pack(float v, int idx) {
+    unsigned int b;
+    memcpy(&b, &v, 4);
+    const unsigned int key = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)key << 32) | (unsigned long long)(0xFFFFFFFFu - (unsigned int)idx);
+}
+__host__ __device__ inline int argmax_unpack(unsigned long long w) { return (int)(0xFFFFFFFFu - (unsigned int)w); }
 
 // ----------------------------------------------------------------- elementwise / small
 
