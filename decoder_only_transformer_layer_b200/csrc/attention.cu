@@ -350,10 +350,12 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             }
         }
     } else if (a.splits > 1) {
-        for (int idx = tid; idx < G; idx += 128) {
-            float* pp = a.part + (((size_t)b * a.nq + g * G + idx) * a.splits + s) * (D + 2);
-            pp[D] = -INFINITY;
-            pp[D + 1] = 0.f;
+        // an empty split still writes a full partial (zero output, zero weight): the merge
+        // reads every split, and the scratch holds whatever an earlier call left there
+        for (int idx = tid; idx < G * (D + 2); idx += 128) {
+            const int r = idx / (D + 2), c = idx % (D + 2);
+            float* pp = a.part + (((size_t)b * a.nq + g * G + r) * a.splits + s) * (D + 2);
+            pp[c] = c == D ? -INFINITY : 0.f;
         }
     }
     if (a.splits == 1) return;

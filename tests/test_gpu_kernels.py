@@ -102,6 +102,15 @@ def test_gqa_decode_mha_and_group_16():
     _check_attn(got, ref, "G=16")
 
 
+def test_gqa_decode_empty_splits_after_another_shape():
+    # Split partials live in scratch that keeps an earlier call's contents; a split with no
+    # pages must not let those values into the merge (0 * -inf is NaN).
+    _attn_case(3, 8, 2, 128, [0, 17, 300], 1, 1, 11)
+    for pos in ([40, 1000], [3, 1000], [1000, 0]):
+        got, ref, _ = _attn_case(2, 9, 3, 64, pos, 1, 1, 21)
+        _check_attn(got, ref, f"d=64 after d=128, pos={pos}")
+
+
 def test_gqa_decode_sweep_shape_ctx2048():
     B, nq, nkv, d = 64, 32, 8, 128
     got, ref, _ = _attn_case(B, nq, nkv, d, [2047] * B, 1, 1, 15)
