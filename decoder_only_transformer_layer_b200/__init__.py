@@ -74,11 +74,12 @@ def lib():
         L.dec_seq_len.argtypes = [_P, _I, _P]
         L.gqa_decode_attn.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, C.c_float, _I,
                                       C.c_float, _P, _P]
+        L.gqa_decode_attn_noalloc.argtypes = L.gqa_decode_attn.argtypes
         L.moe_route_topk.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
         L.weight_gemv.argtypes = [_P, _P, _I, _I, _I, _P, _P]
         for f in ("dec_init", "dec_free", "dec_reset", "dec_prefill", "dec_step", "dec_last_argmax", "dec_kv_read",
                   "dec_kv_write", "dec_last_routes", "dec_last_hidden", "dec_seq_len", "gqa_decode_attn",
-                  "moe_route_topk", "weight_gemv"):
+                  "gqa_decode_attn_noalloc", "moe_route_topk", "weight_gemv"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -233,6 +234,18 @@ def gqa_decode_attn(q, k_new, v_new, k_pool, v_pool, block_table, pos, nq, nkv, 
     _check(lib().gqa_decode_attn(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(block_table),
                                  max_pages, _ptr(pos), B, nq, nkv, d, page_size, float(scale), int(fused_rope),
                                  float(rope_base), _ptr(out), _stream(stream)))
+    return out
+
+
+def gqa_decode_attn_noalloc(q, k_new, v_new, k_pool, v_pool, block_table, pos, nq, nkv, d, scale, fused_rope,
+                            rope_base, out, page_size=16, stream=None):
+    """gqa_decode_attn for callers that must not let the library allocate device memory:
+    the scratch is a fixed array built into the library (same arguments and results)."""
+    B, max_pages = block_table.shape
+    _check(lib().gqa_decode_attn_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+                                         _ptr(block_table), max_pages, _ptr(pos), B, nq, nkv, d, page_size,
+                                         float(scale), int(fused_rope), float(rope_base), _ptr(out),
+                                         _stream(stream)))
     return out
 
 

@@ -407,6 +407,11 @@ int device_smem_cap() {
 
 }  // namespace
 
+namespace dec {
+// Message returned by dec_last_error() for entry points defined in other files.
+void set_last_error(const std::string& msg) { g_err = msg; }
+}  // namespace dec
+
 // =================================================================== ABI
 
 extern "C" {

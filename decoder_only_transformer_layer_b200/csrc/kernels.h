@@ -152,7 +152,9 @@ cudaError_t topk_launch(const float* logits, int T, int E, int k, int renorm, in
 
 }  // namespace dec
 
+#include <string>
 namespace dec {
+void set_last_error(const std::string& msg);
 cudaError_t kv_move_launch(uint16_t* pool_k, uint16_t* pool_v, const int32_t* block_row, int pos0, int n, int nkv,
                            int d, uint16_t* dense_k, uint16_t* dense_v, int to_pool, cudaStream_t st);
 int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn);

@@ -168,6 +168,28 @@ dec_status gqa_decode_attn(const void* q, const void* k_new, const void* v_new, 
                            int32_t nq, int32_t nkv, int32_t d, int32_t page_size, float scale,
                            int32_t fused_rope, float rope_base, void* out, dec_stream_t stream);
 
+/* gqa_decode_attn without any device allocation. The source pages have no
+ * counterpart to this call; it exists for callers that must not let a library
+ * allocate device memory: programs whose device memory is reserved up front by their
+ * own pool allocator, latency-bound loops that cannot absorb the synchronisation a
+ * cudaMalloc/cudaFree may cause, and plugin hosts that forbid allocation after
+ * start-up. Arguments, layout and results are those of gqa_decode_attn.
+ *   - Scratch lives in one fixed array inside the library image, present on every
+ *     device that loads the library until the process exits: room for 16384
+ *     (sequence, kv head) pairs and 1048576 floats of split partials. Shapes that need
+ *     more are refused with DEC_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device looks up the array's device address (a one-time
+ *     set-up per device); make that first call before any stream capture begins.
+ *   - Every call uses the same array. The call clears the merge counters it needs
+ *     (an asynchronous memset on `stream`) before its kernel; calls whose work can
+ *     overlap on the GPU (different streams, or several threads) race on the array
+ *     and must be serialised by the caller.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine. */
+dec_status gqa_decode_attn_noalloc(const void* q, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                                   const int32_t* block_table, int32_t max_pages, const int32_t* pos, int32_t B,
+                                   int32_t nq, int32_t nkv, int32_t d, int32_t page_size, float scale,
+                                   int32_t fused_rope, float rope_base, void* out, dec_stream_t stream);
+
 /* MoE routing (ANEDVD cpu.moeRoute; frink route_top_k; cortiq MoeFfn): for each of
  * T rows of router logits, P = softmax over all E, then the k most probable experts
  * in descending order (lower index first on equal probability); weights P, or P /
