@@ -43,6 +43,23 @@ def peaks():
     return dict(hbm=6650.0, tc=1590.0, tc_sus=1400.0, src="fallback")
 
 
+def measured_traffic():
+    """dram read+write bytes per launch of the roofline kernel, from the committed ncu summary;
+    None when that summary is missing or the kernel source changed since it was captured."""
+    import hashlib
+    import re
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "gemv_llama3-8b_decode_full.md")).read()
+        src = open(os.path.join(ROOT, "decoder_only_transformer_layer_b200", "csrc", "gemv.cu"), "rb").read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch: (\d+)", txt)
+    h = re.search(r"kernel_sha256: ([0-9a-f]+)", txt)
+    if not m or not h or h.group(1) != hashlib.sha256(src).hexdigest():
+        return None
+    return int(m.group(1))
+
+
 def layer_bytes(cfg):
     h, d, nq, nkv, I = cfg["hidden"], cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ffn_inter"]
     qkv = (nq * d + 2 * nkv * d) * h
@@ -335,7 +352,8 @@ def main():
                         global_batch=world, seq_len=PROMPT, model_shape="llama3-8b", layers=cfg["layers"],
                         parallelism=f"replicas x{world}", l2="inputs larger than L2 (15 GB of weights per step)"),
             roofline=dict(bound="hbm", achieved=round(gemv_gbs, 1), peak=P["hbm"], unit="GB/s",
-                          frac=round(gemv_gbs / P["hbm"], 4), traffic=None,
+                          frac=round(gemv_gbs / P["hbm"], 4), traffic=measured_traffic(),
+                          traffic_unit="bytes per launch (ncu dram read+write)",
                           kernel=f"gemv_kernel<1,SWIGLU-shaped> on [{2 * cfg['ffn_inter']}][{cfg['hidden']}] bf16",
                           peak_source=P["src"]),
             step_roofline=dict(bytes_per_step=wbytes + kvbytes / K, achieved_gbs=round(step_gbs, 1),
