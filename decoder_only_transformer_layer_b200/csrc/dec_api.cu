@@ -102,6 +102,10 @@ struct dec_ctx {
     int* h_err = nullptr;
     int act_cols = 0;
     int decode_splits = 1;
+    // MoE step buffers (rows: max_tok tokens, or max_tok * top_k (token, expert) slots)
+    float *moe_logits = nullptr, *moe_w = nullptr, *moe_sgate = nullptr, *moe_y = nullptr, *moe_ys = nullptr;
+    int32_t *moe_routes = nullptr, *moe_perm = nullptr, *moe_inv = nullptr, *moe_groups = nullptr, *moe_ngroups = nullptr;
+    uint16_t* moe_act = nullptr;
     std::map<int, cudaGraphExec_t> graphs;
     int last_rows = 0;
     bool last_was_step = false;
@@ -122,9 +126,14 @@ dec_status check_config(const dec_config* c) {
     if (c->page_size != 16) return fail(DEC_ERR_UNSUPPORTED, "page_size must be 16");
     if (c->max_batch <= 0 || c->max_context <= 0 || c->prefill_chunk <= 0)
         return fail(DEC_ERR_INVALID_ARG, "max_batch, max_context and prefill_chunk must be positive");
-    if (c->n_experts > 0) return fail(DEC_ERR_UNSUPPORTED, "MoE layers are not enabled in this build");
-    if (c->ffn_inter <= 0 || c->ffn_inter % 8 != 0)
+    if (c->n_experts > 0) {
+        if (c->n_experts > 256 || c->top_k <= 0 || c->top_k > 16 || c->top_k > c->n_experts)
+            return fail(DEC_ERR_UNSUPPORTED, "MoE needs n_experts <= 256 and 0 < top_k <= min(16, n_experts)");
+        if (c->expert_inter <= 0 || c->expert_inter % 8 != 0 || c->shared_inter < 0 || c->shared_inter % 8 != 0)
+            return fail(DEC_ERR_UNSUPPORTED, "expert_inter / shared_inter must be multiples of 8");
+    } else if (c->ffn_inter <= 0 || c->ffn_inter % 8 != 0) {
         return fail(DEC_ERR_UNSUPPORTED, "ffn_inter must be a positive multiple of 8");
+    }
     if (!(c->rms_eps > 0.f)) return fail(DEC_ERR_INVALID_ARG, "rms_eps must be positive");
     return DEC_OK;
 }
@@ -198,6 +207,91 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
     a.amax = amax;
     a.err = c->d_err;
     CUDA_TRY(gemm_launch(plan, a, st, true));
+    return DEC_OK;
+}
+
+// ----------------------------------------------------------------- MoE FFN of one layer
+
+// xn = R1(rmsnorm(x)); router logits; top-k + shared gate; permutation by expert; grouped
+// gate/up (SiLU*up) and down over the routed (token, expert) slots; shared expert; combine
+// into the residual: x += sum_j w_j y_j + sigmoid(g . xn) y_shared.
+dec_status moe_ffn(dec_ctx* c, int li, int n, cudaStream_t st) {
+    const dec_config& k = c->c;
+    LayerDev& L = c->L[li];
+    const int h = k.hidden, E = k.n_experts, kk = k.top_k, Ie = k.expert_inter, Is = k.shared_inter;
+    CUDA_TRY(rmsnorm_launch(c->x, L.ffn_norm, n, h, k.rms_eps, c->xn, st, true));
+    dec_status s = run_proj(c, {L.wrouter, E, h}, n, GEMM_STORE, false, nullptr, nullptr, c->xn, c->moe_logits, E,
+                            nullptr, nullptr, 0, st);
+    if (s != DEC_OK) return s;
+    int32_t* idx = c->moe_routes + (size_t)li * c->max_tok * kk;
+    MoeRouteArgs r{};
+    r.logits = c->moe_logits;
+    r.E = E;
+    r.k = kk;
+    r.renorm = k.norm_topk_prob;
+    r.idx = idx;
+    r.w = c->moe_w;
+    r.xn = c->xn;
+    r.gvec = (Is > 0 && k.shared_gate) ? L.sgate_vec : nullptr;
+    r.h = h;
+    r.sgate = c->moe_sgate;
+    CUDA_TRY(moe_route_launch(r, n, st, true));
+    const int nb = grouped_nb_for(n);
+    MoePermArgs p{};
+    p.idx = idx;
+    p.n = n;
+    p.k = kk;
+    p.E = E;
+    p.nb = nb;
+    p.perm_tok = c->moe_perm;
+    p.inv = c->moe_inv;
+    p.groups = c->moe_groups;
+    p.n_groups = c->moe_ngroups;
+    CUDA_TRY(moe_permute_launch(p, st, true));
+    GroupedGemvArgs g{};
+    g.W = L.egu;
+    g.wstride = (size_t)2 * Ie * h;
+    g.M = 2 * Ie;
+    g.K = h;
+    g.groups = c->moe_groups;
+    g.n_groups = c->moe_ngroups;
+    g.x = c->xn;
+    g.x_map = c->moe_perm;
+    g.ldx = h;
+    g.act = c->moe_act;
+    g.ldact = Ie;
+    g.err = c->d_err;
+    g.smem_cap = c->smem_cap;
+    CUDA_TRY(grouped_gemv_launch(g, nb, true, st, c->num_sms, true));
+    g.W = L.edown;
+    g.wstride = (size_t)h * Ie;
+    g.M = h;
+    g.K = Ie;
+    g.x = c->moe_act;
+    g.x_map = nullptr;
+    g.ldx = Ie;
+    g.y = c->moe_y;
+    g.ldy = h;
+    g.act = nullptr;
+    CUDA_TRY(grouped_gemv_launch(g, nb, false, st, c->num_sms, true));
+    if (Is > 0) {
+        s = run_proj(c, {L.sgu, 2 * Is, h}, n, GEMM_SWIGLU, false, nullptr, nullptr, c->xn, nullptr, 0, nullptr,
+                     c->act, Is, st);
+        if (s != DEC_OK) return s;
+        s = run_proj(c, {L.sdown, h, Is}, n, GEMM_STORE, false, nullptr, nullptr, c->act, c->moe_ys, h, nullptr,
+                     nullptr, 0, st);
+        if (s != DEC_OK) return s;
+    }
+    MoeCombineArgs m{};
+    m.x = c->x;
+    m.y = c->moe_y;
+    m.ys = Is > 0 ? c->moe_ys : nullptr;
+    m.w = c->moe_w;
+    m.inv = c->moe_inv;
+    m.sgate = (Is > 0 && k.shared_gate && L.sgate_vec) ? c->moe_sgate : nullptr;
+    m.k = kk;
+    m.h = h;
+    CUDA_TRY(moe_combine_launch(m, n, st, true));
     return DEC_OK;
 }
 
@@ -284,6 +378,11 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
         s = run_proj(c, {L.wo, h, c->qd}, n, GEMM_RESID, false, nullptr, nullptr, c->attn, c->x, h, nullptr, nullptr,
                      0, st);
         if (s != DEC_OK) return s;
+        if (k.n_experts > 0) {
+            s = moe_ffn(c, li, n, st);
+            if (s != DEC_OK) return s;
+            continue;
+        }
         // FFN: norm + fused gate/up + SiLU, then down + residual
         s = run_proj(c, {L.wgu, 2 * k.ffn_inter, h}, n, GEMM_SWIGLU, true, c->x, L.ffn_norm, nullptr, nullptr, 0,
                      nullptr, c->act, c->act_cols, st);
@@ -456,7 +555,7 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     c->max_pages = (k.max_context + 15) / 16;
     c->n_pages = k.n_pages > 0 ? k.n_pages : k.max_batch * c->max_pages;
     c->max_tok = std::max(k.max_batch, k.prefill_chunk);
-    c->act_cols = k.ffn_inter;
+    c->act_cols = std::max(k.ffn_inter, k.shared_inter);
     auto cleanup = [&](dec_status st_) {
         dec_free(c);
         return st_;
@@ -507,10 +606,30 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
         }
         INIT_TRY(dmalloc(&L.wo, (size_t)h * c->qd));
         INIT_TRY(copy_in(L.wo, s_.wo, (size_t)h * c->qd * 2, st));
-        INIT_TRY(dmalloc(&L.wgu, (size_t)2 * k.ffn_inter * h));
-        INIT_TRY(interleave_in(L.wgu, s_.w_gate, s_.w_up, (size_t)k.ffn_inter, h, st));
-        INIT_TRY(dmalloc(&L.wdown, (size_t)h * k.ffn_inter));
-        INIT_TRY(copy_in(L.wdown, s_.w_down, (size_t)h * k.ffn_inter * 2, st));
+        if (k.n_experts > 0) {
+            const size_t E = k.n_experts, Ie = k.expert_inter, Is = k.shared_inter;
+            INIT_TRY(dmalloc(&L.wrouter, E * h));
+            INIT_TRY(copy_in(L.wrouter, s_.w_router, E * h * 2, st));
+            INIT_TRY(dmalloc(&L.egu, E * 2 * Ie * h));  // per expert: gate/up rows interleaved
+            INIT_TRY(interleave_in(L.egu, s_.e_gate, s_.e_up, E * Ie, h, st));
+            INIT_TRY(dmalloc(&L.edown, E * h * Ie));
+            INIT_TRY(copy_in(L.edown, s_.e_down, E * h * Ie * 2, st));
+            if (Is > 0) {
+                INIT_TRY(dmalloc(&L.sgu, 2 * Is * h));
+                INIT_TRY(interleave_in(L.sgu, s_.s_gate, s_.s_up, Is, h, st));
+                INIT_TRY(dmalloc(&L.sdown, (size_t)h * Is));
+                INIT_TRY(copy_in(L.sdown, s_.s_down, (size_t)h * Is * 2, st));
+                if (k.shared_gate && s_.s_gate_vec) {
+                    INIT_TRY(dmalloc(&L.sgate_vec, h));
+                    INIT_TRY(copy_in(L.sgate_vec, s_.s_gate_vec, (size_t)h * 4, st));
+                }
+            }
+        } else {
+            INIT_TRY(dmalloc(&L.wgu, (size_t)2 * k.ffn_inter * h));
+            INIT_TRY(interleave_in(L.wgu, s_.w_gate, s_.w_up, (size_t)k.ffn_inter, h, st));
+            INIT_TRY(dmalloc(&L.wdown, (size_t)h * k.ffn_inter));
+            INIT_TRY(copy_in(L.wdown, s_.w_down, (size_t)h * k.ffn_inter * 2, st));
+        }
         INIT_TRY(dmalloc(&L.k_pool, page_elems));
         INIT_TRY(dmalloc(&L.v_pool, page_elems));
         INIT_TRY(cudaMemsetAsync(L.k_pool, 0, page_elems * 2, st));
@@ -550,6 +669,21 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(dmalloc(&c->qrot, (size_t)T * c->qd));
     INIT_TRY(dmalloc(&c->attn, (size_t)T * c->qd));
     INIT_TRY(dmalloc(&c->act, (size_t)T * c->act_cols));
+    if (k.n_experts > 0) {
+        const size_t E = k.n_experts, kk = k.top_k, slots = (size_t)T * kk;
+        INIT_TRY(dmalloc(&c->moe_logits, (size_t)T * E));
+        INIT_TRY(dmalloc(&c->moe_w, slots));
+        INIT_TRY(dmalloc(&c->moe_sgate, T));
+        INIT_TRY(dmalloc(&c->moe_routes, (size_t)k.layers * slots));
+        INIT_TRY(cudaMemsetAsync(c->moe_routes, 0, (size_t)k.layers * slots * 4, st));
+        INIT_TRY(dmalloc(&c->moe_perm, slots));
+        INIT_TRY(dmalloc(&c->moe_inv, slots));
+        INIT_TRY(dmalloc(&c->moe_groups, 4 * (E + slots)));
+        INIT_TRY(dmalloc(&c->moe_ngroups, 1));
+        INIT_TRY(dmalloc(&c->moe_act, slots * k.expert_inter));
+        INIT_TRY(dmalloc(&c->moe_y, slots * h));
+        INIT_TRY(dmalloc(&c->moe_ys, (size_t)T * h));
+    }
     INIT_TRY(dmalloc(&c->d_err, 1));
     INIT_TRY(cudaMemsetAsync(c->d_err, 0, 4, st));
     INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_stage), sizeof(int32_t) * (2 * T + c->max_pages + 16)));
@@ -574,11 +708,19 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     {
         size_t ws = 0;
         int cnt = 0;
-        const int Ms[5] = {c->qkv_rows, h, 2 * k.ffn_inter, h, k.vocab};
-        const int Ks[5] = {h, c->qd, h, k.ffn_inter, h};
+        // (rows, K) of every projection that can run on the GEMM
+        std::vector<int> Ms = {c->qkv_rows, h, k.vocab}, Ks = {h, c->qd, h};
+        if (k.n_experts > 0) {
+            Ms.insert(Ms.end(), {k.n_experts, 2 * k.shared_inter, h});
+            Ks.insert(Ks.end(), {h, h, k.shared_inter});
+        } else {
+            Ms.insert(Ms.end(), {2 * k.ffn_inter, h});
+            Ks.insert(Ks.end(), {h, k.ffn_inter});
+        }
         // every token count a prefill chunk (tail included) or a decode batch can have
         for (int n = 1; n <= std::max(pre_T, k.max_batch); ++n)
-            for (int j = 0; j < 5; ++j) {
+            for (size_t j = 0; j < Ms.size(); ++j) {
+                if (Ms[j] <= 0 || Ks[j] <= 0) continue;
                 int bn = 0;
                 const int sp = gemm_choose_splits(Ms[j], n, Ks[j], c->num_sms, &bn);
                 if (sp > 1) ws = std::max(ws, (size_t)sp * n * Ms[j]);
@@ -637,6 +779,17 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->attn_cnt);
     cudaFree(c->gemm_ws);
     cudaFree(c->gemm_cnt);
+    cudaFree(c->moe_logits);
+    cudaFree(c->moe_w);
+    cudaFree(c->moe_sgate);
+    cudaFree(c->moe_routes);
+    cudaFree(c->moe_perm);
+    cudaFree(c->moe_inv);
+    cudaFree(c->moe_groups);
+    cudaFree(c->moe_ngroups);
+    cudaFree(c->moe_act);
+    cudaFree(c->moe_y);
+    cudaFree(c->moe_ys);
     cudaFree(c->d_err);
     if (c->h_stage) cudaFreeHost(c->h_stage);
     if (c->h_err) cudaFreeHost(c->h_err);
@@ -826,10 +979,15 @@ dec_status dec_kv_read(dec_ctx* c, int32_t seq, int32_t layer, int32_t pos0, int
 }
 
 dec_status dec_last_routes(dec_ctx* c, int32_t* idx, int32_t B) {
-    (void)idx;
-    (void)B;
-    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
-    return fail(DEC_ERR_UNSUPPORTED, "the model has no MoE layers");
+    if (!c || !idx) return fail(DEC_ERR_INVALID_ARG, "NULL argument");
+    if (c->c.n_experts <= 0) return fail(DEC_ERR_UNSUPPORTED, "the model has no MoE layers");
+    if (B <= 0 || B > c->max_tok) return fail(DEC_ERR_INVALID_ARG, "B out of range");
+    const size_t kk = c->c.top_k;
+    for (int l = 0; l < c->c.layers; ++l)
+        CUDA_TRY(cudaMemcpyAsync(idx + (size_t)l * B * kk, c->moe_routes + (size_t)l * c->max_tok * kk,
+                                 sizeof(int32_t) * B * kk, cudaMemcpyDeviceToHost, c->stream));
+    CUDA_TRY(cudaStreamSynchronize(c->stream));
+    return DEC_OK;
 }
 
 dec_status dec_last_hidden(dec_ctx* c, float* out, int32_t B) {

@@ -155,6 +155,62 @@ cudaError_t topk_launch(const float* logits, int T, int E, int k, int renorm, in
 #include <string>
 namespace dec {
 void set_last_error(const std::string& msg);
+
+// ----------------------------------------------------------------- MoE
+
+struct MoeRouteArgs {
+    const float* logits;  // [n][E]
+    int E, k, renorm;
+    int32_t* idx;         // [n][k]
+    float* w;             // [n][k]
+    const uint16_t* xn;   // [n][h] normalised rows (shared-expert gate input)
+    const float* gvec;    // [h] shared-expert gate vector, or null (gate = 1)
+    int h;
+    float* sgate;         // [n] sigmoid(gvec . xn), or null
+};
+cudaError_t moe_route_launch(const MoeRouteArgs& a, int n, cudaStream_t st, bool pdl);
+
+struct MoePermArgs {
+    const int32_t* idx;   // [n][k]
+    int n, k, E, nb;
+    int32_t* perm_tok;    // [n*k] token of each permuted slot
+    int32_t* inv;         // [n*k] permuted slot of (token, j)
+    int32_t* groups;      // [max_groups][4]: expert, first slot, count, 0
+    int32_t* n_groups;    // [1]
+};
+cudaError_t moe_permute_launch(const MoePermArgs& a, cudaStream_t st, bool pdl);
+
+struct GroupedGemvArgs {
+    const uint16_t* W;    // expert 0 weights [M][K]; expert e at W + e * wstride
+    size_t wstride;
+    int M, K;
+    const int32_t* groups;
+    const int32_t* n_groups;
+    const uint16_t* x;    // token rows (bf16), row of slot p = x_map ? x_map[p] : p
+    const int32_t* x_map;
+    int ldx;
+    float* y;             // STORE: y[p][row]
+    int ldy;
+    uint16_t* act;        // SWIGLU: act[p][row/2]
+    int ldact;
+    int* err;
+    int smem_cap;
+};
+int grouped_nb_for(int n);
+bool grouped_fits(int nb, int K, int smem_cap);
+cudaError_t grouped_gemv_launch(const GroupedGemvArgs& a, int nb, bool swiglu, cudaStream_t st, int num_sms,
+                                bool pdl);
+
+struct MoeCombineArgs {
+    float* x;             // [n][h] residual
+    const float* y;       // [n*k][h] routed slot outputs
+    const float* ys;      // [n][h] shared expert output, or null
+    const float* w;       // [n][k]
+    const int32_t* inv;   // [n][k]
+    const float* sgate;   // [n] or null
+    int k, h;
+};
+cudaError_t moe_combine_launch(const MoeCombineArgs& a, int n, cudaStream_t st, bool pdl);
 cudaError_t kv_move_launch(uint16_t* pool_k, uint16_t* pool_v, const int32_t* block_row, int pos0, int n, int nkv,
                            int d, uint16_t* dense_k, uint16_t* dense_v, int to_pool, cudaStream_t st);
 int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn);
