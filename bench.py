@@ -235,6 +235,164 @@ def run_reference(args):
     return 0
 
 
+WORKLOADS = {
+    # decode over synthetic caches (N(0,1) bf16 rows), greedy continuation
+    "llama3-8b-b32": dict(model="LLAMA3_8B", B=32, ctx=4096),
+    "qwen15-moe-b1": dict(model="QWEN15_MOE_A27B", B=1, ctx=2048),
+    "qwen15-moe-b64": dict(model="QWEN15_MOE_A27B", B=64, ctx=2048),
+    # prefill a prompt (chunks of 128), then batch-1 decode
+    "smollm2-135m": dict(model="SMOLLM2_135M", B=1, ctx=1024, prefill=1024),
+    "tiny": dict(model="TINY", B=1, ctx=16, prefill=16),
+    # standalone decode attention
+    "gqa-sweep": dict(),
+}
+
+
+def decode_step_bytes(cfg, B, ctx_list, experts_touched=None):
+    """Weights read once per step (MoE: only the experts some token picked) + every KV row."""
+    L, h, V = cfg["layers"], cfg["hidden"], cfg["vocab"]
+    d, nq, nkv = cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"]
+    attn = (nq * d + 2 * nkv * d) * h + h * nq * d
+    if cfg.get("n_experts", 0):
+        Ie, Is, E = cfg["expert_inter"], cfg["shared_inter"], cfg["n_experts"]
+        touched = experts_touched if experts_touched is not None else min(E, B * cfg["top_k"])
+        ffn = E * h + 3 * Is * h + touched * 3 * Ie * h
+    else:
+        ffn = 3 * cfg["ffn_inter"] * h
+    w = 2 * (L * (attn + ffn) + V * h)  # the LM head (the embedding when tied) is read once
+    kv = sum(L * c * 2 * nkv * d * 2 for c in ctx_list)
+    return w, kv
+
+
+def run_workload(args, torch, dec):
+    name = args.workload
+    P = peaks()
+    W, K = max(3, args.warmup), max(1, args.steps)
+    if name == "gqa-sweep":
+        return run_gqa_sweep(args, torch, dec, P)
+    spec = WORKLOADS[name]
+    base = getattr(configs, spec["model"])
+    B, ctx = spec["B"], spec["ctx"]
+    cfg = dict(base, max_batch=B, max_context=ctx + W + K + 8, prefill_chunk=128)
+    w = make_device_weights(cfg, torch)
+    d = dec.Decoder(cfg, w)
+    del w
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    extra = {}
+    if "prefill" in spec:
+        prompt = synth.tokens(spec["prefill"], cfg["vocab"], 1000)
+        d.prefill(0, prompt[:min(128, len(prompt))], 0)
+        d.reset(0)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        d.prefill(0, prompt, 0)
+        e1.record(stream)
+        e1.synchronize()
+        pms = e0.elapsed_time(e1)
+        extra["prefill"] = dict(tokens=len(prompt), chunk=128, ms=round(pms, 3),
+                                tok_s=round(len(prompt) / (pms * 1e-3), 1))
+        toks = d.last_argmax(1)
+    else:
+        # synthetic cache rows made on the device (same rows for every sequence and layer)
+        kvd = cfg["n_kv_heads"] * cfg["head_dim"]
+        dl, st = synth.dev_lib(), torch.cuda.current_stream().cuda_stream
+        kb = torch.empty((ctx, kvd), dtype=torch.int16, device="cuda")
+        vb = torch.empty((ctx, kvd), dtype=torch.int16, device="cuda")
+        assert dl.syn_dev_fill_bf16(kb.data_ptr(), kb.numel(), 2000, 0, 0.0, 1.0, st) == 0
+        assert dl.syn_dev_fill_bf16(vb.data_ptr(), vb.numel(), 2000, 1, 0.0, 1.0, st) == 0
+        torch.cuda.synchronize()
+        for b in range(B):
+            for l in range(cfg["layers"]):
+                d.kv_write(b, l, 0, kb, vb)
+        del kb, vb
+        toks = synth.tokens(B, cfg["vocab"], 1000)
+    pos = np.full(B, ctx, np.int32)
+    for _ in range(W):
+        d.step(toks, pos)
+        toks = d.last_argmax(B)
+        pos += 1
+    torch.cuda.synchronize()
+    clk = Clocks(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.3)
+    ctxs = []
+    e0.record(stream)
+    for _ in range(K):
+        d.step(toks, pos)
+        ctxs.extend((pos + 1).tolist())
+        pos += 1
+    e1.record(stream)
+    e1.synchronize()
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1) / K
+    touched = None
+    if cfg.get("n_experts", 0):
+        r = d.last_routes(B)  # [L][B][k] of the last timed step
+        touched = float(np.mean([len(np.unique(r[l])) for l in range(cfg["layers"])]))
+        extra["experts_touched_per_layer"] = round(touched, 2)
+    wb, kvb = decode_step_bytes(cfg, B, ctxs, touched)
+    step_bytes = wb + kvb / K
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    line = dict(metric=f"decode tok/s ({name}, b={B}, ctx {ctx})", value=B / (ms * 1e-3), unit="tok/s", n_gpus=1,
+                steps=K, warmup=W, ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="bf16", data="synthetic",
+                config=dict(workload=f"{spec['model'].lower()} shape, batch {B}, context {ctx}", global_batch=B,
+                            seq_len=ctx, l2="inputs larger than L2"),
+                step_roofline=dict(bytes_per_step=step_bytes, achieved_gbs=round(gbs, 1),
+                                   frac=round(gbs / P["hbm"], 4), peak=P["hbm"], unit="GB/s", peak_source=P["src"]),
+                clocks=clocks, **extra)
+    print(json.dumps(line))
+    d.close()
+    return 0
+
+
+def run_gqa_sweep(args, torch, dec, P):
+    B, nq, nkv, d = 64, 32, 8, 128
+    gen = torch.Generator(device="cuda").manual_seed(2000)
+    rows = []
+    clk = Clocks(int(os.environ.get("LOCAL_RANK", "0")))
+    for ctx in (512, 2048, 8192, 32768):
+        pages = B * ctx // 16
+        kp = torch.randn((pages, nkv, 16, d), device="cuda", generator=gen).to(torch.bfloat16)
+        vp = torch.randn((pages, nkv, 16, d), device="cuda", generator=gen).to(torch.bfloat16)
+        bt = torch.from_numpy(np.random.default_rng(ctx).permutation(pages).astype(np.int32).reshape(B, -1)).cuda()
+        q = torch.randn((B, nq, d), device="cuda", generator=gen).to(torch.bfloat16)
+        kn = torch.randn((B, nkv, d), device="cuda", generator=gen).to(torch.bfloat16)
+        vn = torch.randn((B, nkv, d), device="cuda", generator=gen).to(torch.bfloat16)
+        pos = torch.full((B,), ctx - 1, dtype=torch.int32, device="cuda")
+        out = torch.empty((B, nq, d), dtype=torch.bfloat16, device="cuda")
+        byts = B * ctx * nkv * d * 2 * 2
+        for rope in (0, 1):
+            def call():
+                dec.gqa_decode_attn(q, kn if rope else None, vn if rope else None, kp, vp, bt, pos, nq, nkv, d,
+                                    1 / math.sqrt(d), rope, 10000.0, out)
+            for _ in range(max(3, args.warmup)):
+                call()
+            s = torch.cuda.current_stream()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(s)
+            reps = max(1, args.steps)
+            for _ in range(reps):
+                call()
+            e1.record(s)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) / reps * 1e3
+            gbs = byts / (us * 1e-6) / 1e9
+            rows.append(dict(ctx=ctx, fused_rope=rope, us=round(us, 1), gbs=round(gbs, 1),
+                             frac=round(gbs / P["hbm"], 4)))
+        del kp, vp
+        torch.cuda.empty_cache()
+    clocks = clk.stop()
+    gm = math.exp(sum(math.log(r["gbs"]) for r in rows) / len(rows))
+    print(json.dumps(dict(metric="GQA decode attention sweep (B=64, 32q/8kv, d=128, paged 16), GB/s geomean",
+                          value=gm, unit="GB/s", n_gpus=1, steps=args.steps, warmup=args.warmup,
+                          higher_is_better=True, dtype="bf16", data="synthetic", peak=P["hbm"],
+                          peak_source=P["src"], points=rows, clocks=clocks)))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -243,6 +401,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling only; not a bench number)")
+    ap.add_argument("--workload", default="llama3-8b", choices=["llama3-8b"] + sorted(WORKLOADS),
+                    help="llama3-8b: the headline line (prefill 4096 + batch-1 decode); others: one extra line each")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -251,6 +411,9 @@ def main():
     import torch.distributed as dist
 
     import decoder_only_transformer_layer_b200 as dec
+
+    if args.workload != "llama3-8b":
+        return run_workload(args, torch, dec)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

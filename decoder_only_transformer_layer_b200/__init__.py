@@ -202,9 +202,11 @@ class Decoder:
 
     # ------------------------------------------------------------------ test hooks
     def kv_write(self, seq, layer, pos0, k, v):
-        k = np.ascontiguousarray(k, np.uint16)
-        v = np.ascontiguousarray(v, np.uint16)
-        _check(lib().dec_kv_write(self.h, seq, layer, pos0, k.shape[0], k.ctypes.data, v.ctypes.data))
+        """k, v: bf16 rows [n][nkv*d] as uint16 numpy arrays (host) or 16-bit torch tensors."""
+        if not hasattr(k, "data_ptr"):
+            k = np.ascontiguousarray(k, np.uint16)
+            v = np.ascontiguousarray(v, np.uint16)
+        _check(lib().dec_kv_write(self.h, seq, layer, pos0, k.shape[0], _ptr(k), _ptr(v)))
 
     def kv_read(self, seq, layer, pos0, n):
         kvd = self.cfg["n_kv_heads"] * self.cfg["head_dim"]
