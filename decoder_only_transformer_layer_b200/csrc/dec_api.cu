@@ -93,10 +93,6 @@ struct dec_ctx {
     int* attn_cnt = nullptr;
     size_t attn_part_floats = 0;
     int attn_cnt_n = 0;
-    float* gemm_ws = nullptr;
-    size_t gemm_ws_n = 0;
-    int* gemm_cnt = nullptr;
-    int gemm_cnt_n = 0;
     int* d_err = nullptr;
     int32_t* h_stage = nullptr;  // pinned: tokens, positions, block rows
     int* h_err = nullptr;
@@ -193,8 +189,6 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
     }
     GemmPlan plan;
     CUDA_TRY(gemm_plan(&plan, p.W, p.M, p.K, in, n, c->num_sms));
-    if (gemm_ws_floats(plan) > c->gemm_ws_n || gemm_tiles(plan) > c->gemm_cnt_n)
-        return fail(DEC_ERR_UNSUPPORTED, "GEMM workspace too small for this shape");
     GemmArgs a{};
     a.epi = epi;
     a.y = y;
@@ -202,8 +196,6 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
     a.bias = bias;
     a.act = act;
     a.ldact = ldact;
-    a.ws = c->gemm_ws;
-    a.counters = c->gemm_cnt;
     a.amax = amax;
     a.err = c->d_err;
     CUDA_TRY(gemm_launch(plan, a, st, true));
@@ -704,34 +696,6 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(dmalloc(&c->attn_cnt, c->attn_cnt_n));
     INIT_TRY(cudaMemsetAsync(c->attn_cnt, 0, (size_t)c->attn_cnt_n * 4, st));
 
-    // GEMM split workspace: the largest projection at the largest token count that uses the GEMM
-    {
-        size_t ws = 0;
-        int cnt = 0;
-        // (rows, K) of every projection that can run on the GEMM
-        std::vector<int> Ms = {c->qkv_rows, h, k.vocab}, Ks = {h, c->qd, h};
-        if (k.n_experts > 0) {
-            Ms.insert(Ms.end(), {k.n_experts, 2 * k.shared_inter, h});
-            Ks.insert(Ks.end(), {h, h, k.shared_inter});
-        } else {
-            Ms.insert(Ms.end(), {2 * k.ffn_inter, h});
-            Ks.insert(Ks.end(), {h, k.ffn_inter});
-        }
-        // every token count a prefill chunk (tail included) or a decode batch can have
-        for (int n = 1; n <= std::max(pre_T, k.max_batch); ++n)
-            for (size_t j = 0; j < Ms.size(); ++j) {
-                if (Ms[j] <= 0 || Ks[j] <= 0) continue;
-                int bn = 0;
-                const int sp = gemm_choose_splits(Ms[j], n, Ks[j], c->num_sms, &bn);
-                if (sp > 1) ws = std::max(ws, (size_t)sp * n * Ms[j]);
-                cnt = std::max(cnt, ((Ms[j] + 127) / 128) * ((n + bn - 1) / bn));
-            }
-        c->gemm_ws_n = ws;
-        c->gemm_cnt_n = cnt;
-        INIT_TRY(dmalloc(&c->gemm_ws, ws));
-        INIT_TRY(dmalloc(&c->gemm_cnt, cnt));
-        INIT_TRY(cudaMemsetAsync(c->gemm_cnt, 0, (size_t)cnt * 4, st));
-    }
     INIT_TRY(cudaStreamSynchronize(st));
 #undef INIT_TRY
     *out = c;
@@ -777,8 +741,6 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->act);
     cudaFree(c->attn_part);
     cudaFree(c->attn_cnt);
-    cudaFree(c->gemm_ws);
-    cudaFree(c->gemm_cnt);
     cudaFree(c->moe_logits);
     cudaFree(c->moe_w);
     cudaFree(c->moe_sgate);
@@ -1089,14 +1051,10 @@ dec_status weight_gemv(const void* W, const void* x, int32_t B, int32_t N, int32
     }
     GemmPlan plan;
     CUDA_TRY(gemm_plan(&plan, static_cast<const uint16_t*>(W), N, K, static_cast<const uint16_t*>(x), B, sms));
-    CUDA_TRY(grow(&S.ws, &S.ws_n, std::max<size_t>(1, gemm_ws_floats(plan)), false));
-    CUDA_TRY(grow(&S.cnt, &S.cnt_n, (size_t)gemm_tiles(plan), true));
     GemmArgs a{};
     a.epi = GEMM_STORE;
     a.y = y;
     a.ldy = N;
-    a.ws = S.ws;
-    a.counters = S.cnt;
     a.err = S.err;
     CUDA_TRY(gemm_launch(plan, a, st, false));
     return DEC_OK;

@@ -102,6 +102,42 @@ DEC_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.ld of 16 columns without waiting; the values are valid after tmem_ld_wait32.
+DEC_DEVINL void tmem_ld16_issue(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Wait for outstanding tcgen05.ld; the registers are in-out operands so no use of them can
+// be scheduled before the wait.
+DEC_DEVINL void tmem_ld_wait32(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// Barrier across every CTA of the cluster, with release/acquire ordering of shared memory.
+DEC_DEVINL void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 16-byte store into the shared memory of CTA `rank` of this cluster, at the same offset as
+// the local shared address `saddr` (fire-and-forget; ordered by the next cluster barrier).
+DEC_DEVINL void dsmem_st4(uint32_t saddr, int rank, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(saddr), "r"(rank));
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
 // Apply the epilogue to the 16 values v[j] of (row, t0 + j). All lanes of the warp call
 // it together (the SwiGLU pairing uses a shuffle). Every global load of a chunk is issued
 // before any store, so the 16 accesses overlap instead of waiting on one another.
@@ -235,24 +271,39 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();
     const bool acc_ready = mbar_wait_bounded(accb, 0, a.err);
     tc_fence_after();
-    const int row = m0 + warp * 32 + lane;
+    const int rloc = warp * 32 + lane;
+    const int row = m0 + rloc;
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(lane_base + (uint32_t)c0, r);
+    // Split-K: the a.splits CTAs of this tile form one cluster. CTA r owns rows
+    // [r*rp, r*rp + rp) of the tile; every CTA pushes its partial of those rows into the
+    // owner's receive buffer (drained stage ring, [split][row][BN + 4] fp32, vector stores
+    // to distributed shared memory, no waiting), then after one cluster barrier each owner
+    // sums its rows over the splits in split order from local shared memory (deterministic).
+    const int S = a.splits;
+    const int rp = (((BM + S - 1) / S) + 1) & ~1;  // even, so SwiGLU pairs stay in one slice
+    constexpr int LDR = BN + 4;                    // padded row: conflict-free vector access
+    const uint32_t recv = smem_u32(smem);
+    const int owner = rloc / rp, lr = rloc - owner * rp;
+    if (S > 1) cluster_sync();  // every CTA's stage ring is drained before any partial lands in it
+    for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld16_issue(lane_base + (uint32_t)c0, r);
+        tmem_ld16_issue(lane_base + (uint32_t)c0 + 16, r + 16);
+        tmem_ld_wait32(r);
         if (!acc_ready) continue;
-        float v[16];
+        if (S == 1) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-        if (a.splits == 1) {
-            epilogue16(a, row, n0 + c0, v);
-            if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0, v);
-        } else if (row < a.M) {
+            for (int h = 0; h < 2; ++h) {
+                float v[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int t = n0 + c0 + j;
-                if (t < a.N) a.ws[((size_t)z * a.N + t) * a.M + row] = v[j];
+                for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[16 * h + j]);
+                epilogue16(a, row, n0 + c0 + 16 * h, v);
+                if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0 + 16 * h, v);
             }
+        } else {
+            const uint32_t dst = recv + (uint32_t)(((z * rp + lr) * LDR + c0) * 4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dsmem_st4(dst + q * 16, owner, r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
         }
     }
     tc_fence_before();
@@ -263,36 +314,61 @@ __global__ void __launch_bounds__(128, 1)
                      : "memory");
     }
     (void)ok;
-    if (a.splits == 1 || !acc_ready) return;
+    (void)ticket;
+    if (S == 1) return;
 
-    // ---------------------------------------------------- split-K: last CTA of the tile reduces
-    __threadfence();
-    __syncthreads();
-    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-    if (threadIdx.x == 0) *ticket = atomicAdd(&a.counters[tile], 1);
-    __syncthreads();
-    if (*ticket != a.splits - 1) return;
-    __threadfence();
-    const int ncols = min(BN, a.N - n0);
-    for (int c0 = 0; c0 < ncols; c0 += 16) {
-        float v[16];
+    cluster_sync();  // all partials have arrived; from here on only local shared memory is read
+    const int r_lo = min(BM, z * rp), nr = min(BM, r_lo + rp) - r_lo;
+    const float* rb = reinterpret_cast<const float*>(smem);
+    if (!acc_ready || nr <= 0) return;
+    if (a.epi == GEMM_SWIGLU) {
+        const int np = nr / 2;
+        for (int i = threadIdx.x; i < np * (BN / 4); i += 128) {
+            const int lp = 2 * (i % np), c4 = 4 * (i / np);
+            float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
+            for (int s2 = 0; s2 < S; ++s2) {
+                const float4 pg = *reinterpret_cast<const float4*>(rb + (s2 * rp + lp) * LDR + c4);
+                const float4 pu = *reinterpret_cast<const float4*>(rb + (s2 * rp + lp + 1) * LDR + c4);
+                g.x += pg.x, g.y += pg.y, g.z += pg.z, g.w += pg.w;
+                u.x += pu.x, u.y += pu.y, u.z += pu.z, u.w += pu.w;
+            }
+            const int grow = m0 + r_lo + lp;
+            if (grow >= a.M) continue;
+            const float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.f;
-        if (row < a.M) {
-            // splits summed in split order; all loads of a split are independent
-            for (int s = 0; s < a.splits; ++s) {
-                float p[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    p[j] = c0 + j < ncols ? __ldcg(a.ws + ((size_t)s * a.N + n0 + c0 + j) * a.M + row) : 0.f;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] += p[j];
+            for (int q = 0; q < 4; ++q) {
+                const int t = n0 + c4 + q;
+                if (t >= a.N) continue;
+                const float sg = gv[q] * (1.0f / (1.0f + expf(-gv[q])));
+                a.act[(size_t)t * a.ldact + (grow >> 1)] = f2bf(sg * uv[q]);
             }
         }
-        epilogue16(a, row, n0 + c0, v);
-        if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0, v);
+    } else {
+        for (int i = threadIdx.x; i < nr * (BN / 4); i += 128) {
+            const int l = i % nr, c4 = 4 * (i / nr);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s2 = 0; s2 < S; ++s2) {
+                const float4 p = *reinterpret_cast<const float4*>(rb + (s2 * rp + l) * LDR + c4);
+                v.x += p.x, v.y += p.y, v.z += p.z, v.w += p.w;
+            }
+            const int grow = m0 + r_lo + l;
+            if (grow >= a.M) continue;
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+            const float bias = (a.epi == GEMM_STORE && a.bias) ? a.bias[grow] : 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = n0 + c4 + q;
+                if (t >= a.N) continue;
+                float* dst = a.y + (size_t)t * a.ldy + grow;
+                if (a.epi == GEMM_RESID) {
+                    *dst += vv[q];
+                } else {
+                    *dst = vv[q] + bias;
+                    if (a.amax) atomicMax(&a.amax[(size_t)t * 32], argmax_pack(vv[q] + bias, grow));
+                }
+            }
+        }
     }
-    if (threadIdx.x == 0) a.counters[tile] = 0;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -334,19 +410,28 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (p.splits > 1) {  // the split CTAs of a tile form one cluster (reduction through DSMEM)
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = p.splits;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, a);
 }
 
 }  // namespace
 
 int gemm_tiles(const GemmPlan& p) { return ((p.M + BM - 1) / BM) * ((p.N + p.bn - 1) / p.bn); }
-
-size_t gemm_ws_floats(const GemmPlan& p) { return p.splits > 1 ? (size_t)p.splits * p.N * p.M : 0; }
 
 int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn_out) {
     const int bn = N <= 32 ? 32 : N <= 64 ? 64 : 128;

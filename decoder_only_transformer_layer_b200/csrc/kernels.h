@@ -53,16 +53,13 @@ struct GemmArgs {
     const float* bias;
     uint16_t* act;
     int ldact;
-    int splits;
-    float* ws;        // split partials [splits][N][M] fp32
-    int* counters;    // [tiles], zero on entry, left zero on exit
+    int splits;       // K splits: the split CTAs of a tile form one cluster (<= 8)
     unsigned long long* amax;  // STORE: per token, packed greedy argmax of y (null = off)
     int* err;
 };
 
 // Build the tensor maps for one GEMM shape (host; encodes A and B addresses).
 cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms);
-size_t gemm_ws_floats(const GemmPlan& p);
 int gemm_tiles(const GemmPlan& p);
 cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl);
 
