@@ -440,19 +440,114 @@ __global__ void __launch_bounds__(128) rope_append_kernel(RopeAppendArgs a) {
 
 // ================================================================== prefill attention
 
-constexpr int kPrefRows = 64;   // (token, head) rows per CTA: 4 warps x 16
-constexpr int kPrefKeys = 64;   // keys per shared block (4 pages)
+constexpr int kPrefRows = 64;      // (token, head) rows per CTA: 4 warps x 16
+constexpr int kPrefKeys = 64;      // keys per shared block (4 pages)
+constexpr int kPrefMaxSplits = 8;  // key splits of one row block: the CTAs of one cluster
 
+// K and V blocks, double-buffered, rows padded to D + 8 (conflict-free ldmatrix).
 template <int D>
-__global__ void __launch_bounds__(128) attn_prefill_kernel(AttnPrefillArgs a) {
+constexpr size_t prefill_smem() {
+    return (size_t)2 * 2 * kPrefKeys * (D + 8) * 2;
+}
+
+// S = Q K^T for one 64-key block: sc[nt] holds keys 8 nt .. 8 nt + 7 of the block.
+template <int D, int LD>
+DEC_DEVINL void qk_block(const uint32_t (&qf)[D / 16][4], const uint16_t* kd, float (&sc)[8][4]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    const int key = (lane & 7) + (lane >> 4) * 8;
+    const int col = ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+#pragma unroll
+        for (int kp = 0; kp < 4; ++kp) {
+            uint32_t kb[4];
+            ldsm_x4(kb, kd + (kp * 16 + key) * LD + ks * 16 + col);
+            const uint32_t b0[2] = {kb[0], kb[1]}, b1[2] = {kb[2], kb[3]};
+            mma_bf16_16816(sc[2 * kp], qf[ks], b0);
+            mma_bf16_16816(sc[2 * kp + 1], qf[ks], b1);
+        }
+    }
+}
+
+// Online-softmax update over one 64-key block (log2 units; masked entries -inf).
+// Rows g (r = 0) and g + 8 (r = 1) of the warp's 16; the quad's four threads hold
+// the block's 64 columns of a row. Returns P in sc and the rescale factor of o.
+DEC_DEVINL void softmax_block(float (&sc)[8][4], float (&m)[2], float (&l)[2], float (&corr)[2]) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][2 * r], sc[nt][2 * r + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mn = fmaxf(m[r], mx);
+        if (mn == -INFINITY) {  // every key so far masked for this row
+            corr[r] = 1.f;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) sc[nt][2 * r] = sc[nt][2 * r + 1] = 0.f;
+            continue;
+        }
+        corr[r] = exp2f(m[r] - mn);
+        m[r] = mn;
+        float sum = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float p = exp2f(sc[nt][2 * r + c] - mn);
+                sc[nt][2 * r + c] = p;
+                sum += p;
+            }
+        l[r] = l[r] * corr[r] + sum;
+    }
+}
+
+// O += P V for one 64-key block; P enters as bf16 hi + lo parts.
+template <int D, int LD>
+DEC_DEVINL void pv_block(const float (&sc)[8][4], const uint16_t* vd, float (&o)[D / 8][4]) {
+    const int lane = threadIdx.x & 31;
+    const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int col = (lane >> 4) * 8;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float v[8] = {sc[2 * j][0],     sc[2 * j][1],     sc[2 * j][2],     sc[2 * j][3],
+                            sc[2 * j + 1][0], sc[2 * j + 1][1], sc[2 * j + 1][2], sc[2 * j + 1][3]};
+        uint32_t ph[4], pl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float x = v[2 * i], y = v[2 * i + 1];
+            const float xh = round_bf(x), yh = round_bf(y);
+            ph[i] = pack_bf2(xh, yh);
+            pl[i] = pack_bf2(x - xh, y - yh);
+        }
+#pragma unroll
+        for (int dt2 = 0; dt2 < D / 16; ++dt2) {
+            uint32_t vb[4];
+            ldsm_x4_trans(vb, vd + (j * 16 + key) * LD + dt2 * 16 + col);
+            const uint32_t b0[2] = {vb[0], vb[1]}, b1[2] = {vb[2], vb[3]};
+            mma_bf16_16816(o[2 * dt2], ph, b0);
+            mma_bf16_16816(o[2 * dt2 + 1], ph, b1);
+            mma_bf16_16816(o[2 * dt2], pl, b0);
+            mma_bf16_16816(o[2 * dt2 + 1], pl, b1);
+        }
+    }
+}
+
+// One CTA: 64 (token, head) rows of kv head g -- row r is token r / G, head g G + r % G --
+// against key split blockIdx.z of the keys those rows may see. With several splits the
+// split CTAs form one cluster: after the key loop each pushes its unnormalised rows
+// (o, running max m, sum l) into the shared memory of the CTA that owns the row, and
+// the owners merge the splits in rank order.
+template <int D>
+__global__ void __launch_bounds__(128, 3) attn_prefill_kernel(AttnPrefillArgs a) {
     constexpr int LD = D + 8;
     extern __shared__ __align__(16) uint8_t dyn[];
-    uint16_t* qsm = reinterpret_cast<uint16_t*>(dyn);   // [4][16][LD]
-    uint16_t* kb = qsm + 4 * 16 * LD;                   // [2][64][LD]
-    uint16_t* vb = kb + 2 * kPrefKeys * LD;             // [2][64][LD]
-    __shared__ int ticket_s;
+    uint16_t* kb = reinterpret_cast<uint16_t*>(dyn);  // [2][64][LD]
+    uint16_t* vb = kb + 2 * kPrefKeys * LD;           // [2][64][LD]
 
-    const int qb = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int qb = blockIdx.x, g = blockIdx.y, s = blockIdx.z, S = gridDim.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int G = a.nq / a.nkv;
     const int R = a.T * G;
@@ -462,34 +557,36 @@ __global__ void __launch_bounds__(128) attn_prefill_kernel(AttnPrefillArgs a) {
     const int rbase = qb * kPrefRows;
     const int t_last = min(a.T - 1, (rbase + kPrefRows - 1) / G);
     const int n_cta = a.pos0 + t_last + 1;  // keys any row of this CTA may see
-    const int np = (n_cta + kPage - 1) / kPage;
-    const int pps = (np + a.splits - 1) / a.splits;
-    const int pg0 = s * pps, pg1 = min(np, pg0 + pps);
+    const int nblk = (n_cta + kPrefKeys - 1) / kPrefKeys;
+    const int bps = (nblk + S - 1) / S;
+    const int blk0 = s * bps, blk1 = min(nblk, blk0 + bps);
 
-    // this warp's rows
+    // this thread's rows (g and g + 8 of the warp's 16) and their last visible key
     const int r0 = rbase + warp * 16;
     const int gr = lane >> 2, t4 = lane & 3;
-    const int ra = r0 + gr, rb2 = r0 + gr + 8;  // rows held by this thread
+    const int ra = r0 + gr, rb = r0 + gr + 8;
     const int lim_a = ra < R ? a.pos0 + ra / G : -1;
-    const int lim_b = rb2 < R ? a.pos0 + rb2 / G : -1;
-    const int warp_max_row = min(R - 1, r0 + 15);
-    const int warp_lim = r0 < R ? a.pos0 + warp_max_row / G : -1;
+    const int lim_b = rb < R ? a.pos0 + rb / G : -1;
+    const int warp_hi = r0 < R ? a.pos0 + min(R - 1, r0 + 15) / G : -1;  // largest limit of the warp
+    const int warp_lo = r0 + 15 < R ? a.pos0 + r0 / G : -1;              // smallest (-1: padding rows)
 
-    // q rows -> shared -> fragments
-    uint16_t* qw = qsm + warp * 16 * LD;
-    for (int i = lane; i < 16 * (D / 8); i += 32) {
-        const int rr = i / (D / 8), col = (i % (D / 8)) * 8;
-        const int r = r0 + rr;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < R) {
-            const int t = r / G, h = g * G + r % G;
-            v = *reinterpret_cast<const uint4*>(a.q + ((size_t)t * a.nq + h) * D + col);
-        }
-        *reinterpret_cast<uint4*>(qw + rr * LD + col) = v;
-    }
-    __syncwarp();
+    // Q fragments straight from global memory (A layout of m16n8k16)
     uint32_t qf[D / 16][4];
-    load_q_frags<D, LD>(qw, qf);
+    {
+        const uint32_t* qa = ra < R ? reinterpret_cast<const uint32_t*>(
+                                          a.q + ((size_t)(ra / G) * a.nq + g * G + ra % G) * D)
+                                    : nullptr;
+        const uint32_t* qbp = rb < R ? reinterpret_cast<const uint32_t*>(
+                                           a.q + ((size_t)(rb / G) * a.nq + g * G + rb % G) * D)
+                                     : nullptr;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            qf[ks][0] = qa ? __ldg(qa + ks * 8 + t4) : 0u;
+            qf[ks][1] = qbp ? __ldg(qbp + ks * 8 + t4) : 0u;
+            qf[ks][2] = qa ? __ldg(qa + ks * 8 + 4 + t4) : 0u;
+            qf[ks][3] = qbp ? __ldg(qbp + ks * 8 + 4 + t4) : 0u;
+        }
+    }
 
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     float o[D / 8][4];
@@ -497,51 +594,57 @@ __global__ void __launch_bounds__(128) attn_prefill_kernel(AttnPrefillArgs a) {
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     const float sl2 = a.scale * kLog2e;
 
-    auto load_block = [&](int blk_pg, int buf) {
+    // keys at or past n_cta are not read: their rows are zero-filled (weight 0, finite)
+    auto load_block = [&](int blk, int buf) {
         uint16_t* kd = kb + buf * kPrefKeys * LD;
         uint16_t* vd = vb + buf * kPrefKeys * LD;
         constexpr int CH = kPrefKeys * D / 8;
         for (int c = tid; c < CH; c += 128) {
             const int key = c / (D / 8), col = (c % (D / 8)) * 8;
-            const int pg = blk_pg + key / kPage;
-            if (pg < pg1) {
-                const int phys = a.block_row[pg];
-                const size_t off = (((size_t)phys * a.nkv + g) * kPage + key % kPage) * D + col;
+            const int kg = blk * kPrefKeys + key;
+            if (kg < n_cta) {
+                const int phys = a.block_row[kg / kPage];
+                const size_t off = (((size_t)phys * a.nkv + g) * kPage + kg % kPage) * D + col;
                 cp_async16(kd + key * LD + col, a.k_pool + off);
                 cp_async16(vd + key * LD + col, a.v_pool + off);
+            } else {
+                *reinterpret_cast<uint4*>(kd + key * LD + col) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(vd + key * LD + col) = make_uint4(0, 0, 0, 0);
             }
         }
         cp_async_commit();
     };
 
-    const int kpp = kPrefKeys / kPage;
     int buf = 0;
-    if (pg0 < pg1) load_block(pg0, 0);
-    for (int bp = pg0; bp < pg1; bp += kpp) {
-        if (bp + kpp < pg1) {
-            load_block(bp + kpp, buf ^ 1);
+    if (blk0 < blk1) load_block(blk0, 0);
+    for (int blk = blk0; blk < blk1; ++blk) {
+        if (blk + 1 < blk1) {
+            load_block(blk + 1, buf ^ 1);
             cp_async_wait<1>();
         } else {
             cp_async_wait<0>();
         }
         __syncthreads();
-        const uint16_t* kd = kb + buf * kPrefKeys * LD;
-        const uint16_t* vd = vb + buf * kPrefKeys * LD;
-        for (int pi = 0; pi < kpp; ++pi) {
-            const int pg = bp + pi;
-            if (pg >= pg1 || pg * kPage > warp_lim) break;  // fully masked for this warp
-            float sc[2][4];
-            qk_page<D, LD>(qf, kd + pi * kPage * LD, sc);
+        const int k0 = blk * kPrefKeys;
+        if (k0 <= warp_hi) {  // else every key of the block is masked for this warp's rows
+            float sc[8][4];
+            qk_block<D, LD>(qf, kb + buf * kPrefKeys * LD, sc);
+            if (k0 + kPrefKeys - 1 > warp_lo) {  // the causal edge (or padding rows) cross the block
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int key = pg * kPage + nt * 8 + 2 * t4 + (c & 1);
-                    const int lim = c < 2 ? lim_a : lim_b;
-                    sc[nt][c] = key <= lim ? sc[nt][c] * sl2 : -INFINITY;
-                }
+                    for (int c = 0; c < 4; ++c) {
+                        const int key = k0 + nt * 8 + 2 * t4 + (c & 1);
+                        sc[nt][c] = key <= (c < 2 ? lim_a : lim_b) ? sc[nt][c] * sl2 : -INFINITY;
+                    }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sc[nt][c] *= sl2;
+            }
             float corr[2];
-            softmax_page(sc, m, l, corr);
+            softmax_block(sc, m, l, corr);
 #pragma unroll
             for (int i = 0; i < D / 8; ++i) {
                 o[i][0] *= corr[0];
@@ -549,7 +652,7 @@ __global__ void __launch_bounds__(128) attn_prefill_kernel(AttnPrefillArgs a) {
                 o[i][2] *= corr[1];
                 o[i][3] *= corr[1];
             }
-            pv_page<D, LD>(sc, vd + pi * kPage * LD, o);
+            pv_block<D, LD>(sc, vb + buf * kPrefKeys * LD, o);
         }
         __syncthreads();  // buffer reuse
         buf ^= 1;
@@ -560,62 +663,64 @@ __global__ void __launch_bounds__(128) attn_prefill_kernel(AttnPrefillArgs a) {
         l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
     }
 
-    // ---- write rows (or split partials)
+    if (S == 1) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int r = hr == 0 ? ra : rb;
+            if (r >= R) continue;
+            const int t = r / G, h = g * G + r % G;
+            const float inv = 1.0f / l[hr];
+            uint32_t* dst = reinterpret_cast<uint32_t*>(a.out + (size_t)t * a.nq * D + (size_t)h * D);
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) dst[i * 4 + t4] = pack_bf2(o[i][2 * hr] * inv, o[i][2 * hr + 1] * inv);
+        }
+        return;
+    }
+
+    // ---- split merge inside the cluster; the K/V buffers become the receive area
+    constexpr int LDR = D + 4;  // o[D], m, l, 2 pad: 16-byte aligned rows
+    const int rp = (kPrefRows + S - 1) / S;  // rows owned by each CTA of the cluster
+    const int rank = (int)cluster_rank();
+    float* recv = reinterpret_cast<float*>(dyn);  // [S][rp][LDR]
+    cluster_sync();  // every CTA's key loop is done before partials land in its buffers
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
-        const int r = hr == 0 ? ra : rb2;
-        if (r >= R) continue;
-        const int t = r / G, h = g * G + r % G;
-        if (a.splits == 1) {
-            const float inv = 1.0f / l[hr];
-            uint16_t* dst = a.out + (size_t)t * a.nq * D + (size_t)h * D;
+        const int lr = warp * 16 + gr + 8 * hr;
+        const int owner = lr / rp, orow = lr - owner * rp;
+        const uint32_t dst = smem_u32(recv + ((size_t)rank * rp + orow) * LDR);
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                dst[i * 8 + 2 * t4] = f2bf(o[i][2 * hr] * inv);
-                dst[i * 8 + 2 * t4 + 1] = f2bf(o[i][2 * hr + 1] * inv);
-            }
-        } else {
-            float* pp = a.part + ((size_t)s * a.T * a.nq + (size_t)t * a.nq + h) * (D + 2);
-#pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                pp[i * 8 + 2 * t4] = o[i][2 * hr];
-                pp[i * 8 + 2 * t4 + 1] = o[i][2 * hr + 1];
-            }
-            if (t4 == 0) {
-                pp[D] = m[hr];
-                pp[D + 1] = l[hr];
-            }
-        }
+        for (int i = 0; i < D / 8; ++i) dsmem_st2f(dst + (i * 8 + 2 * t4) * 4, owner, o[i][2 * hr], o[i][2 * hr + 1]);
+        if (t4 == 0) dsmem_st2f(dst + D * 4, owner, m[hr], l[hr]);
     }
-    if (a.splits == 1) return;
-
-    __threadfence();
-    __syncthreads();
-    const int cidx = qb * a.nkv + g;
-    if (tid == 0) ticket_s = atomicAdd(&a.counters[cidx], 1);
-    __syncthreads();
-    if (ticket_s != a.splits - 1) return;
-    __threadfence();
-    const int nrows = min(kPrefRows, R - rbase);
-    for (int idx = tid; idx < nrows * D; idx += 128) {
-        const int r = rbase + idx / D, c = idx % D;
-        const int t = r / G, h = g * G + r % G;
-        const size_t row = (size_t)t * a.nq + h;
+    cluster_sync();  // all partials have arrived; only local shared memory is read below
+    const int lr0 = rank * rp, nr = min(kPrefRows, lr0 + rp) - lr0;
+    for (int idx = tid; idx < nr * (D / 4); idx += 128) {
+        const int orow = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+        const int r = rbase + lr0 + orow;
+        if (r >= R) continue;
         float M = -INFINITY;
-        for (int z = 0; z < a.splits; ++z)
-            M = fmaxf(M, __ldcg(a.part + ((size_t)z * a.T * a.nq + row) * (D + 2) + D));
-        float L = 0.f, O = 0.f;
-        for (int z = 0; z < a.splits; ++z) {
-            const float* pp = a.part + ((size_t)z * a.T * a.nq + row) * (D + 2);
-            const float mz = __ldcg(pp + D);
+        for (int z = 0; z < S; ++z) M = fmaxf(M, recv[((size_t)z * rp + orow) * LDR + D]);
+        float L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int z = 0; z < S; ++z) {
+            const float* pz = recv + ((size_t)z * rp + orow) * LDR;
+            const float mz = pz[D];
             if (mz == -INFINITY) continue;
             const float f = exp2f(mz - M);
-            L += f * __ldcg(pp + D + 1);
-            O += f * __ldcg(pp + c);
+            L += f * pz[D + 1];
+            const float4 v = *reinterpret_cast<const float4*>(pz + c4);
+            O.x += f * v.x;
+            O.y += f * v.y;
+            O.z += f * v.z;
+            O.w += f * v.w;
         }
-        a.out[(size_t)t * a.nq * D + (size_t)h * D + c] = f2bf(O / L);
+        const float inv = 1.0f / L;
+        const int t = r / G, h = g * G + r % G;
+        uint2 pk;
+        pk.x = pack_bf2(O.x * inv, O.y * inv);
+        pk.y = pack_bf2(O.z * inv, O.w * inv);
+        *reinterpret_cast<uint2*>(a.out + (size_t)t * a.nq * D + (size_t)h * D + c4) = pk;
     }
-    if (tid == 0) a.counters[cidx] = 0;
 }
 
 template <typename K, typename Args>
@@ -680,39 +785,56 @@ cudaError_t rope_append_launch(const RopeAppendArgs& a, cudaStream_t st, bool pd
     return cudaErrorInvalidValue;
 }
 
+// Key splits per 64-row block so that the grid fills about one wave at three CTAs per SM;
+// at most one split per 64-key block and at most a portable cluster (8).
 int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms) {
     const int G = nq / nkv;
     const int qblocks = (T * G + kPrefRows - 1) / kPrefRows;
     const int ctas = qblocks * nkv;
-    int s = (2 * num_sms + ctas - 1) / ctas;
+    int s = (3 * num_sms) / ctas;
     const int blocks = (ctx + kPrefKeys - 1) / kPrefKeys;
     if (s > blocks) s = blocks;
+    if (s > kPrefMaxSplits) s = kPrefMaxSplits;
     if (s < 1) s = 1;
     return s;
 }
 
-size_t attn_prefill_part_floats(int T, int nq, int d, int splits) {
-    return splits > 1 ? (size_t)splits * T * nq * (d + 2) : 0;
+template <int D>
+cudaError_t prefill_launch_d(const AttnPrefillArgs& a, cudaStream_t st, bool pdl) {
+    const int G = a.nq / a.nkv;
+    const int qblocks = (a.T * G + kPrefRows - 1) / kPrefRows;
+    const size_t smem = prefill_smem<D>();
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(qblocks, a.nkv, a.splits);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (a.splits > 1) {  // the key splits of a row block form one cluster (merge through DSMEM)
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = a.splits;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, attn_prefill_kernel<D>, a);
 }
 
 cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl) {
-    const int G = a.nq / a.nkv;
-    const int qblocks = (a.T * G + kPrefRows - 1) / kPrefRows;
-    const dim3 grid(qblocks, a.nkv, a.splits);
-    if (a.d == 128) {
-        const size_t smem = ((size_t)4 * 16 + 4 * kPrefKeys) * (128 + 8) * 2;
-        cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_ex(attn_prefill_kernel<128>, grid, dim3(128), smem, st, pdl, a);
-    }
-    if (a.d == 64) {
-        const size_t smem = ((size_t)4 * 16 + 4 * kPrefKeys) * (64 + 8) * 2;
-        cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_ex(attn_prefill_kernel<64>, grid, dim3(128), smem, st, pdl, a);
-    }
+    if (a.T <= 0) return cudaSuccess;
+    if (a.splits < 1 || a.splits > kPrefMaxSplits) return cudaErrorInvalidValue;
+    if (a.d == 128) return prefill_launch_d<128>(a, st, pdl);
+    if (a.d == 64) return prefill_launch_d<64>(a, st, pdl);
     return cudaErrorInvalidValue;
 }
 

@@ -153,6 +153,39 @@ DEC_DEVINL void ldsm_x4_trans(uint32_t* r, const void* p) {
                  : "r"(smem_u32(p)));
 }
 
+// ----------------------------------------------------------------- thread-block clusters
+
+// Barrier across every CTA of the cluster, with release/acquire ordering of shared memory.
+DEC_DEVINL void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+DEC_DEVINL uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+DEC_DEVINL uint32_t dsmem_map(uint32_t saddr, int rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(saddr), "r"(rank));
+    return remote;
+}
+
+// 16-byte store into the shared memory of CTA `rank` of this cluster, at the same offset as
+// the local shared address `saddr` (fire-and-forget; ordered by the next cluster barrier).
+DEC_DEVINL void dsmem_st4(uint32_t saddr, int rank, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    const uint32_t remote = dsmem_map(saddr, rank);
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// 8-byte store of two floats into CTA `rank`'s shared memory (see dsmem_st4).
+DEC_DEVINL void dsmem_st2f(uint32_t saddr, int rank, float a, float b) {
+    const uint32_t remote = dsmem_map(saddr, rank);
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(a), "f"(b) : "memory");
+}
+
 // ----------------------------------------------------------------- RoPE angle
 
 // cos/sin of pos * base^(-2i/d), evaluated in fp64 and rounded to fp32.

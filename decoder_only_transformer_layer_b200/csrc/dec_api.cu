@@ -358,10 +358,6 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
             a.d = d;
             a.scale = scale;
             a.splits = attn_prefill_splits(n, k.n_q_heads, k.n_kv_heads, pos0 + n, c->num_sms);
-            while (a.splits > 1 && attn_prefill_part_floats(n, k.n_q_heads, d, a.splits) > c->attn_part_floats)
-                --a.splits;
-            a.part = c->attn_part;
-            a.counters = c->attn_cnt;
             a.out = c->attn;
             a.err = c->d_err;
             CUDA_TRY(attn_prefill_launch(a, st, true));
@@ -682,17 +678,12 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_err), sizeof(int)));
     *c->h_err = 0;
 
-    // attention scratch: decode splits over max_context for max_batch; prefill splits over a chunk
+    // decode attention scratch: split partials over max_context for max_batch (prefill
+    // attention merges its splits inside a cluster and needs none)
     c->decode_splits = attn_decode_splits(k.max_batch, k.n_kv_heads, k.max_context, c->num_sms);
-    size_t dec_part = c->decode_splits > 1 ? (size_t)k.max_batch * k.n_q_heads * c->decode_splits * (d + 2) : 0;
-    const int pre_T = std::min(k.prefill_chunk, k.max_context);
-    const int pre_s = attn_prefill_splits(pre_T, k.n_q_heads, k.n_kv_heads, k.max_context, c->num_sms);
-    size_t pre_part = attn_prefill_part_floats(pre_T, k.n_q_heads, d, pre_s);
-    c->attn_part_floats = std::max(dec_part, pre_part);
+    c->attn_part_floats = c->decode_splits > 1 ? (size_t)k.max_batch * k.n_q_heads * c->decode_splits * (d + 2) : 1;
     INIT_TRY(dmalloc(&c->attn_part, c->attn_part_floats));
-    const int G = k.n_q_heads / k.n_kv_heads;
-    const int qblocks = (pre_T * G + 63) / 64;
-    c->attn_cnt_n = std::max(k.max_batch * k.n_kv_heads, qblocks * k.n_kv_heads);
+    c->attn_cnt_n = k.max_batch * k.n_kv_heads;
     INIT_TRY(dmalloc(&c->attn_cnt, c->attn_cnt_n));
     INIT_TRY(cudaMemsetAsync(c->attn_cnt, 0, (size_t)c->attn_cnt_n * 4, st));
 

@@ -124,19 +124,6 @@ DEC_DEVINL void tmem_ld_wait32(uint32_t (&r)[32]) {
                  : "memory");
 }
 
-// Barrier across every CTA of the cluster, with release/acquire ordering of shared memory.
-DEC_DEVINL void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// 16-byte store into the shared memory of CTA `rank` of this cluster, at the same offset as
-// the local shared address `saddr` (fire-and-forget; ordered by the next cluster barrier).
-DEC_DEVINL void dsmem_st4(uint32_t saddr, int rank, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(saddr), "r"(rank));
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
 
 // Apply the epilogue to the 16 values v[j] of (row, t0 + j). All lanes of the warp call
 // it together (the SwiGLU pairing uses a shuffle). Every global load of a chunk is issued

@@ -117,15 +117,12 @@ struct AttnPrefillArgs {
     const int32_t* block_row;
     int T, pos0, nq, nkv, d;
     float scale;
-    int splits;
-    float* part;        // [splits][T*nq][d+2]
-    int* counters;      // [qblocks*nkv]
+    int splits;         // key splits (1..8): the split CTAs of a row block form one cluster
     uint16_t* out;      // [T][nq*d]
     int* err;
 };
 cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl);
 int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms);
-size_t attn_prefill_part_floats(int T, int nq, int d, int splits);
 
 // Greedy argmax as one 64-bit word per row: high half an order-preserving key of the
 // fp32 value, low half ~index (so on equal values the lowest index is the largest word).
