@@ -763,15 +763,14 @@ cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pd
     if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64>()) return cudaErrorInvalidValue;
     if (a.d == 128) {
         const size_t smem = decode_smem<128>();
-        cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<128>), (int)smem);
         if (e != cudaSuccess) return e;
         return launch_ex(attn_decode_kernel<128>, grid, dim3(128), smem, st, pdl, a);
     }
     if (a.d == 64) {
         const size_t smem = decode_smem<64>();
         cudaError_t e =
-            cudaFuncSetAttribute(attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<64>), (int)smem);
         if (e != cudaSuccess) return e;
         return launch_ex(attn_decode_kernel<64>, grid, dim3(128), smem, st, pdl, a);
     }
@@ -804,7 +803,7 @@ cudaError_t prefill_launch_d(const AttnPrefillArgs& a, cudaStream_t st, bool pdl
     const int G = a.nq / a.nkv;
     const int qblocks = (a.T * G + kPrefRows - 1) / kPrefRows;
     const size_t smem = prefill_smem<D>();
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_prefill_kernel<D>), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(qblocks, a.nkv, a.splits);

@@ -93,8 +93,13 @@ struct dec_ctx {
     int* attn_cnt = nullptr;
     size_t attn_part_floats = 0;
     int attn_cnt_n = 0;
+    float* gemm_ws = nullptr;  // tensor-core GEMM: pieces of tiles shared between CTAs
+    int* gemm_cnt = nullptr;   // and their arrival counters (zero between launches)
+    int gemm_cnt_n = 0;
     int* d_err = nullptr;
     int32_t* h_stage = nullptr;  // pinned: tokens, positions, block rows
+    int32_t* h_prompt = nullptr; // pinned [max_context]: one prefill's tokens
+    int32_t* d_prompt = nullptr; // [max_context]
     int* h_err = nullptr;
     int act_cols = 0;
     int decode_splits = 1;
@@ -188,7 +193,7 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
         in = c->xn;
     }
     GemmPlan plan;
-    CUDA_TRY(gemm_plan(&plan, p.W, p.M, p.K, in, n, c->num_sms));
+    CUDA_TRY(gemm_plan(&plan, p.W, p.M, p.K, in, n, c->num_sms, c->gemm_ws));
     GemmArgs a{};
     a.epi = epi;
     a.y = y;
@@ -197,7 +202,9 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
     a.act = act;
     a.ldact = ldact;
     a.amax = amax;
+    a.cnt = c->gemm_cnt;
     a.err = c->d_err;
+    if (gemm_cnt_needed(p.M, n) > c->gemm_cnt_n) return fail(DEC_ERR_UNSUPPORTED, "GEMM tile counters too small");
     CUDA_TRY(gemm_launch(plan, a, st, true));
     return DEC_OK;
 }
@@ -636,8 +643,17 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     // ---- step buffers
     const int T = c->max_tok;
     INIT_TRY(dmalloc(&c->d_tok, T));
+    INIT_TRY(dmalloc(&c->d_prompt, (size_t)k.max_context));
     INIT_TRY(dmalloc(&c->d_pos, T));
     INIT_TRY(dmalloc(&c->d_amax, (size_t)32 * k.max_batch));
+    {
+        const int qkv_rows = k.n_q_heads * d + 2 * k.n_kv_heads * d;
+        const int m_max = std::max({k.vocab, qkv_rows, k.hidden, 2 * k.ffn_inter, 2 * k.shared_inter, k.n_experts});
+        c->gemm_cnt_n = gemm_cnt_needed(m_max, T);
+        INIT_TRY(dmalloc(&c->gemm_ws, gemm_ws_floats(c->num_sms)));
+        INIT_TRY(dmalloc(&c->gemm_cnt, c->gemm_cnt_n));
+        INIT_TRY(cudaMemsetAsync(c->gemm_cnt, 0, (size_t)c->gemm_cnt_n * 4, st));
+    }
     {
         // RoPE angles pos * base^(-2i/d), cos and sin evaluated in fp64, stored as fp32
         std::vector<float2> tab((size_t)k.max_context * (d / 2));
@@ -675,6 +691,7 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(dmalloc(&c->d_err, 1));
     INIT_TRY(cudaMemsetAsync(c->d_err, 0, 4, st));
     INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_stage), sizeof(int32_t) * (2 * T + c->max_pages + 16)));
+    INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_prompt), sizeof(int32_t) * (size_t)k.max_context));
     INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_err), sizeof(int)));
     *c->h_err = 0;
 
@@ -720,6 +737,7 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->final_norm);
     cudaFree(c->d_bt);
     cudaFree(c->d_tok);
+    cudaFree(c->d_prompt);
     cudaFree(c->d_pos);
     cudaFree(c->d_amax);
     cudaFree(c->rope_tab);
@@ -732,6 +750,8 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->act);
     cudaFree(c->attn_part);
     cudaFree(c->attn_cnt);
+    cudaFree(c->gemm_ws);
+    cudaFree(c->gemm_cnt);
     cudaFree(c->moe_logits);
     cudaFree(c->moe_w);
     cudaFree(c->moe_sgate);
@@ -745,6 +765,7 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->moe_ys);
     cudaFree(c->d_err);
     if (c->h_stage) cudaFreeHost(c->h_stage);
+    if (c->h_prompt) cudaFreeHost(c->h_prompt);
     if (c->h_err) cudaFreeHost(c->h_err);
     if (c->bridge) {
         if (c->stream) cudaStreamDestroy(c->stream);
@@ -792,16 +813,16 @@ dec_status dec_prefill(dec_ctx* c, int32_t seq, const int32_t* tokens, int32_t T
     if (s != DEC_OK) return s;
     const int C = k.prefill_chunk;
     int last_rows = 0;
+    // all the tokens in one copy (the pinned buffer is reused only after this call has
+    // synchronised), then the chunks back to back with no host wait between them
+    memcpy(c->h_prompt, tokens, sizeof(int32_t) * T);
+    CUDA_TRY(cudaMemcpyAsync(c->d_prompt, c->h_prompt, sizeof(int32_t) * T, cudaMemcpyHostToDevice, st));
     for (int done = 0; done < T; done += C) {
         const int n = std::min(C, T - done);
-        memcpy(c->h_stage, tokens + done, sizeof(int32_t) * n);
-        CUDA_TRY(cudaMemcpyAsync(c->d_tok, c->h_stage, sizeof(int32_t) * n, cudaMemcpyHostToDevice, st));
-        CUDA_TRY(embed_launch(c->embed, c->d_tok, n, k.hidden, c->x, st, false));
+        CUDA_TRY(embed_launch(c->embed, c->d_prompt + done, n, k.hidden, c->x, st, false));
         s = forward_layers(c, n, false, seq, pos0 + done, st);
         if (s != DEC_OK) return s;
         last_rows = n;
-        // the staging buffer is rewritten by the next chunk
-        CUDA_TRY(cudaStreamSynchronize(st));
     }
     s = head(c, last_rows - 1, 1, st);
     if (s != DEC_OK) return s;
@@ -1040,12 +1061,15 @@ dec_status weight_gemv(const void* W, const void* x, int32_t B, int32_t N, int32
         CUDA_TRY(gemv_launch(a, GEMV_STORE, st, sms, false));
         return DEC_OK;
     }
+    CUDA_TRY(grow(&S.ws, &S.ws_n, gemm_ws_floats(sms), false));
+    CUDA_TRY(grow(&S.cnt, &S.cnt_n, (size_t)gemm_cnt_needed(N, B), true));
     GemmPlan plan;
-    CUDA_TRY(gemm_plan(&plan, static_cast<const uint16_t*>(W), N, K, static_cast<const uint16_t*>(x), B, sms));
+    CUDA_TRY(gemm_plan(&plan, static_cast<const uint16_t*>(W), N, K, static_cast<const uint16_t*>(x), B, sms, S.ws));
     GemmArgs a{};
     a.epi = GEMM_STORE;
     a.y = y;
     a.ldy = N;
+    a.cnt = S.cnt;
     a.err = S.err;
     CUDA_TRY(gemm_launch(plan, a, st, false));
     return DEC_OK;

@@ -8,19 +8,23 @@
 // dense contraction.
 //
 // B200 design (sm_100a, tcgen05):
-//  * one 128 x BN output tile per CTA (BN = 32/64/128 tokens), split over K when
-//    the tile count would leave SMs idle; split partials are summed in split order
-//    by the last CTA of the tile (deterministic, no atomics on data);
-//  * warp 0 / lane 0 drives TMA: 128B-swizzled 64-wide K slices of A and B into a
+//  * persistent: one CTA per SM; the (128 x BN tile, 64-wide k block) units of the
+//    product (BN = 32/64/128 tokens) are cut into equal contiguous ranges, one per
+//    CTA (stream-K), so every SM streams the same share of the weights whatever the
+//    tile count; a tile shared by several CTAs is finished by the CTA whose piece
+//    arrives last, which sums the fp32 pieces in k order (deterministic, no atomics
+//    on data);
+//  * warp 4 / lane 0 drives TMA: 128B-swizzled 64-wide K slices of A and B into a
 //    6-8 stage shared-memory ring (mbarrier complete_tx); the weight slices of
 //    the first stages are issued before griddepcontrol.wait (they do not depend
 //    on the previous kernel), the activation slices after it;
-//  * warp 1 / lane 0 issues tcgen05.mma.cta_group::1.kind::f16 (M=128, N=BN,
+//  * warp 5 / lane 0 issues tcgen05.mma.cta_group::1.kind::f16 (M=128, N=BN,
 //    K=16 per instruction, fp32 accumulator in TMEM) and frees each stage with
-//    tcgen05.commit;
-//  * all 4 warps read the accumulator with tcgen05.ld (warp w owns TMEM lanes
-//    32w..32w+31 = weight rows) and apply the epilogue: store (+bias), residual
-//    add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
+//    tcgen05.commit; the accumulator is double-buffered in TMEM (2 x BN columns),
+//    so one tile's epilogue overlaps the next tile's main loop;
+//  * warps 0-3 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
+//    32w..32w+31 = weight rows) and apply the epilogue: store (+bias, + greedy
+//    argmax), residual add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -38,7 +42,7 @@ struct Cfg {
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int STAGES = BN <= 64 ? 8 : 6;
-    static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
+    static constexpr int TMEM_COLS = 2 * BN;  // two accumulator buffers (64/128/256 columns)
     static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
 };
 
@@ -93,15 +97,6 @@ DEC_DEVINL void tc_commit(uint64_t* bar) {
                  : "memory");
 }
 
-DEC_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 // tcgen05.ld of 16 columns without waiting; the values are valid after tmem_ld_wait32.
 DEC_DEVINL void tmem_ld16_issue(uint32_t taddr, uint32_t* r) {
     asm volatile(
@@ -131,12 +126,18 @@ DEC_DEVINL void tmem_ld_wait32(uint32_t (&r)[32]) {
 DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v)[16]) {
     const bool row_ok = row < a.M;
     if (a.epi == GEMM_SWIGLU) {
+        // rows 2i (gate) and 2i+1 (up) sit in adjacent lanes; the even lane finishes the
+        // even tokens and the odd lane the odd ones, so every lane evaluates 8 SiLUs
+        const bool odd = (threadIdx.x & 1) != 0;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const float partner = __shfl_xor_sync(0xffffffffu, v[j], 1);
-            if (row_ok && (row & 1) == 0 && t0 + j < a.N) {
-                const float sg = v[j] * (1.0f / (1.0f + expf(-v[j])));
-                a.act[(size_t)(t0 + j) * a.ldact + (row >> 1)] = f2bf(sg * partner);
+        for (int jj = 0; jj < 8; ++jj) {
+            const float own = odd ? v[2 * jj + 1] : v[2 * jj];
+            const float other = __shfl_xor_sync(0xffffffffu, odd ? v[2 * jj] : v[2 * jj + 1], 1);
+            const float g = odd ? other : own, u = odd ? own : other;
+            const int t = t0 + 2 * jj + (odd ? 1 : 0);
+            if (row_ok && t < a.N) {
+                const float sg = g * (1.0f / (1.0f + expf(-g)));
+                a.act[(size_t)t * a.ldact + (row >> 1)] = f2bf(sg * u);
             }
         }
         return;
@@ -174,33 +175,327 @@ DEC_DEVINL void argmax16(const GemmArgs& a, int row, int t0, const float (&v)[16
     }
 }
 
+// ----------------------------------------------------------------- stream-K work split
+//
+// The (tile, 64-wide k block) units of the whole product, tile-major, are cut into
+// gridDim.x equal contiguous ranges, one per persistent CTA. A CTA's range is a run of
+// segments, one per tile it touches: whole tiles in the middle, and at its two ends
+// pieces of tiles it shares with the neighbouring CTAs.
+struct Work {
+    long long U;  // units
+    int nkb, tiles_n, bn, nc;
+};
+
+DEC_DEVINL Work make_work(const GemmArgs& a, int bn) {
+    Work w;
+    w.nkb = (a.K + BK - 1) / BK;
+    w.tiles_n = (a.N + bn - 1) / bn;
+    w.U = (long long)((a.M + BM - 1) / BM) * w.tiles_n * w.nkb;
+    w.bn = bn;
+    w.nc = gridDim.x;
+    return w;
+}
+
+DEC_DEVINL long long unit0(const Work& w, int c) { return w.U * c / w.nc; }
+// CTA whose range holds unit u.
+DEC_DEVINL int cta_of(const Work& w, long long u) { return (int)(((u + 1) * w.nc - 1) / w.U); }
+
+struct Range {
+    long long u0, u1;
+    int tf, nseg, iters;
+};
+
+DEC_DEVINL Range cta_range(const Work& w, int c) {
+    Range r;
+    r.u0 = unit0(w, c);
+    r.u1 = unit0(w, c + 1);
+    r.iters = (int)(r.u1 - r.u0);
+    r.tf = (int)(r.u0 / w.nkb);
+    r.nseg = r.u1 > r.u0 ? (int)((r.u1 - 1) / w.nkb) - r.tf + 1 : 0;
+    return r;
+}
+
+struct Seg {
+    int tile, kb0, kb1, slot;  // slot: 0 = first tile of the range, 1 = any later one
+};
+
+// The j-th segment in processing order: the pieces at the two ends of the range come
+// first (their tiles are finished by whichever CTA completes its piece last, so those
+// reductions overlap the whole tiles processed afterwards), then the middle tiles.
+DEC_DEVINL Seg segment(const Work& w, const Range& r, int j) {
+    int i = j;
+    if (r.nseg >= 2) i = j == 0 ? r.nseg - 1 : j - 1;
+    Seg s;
+    s.tile = r.tf + i;
+    const long long t0 = (long long)s.tile * w.nkb;
+    s.kb0 = (int)((r.u0 > t0 ? r.u0 : t0) - t0);
+    s.kb1 = (int)((r.u1 < t0 + w.nkb ? r.u1 : t0 + w.nkb) - t0);
+    s.slot = i == 0 ? 0 : 1;
+    return s;
+}
+
+// Workspace slot of CTA cc's piece of `tile`.
+DEC_DEVINL int piece_slot(const Work& w, int cc, int tile) { return (int)(unit0(w, cc) / w.nkb) == tile ? 0 : 1; }
+
+// Walks the k blocks of a range in processing order (the producer's view).
+struct SegIter {
+    Work w;
+    Range r;
+    Seg s;
+    int j, kb, m0, n0;
+    DEC_DEVINL SegIter(const Work& w_, const Range& r_) : w(w_), r(r_), j(0) { load(); }
+    DEC_DEVINL void load() {
+        if (j >= r.nseg) return;
+        s = segment(w, r, j);
+        kb = s.kb0;
+        m0 = s.tile / w.tiles_n * BM;
+        n0 = s.tile % w.tiles_n * w.bn;
+    }
+    DEC_DEVINL void next() {
+        if (++kb >= s.kb1) {
+            ++j;
+            load();
+        }
+    }
+};
+
+// Barrier of the four epilogue warps only.
+DEC_DEVINL void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+DEC_DEVINL int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Whether every piece of a shared tile has been published (tile counter >= P), waiting
+// for it (bounded: on time-out sets the error flag and returns false).
+DEC_DEVINL bool tile_ready(const GemmArgs& a, int tile, int P, volatile int* flag_s) {
+    if (threadIdx.x == 0) {
+        int r = 1;
+        const long long st = clock64();
+        while (ld_acquire_gpu(&a.cnt[tile]) < P) {
+            if (clock64() - st > (1ll << 31)) {
+                atomicExch(a.err, 1);
+                r = 0;
+                break;
+            }
+        }
+        // the pieces were written through the generic proxy; they are read by TMA below
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        *flag_s = r;
+    }
+    epi_bar();
+    const int r = *flag_s;
+    epi_bar();
+    return r != 0;
+}
+
+// Cooperative finish of a tile shared by CTAs c_lo..c_hi (k order), once all of them have
+// published their pieces: CTA c takes a slice of the tile's rows, fetches that slice of
+// every piece into shared memory with TMA (32-row boxes, [column][row] fp32), sums the
+// pieces in k order (deterministic) and applies the epilogue; lane = row and warp w
+// = 16-column chunks w, w + 4, as in the accumulator epilogue. The tile counter goes from
+// 0 to P (pieces published) and on to 2P (slices done); the CTA that completes it resets
+// it to 0. `buf` is the drained operand ring, room for `cap` boxes.
 template <int BN>
-__global__ void __launch_bounds__(128, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+DEC_DEVINL bool reduce_slice(const GemmArgs& a, const Work& w, int c, int tile, const CUtensorMap* tmW,
+                             uint8_t* buf, int cap, uint64_t* redb, uint32_t& red_phase) {
+    constexpr int BOX = 32 * BN * 4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long t0 = (long long)tile * w.nkb;
+    const int c_lo = cta_of(w, t0), c_hi = cta_of(w, t0 + w.nkb - 1);
+    const int P = c_hi - c_lo + 1;
+    // every CTA after the first starts inside the tile (its slot 0); the first holds the
+    // tile in slot 0 only if its range starts exactly at the tile
+    const int slot_lo = piece_slot(w, c_lo, tile);
+    const int rs = (((BM + P - 1) / P) + 3) & ~3;  // multiple of 4 rows: 16-byte TMA x
+    const int r0 = min(BM, (c - c_lo) * rs), r1 = min(BM, r0 + rs);
+    const int m0 = tile / w.tiles_n * BM, n0 = tile % w.tiles_n * BN;
+    for (int rb = r0; rb < r1; rb += 32) {
+        float acc[2][16];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) acc[h][q] = 0.f;
+        for (int cb = c_lo; cb <= c_hi; cb += cap) {
+            const int n = min(cap, c_hi - cb + 1);
+            if (threadIdx.x == 0) {
+                mbar_arrive_expect_tx(redb, (uint32_t)(n * BOX));
+                for (int u = 0; u < n; ++u) {
+                    const int cc = cb + u;
+                    tma_load_2d(buf + u * BOX, tmW, rb, (cc * 2 + (cc == c_lo ? slot_lo : 0)) * BN, redb);
+                }
+            }
+            if (!mbar_wait_bounded(redb, red_phase & 1u, a.err)) return false;
+            ++red_phase;
+            for (int u = 0; u < n; ++u) {
+                const float* bx = reinterpret_cast<const float*>(buf + u * BOX);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int ch = warp + 4 * h;
+                    if (ch * 16 < BN) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) acc[h][q] += bx[(ch * 16 + q) * 32 + lane];
+                    }
+                }
+            }
+            epi_bar();  // every thread is done with the boxes before the next batch lands
+        }
+        const int rl = rb + lane;
+        const int row = rl < r1 ? m0 + rl : 0x3fffffff;  // rows outside the slice write nothing
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int ch = warp + 4 * h;
+            if (ch * 16 < BN) {
+                epilogue16(a, row, n0 + ch * 16, acc[h]);
+                if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + ch * 16, acc[h]);
+            }
+        }
+    }
+    epi_bar();
+    if (threadIdx.x == 0 && atomicAdd(&a.cnt[tile], 1) == 2 * P - 1) atomicExch(&a.cnt[tile], 0);
+    return true;
+}
+
+// The slice of a shared tile that CTA c finishes (see reduce_slice).
+struct RedPlan {
+    int tile, c_lo, c_hi, slot_lo, r0, r1;
+};
+
+DEC_DEVINL RedPlan red_plan(const Work& w, int c, int tile) {
+    RedPlan r;
+    const long long t0 = (long long)tile * w.nkb;
+    r.tile = tile;
+    r.c_lo = cta_of(w, t0);
+    r.c_hi = cta_of(w, t0 + w.nkb - 1);
+    const int P = r.c_hi - r.c_lo + 1;
+    r.slot_lo = piece_slot(w, r.c_lo, tile);
+    const int rs = (((BM + P - 1) / P) + 3) & ~3;
+    r.r0 = min(BM, (c - r.c_lo) * rs);
+    r.r1 = min(BM, r.r0 + rs);
+    return r;
+}
+
+DEC_DEVINL int red_boxes(const RedPlan& r) { return ((r.r1 - r.r0 + 31) / 32) * (r.c_hi - r.c_lo + 1); }
+
+// Thread 0 issues the boxes of every plan in one batch (plan, row box, piece order).
+template <int BN>
+DEC_DEVINL void red_issue(const RedPlan* rp, int n, int total, const CUtensorMap* tmW, uint8_t* buf,
+                          uint64_t* redb) {
+    constexpr int BOX = 32 * BN * 4;
+    if (threadIdx.x != 0) return;
+    mbar_arrive_expect_tx(redb, (uint32_t)(total * BOX));
+    int k = 0;
+    for (int i = 0; i < n; ++i)
+        for (int rb = rp[i].r0; rb < rp[i].r1; rb += 32)
+            for (int cc = rp[i].c_lo; cc <= rp[i].c_hi; ++cc, ++k)
+                tma_load_2d(buf + k * BOX, tmW, rb, (cc * 2 + (cc == rp[i].c_lo ? rp[i].slot_lo : 0)) * BN, redb);
+}
+
+// Sums the boxes issued by red_issue in k order, applies the epilogue and advances the
+// tile counters (see reduce_slice).
+template <int BN>
+DEC_DEVINL void red_finish(const GemmArgs& a, const Work& w, const RedPlan* rp, int n, const uint8_t* buf) {
+    constexpr int BOX = 32 * BN * 4;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int k = 0;
+    for (int i = 0; i < n; ++i) {
+        const RedPlan& r = rp[i];
+        const int m0 = r.tile / w.tiles_n * BM, n0 = r.tile % w.tiles_n * BN;
+        for (int rb = r.r0; rb < r.r1; rb += 32) {
+            float acc[2][16];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int q = 0; q < 16; ++q) acc[h][q] = 0.f;
+            for (int cc = r.c_lo; cc <= r.c_hi; ++cc, ++k) {
+                const float* bx = reinterpret_cast<const float*>(buf + k * BOX);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int ch = warp + 4 * h;
+                    if (ch * 16 < BN) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) acc[h][q] += bx[(ch * 16 + q) * 32 + lane];
+                    }
+                }
+            }
+            const int rl = rb + lane;
+            const int row = rl < r.r1 ? m0 + rl : 0x3fffffff;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int ch = warp + 4 * h;
+                if (ch * 16 < BN) {
+                    epilogue16(a, row, n0 + ch * 16, acc[h]);
+                    if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + ch * 16, acc[h]);
+                }
+            }
+        }
+    }
+    epi_bar();
+    if (threadIdx.x == 0)
+        for (int i = 0; i < n; ++i) {
+            const int P = rp[i].c_hi - rp[i].c_lo + 1;
+            if (atomicAdd(&a.cnt[rp[i].tile], 1) == 2 * P - 1) atomicExch(&a.cnt[rp[i].tile], 0);
+        }
+}
+
+DEC_DEVINL int tile_pieces(const Work& w, int tile) {
+    const long long t0 = (long long)tile * w.nkb;
+    return cta_of(w, t0 + w.nkb - 1) - cta_of(w, t0) + 1;
+}
+
+// Waits until every pending shared tile has all its pieces, then (when their boxes fit
+// the ring) issues the fetch of all of them in one batch. `issued` = boxes in flight, or
+// 0 when they do not fit (reduce_slice then fetches tile by tile).
+template <int BN>
+DEC_DEVINL bool begin_reductions(const GemmArgs& a, const Work& w, int c, const int* pend, int npend,
+                                 RedPlan* plans, const CUtensorMap* tmW, uint8_t* buf, int cap, uint64_t* redb,
+                                 volatile int* flag_s, int& issued) {
+    int total = 0;
+    for (int i = 0; i < npend; ++i) {
+        if (!tile_ready(a, pend[i], tile_pieces(w, pend[i]), flag_s)) return false;
+        plans[i] = red_plan(w, c, pend[i]);
+        total += red_boxes(plans[i]);
+    }
+    issued = total <= cap ? total : 0;
+    if (issued > 0) red_issue<BN>(plans, npend, total, tmW, buf, redb);
+    return true;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmW, GemmArgs a) {
     using C = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
     uint64_t* empty = full + C::STAGES;
-    uint64_t* accb = empty + C::STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
-    int* ticket = reinterpret_cast<int*>(tmem_slot + 1);
+    uint64_t* accf = empty + C::STAGES;  // [2] accumulator buffer ready for the epilogue
+    uint64_t* acce = accf + 2;           // [2] accumulator buffer drained by the epilogue
+    uint64_t* redb = acce + 2;           // reduction boxes landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redb + 1);
+    int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);  // reduction wait timed out
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN, z = blockIdx.z;
-    const int nkb = (a.K + BK - 1) / BK;
-    const int kb0 = (int)((int64_t)z * nkb / a.splits), kb1 = (int)((int64_t)(z + 1) * nkb / a.splits);
-    const int nk = kb1 - kb0;
+    const Work w = make_work(a, BN);
+    const int c = blockIdx.x;
+    const Range rg = cta_range(w, c);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accb, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 128);
+        }
+        mbar_init(redb, 1);
         fence_mbar_init();
     }
-    if (warp == 2) {
+    if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(C::TMEM_COLS)
                      : "memory");
@@ -212,149 +507,145 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem = *tmem_slot;
     pdl_trigger();
 
-    bool ok = true;
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------ TMA producer
-        const uint64_t pol = policy_evict_first();
-        const int pre = nk < C::STAGES ? nk : C::STAGES;
-        for (int i = 0; i < pre; ++i) {
-            mbar_arrive_expect_tx(&full[i], C::STAGE);
-            tma_load_2d_hint(smem + i * C::STAGE, &tmA, (kb0 + i) * BK, m0, &full[i], pol);
+    if (warp == 4) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            const uint64_t pol = policy_evict_first();
+            const int total = rg.iters;
+            const int pre = total < C::STAGES ? total : C::STAGES;
+            // the weight slices of the first stages do not depend on the previous kernel
+            SegIter it(w, rg);
+            for (int i = 0; i < pre; ++i, it.next()) {
+                mbar_arrive_expect_tx(&full[i], C::STAGE);
+                tma_load_2d_hint(smem + i * C::STAGE, &tmA, it.kb * BK, it.m0, &full[i], pol);
+            }
+            pdl_wait();
+            SegIter jt(w, rg);
+            for (int i = 0; i < pre; ++i, jt.next())
+                tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, jt.kb * BK, jt.n0, &full[i]);
+            for (int i = pre; i < total; ++i, it.next()) {
+                const int s = i % C::STAGES;
+                const uint32_t u = (uint32_t)(i / C::STAGES);
+                if (!mbar_wait_bounded(&empty[s], (u & 1u) ^ 1u, a.err)) break;
+                mbar_arrive_expect_tx(&full[s], C::STAGE);
+                tma_load_2d_hint(smem + s * C::STAGE, &tmA, it.kb * BK, it.m0, &full[s], pol);
+                tma_load_2d(smem + s * C::STAGE + C::A_BYTES, &tmB, it.kb * BK, it.n0, &full[s]);
+            }
         }
+        __syncwarp();
+    } else if (warp == 5) {
         pdl_wait();
-        for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, (kb0 + i) * BK, n0, &full[i]);
-        for (int i = pre; i < nk; ++i) {
-            const int s = i % C::STAGES;
-            const uint32_t u = (uint32_t)(i / C::STAGES);
-            if (!mbar_wait_bounded(&empty[s], (u & 1u) ^ 1u, a.err)) break;
-            mbar_arrive_expect_tx(&full[s], C::STAGE);
-            tma_load_2d_hint(smem + s * C::STAGE, &tmA, (kb0 + i) * BK, m0, &full[s], pol);
-            tma_load_2d(smem + s * C::STAGE + C::A_BYTES, &tmB, (kb0 + i) * BK, n0, &full[s]);
-        }
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = idesc_bf16<BN>();
-        const uint32_t sbase = smem_u32(smem);
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % C::STAGES;
-            const uint32_t u = (uint32_t)(i / C::STAGES);
-            if (!mbar_wait_bounded(&full[s], u & 1u, a.err)) {
-                ok = false;
-                break;
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_bf16<BN>();
+            const uint32_t sbase = smem_u32(smem);
+            int i = 0;
+            bool ok = true;
+            for (int j = 0; j < rg.nseg && ok; ++j) {
+                const Seg sg = segment(w, rg, j);
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait_bounded(&acce[buf], (uint32_t)(((j >> 1) - 1) & 1), a.err)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * BN);
+                for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++i) {
+                    const int s = i % C::STAGES;
+                    const uint32_t u = (uint32_t)(i / C::STAGES);
+                    if (!mbar_wait_bounded(&full[s], u & 1u, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t abase = sbase + s * C::STAGE, bbase = abase + C::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc_mma(d, sdesc_sw128(abase + kk * 32), sdesc_sw128(bbase + kk * 32), idesc,
+                               (kb > sg.kb0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                }
+                tc_commit(&accf[buf]);
             }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (warps 0-3: TMEM lanes 32w..)
+        pdl_wait();
+        const int rloc = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        int pend_tile[2], npend = 0;
+        RedPlan plans[2];
+        int issued = -1;  // reduction boxes fetched in one batch (0: too many, per-tile batches)
+        const int cap = (C::STAGES * C::STAGE) / (32 * BN * 4);
+        bool ok = true;
+        for (int j = 0; j < rg.nseg && ok; ++j) {
+            const Seg sg = segment(w, rg, j);
+            const int buf = j & 1;
+            if (!mbar_wait_bounded(&accf[buf], (uint32_t)((j >> 1) & 1), a.err)) break;
             tc_fence_after();
-            const uint32_t abase = sbase + s * C::STAGE, bbase = abase + C::A_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-                tc_mma(tmem, sdesc_sw128(abase + kk * 32), sdesc_sw128(bbase + kk * 32), idesc,
-                       (i > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&empty[s]);
-        }
-        tc_commit(accb);
-    }
-    if (warp != 0) pdl_wait();  // every thread passes the grid dependency before finishing
-
-    // ---------------------------------------------------- epilogue
-    __syncwarp();
-    const bool acc_ready = mbar_wait_bounded(accb, 0, a.err);
-    tc_fence_after();
-    const int rloc = warp * 32 + lane;
-    const int row = m0 + rloc;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    // Split-K: the a.splits CTAs of this tile form one cluster. CTA r owns rows
-    // [r*rp, r*rp + rp) of the tile; every CTA pushes its partial of those rows into the
-    // owner's receive buffer (drained stage ring, [split][row][BN + 4] fp32, vector stores
-    // to distributed shared memory, no waiting), then after one cluster barrier each owner
-    // sums its rows over the splits in split order from local shared memory (deterministic).
-    const int S = a.splits;
-    const int rp = (((BM + S - 1) / S) + 1) & ~1;  // even, so SwiGLU pairs stay in one slice
-    constexpr int LDR = BN + 4;                    // padded row: conflict-free vector access
-    const uint32_t recv = smem_u32(smem);
-    const int owner = rloc / rp, lr = rloc - owner * rp;
-    if (S > 1) cluster_sync();  // every CTA's stage ring is drained before any partial lands in it
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld16_issue(lane_base + (uint32_t)c0, r);
-        tmem_ld16_issue(lane_base + (uint32_t)c0 + 16, r + 16);
-        tmem_ld_wait32(r);
-        if (!acc_ready) continue;
-        if (S == 1) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float v[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[16 * h + j]);
-                epilogue16(a, row, n0 + c0 + 16 * h, v);
-                if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0 + 16 * h, v);
+            const uint32_t acc = tmem + lane_off + (uint32_t)(buf * BN);
+            const bool whole = sg.kb0 == 0 && sg.kb1 == w.nkb;
+            if (whole && j == rg.nseg - 1 && npend > 0) {
+                // every piece of this CTA is published and the operand ring is drained
+                // (the last MMA has completed): start fetching the shared tiles' pieces now,
+                // so the fetch overlaps this tile's epilogue
+                ok = begin_reductions<BN>(a, w, c, pend_tile, npend, plans, &tmW, smem, cap, redb, flag_s, issued);
             }
-        } else {
-            const uint32_t dst = recv + (uint32_t)(((z * rp + lr) * LDR + c0) * 4);
+            if (whole) {
+                const int row = sg.tile / w.tiles_n * BM + rloc, n0 = sg.tile % w.tiles_n * BN;
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld16_issue(acc + (uint32_t)c0, r);
+                    tmem_ld16_issue(acc + (uint32_t)c0 + 16, r + 16);
+                    tmem_ld_wait32(r);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) dsmem_st4(dst + q * 16, owner, r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                    for (int h = 0; h < 2; ++h) {
+                        float v[16];
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[16 * h + q]);
+                        epilogue16(a, row, n0 + c0 + 16 * h, v);
+                        if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0 + 16 * h, v);
+                    }
+                }
+            } else {
+                // publish this piece ([column][row] fp32, coalesced) and free the accumulator
+                float* mine = a.ws + ((size_t)c * 2 + sg.slot) * (BM * BN);
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld16_issue(acc + (uint32_t)c0, r);
+                    tmem_ld16_issue(acc + (uint32_t)c0 + 16, r + 16);
+                    tmem_ld_wait32(r);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) __stcg(mine + (size_t)(c0 + q) * BM + rloc, __uint_as_float(r[q]));
+                }
+                asm volatile("fence.proxy.async.global;" ::: "memory");  // read back by TMA
+                __threadfence();
+                pend_tile[npend++] = sg.tile;
+            }
+            tc_fence_before();
+            mbar_arrive(&acce[buf]);
+            if (!whole) {
+                epi_bar();
+                if (threadIdx.x == 0) atomicAdd(&a.cnt[sg.tile], 1);
+            }
+        }
+        // the shared tiles are finished once this CTA's own work is done: its pieces were
+        // published first, so no CTA ever waits on another CTA's wait, and the operand
+        // ring is free to receive the pieces
+        if (ok && npend > 0 && issued < 0)
+            ok = begin_reductions<BN>(a, w, c, pend_tile, npend, plans, &tmW, smem, cap, redb, flag_s, issued);
+        if (ok && issued > 0) {
+            if (mbar_wait_bounded(redb, 0, a.err)) red_finish<BN>(a, w, plans, npend, smem);
+        } else if (ok && issued == 0) {
+            uint32_t red_phase = 0;
+            for (int i = 0; i < npend && ok; ++i)
+                ok = reduce_slice<BN>(a, w, c, pend_tile[i], &tmW, smem, cap, redb, red_phase);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
                      : "memory");
-    }
-    (void)ok;
-    (void)ticket;
-    if (S == 1) return;
-
-    cluster_sync();  // all partials have arrived; from here on only local shared memory is read
-    const int r_lo = min(BM, z * rp), nr = min(BM, r_lo + rp) - r_lo;
-    const float* rb = reinterpret_cast<const float*>(smem);
-    if (!acc_ready || nr <= 0) return;
-    if (a.epi == GEMM_SWIGLU) {
-        const int np = nr / 2;
-        for (int i = threadIdx.x; i < np * (BN / 4); i += 128) {
-            const int lp = 2 * (i % np), c4 = 4 * (i / np);
-            float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
-            for (int s2 = 0; s2 < S; ++s2) {
-                const float4 pg = *reinterpret_cast<const float4*>(rb + (s2 * rp + lp) * LDR + c4);
-                const float4 pu = *reinterpret_cast<const float4*>(rb + (s2 * rp + lp + 1) * LDR + c4);
-                g.x += pg.x, g.y += pg.y, g.z += pg.z, g.w += pg.w;
-                u.x += pu.x, u.y += pu.y, u.z += pu.z, u.w += pu.w;
-            }
-            const int grow = m0 + r_lo + lp;
-            if (grow >= a.M) continue;
-            const float gv[4] = {g.x, g.y, g.z, g.w}, uv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int t = n0 + c4 + q;
-                if (t >= a.N) continue;
-                const float sg = gv[q] * (1.0f / (1.0f + expf(-gv[q])));
-                a.act[(size_t)t * a.ldact + (grow >> 1)] = f2bf(sg * uv[q]);
-            }
-        }
-    } else {
-        for (int i = threadIdx.x; i < nr * (BN / 4); i += 128) {
-            const int l = i % nr, c4 = 4 * (i / nr);
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s2 = 0; s2 < S; ++s2) {
-                const float4 p = *reinterpret_cast<const float4*>(rb + (s2 * rp + l) * LDR + c4);
-                v.x += p.x, v.y += p.y, v.z += p.z, v.w += p.w;
-            }
-            const int grow = m0 + r_lo + l;
-            if (grow >= a.M) continue;
-            const float vv[4] = {v.x, v.y, v.z, v.w};
-            const float bias = (a.epi == GEMM_STORE && a.bias) ? a.bias[grow] : 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int t = n0 + c4 + q;
-                if (t >= a.N) continue;
-                float* dst = a.y + (size_t)t * a.ldy + grow;
-                if (a.epi == GEMM_RESID) {
-                    *dst += vv[q];
-                } else {
-                    *dst = vv[q] + bias;
-                    if (a.amax) atomicMax(&a.amax[(size_t)t * 32], argmax_pack(vv[q] + bias, grow));
-                }
-            }
-        }
     }
 }
 
@@ -387,76 +678,81 @@ cudaError_t encode_2d(CUtensorMap* tm, const uint16_t* base, int rows, int K, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The stream-K pieces: fp32 [slot * bn + column][BM rows], read back in boxes of 32 rows
+// x bn columns.
+cudaError_t encode_ws(CUtensorMap* tm, const float* ws, int slots, int bn) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    cuuint64_t dims[2] = {(cuuint64_t)BM, (cuuint64_t)slots * bn};
+    cuuint64_t strides[1] = {(cuuint64_t)BM * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)bn};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ws), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int BN>
 cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, bool pdl) {
     using C = Cfg<BN>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(gemm_tc_kernel<BN>), C::SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((p.M + BM - 1) / BM, (p.N + BN - 1) / BN, p.splits);
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3(p.nc);
+    cfg.blockDim = dim3(192);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    int na = 0;
-    if (pdl) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
-    if (p.splits > 1) {  // the split CTAs of a tile form one cluster (reduction through DSMEM)
-        attr[na].id = cudaLaunchAttributeClusterDimension;
-        attr[na].val.clusterDim.x = 1;
-        attr[na].val.clusterDim.y = 1;
-        attr[na].val.clusterDim.z = p.splits;
-        ++na;
-    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, a);
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, p.tmW, a);
 }
 
 }  // namespace
 
 int gemm_tiles(const GemmPlan& p) { return ((p.M + BM - 1) / BM) * ((p.N + p.bn - 1) / p.bn); }
 
-int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn_out) {
-    const int bn = N <= 32 ? 32 : N <= 64 ? 64 : 128;
-    if (bn_out) *bn_out = bn;
-    const int tiles = ((M + BM - 1) / BM) * ((N + bn - 1) / bn);
-    const int nkb = (K + BK - 1) / BK;
-    int best = 1;
-    double best_eff = 0.0;
-    for (int s = 1; s <= 8 && s <= nkb / 4 + 1; ++s) {
-        const int ctas = tiles * s;
-        const int waves = (ctas + num_sms - 1) / num_sms;
-        const double eff = (double)ctas / ((double)waves * num_sms);
-        if (eff > best_eff + 0.05) {
-            best_eff = eff;
-            best = s;
-        }
-        if (eff >= 0.85) break;
-    }
-    if (best > nkb) best = nkb;
-    return best;
+int gemm_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : 128; }
+
+// One persistent CTA per SM, each with at least 8 k blocks of work.
+int gemm_ctas(int M, int N, int K, int num_sms) {
+    const int bn = gemm_bn(N);
+    const long long units = (long long)((M + BM - 1) / BM) * ((N + bn - 1) / bn) * ((K + BK - 1) / BK);
+    long long nc = units / 8;
+    if (nc > num_sms) nc = num_sms;
+    if (nc < 1) nc = 1;
+    return (int)nc;
 }
 
-cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms) {
-    if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0) return cudaErrorInvalidValue;
+size_t gemm_ws_floats(int num_sms) { return (size_t)2 * num_sms * BM * 128; }
+
+int gemm_cnt_needed(int M, int N) { return ((M + BM - 1) / BM) * ((N + 31) / 32); }
+
+cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms,
+                      const float* ws) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0 || !ws) return cudaErrorInvalidValue;
     p->M = M;
     p->N = N;
     p->K = K;
-    p->splits = gemm_choose_splits(M, N, K, num_sms, &p->bn);
+    p->bn = gemm_bn(N);
+    p->nc = gemm_ctas(M, N, K, num_sms);
+    p->ws = ws;
     cudaError_t e = encode_2d(&p->tmA, A, M, K, BM);
     if (e != cudaSuccess) return e;
-    return encode_2d(&p->tmB, B, N, K, p->bn);
+    e = encode_2d(&p->tmB, B, N, K, p->bn);
+    if (e != cudaSuccess) return e;
+    return encode_ws(&p->tmW, ws, 2 * p->nc, p->bn);
 }
 
 cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl) {
     a.M = p.M;
     a.N = p.N;
     a.K = p.K;
-    a.splits = p.splits;
+    a.ws = const_cast<float*>(p.ws);
+    if (!a.cnt) return cudaErrorInvalidValue;
     switch (p.bn) {
         case 32: return launch_bn<32>(p, a, st, pdl);
         case 64: return launch_bn<64>(p, a, st, pdl);

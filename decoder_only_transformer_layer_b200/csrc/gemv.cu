@@ -267,7 +267,7 @@ cudaError_t launch_nb(const GemvArgs& a0, cudaStream_t st, int num_sms, bool pdl
     const Layout L = make_layout(NB, a.K, a.smem_cap);
     if (L.stages < 3) return cudaErrorInvalidValue;
     auto kern = gemv_kernel<NB, EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)L.total);
     if (e != cudaSuccess) return e;
     const int nrb = (a.N + kRows - 1) / kRows;
     const int grid = nrb < num_sms ? nrb : num_sms;

@@ -42,7 +42,9 @@ enum GemmEpi { GEMM_STORE = 0, GEMM_RESID = 1, GEMM_SWIGLU = 2 };
 struct GemmPlan {
     CUtensorMap tmA;  // weights [M][K], box 64 x 128
     CUtensorMap tmB;  // activations [N][K], box 64 x BN
-    int M, N, K, bn, splits;
+    CUtensorMap tmW;  // stream-K pieces (fp32 workspace), box 32 rows x BN
+    const float* ws;
+    int M, N, K, bn, nc;  // nc: persistent CTAs (stream-K ranges)
 };
 
 struct GemmArgs {
@@ -53,14 +55,19 @@ struct GemmArgs {
     const float* bias;
     uint16_t* act;
     int ldact;
-    int splits;       // K splits: the split CTAs of a tile form one cluster (<= 8)
     unsigned long long* amax;  // STORE: per token, packed greedy argmax of y (null = off)
+    float* ws;        // set from the plan: fp32 pieces of tiles shared between CTAs
+    int* cnt;         // gemm_cnt_needed(M, N) zeroed tile counters (left zeroed)
     int* err;
 };
 
-// Build the tensor maps for one GEMM shape (host; encodes A and B addresses).
-cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms);
+// Build the tensor maps for one GEMM shape (host; encodes the A, B and workspace
+// addresses). ws holds gemm_ws_floats(num_sms) floats.
+cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms,
+                      const float* ws);
 int gemm_tiles(const GemmPlan& p);
+size_t gemm_ws_floats(int num_sms);
+int gemm_cnt_needed(int M, int N);
 cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl);
 
 // ----------------------------------------------------------------- attention
@@ -146,9 +153,29 @@ cudaError_t topk_launch(const float* logits, int T, int E, int k, int renorm, in
 
 }  // namespace dec
 
+#include <map>
+#include <mutex>
 #include <string>
+#include <utility>
 namespace dec {
 void set_last_error(const std::string& msg);
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) only when a kernel needs more dynamic
+// shared memory on this device than already granted (the call costs host time on every
+// launch otherwise).
+inline cudaError_t ensure_smem(const void* fn, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, int> granted;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    int& g = granted[std::make_pair(fn, dev)];
+    if (g >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) g = bytes;
+    return e;
+}
 
 // ----------------------------------------------------------------- MoE
 
@@ -207,5 +234,4 @@ struct MoeCombineArgs {
 cudaError_t moe_combine_launch(const MoeCombineArgs& a, int n, cudaStream_t st, bool pdl);
 cudaError_t kv_move_launch(uint16_t* pool_k, uint16_t* pool_v, const int32_t* block_row, int pos0, int n, int nkv,
                            int d, uint16_t* dense_k, uint16_t* dense_v, int to_pool, cudaStream_t st);
-int gemm_choose_splits(int M, int N, int K, int num_sms, int* bn);
 }  // namespace dec

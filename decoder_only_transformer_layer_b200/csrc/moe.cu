@@ -362,7 +362,7 @@ cudaError_t launch_grouped_nb(const GroupedGemvArgs& a, cudaStream_t st, int num
     const Layout L = make_layout(NB, a.K, a.smem_cap);
     if (L.stages < 3) return cudaErrorInvalidValue;
     auto kern = grouped_gemv_kernel<NB, SW>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)L.total);
     if (e != cudaSuccess) return e;
     return launch_ex(kern, dim3(num_sms), dim3(kThreads), L.total, st, pdl, a);
 }
