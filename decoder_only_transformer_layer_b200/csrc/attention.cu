@@ -35,6 +35,7 @@ namespace {
 
 constexpr int kPage = 16;
 constexpr int kRing = 3;  // pages in flight per warp in the decode kernel
+constexpr int kDecodeMaxSplits = 16;  // context splits of one (sequence, kv head): one cluster
 constexpr float kLog2e = 1.4426950408889634f;
 
 // A warp transforms one head vector of D fp32 values: optional RMSNorm with weight
@@ -189,27 +190,55 @@ template <int D>
 __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     constexpr int LD = D + 8;
     constexpr int PAGE = kPage * LD;
+    constexpr int LDR = D + 4;  // receive rows: o[D], m, l, 2 pad (16-byte aligned)
     __shared__ __align__(16) uint16_t qs[16 * LD];
+    __shared__ __align__(16) uint16_t newkv[2][D];  // the appended k and v rows (bf16)
     __shared__ float wm[4][16], wl[4][16];
-    __shared__ int ticket_s;
     extern __shared__ __align__(16) uint8_t dyn[];
-    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [4 warps][2 bufs][K,V][16][LD]
+    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [4 warps][kRing][K,V][16][LD]
+    float* wo = reinterpret_cast<float*>(dyn);           // [4][16][D] after the page loop
+    float* recv = wo + 4 * 16 * D;                       // [rows owned][splits][LDR]
 
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z, S = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int G = a.nq / a.nkv;
-    pdl_trigger();
-    pdl_wait();
+    // Without a scratch buffer the splits of one (sequence, kv head) form a cluster and
+    // merge in distributed shared memory; mark this CTA as running before any other CTA
+    // of the cluster writes into its shared memory.
+    const bool cl = S > 1 && a.part == nullptr;
+    if (cl) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    __shared__ int ticket_s;
 
+    // ---- independent of the previous kernel: positions, block table and the cache pages
+    // (the row being appended is patched in after it is written, below)
     const int p = a.pos[b];
     const int n = p + 1;
     const int np = (n + kPage - 1) / kPage;
-    const int pps = (np + a.splits - 1) / a.splits;
+    const int pps = (np + S - 1) / S;
     const int pg0 = s * pps, pg1 = min(np, pg0 + pps);
     const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
     const bool has_last = pg0 < pg1 && pg1 == np;
     const float sl2 = a.scale * kLog2e;
+    // this warp's pages: pg0 + warp + 4 i, i < cnt; the first kRing are fetched now
+    uint16_t* wbuf = kvbuf + (size_t)warp * kRing * 2 * PAGE;
+    const int cnt = pg0 + warp < pg1 ? (pg1 - pg0 - warp + 3) / 4 : 0;
+    int issued = 0;
+    for (; issued < cnt && issued < kRing; ++issued) {
+        uint16_t* slot = wbuf + (size_t)issued * 2 * PAGE;
+        load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg0 + warp + 4 * issued], a.nkv, g, slot, slot + PAGE);
+    }
+
+    pdl_trigger();
+    pdl_wait();
     const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
+    const bool have_new = a.qkv != nullptr || a.k_new != nullptr;
+    const size_t off_p = has_last ? (((size_t)bt[p / kPage] * a.nkv + g) * kPage + (p % kPage)) * D : 0;
+
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    const int t4 = lane & 3, gr = lane >> 2;
 
     if (pg0 < pg1) {
         // ---- q tile of the group (rows >= G are zero); the split holding row p appends it
@@ -227,55 +256,53 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
                 for (int i = lane; i < D; i += 32) dst[i] = 0;
             }
         }
-        const bool have_new = a.qkv != nullptr || a.k_new != nullptr;
         if (has_last && have_new && warp < 2) {
-            const int phys = bt[p / kPage];
-            const size_t off = (((size_t)phys * a.nkv + g) * kPage + (p % kPage)) * D;
-            if (warp == 0) {  // k: QK-norm, RoPE, bf16
+            // the new row: k gets QK-norm and RoPE, v is only rounded; staged in shared
+            // memory (patched into the page fetched before it existed) and appended to the cache
+            if (warp == 0) {
                 if (a.qkv)
                     head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + g) * D, false, nullptr, a.k_norm,
-                                      a.eps, a.rope, p, a.rope_base, a.k_pool + off, tab);
+                                      a.eps, a.rope, p, a.rope_base, newkv[0], tab);
                 else
                     head_transform<D>(nullptr, true, a.k_new + ((size_t)b * a.nkv + g) * D, nullptr, a.eps, a.rope, p,
-                                      a.rope_base, a.k_pool + off);
-            } else {  // v: bf16 only
+                                      a.rope_base, newkv[0]);
+            } else {
                 if (a.qkv)
                     head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + a.nkv + g) * D, false, nullptr,
-                                      nullptr, a.eps, false, p, a.rope_base, a.v_pool + off);
+                                      nullptr, a.eps, false, p, a.rope_base, newkv[1], tab);
                 else
                     head_transform<D>(nullptr, true, a.v_new + ((size_t)b * a.nkv + g) * D, nullptr, a.eps, false, p,
-                                      a.rope_base, a.v_pool + off);
+                                      a.rope_base, newkv[1]);
             }
+            __syncwarp();
+            uint16_t* dst = (warp == 0 ? a.k_pool : a.v_pool) + off_p;
+            for (int c = lane * 8; c < D; c += 256)
+                *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(&newkv[warp][c]);
         }
-        __syncthreads();  // q tile ready; the appended row is visible to the block's cp.async reads
+        __syncthreads();  // q tile and the staged row are ready
 
         uint32_t qf[D / 16][4];
         load_q_frags<D, LD>(qs, qf);
 
-        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-        float o[D / 8][4];
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-
-        // each warp streams its pages (pg0 + warp, +4, ...) through a 3-page cp.async ring
-        uint16_t* wbuf = kvbuf + (size_t)warp * kRing * 2 * PAGE;
-        int pg = pg0 + warp, buf = 0;
-        if (pg < pg1) load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg], a.nkv, g, wbuf, wbuf + PAGE);
-        if (pg + 4 < pg1)
-            load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg + 4], a.nkv, g, wbuf + 2 * PAGE, wbuf + 3 * PAGE);
-        const int t4 = lane & 3;
-        for (; pg < pg1; pg += 4) {
-            if (pg + 8 < pg1) {
-                uint16_t* nb = wbuf + ((buf + 2) % kRing) * 2 * PAGE;
-                load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg + 8], a.nkv, g, nb, nb + PAGE);
-                cp_async_wait<2>();
-            } else if (pg + 4 < pg1) {
-                cp_async_wait<1>();
-            } else {
-                cp_async_wait<0>();
+        // each warp streams its pages through a kRing-page cp.async ring; a slot is refilled
+        // as soon as its page has been used
+        for (int i = 0; i < cnt; ++i) {
+            const int pg = pg0 + warp + 4 * i;
+            switch (issued - i - 1) {  // groups that may stay in flight
+                case 0: cp_async_wait<0>(); break;
+                case 1: cp_async_wait<1>(); break;
+                case 2: cp_async_wait<2>(); break;
+                default: cp_async_wait<3>(); break;
             }
             __syncwarp();
-            const uint16_t* kd = wbuf + buf * 2 * PAGE;
+            uint16_t* kd = wbuf + (size_t)(i % kRing) * 2 * PAGE;
+            if (pg == np - 1 && has_last && have_new) {
+                // the page was fetched before row p existed: copy the staged row in
+                uint16_t* row = kd + (lane < 16 ? 0 : PAGE) + (p % kPage) * LD;
+                for (int c = (lane & 15) * 8; c < D; c += 128)
+                    *reinterpret_cast<uint4*>(row + c) = *reinterpret_cast<const uint4*>(&newkv[lane >> 4][c]);
+                __syncwarp();
+            }
             float sc[2][4];
             qk_page<D, LD>(qf, kd, sc);
 #pragma unroll
@@ -288,113 +315,152 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             float corr[2];
             softmax_page(sc, m, l, corr);
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                o[i][0] *= corr[0];
-                o[i][1] *= corr[0];
-                o[i][2] *= corr[1];
-                o[i][3] *= corr[1];
+            for (int q = 0; q < D / 8; ++q) {
+                o[q][0] *= corr[0];
+                o[q][1] *= corr[0];
+                o[q][2] *= corr[1];
+                o[q][3] *= corr[1];
             }
             pv_page<D, LD>(sc, kd + PAGE, o);
             __syncwarp();
-            buf = (buf + 1) % kRing;
+            if (issued < cnt) {
+                load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg0 + warp + 4 * issued], a.nkv, g, kd, kd + PAGE);
+                ++issued;
+            }
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
             l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
         }
+    }
 
-        // ---- merge the 4 warps of the CTA through shared memory
-        __syncthreads();  // page buffers are free
-        float* wo = reinterpret_cast<float*>(kvbuf);  // [4][16][D]
-        const int gr = lane >> 2;
-        if (t4 == 0) {
-            wm[warp][gr] = m[0];
-            wm[warp][gr + 8] = m[1];
-            wl[warp][gr] = l[0];
-            wl[warp][gr + 8] = l[1];
+    // ---- merge the 4 warps of the CTA through shared memory (a CTA without pages
+    // contributes m = -inf, l = 0, o = 0)
+    __syncthreads();  // page buffers are free
+    if (t4 == 0) {
+        wm[warp][gr] = m[0];
+        wm[warp][gr + 8] = m[1];
+        wl[warp][gr] = l[0];
+        wl[warp][gr + 8] = l[1];
+    }
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+        float* r0 = wo + ((size_t)warp * 16 + gr) * D + i * 8 + 2 * t4;
+        float* r1 = wo + ((size_t)warp * 16 + gr + 8) * D + i * 8 + 2 * t4;
+        r0[0] = o[i][0];
+        r0[1] = o[i][1];
+        r1[0] = o[i][2];
+        r1[1] = o[i][3];
+    }
+    __syncthreads();
+    // Split partial of row r: o (relative to M) and M, L. In a cluster, row r is finished
+    // by CTA r % S, which receives every split's partial of it in slot [r / S][s];
+    // otherwise the partials go to the scratch and the last CTA of (b, g) merges them.
+    if (cl) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA is running
+    for (int idx = tid; idx < G * (D / 4); idx += 128) {
+        const int r = idx / (D / 4), c = (idx % (D / 4)) * 4;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][r]);
+        float L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            if (wm[w][r] == -INFINITY) continue;
+            const float f = exp2f(wm[w][r] - M);
+            L += f * wl[w][r];
+            const float4 v = *reinterpret_cast<const float4*>(wo + ((size_t)w * 16 + r) * D + c);
+            O.x += f * v.x;
+            O.y += f * v.y;
+            O.z += f * v.z;
+            O.w += f * v.w;
         }
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-            float* r0 = wo + ((size_t)warp * 16 + gr) * D + i * 8 + 2 * t4;
-            float* r1 = wo + ((size_t)warp * 16 + gr + 8) * D + i * 8 + 2 * t4;
-            r0[0] = o[i][0];
-            r0[1] = o[i][1];
-            r1[0] = o[i][2];
-            r1[1] = o[i][3];
-        }
-        __syncthreads();
-        for (int idx = tid; idx < G * D; idx += 128) {
-            const int r = idx / D, c = idx % D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][r]);
-            float L = 0.f, O = 0.f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                if (wm[w][r] == -INFINITY) continue;
-                const float f = exp2f(wm[w][r] - M);
-                L += f * wl[w][r];
-                O += f * wo[((size_t)w * 16 + r) * D + c];
+        if (S == 1) {
+            const float inv = 1.0f / L;
+            uint2 pk;
+            pk.x = pack_bf2(O.x * inv, O.y * inv);
+            pk.y = pack_bf2(O.z * inv, O.w * inv);
+            *reinterpret_cast<uint2*>(a.out + (size_t)b * a.nq * D + (size_t)(g * G + r) * D + c) = pk;
+        } else if (cl) {
+            const uint32_t dst = smem_u32(recv + ((size_t)(r / S) * S + s) * LDR);
+            dsmem_st4(dst + c * 4, r % S, __float_as_uint(O.x), __float_as_uint(O.y), __float_as_uint(O.z),
+                      __float_as_uint(O.w));
+            if (c == 0) dsmem_st2f(dst + D * 4, r % S, M, L);
+        } else {
+            float* pp = a.part + (((size_t)b * a.nq + g * G + r) * S + s) * (D + 2);
+            pp[c] = O.x;
+            pp[c + 1] = O.y;
+            pp[c + 2] = O.z;
+            pp[c + 3] = O.w;
+            if (c == 0) {
+                pp[D] = M;
+                pp[D + 1] = L;
             }
-            const int h = g * G + r;
-            if (a.splits == 1) {
-                a.out[(size_t)b * a.nq * D + (size_t)h * D + c] = f2bf(O / L);
-            } else {
-                float* pp = a.part + (((size_t)b * a.nq + h) * a.splits + s) * (D + 2);
-                pp[c] = O;
-                if (c == 0) {
-                    pp[D] = M;
-                    pp[D + 1] = L;
-                }
-            }
-        }
-    } else if (a.splits > 1) {
-        // an empty split still writes a full partial (zero output, zero weight): the merge
-        // reads every split, and the scratch holds whatever an earlier call left there
-        for (int idx = tid; idx < G * (D + 2); idx += 128) {
-            const int r = idx / (D + 2), c = idx % (D + 2);
-            float* pp = a.part + (((size_t)b * a.nq + g * G + r) * a.splits + s) * (D + 2);
-            pp[c] = c == D ? -INFINITY : 0.f;
         }
     }
-    if (a.splits == 1) return;
+    if (S == 1) return;
+
+    if (cl) {
+        cluster_sync();  // all partials have arrived
+        // rows r = s, s + S, ...: weighted sum over the splits in split order
+        for (int r = s; r < G; r += S) {
+            const float* rv = recv + (size_t)(r / S) * S * LDR;
+            float M = -INFINITY;
+            for (int z = 0; z < S; ++z) M = fmaxf(M, rv[(size_t)z * LDR + D]);
+            float L = 0.f;
+            for (int z = 0; z < S; ++z) {
+                const float mz = rv[(size_t)z * LDR + D];
+                if (mz != -INFINITY) L += exp2f(mz - M) * rv[(size_t)z * LDR + D + 1];
+            }
+            const float invL = 1.0f / L;
+            for (int c = tid; c < D; c += 128) {
+                float O = 0.f;
+                for (int z = 0; z < S; ++z) {
+                    const float mz = rv[(size_t)z * LDR + D];
+                    if (mz != -INFINITY) O += exp2f(mz - M) * rv[(size_t)z * LDR + c];
+                }
+                a.out[(size_t)b * a.nq * D + (size_t)(g * G + r) * D + c] = f2bf(O * invL);
+            }
+        }
+        return;
+    }
 
     // ---- the last CTA of (b, g) merges the splits in split order
     __threadfence();
     __syncthreads();
     if (tid == 0) ticket_s = atomicAdd(&a.counters[b * a.nkv + g], 1);
     __syncthreads();
-    if (ticket_s != a.splits - 1) return;
+    if (ticket_s != S - 1) return;
     __threadfence();
     // weights of each split: f_z = exp2(m_z - M) / sum_z exp2(m_z - M) l_z (one warp per head)
     float* fz = reinterpret_cast<float*>(kvbuf);  // [G][splits]
     for (int r = warp; r < G; r += 4) {
-        const float* pp = a.part + ((size_t)b * a.nq + g * G + r) * a.splits * (D + 2);
+        const float* pp = a.part + ((size_t)b * a.nq + g * G + r) * S * (D + 2);
         float M = -INFINITY;
-        for (int z = lane; z < a.splits; z += 32) M = fmaxf(M, __ldcg(pp + (size_t)z * (D + 2) + D));
+        for (int z = lane; z < S; z += 32) M = fmaxf(M, __ldcg(pp + (size_t)z * (D + 2) + D));
         M = warp_max(M);
         float L = 0.f;
-        for (int z = lane; z < a.splits; z += 32) {
+        for (int z = lane; z < S; z += 32) {
             const float mz = __ldcg(pp + (size_t)z * (D + 2) + D);
             const float f = mz == -INFINITY ? 0.f : exp2f(mz - M);
-            fz[r * a.splits + z] = f;
+            fz[r * S + z] = f;
             L += f * __ldcg(pp + (size_t)z * (D + 2) + D + 1);
         }
         L = warp_sum(L);
         __syncwarp();
-        for (int z = lane; z < a.splits; z += 32) fz[r * a.splits + z] /= L;
+        for (int z = lane; z < S; z += 32) fz[r * S + z] /= L;
     }
     __syncthreads();
     // weighted sum over splits in split order; loads of one split are coalesced across threads
     for (int idx = tid; idx < G * D; idx += 128) {
         const int r = idx / D, c = idx % D;
         const int h = g * G + r;
-        const float* pp = a.part + ((size_t)b * a.nq + h) * a.splits * (D + 2) + c;
-        const float* f = fz + r * a.splits;
+        const float* pp = a.part + ((size_t)b * a.nq + h) * S * (D + 2) + c;
+        const float* f = fz + r * S;
         float O = 0.f;
         int z = 0;
-        for (; z + 4 <= a.splits; z += 4) {
+        for (; z + 4 <= S; z += 4) {
             const float p0 = __ldcg(pp + (size_t)z * (D + 2)), p1 = __ldcg(pp + (size_t)(z + 1) * (D + 2));
             const float p2 = __ldcg(pp + (size_t)(z + 2) * (D + 2)), p3 = __ldcg(pp + (size_t)(z + 3) * (D + 2));
             O += f[z] * p0;
@@ -402,7 +468,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             O += f[z + 2] * p2;
             O += f[z + 3] * p3;
         }
-        for (; z < a.splits; ++z) O += f[z] * __ldcg(pp + (size_t)z * (D + 2));
+        for (; z < S; ++z) O += f[z] * __ldcg(pp + (size_t)z * (D + 2));
         a.out[(size_t)b * a.nq * D + (size_t)h * D + c] = f2bf(O);
     }
     if (tid == 0) a.counters[b * a.nkv + g] = 0;
@@ -740,40 +806,72 @@ cudaError_t launch_ex(K kern, dim3 grid, dim3 block, size_t smem, cudaStream_t s
 
 }  // namespace
 
-// One wave of (sequence, kv head, split) CTAs, each split at least 8 pages long.
-int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms) {
+// One wave of (sequence, kv head, split) CTAs, each split at least 8 pages long; merged
+// in a cluster, at most kDecodeMaxSplits (the CTAs of one cluster).
+int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms, bool cluster) {
     const int ctas = B * nkv;
     int s = (num_sms + ctas - 1) / ctas;
     const int pages = (max_ctx + kPage - 1) / kPage;
     const int max_s = (pages + 7) / 8;
     if (s > max_s) s = max_s;
+    if (cluster && s > kDecodeMaxSplits) s = kDecodeMaxSplits;
     if (s < 1) s = 1;
     return s;
 }
 
 template <int D>
-size_t decode_smem() {
+size_t decode_smem(int G, int splits) {
     const size_t ring = (size_t)4 * kRing * 2 * kPage * (D + 8) * 2;  // page rings of 4 warps
-    const size_t merge = (size_t)4 * 16 * D * 4;                     // per-warp partial outputs
+    const size_t rows_owned = (size_t)(G + splits - 1) / splits;
+    const size_t merge = (size_t)4 * 16 * D * 4 + rows_owned * splits * (D + 4) * 4;  // warp partials + receive
     return ring > merge ? ring : merge;
 }
 
+template <int D>
+cudaError_t decode_launch_d(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
+    const int G = a.nq / a.nkv;
+    const size_t smem = decode_smem<D>(G, a.splits);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<D>), (int)smem);
+    if (e != cudaSuccess) return e;
+    const bool cl = a.splits > 1 && a.part == nullptr;
+    if (cl && a.splits > 8) {
+        static std::once_flag once;
+        static cudaError_t ce = cudaSuccess;
+        std::call_once(once, [] {
+            ce = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        });
+        if (ce != cudaSuccess) return ce;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.splits, a.nkv, a.B);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (cl) {  // the splits of a (sequence, kv head) merge inside one cluster
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = a.splits;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, attn_decode_kernel<D>, a);
+}
+
 cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
-    const dim3 grid(a.splits, a.nkv, a.B);
-    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64>()) return cudaErrorInvalidValue;
-    if (a.d == 128) {
-        const size_t smem = decode_smem<128>();
-        cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<128>), (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_ex(attn_decode_kernel<128>, grid, dim3(128), smem, st, pdl, a);
-    }
-    if (a.d == 64) {
-        const size_t smem = decode_smem<64>();
-        cudaError_t e =
-            ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<64>), (int)smem);
-        if (e != cudaSuccess) return e;
-        return launch_ex(attn_decode_kernel<64>, grid, dim3(128), smem, st, pdl, a);
-    }
+    if (a.splits < 1 || a.nkv <= 0 || a.nq % a.nkv != 0 || a.nq / a.nkv > 16) return cudaErrorInvalidValue;
+    if (a.splits > 1 && a.part == nullptr && a.splits > kDecodeMaxSplits) return cudaErrorInvalidValue;
+    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64>(a.nq / a.nkv, a.splits)) return cudaErrorInvalidValue;
+    if (a.d == 128) return decode_launch_d<128>(a, st, pdl);
+    if (a.d == 64) return decode_launch_d<64>(a, st, pdl);
     return cudaErrorInvalidValue;
 }
 

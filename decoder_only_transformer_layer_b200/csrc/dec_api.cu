@@ -89,10 +89,6 @@ struct dec_ctx {
     float2* rope_tab = nullptr;            // [max_context][d/2] (cos, sin): fp64 on the host, stored fp32
     float *x = nullptr, *qkv = nullptr, *logits = nullptr;
     uint16_t *xn = nullptr, *qrot = nullptr, *attn = nullptr, *act = nullptr;
-    float* attn_part = nullptr;
-    int* attn_cnt = nullptr;
-    size_t attn_part_floats = 0;
-    int attn_cnt_n = 0;
     float* gemm_ws = nullptr;  // tensor-core GEMM: pieces of tiles shared between CTAs
     int* gemm_cnt = nullptr;   // and their arrival counters (zero between launches)
     int gemm_cnt_n = 0;
@@ -102,7 +98,6 @@ struct dec_ctx {
     int32_t* d_prompt = nullptr; // [max_context]
     int* h_err = nullptr;
     int act_cols = 0;
-    int decode_splits = 1;
     // MoE step buffers (rows: max_tok tokens, or max_tok * top_k (token, expert) slots)
     float *moe_logits = nullptr, *moe_w = nullptr, *moe_sgate = nullptr, *moe_y = nullptr, *moe_ys = nullptr;
     int32_t *moe_routes = nullptr, *moe_perm = nullptr, *moe_inv = nullptr, *moe_groups = nullptr, *moe_ngroups = nullptr;
@@ -164,7 +159,8 @@ struct Proj {
 dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, const float* xr, const float* g,
                     const uint16_t* xb, float* y, int ldy, const float* bias, uint16_t* act, int ldact,
                     cudaStream_t st, unsigned long long* amax = nullptr) {
-    if (n <= 8 && gemv_fits(n, p.K, c->smem_cap)) {
+    const int cap = c->smem_cap;
+    if (n <= 8 && gemv_fits(n, p.K, cap)) {
         GemvArgs a{};
         a.W = p.W;
         a.N = p.M;
@@ -182,7 +178,7 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
         a.ldact = ldact;
         a.amax = amax;
         a.err = c->d_err;
-        a.smem_cap = c->smem_cap;
+        a.smem_cap = cap;
         const int ge = epi == GEMM_STORE ? GEMV_STORE : epi == GEMM_RESID ? GEMV_RESID : GEMV_SWIGLU;
         CUDA_TRY(gemv_launch(a, ge, st, c->num_sms, true));
         return DEC_OK;
@@ -328,9 +324,10 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
             a.nkv = k.n_kv_heads;
             a.d = d;
             a.scale = scale;
-            a.splits = c->decode_splits;
-            a.part = c->attn_part;
-            a.counters = c->attn_cnt;
+            // context splits merged inside a cluster: no scratch, chosen per batch size
+            a.splits = attn_decode_splits(n, k.n_kv_heads, k.max_context, c->num_sms, true);
+            a.part = nullptr;
+            a.counters = nullptr;
             a.out = c->attn;
             a.err = c->d_err;
             CUDA_TRY(attn_decode_launch(a, st, true));
@@ -695,15 +692,6 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_err), sizeof(int)));
     *c->h_err = 0;
 
-    // decode attention scratch: split partials over max_context for max_batch (prefill
-    // attention merges its splits inside a cluster and needs none)
-    c->decode_splits = attn_decode_splits(k.max_batch, k.n_kv_heads, k.max_context, c->num_sms);
-    c->attn_part_floats = c->decode_splits > 1 ? (size_t)k.max_batch * k.n_q_heads * c->decode_splits * (d + 2) : 1;
-    INIT_TRY(dmalloc(&c->attn_part, c->attn_part_floats));
-    c->attn_cnt_n = k.max_batch * k.n_kv_heads;
-    INIT_TRY(dmalloc(&c->attn_cnt, c->attn_cnt_n));
-    INIT_TRY(cudaMemsetAsync(c->attn_cnt, 0, (size_t)c->attn_cnt_n * 4, st));
-
     INIT_TRY(cudaStreamSynchronize(st));
 #undef INIT_TRY
     *out = c;
@@ -748,8 +736,6 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->qrot);
     cudaFree(c->attn);
     cudaFree(c->act);
-    cudaFree(c->attn_part);
-    cudaFree(c->attn_cnt);
     cudaFree(c->gemm_ws);
     cudaFree(c->gemm_cnt);
     cudaFree(c->moe_logits);
@@ -991,7 +977,7 @@ dec_status gqa_decode_attn(const void* q, const void* k_new, const void* v_new, 
     cudaGetDevice(&dev);
     Scratch& S = g_scratch[dev];
     const int sms = device_sms();
-    const int splits = attn_decode_splits(B, nkv, max_pages * 16, sms);
+    const int splits = attn_decode_splits(B, nkv, max_pages * 16, sms, false);
     CUDA_TRY(grow(&S.attn_part, &S.attn_part_n, (size_t)B * nq * splits * (d + 2), false));
     CUDA_TRY(grow(&S.attn_cnt, &S.attn_cnt_n, (size_t)B * nkv, true));
     size_t one = 0;

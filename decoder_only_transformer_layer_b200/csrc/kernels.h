@@ -93,13 +93,13 @@ struct AttnDecodeArgs {
     int B, nq, nkv, d;
     float scale;
     int splits;
-    float* part;            // [B][nq][splits][d+2]
-    int* counters;          // [B][nkv]
+    float* part;            // [B][nq][splits][d+2], or null: the splits merge inside a cluster (<= 16)
+    int* counters;          // [B][nkv] (with part)
     uint16_t* out;          // [B][nq*d]
     int* err;
 };
 cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl);
-int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms);
+int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms, bool cluster);
 
 struct RopeAppendArgs {
     const float* qkv;  // [T][ld]

@@ -56,7 +56,7 @@ extern "C" dec_status gqa_decode_attn_noalloc(const void* q, const void* k_new, 
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return bad(DEC_ERR_CUDA, "no current device");
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // Same split choice as gqa_decode_attn, so both calls sum in the same order.
-    const int splits = dec::attn_decode_splits(B, nkv, max_pages * 16, sms);
+    const int splits = dec::attn_decode_splits(B, nkv, max_pages * 16, sms, false);
     const size_t counters = (size_t)B * nkv;
     const size_t partials = splits > 1 ? (size_t)B * nq * splits * (d + 2) : 0;
     if (counters > kCounterCap)
