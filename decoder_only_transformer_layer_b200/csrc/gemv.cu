@@ -10,11 +10,12 @@
 // Design (B200):
 //  * one CTA per SM (persistent over a contiguous range of 4-row blocks), 8
 //    consumer warps + 1 producer warp;
-//  * the producer streams 4-row x KC-column weight stages (KC <= 4096, so one
-//    bulk copy moves up to 8 KB of a row) into a shared-memory ring with
-//    cp.async.bulk (TMA engine, L2 evict-first), up to 8 stages in flight per
-//    SM. Large copies matter: 2 KB copies held the kernel near 60% of HBM
-//    bandwidth, 4-8 KB copies above 90%. The producer starts BEFORE
+//  * the producer streams 4-row x KC-column weight stages (KC <= 4096) into a
+//    shared-memory ring with cp.async.bulk (TMA engine, L2 evict-first), up to 8
+//    stages in flight per SM. Large copies matter: 2 KB copies held the kernel near
+//    60% of HBM bandwidth and 8 KB copies near 6.6 TB/s on a pure read, while 32 KB
+//    copies reach 7.2-7.4 TB/s; when a stage holds whole rows (K <= 4096) its 4 rows
+//    are one contiguous block and move in one copy, else one copy per row. The producer starts BEFORE
 //    griddepcontrol.wait: weights do not depend on the previous kernel, so their
 //    stream overlaps its tail;
 //  * the input columns sit in shared memory as bf16; with a fused RMSNorm they
@@ -116,9 +117,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvArgs a) {
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1, a.err)) goto producer_done;
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * kcols * 2));
                     uint8_t* dst = ring + (size_t)s * L.stage_bytes;
-                    for (int r = 0; r < nrows; ++r)
-                        bulk_g2s_stream(dst + (size_t)r * L.kc * 2, a.W + (size_t)(r0 + r) * a.K + k0,
-                                        (uint32_t)kcols * 2, &full[s], pol);
+                    if (kcols == a.K) {  // whole rows: the stage is one contiguous block
+                        bulk_g2s_stream(dst, a.W + (size_t)r0 * a.K, (uint32_t)(nrows * kcols * 2), &full[s], pol);
+                    } else {
+                        for (int r = 0; r < nrows; ++r)
+                            bulk_g2s_stream(dst + (size_t)r * L.kc * 2, a.W + (size_t)(r0 + r) * a.K + k0,
+                                            (uint32_t)kcols * 2, &full[s], pol);
+                    }
                     if (++s == L.stages) {
                         s = 0;
                         ph ^= 1;

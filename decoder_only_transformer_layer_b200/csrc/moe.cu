@@ -245,9 +245,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(GroupedGemvAr
                     if (!mbar_wait_bounded(&empty[s], ph ^ 1, a.err)) return;
                     mbar_arrive_expect_tx(&full[s], (uint32_t)(nrows * kcols * 2));
                     uint8_t* dst = ring + (size_t)s * L.stage_bytes;
-                    for (int r = 0; r < nrows; ++r)
-                        bulk_g2s_stream(dst + (size_t)r * L.kc * 2, W + (size_t)(r0 + r) * a.K + k0,
-                                        (uint32_t)kcols * 2, &full[s], pol);
+                    if (kcols == a.K) {  // whole rows: one contiguous block
+                        bulk_g2s_stream(dst, W + (size_t)r0 * a.K, (uint32_t)(nrows * kcols * 2), &full[s], pol);
+                    } else {
+                        for (int r = 0; r < nrows; ++r)
+                            bulk_g2s_stream(dst + (size_t)r * L.kc * 2, W + (size_t)(r0 + r) * a.K + k0,
+                                            (uint32_t)kcols * 2, &full[s], pol);
+                    }
                     if (++s == L.stages) {
                         s = 0;
                         ph ^= 1;
