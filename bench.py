@@ -245,6 +245,10 @@ WORKLOADS = {
     "tiny": dict(model="TINY", B=1, ctx=16, prefill=16),
     # standalone decode attention
     "gqa-sweep": dict(),
+    # 4096-token prefill of the Llama-3-8B shape with longer chunks: the projections become
+    # compute-bound GEMMs (the chunk-128 line is HBM-bound)
+    "llama3-8b-prefill-c512": dict(prefill_chunk=512),
+    "llama3-8b-prefill-c4096": dict(prefill_chunk=4096),
 }
 
 
@@ -264,12 +268,65 @@ def decode_step_bytes(cfg, B, ctx_list, experts_touched=None):
     return w, kv
 
 
+def run_prefill_workload(args, torch, dec, P):
+    """Prefill of a 4096-token prompt, Llama-3-8B shape, with prefill_chunk C (512 or 4096):
+    each timed run is one dec_prefill from position 0 (the sequence is reset between runs,
+    outside the timed region)."""
+    name = args.workload
+    C = WORKLOADS[name]["prefill_chunk"]
+    PROMPT = 4096
+    runs = max(2, min(args.steps, 4))
+    cfg = dict(configs.LLAMA3_8B, max_context=PROMPT + 8, max_batch=1, prefill_chunk=C)
+    w = make_device_weights(cfg, torch)
+    d = dec.Decoder(cfg, w)
+    del w
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+    prompt = synth.tokens(PROMPT, cfg["vocab"], 1000)
+    for _ in range(max(1, min(args.warmup, 2))):
+        d.prefill(0, prompt, 0)
+        d.reset(0)
+    torch.cuda.synchronize()
+    clk = Clocks(int(os.environ.get("LOCAL_RANK", "0")))
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(runs):
+        e0.record(stream)
+        d.prefill(0, prompt, 0)
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+        d.reset(0)
+    clocks = clk.stop()
+    ms = statistics.mean(times)
+    flops = gemm_flops_per_token(cfg) * PROMPT + attn_flops_prefill(cfg, PROMPT)
+    tflops = flops / (ms * 1e-3) / 1e12
+    hbm_floor_ms = (PROMPT / C) * (cfg["layers"] * layer_bytes(cfg)) / (P["hbm"] * 1e9) * 1e3
+    tc_floor_ms = flops / (P["tc_sus"] * 1e12) * 1e3
+    line = dict(metric=f"prefill tok/s ({name}, 4096 tokens, chunk {C})", value=PROMPT / (ms * 1e-3), unit="tok/s",
+                n_gpus=1, steps=runs, warmup=max(1, min(args.warmup, 2)), ms_per_step=ms, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+                config=dict(workload=f"llama3_8b shape, 4096-token prefill, chunk {C}", global_batch=1,
+                            seq_len=PROMPT, l2="inputs larger than L2"),
+                prefill=dict(tokens=PROMPT, chunk=C, ms=round(ms, 2), tflops=round(tflops, 1),
+                             tc_frac=round(tflops / P["tc_sus"], 4), tc_peak_tflops=P["tc_sus"],
+                             hbm_floor_ms=round(hbm_floor_ms, 2), tc_floor_ms=round(tc_floor_ms, 2),
+                             attainable_frac=round(max(hbm_floor_ms, tc_floor_ms) / ms, 4)),
+                clocks=clocks)
+    print(json.dumps(line))
+    d.close()
+    return 0
+
+
 def run_workload(args, torch, dec):
     name = args.workload
     P = peaks()
     W, K = max(3, args.warmup), max(1, args.steps)
     if name == "gqa-sweep":
         return run_gqa_sweep(args, torch, dec, P)
+    if "prefill_chunk" in WORKLOADS[name]:
+        return run_prefill_workload(args, torch, dec, P)
     spec = WORKLOADS[name]
     base = getattr(configs, spec["model"])
     B, ctx = spec["B"], spec["ctx"]

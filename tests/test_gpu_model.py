@@ -86,6 +86,13 @@ def test_smollm2_shape_4_layers_ragged_chunks():
     check_model(cfg, 300, 3)  # chunks 128 + 128 + 44
 
 
+def test_smollm2_shape_2_layers_chunk512():
+    # prefill_chunk 512: tensor-core GEMMs over several 128-token column tiles (N = 512, then
+    # a ragged N = 188) and prefill attention over 512-token chunks
+    cfg = configs.with_layers(configs.SMOLLM2_135M, 2, max_context=1024, prefill_chunk=512)
+    check_model(cfg, 700, 2)  # chunks 512 + 188
+
+
 def test_llama8b_shape_1_layer_chunk_tail():
     cfg = configs.with_layers(configs.LLAMA3_8B, 1, max_context=256, max_batch=1)
     check_model(cfg, 136, 2)  # chunks 128 + 8
