@@ -37,13 +37,18 @@ namespace {
 
 constexpr int BM = 128, BK = 64;
 
+// 16-column chunks of a BN-wide tile that each of the 4 epilogue warps handles in the
+// reductions (warp w takes chunks w, w + 4, ...; BN < 128 leaves some warps idle).
+template <int BN>
+constexpr int kChunks = BN >= 128 ? BN / 64 : 2;
+
 template <int BN>
 struct Cfg {
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = BN <= 64 ? 8 : 6;
-    static constexpr int TMEM_COLS = 2 * BN;  // two accumulator buffers (64/128/256 columns)
+    static constexpr int STAGES = BN <= 64 ? 8 : BN <= 128 ? 6 : 4;
+    static constexpr int TMEM_COLS = 2 * BN;  // two accumulator buffers (64/128/256/512 columns)
     static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
 };
 
@@ -245,9 +250,9 @@ DEC_DEVINL bool reduce_slice(const GemmArgs& a, const Work& w, int c, int tile, 
     const int r0 = min(BM, (c - c_lo) * rs), r1 = min(BM, r0 + rs);
     const int m0 = tile / w.tiles_n * BM, n0 = tile % w.tiles_n * BN;
     for (int rb = r0; rb < r1; rb += 32) {
-        float acc[2][16];
+        float acc[kChunks<BN>][16];
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < kChunks<BN>; ++h)
 #pragma unroll
             for (int q = 0; q < 16; ++q) acc[h][q] = 0.f;
         for (int cb = c_lo; cb <= c_hi; cb += cap) {
@@ -264,7 +269,7 @@ DEC_DEVINL bool reduce_slice(const GemmArgs& a, const Work& w, int c, int tile, 
             for (int u = 0; u < n; ++u) {
                 const float* bx = reinterpret_cast<const float*>(buf + u * BOX);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < kChunks<BN>; ++h) {
                     const int ch = warp + 4 * h;
                     if (ch * 16 < BN) {
 #pragma unroll
@@ -277,7 +282,7 @@ DEC_DEVINL bool reduce_slice(const GemmArgs& a, const Work& w, int c, int tile, 
         const int rl = rb + lane;
         const int row = rl < r1 ? m0 + rl : 0x3fffffff;  // rows outside the slice write nothing
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kChunks<BN>; ++h) {
             const int ch = warp + 4 * h;
             if (ch * 16 < BN) {
                 epilogue16(a, row, n0 + ch * 16, acc[h]);
@@ -336,15 +341,15 @@ DEC_DEVINL void red_finish(const GemmArgs& a, const Work& w, const RedPlan* rp, 
         const RedPlan& r = rp[i];
         const int m0 = r.tile / w.tiles_n * BM, n0 = r.tile % w.tiles_n * BN;
         for (int rb = r.r0; rb < r.r1; rb += 32) {
-            float acc[2][16];
+            float acc[kChunks<BN>][16];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < kChunks<BN>; ++h)
 #pragma unroll
                 for (int q = 0; q < 16; ++q) acc[h][q] = 0.f;
             for (int cc = r.c_lo; cc <= r.c_hi; ++cc, ++k) {
                 const float* bx = reinterpret_cast<const float*>(buf + k * BOX);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < kChunks<BN>; ++h) {
                     const int ch = warp + 4 * h;
                     if (ch * 16 < BN) {
 #pragma unroll
@@ -355,7 +360,7 @@ DEC_DEVINL void red_finish(const GemmArgs& a, const Work& w, const RedPlan* rp, 
             const int rl = rb + lane;
             const int row = rl < r.r1 ? m0 + rl : 0x3fffffff;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < kChunks<BN>; ++h) {
                 const int ch = warp + 4 * h;
                 if (ch * 16 < BN) {
                     epilogue16(a, row, n0 + ch * 16, acc[h]);
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_ld16_issue(acc + (uint32_t)c0 + 16, r + 16);
                     tmem_ld_wait32(r);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int h = 0; h < 2; ++h) {  // the two 16-column halves of r
                         float v[16];
 #pragma unroll
                         for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[16 * h + q]);
@@ -647,7 +652,9 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
 
 int gemm_tiles(const GemmPlan& p) { return ((p.M + BM - 1) / BM) * ((p.N + p.bn - 1) / p.bn); }
 
-int gemm_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : 128; }
+// Column tile: the whole batch up to 128 tokens; 256 beyond (more work per operand byte
+// once the product is compute-bound).
+int gemm_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }
 
 // One persistent CTA per SM, each with at least 8 k blocks of work.
 int gemm_ctas(int M, int N, int K, int num_sms) {
@@ -659,7 +666,7 @@ int gemm_ctas(int M, int N, int K, int num_sms) {
     return (int)nc;
 }
 
-size_t gemm_ws_floats(int num_sms) { return (size_t)2 * num_sms * BM * 128; }
+size_t gemm_ws_floats(int num_sms) { return (size_t)2 * num_sms * BM * 256; }
 
 int gemm_cnt_needed(int M, int N) { return ((M + BM - 1) / BM) * ((N + 31) / 32); }
 
@@ -689,6 +696,7 @@ cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl
         case 32: return launch_bn<32>(p, a, st, pdl);
         case 64: return launch_bn<64>(p, a, st, pdl);
         case 128: return launch_bn<128>(p, a, st, pdl);
+        case 256: return launch_bn<256>(p, a, st, pdl);
         default: return cudaErrorInvalidValue;
     }
 }

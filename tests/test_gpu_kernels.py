@@ -19,7 +19,8 @@ KERNEL_REL = 2e-5
 GEMV_CASES = [(1, 6152, 4096), (1, 1000, 688), (1, 4100, 576), (2, 517, 1408), (3, 999, 2048), (4, 300, 14336),
               (8, 256, 576), (8, 129, 4096), (1, 9, 64)]
 GEMM_CASES = [(9, 300, 704), (16, 1024, 4096), (32, 777, 2048), (64, 1500, 1408), (100, 640, 576),
-              (128, 6144, 4096), (160, 2100, 448), (256, 512, 1024), (33, 129, 14336)]
+              (128, 6144, 4096), (160, 2100, 448), (256, 512, 1024), (33, 129, 14336), (300, 1000, 2048),
+              (512, 768, 4096)]
 
 
 @pytest.mark.parametrize("B,N,K", GEMV_CASES + GEMM_CASES)
