@@ -277,6 +277,8 @@ def run_prefill_workload(args, torch, dec, P):
     PROMPT = 4096
     runs = max(2, min(args.steps, 4))
     cfg = dict(configs.LLAMA3_8B, max_context=PROMPT + 8, max_batch=1, prefill_chunk=C)
+    if args.layers:  # profiling only: fewer layers of the same shape
+        cfg = configs.with_layers(cfg, args.layers)
     w = make_device_weights(cfg, torch)
     d = dec.Decoder(cfg, w)
     del w

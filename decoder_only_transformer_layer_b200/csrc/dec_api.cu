@@ -1014,7 +1014,15 @@ dec_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k, 
     if (!logits || !idx_out || !w_out) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
     if (T <= 0 || E <= 0 || k <= 0 || k > E) return fail(DEC_ERR_INVALID_ARG, "bad T / E / k");
     if (E > 256 || k > 16) return fail(DEC_ERR_UNSUPPORTED, "E <= 256 and k <= 16");
-    CUDA_TRY(topk_launch(logits, T, E, k, renorm, idx_out, w_out, reinterpret_cast<cudaStream_t>(stream), false));
+    // the same routing kernel as the MoE layer, without the shared-expert gate
+    MoeRouteArgs r{};
+    r.logits = logits;
+    r.E = E;
+    r.k = k;
+    r.renorm = renorm;
+    r.idx = idx_out;
+    r.w = w_out;
+    CUDA_TRY(moe_route_launch(r, T, reinterpret_cast<cudaStream_t>(stream), false));
     return DEC_OK;
 }
 

@@ -3,9 +3,9 @@
 //    embed scale 1;
 //  * RMSNorm of fp32 residual rows to bf16 (ANEDVD rmsnormColumn / rmsnormChunk:
 //    x * (1/sqrt(mean(x^2) + eps)) * w, written in the device input precision);
-//  * greedy argmax over logits, lowest index on ties;
-//  * MoE routing: softmax over all experts, top-k, optional renormalisation
-//    (ANEDVD cpu.moeRoute; frink route_top_k; cortiq MoeFfn).
+//  * moving cache rows between the paged pool and dense arrays (test hooks).
+// The greedy argmax is folded into the LM-head epilogues (gemv.cu, gemm_tc.cu) and the
+// MoE routing lives in moe.cu.
 #include <math.h>
 
 #include "common.cuh"
@@ -92,127 +92,6 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
     }
 }
 
-struct ArgmaxArgs {
-    const float* logits;
-    int V;
-    int32_t* out;
-};
-
-__global__ void __launch_bounds__(1024) argmax_kernel(ArgmaxArgs a) {
-    __shared__ float bv[32];
-    __shared__ int bi[32];
-    pdl_trigger();
-    pdl_wait();
-    const int b = blockIdx.x;
-    const float* l = a.logits + (size_t)b * a.V;
-    float best = -INFINITY;
-    int idx = 0x7fffffff;
-    for (int i = threadIdx.x; i < a.V; i += blockDim.x) {
-        const float v = l[i];
-        if (v > best || (v == best && i < idx)) {
-            best = v;
-            idx = i;
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, idx, o);
-        if (ov > best || (ov == best && oi < idx)) {
-            best = ov;
-            idx = oi;
-        }
-    }
-    const int w = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) == 0) {
-        bv[w] = best;
-        bi[w] = idx;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int nw = blockDim.x >> 5;
-        for (int k = 1; k < nw; ++k)
-            if (bv[k] > best || (bv[k] == best && bi[k] < idx)) {
-                best = bv[k];
-                idx = bi[k];
-            }
-        a.out[b] = idx;
-    }
-}
-
-struct TopkArgs {
-    const float* logits;
-    int E, k, renorm;
-    int32_t* idx;
-    float* w;
-};
-
-// One warp per row: E <= 256 logits held 8 per lane.
-__global__ void __launch_bounds__(32) topk_kernel(TopkArgs a) {
-    pdl_trigger();
-    pdl_wait();
-    const int t = blockIdx.x, lane = threadIdx.x;
-    const float* r = a.logits + (size_t)t * a.E;
-    float v[8];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        v[j] = e < a.E ? r[e] : -INFINITY;
-        mx = fmaxf(mx, v[j]);
-    }
-    mx = warp_max(mx);
-    float p[8], sum = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        p[j] = e < a.E ? expf(v[j] - mx) : 0.f;
-        sum += p[j];
-    }
-    sum = warp_sum(sum);
-    const float inv = 1.0f / sum;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) p[j] *= inv;
-    bool taken[8] = {false, false, false, false, false, false, false, false};
-    float sel_p[16];
-    int sel_i[16];
-    float tot = 0.f;
-    for (int q = 0; q < a.k; ++q) {
-        float bp = -1.f;
-        int be = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            if (e < a.E && !taken[j] && (p[j] > bp || (p[j] == bp && e < be))) {
-                bp = p[j];
-                be = e;
-
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float op = __shfl_xor_sync(0xffffffffu, bp, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            if (op > bp || (op == bp && oe < be)) {
-                bp = op;
-                be = oe;
-            }
-        }
-        if ((be & 31) == lane) taken[be >> 5] = true;
-
-        if (q < 16) {
-            sel_p[q] = bp;
-            sel_i[q] = be;
-        }
-        tot += bp;
-    }
-    if (lane == 0) {
-        for (int q = 0; q < a.k && q < 16; ++q) {
-            a.idx[(size_t)t * a.k + q] = sel_i[q];
-            a.w[(size_t)t * a.k + q] = a.renorm ? sel_p[q] / tot : sel_p[q];
-        }
-    }
-}
 
 }  // namespace
 
@@ -227,17 +106,6 @@ cudaError_t rmsnorm_launch(const float* x, const float* g, int T, int h, float e
     return launch_ex(rmsnorm_kernel, dim3(T), dim3(256), 0, st, pdl, a);
 }
 
-cudaError_t argmax_launch(const float* logits, int B, int V, int32_t* out, cudaStream_t st, bool pdl) {
-    ArgmaxArgs a{logits, V, out};
-    return launch_ex(argmax_kernel, dim3(B), dim3(1024), 0, st, pdl, a);
-}
-
-cudaError_t topk_launch(const float* logits, int T, int E, int k, int renorm, int32_t* idx, float* w,
-                        cudaStream_t st, bool pdl) {
-    if (E > 256 || k > 16 || k > E || k <= 0) return cudaErrorInvalidValue;
-    TopkArgs a{logits, E, k, renorm, idx, w};
-    return launch_ex(topk_kernel, dim3(T), dim3(32), 0, st, pdl, a);
-}
 
 }  // namespace dec
 

@@ -650,8 +650,6 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
 
 }  // namespace
 
-int gemm_tiles(const GemmPlan& p) { return ((p.M + BM - 1) / BM) * ((p.N + p.bn - 1) / p.bn); }
-
 // Column tile: the whole batch up to 128 tokens; 256 beyond (more work per operand byte
 // once the product is compute-bound).
 int gemm_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }

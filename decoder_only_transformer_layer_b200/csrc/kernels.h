@@ -65,7 +65,6 @@ struct GemmArgs {
 // addresses). ws holds gemm_ws_floats(num_sms) floats.
 cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16_t* B, int N, int num_sms,
                       const float* ws);
-int gemm_tiles(const GemmPlan& p);
 size_t gemm_ws_floats(int num_sms);
 int gemm_cnt_needed(int M, int N);
 cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl);
@@ -147,9 +146,6 @@ __host__ __device__ inline int argmax_unpack(unsigned long long w) { return (int
 cudaError_t embed_launch(const uint16_t* E, const int32_t* tok, int B, int h, float* x, cudaStream_t st, bool pdl);
 cudaError_t rmsnorm_launch(const float* x, const float* g, int T, int h, float eps, uint16_t* out, cudaStream_t st,
                            bool pdl);
-cudaError_t argmax_launch(const float* logits, int B, int V, int32_t* out, cudaStream_t st, bool pdl);
-cudaError_t topk_launch(const float* logits, int T, int E, int k, int renorm, int32_t* idx, float* w,
-                        cudaStream_t st, bool pdl);
 
 }  // namespace dec
 
