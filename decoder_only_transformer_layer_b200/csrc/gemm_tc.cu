@@ -119,36 +119,48 @@ DEC_DEVINL void argmax16(const GemmArgs& a, int row, int t0, const float (&v)[16
 // segments, one per tile it touches: whole tiles in the middle, and at its two ends
 // pieces of tiles it shares with the neighbouring CTAs.
 struct Work {
-    long long U;  // units
+    long long U;  // stream-K units (the first tsk tiles x nkb)
     int nkb, tiles_n, bn, nc;
+    int tsk;      // tiles split by stream-K (tiles [0, tsk))
+    int dp;       // whole tiles per CTA after them, round-robin: CTA c takes tsk + c + j nc
 };
 
+// With several column tiles (N > BN) and at least two tiles per CTA, all but about one
+// round of tiles go round-robin, so the CTAs working at the same time share weight blocks
+// in L2; the rest (at least one tile per CTA, so no piece is shorter than a tile's worth of
+// k blocks on average) is split by stream-K and processed first. With one column tile
+// every tile is split by stream-K.
 DEC_DEVINL Work make_work(const GemmArgs& a, int bn) {
     Work w;
     w.nkb = (a.K + BK - 1) / BK;
     w.tiles_n = (a.N + bn - 1) / bn;
-    w.U = (long long)((a.M + BM - 1) / BM) * w.tiles_n * w.nkb;
     w.bn = bn;
     w.nc = gridDim.x;
+    const int T = ((a.M + BM - 1) / BM) * w.tiles_n;
+    w.dp = (w.tiles_n > 1 && T >= 2 * w.nc) ? T / w.nc - 1 : 0;
+    w.tsk = T - w.dp * w.nc;
+    w.U = (long long)w.tsk * w.nkb;
     return w;
 }
 
 DEC_DEVINL long long unit0(const Work& w, int c) { return w.U * c / w.nc; }
-// CTA whose range holds unit u.
+// CTA whose range holds stream-K unit u (w.U > 0).
 DEC_DEVINL int cta_of(const Work& w, long long u) { return (int)(((u + 1) * w.nc - 1) / w.U); }
 
 struct Range {
     long long u0, u1;
-    int tf, nseg, iters;
+    int c, tf, nsk, nseg, iters;  // nsk: stream-K segments, then w.dp whole tiles
 };
 
 DEC_DEVINL Range cta_range(const Work& w, int c) {
     Range r;
+    r.c = c;
     r.u0 = unit0(w, c);
     r.u1 = unit0(w, c + 1);
-    r.iters = (int)(r.u1 - r.u0);
     r.tf = (int)(r.u0 / w.nkb);
-    r.nseg = r.u1 > r.u0 ? (int)((r.u1 - 1) / w.nkb) - r.tf + 1 : 0;
+    r.nsk = r.u1 > r.u0 ? (int)((r.u1 - 1) / w.nkb) - r.tf + 1 : 0;
+    r.nseg = r.nsk + w.dp;
+    r.iters = (int)(r.u1 - r.u0) + w.dp * w.nkb;
     return r;
 }
 
@@ -156,13 +168,21 @@ struct Seg {
     int tile, kb0, kb1, slot;  // slot: 0 = first tile of the range, 1 = any later one
 };
 
-// The j-th segment in processing order: the pieces at the two ends of the range come
-// first (their tiles are finished by whichever CTA completes its piece last, so those
-// reductions overlap the whole tiles processed afterwards), then the middle tiles.
+// The j-th segment in processing order: the stream-K pieces at the two ends of the range
+// come first (their tiles are finished by whichever CTA completes its piece last, so those
+// reductions overlap the whole tiles processed afterwards), then the middle tiles, then
+// the round-robin whole tiles.
 DEC_DEVINL Seg segment(const Work& w, const Range& r, int j) {
-    int i = j;
-    if (r.nseg >= 2) i = j == 0 ? r.nseg - 1 : j - 1;
     Seg s;
+    if (j >= r.nsk) {
+        s.tile = w.tsk + r.c + (j - r.nsk) * w.nc;
+        s.kb0 = 0;
+        s.kb1 = w.nkb;
+        s.slot = 1;
+        return s;
+    }
+    int i = j;
+    if (r.nsk >= 2) i = j == 0 ? r.nsk - 1 : j - 1;
     s.tile = r.tf + i;
     const long long t0 = (long long)s.tile * w.nkb;
     s.kb0 = (int)((r.u0 > t0 ? r.u0 : t0) - t0);
@@ -171,7 +191,7 @@ DEC_DEVINL Seg segment(const Work& w, const Range& r, int j) {
     return s;
 }
 
-// Workspace slot of CTA cc's piece of `tile`.
+// Workspace slot of CTA cc's piece of (stream-K) `tile`.
 DEC_DEVINL int piece_slot(const Work& w, int cc, int tile) { return (int)(unit0(w, cc) / w.nkb) == tile ? 0 : 1; }
 
 // Walks the k blocks of a range in processing order (the producer's view).
@@ -447,14 +467,23 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 4) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
+            // A weight block read by one column tile only streams through L2 (evict-first);
+            // with several column tiles it is read again, so it keeps the normal policy.
             const uint64_t pol = policy_evict_first();
+            const bool once = w.tiles_n == 1;
+            auto load_a = [&](void* dst, int kb, int m0, uint64_t* bar) {
+                if (once)
+                    tma_load_2d_hint(dst, &tmA, kb * BK, m0, bar, pol);
+                else
+                    tma_load_2d(dst, &tmA, kb * BK, m0, bar);
+            };
             const int total = rg.iters;
             const int pre = total < C::STAGES ? total : C::STAGES;
             // the weight slices of the first stages do not depend on the previous kernel
             SegIter it(w, rg);
             for (int i = 0; i < pre; ++i, it.next()) {
                 mbar_arrive_expect_tx(&full[i], C::STAGE);
-                tma_load_2d_hint(smem + i * C::STAGE, &tmA, it.kb * BK, it.m0, &full[i], pol);
+                load_a(smem + i * C::STAGE, it.kb, it.m0, &full[i]);
             }
             pdl_wait();
             SegIter jt(w, rg);
@@ -465,7 +494,7 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t u = (uint32_t)(i / C::STAGES);
                 if (!mbar_wait_bounded(&empty[s], (u & 1u) ^ 1u, a.err)) break;
                 mbar_arrive_expect_tx(&full[s], C::STAGE);
-                tma_load_2d_hint(smem + s * C::STAGE, &tmA, it.kb * BK, it.m0, &full[s], pol);
+                load_a(smem + s * C::STAGE, it.kb, it.m0, &full[s]);
                 tma_load_2d(smem + s * C::STAGE + C::A_BYTES, &tmB, it.kb * BK, it.n0, &full[s]);
             }
         }
