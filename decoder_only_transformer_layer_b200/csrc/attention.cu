@@ -613,7 +613,9 @@ __global__ void __launch_bounds__(128, 3) attn_prefill_kernel(AttnPrefillArgs a)
     uint16_t* kb = reinterpret_cast<uint16_t*>(dyn);  // [2][64][LD]
     uint16_t* vb = kb + 2 * kPrefKeys * LD;           // [2][64][LD]
 
-    const int qb = blockIdx.x, g = blockIdx.y, s = blockIdx.z, S = gridDim.z;
+    // row blocks in reverse: under the causal mask the last rows see the most keys, so the
+    // longest CTAs are dispatched first and the shortest fill the tail
+    const int qb = gridDim.x - 1 - blockIdx.x, g = blockIdx.y, s = blockIdx.z, S = gridDim.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int G = a.nq / a.nkv;
     const int R = a.T * G;
