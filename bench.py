@@ -34,6 +34,30 @@ METRIC = "decode tok/s + % HBM roofline (8B-shape, b=1); prefill tok/s + % bf16 
 PROMPT = 4096
 
 
+def main_config(world, layers):
+    """The `config` of the default line, shared by both arms (ours and the reference)."""
+    return dict(workload="llama3-8b-shape decode b=1 at context 4096 after a 4096-token prefill (chunk 128)",
+                global_batch=world, seq_len=PROMPT, model_shape="llama3-8b", layers=layers,
+                parallelism=f"replicas x{world}", l2="inputs larger than L2 (15 GB of weights per step)")
+
+
+def max_over_ranks(values, device=None):
+    """Replicas: every rank times its own copy of the workload; the job's time is the max
+    over ranks (a collective on the timings only, never on the data path)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(units_per_rank, world, ms):
+    """Whole-job throughput of N replicas: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -228,8 +252,7 @@ def run_reference(args):
     line = dict(metric=METRIC, value=val, unit="tok/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
                 ms_per_step=1000.0 / val, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
                 data="synthetic", impl="reference",
-                config=dict(workload="llama3-8b-shape decode b=1 ctx 4096 (oracle, bounded sample)",
-                            global_batch=1, seq_len=PROMPT),
+                config=main_config(args.gpus, cfg["layers"]),
                 cpu_baseline=cb, e2e=dict(value=val, unit="tok/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line))
     return 0
@@ -534,9 +557,7 @@ def main():
     decode_ms = e0.elapsed_time(e1)
     ms_step = decode_ms / K
     if world > 1:
-        t = torch.tensor([ms_step, prefill_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, prefill_ms = t.tolist()
+        ms_step, prefill_ms = max_over_ranks([ms_step, prefill_ms], "cuda")
 
     # ---- end to end through the C ABI with host buffers (tokens in, logits out per step)
     host_logits = torch.empty((1, cfg["vocab"]), dtype=torch.float32).pin_memory().numpy()
@@ -548,6 +569,8 @@ def main():
         tok = int(np.argmax(host_logits[0]))
         pos += 1
     e2e_s = (time.perf_counter() - t0) / e2e_steps
+    if world > 1:
+        (e2e_s,) = max_over_ranks([e2e_s], "cuda")
 
     # ---- dominant kernel alone: weight-streaming GEMV on the fused gate/up matrix
     P = peaks()
@@ -556,8 +579,8 @@ def main():
 
     wbytes, kvbytes = step_bytes(cfg, 1, ctx_list)
     step_gbs = (wbytes + kvbytes / K) / (ms_step * 1e-3) / 1e9
-    value = world * 1.0 / (ms_step * 1e-3)
-    pf_tok_s = world * PROMPT / (prefill_ms * 1e-3)
+    value = replica_throughput(1, world, ms_step)
+    pf_tok_s = replica_throughput(PROMPT, world, prefill_ms)
     pf_flops = gemm_flops_per_token(cfg) * PROMPT + attn_flops_prefill(cfg, PROMPT)
     pf_tflops = pf_flops / (prefill_ms * 1e-3) / 1e12
     chunk_hbm_floor_ms = (PROMPT / 128) * (cfg["layers"] * layer_bytes(cfg)) / (P["hbm"] * 1e9) * 1e3
@@ -570,9 +593,7 @@ def main():
         line = dict(
             metric=METRIC, value=value, unit="tok/s", n_gpus=world, steps=K, warmup=W, ms_per_step=ms_step,
             higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-            config=dict(workload="llama3-8b-shape decode b=1 at context 4096 after a 4096-token prefill (chunk 128)",
-                        global_batch=world, seq_len=PROMPT, model_shape="llama3-8b", layers=cfg["layers"],
-                        parallelism=f"replicas x{world}", l2="inputs larger than L2 (15 GB of weights per step)"),
+            config=main_config(world, cfg["layers"]),
             roofline=dict(bound="hbm", achieved=round(gemv_gbs, 1), peak=P["hbm"], unit="GB/s",
                           frac=round(gemv_gbs / P["hbm"], 4), traffic=measured_traffic(),
                           traffic_unit="bytes per launch (ncu dram read+write)",
