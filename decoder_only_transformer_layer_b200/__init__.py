@@ -14,7 +14,7 @@ import numpy as np
 
 from ._build import LIB, build, stale  # noqa: F401
 
-__all__ = ["lib", "Decoder", "DecError", "gqa_decode_attn", "moe_route_topk", "weight_gemv", "STATUS"]
+__all__ = ["lib", "Decoder", "DecError", "gqa_decode_attn", "moe_route_topk", "moe_experts", "weight_gemv", "STATUS"]
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "CONTEXT_OVERFLOW", 3: "PAGES_EXHAUSTED", 4: "OOM", 5: "CUDA",
           6: "TIMEOUT", 7: "UNSUPPORTED"}
@@ -77,9 +77,10 @@ def lib():
         L.gqa_decode_attn_noalloc.argtypes = L.gqa_decode_attn.argtypes
         L.moe_route_topk.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
         L.weight_gemv.argtypes = [_P, _P, _I, _I, _I, _P, _P]
+        L.moe_experts.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]
         for f in ("dec_init", "dec_free", "dec_reset", "dec_prefill", "dec_step", "dec_last_argmax", "dec_kv_read",
                   "dec_kv_write", "dec_last_routes", "dec_last_hidden", "dec_seq_len", "gqa_decode_attn",
-                  "gqa_decode_attn_noalloc", "moe_route_topk", "weight_gemv"):
+                  "gqa_decode_attn_noalloc", "moe_route_topk", "moe_experts", "weight_gemv"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -256,6 +257,17 @@ def moe_route_topk(logits, k, renorm, idx_out, w_out, stream=None):
     T, E = logits.shape
     _check(lib().moe_route_topk(_ptr(logits), T, E, k, int(renorm), _ptr(idx_out), _ptr(w_out), _stream(stream)))
     return idx_out, w_out
+
+
+def moe_experts(x, idx, w, Wgu, Wd, out, stream=None):
+    """Device tensors: x bf16 [T][h]; idx int32 [T][k]; w fp32 [T][k]; Wgu bf16 [E][2I][h]
+    (gate row i at 2i, up row i at 2i+1); Wd bf16 [E][h][I]; out fp32 [T][h]."""
+    T, h = x.shape
+    k = idx.shape[1]
+    E, I2, _ = Wgu.shape
+    _check(lib().moe_experts(_ptr(x), _ptr(idx), _ptr(w), T, h, E, k, I2 // 2, _ptr(Wgu), _ptr(Wd), _ptr(out),
+                             _stream(stream)))
+    return out
 
 
 def weight_gemv(W, x, y, stream=None):

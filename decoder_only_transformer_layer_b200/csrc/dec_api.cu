@@ -248,6 +248,7 @@ dec_status moe_ffn(dec_ctx* c, int li, int n, cudaStream_t st) {
     g.wstride = (size_t)2 * Ie * h;
     g.M = 2 * Ie;
     g.K = h;
+    g.E = E;
     g.groups = c->moe_groups;
     g.n_groups = c->moe_ngroups;
     g.x = c->xn;
@@ -462,6 +463,12 @@ struct Scratch {
     int* cnt = nullptr;
     size_t cnt_n = 0;
     int* err = nullptr;
+    int32_t* moe_i = nullptr;  // perm [Tk] | inv [Tk] | groups [4 Tk] | n_groups [1]
+    size_t moe_i_n = 0;
+    uint16_t* moe_act = nullptr;
+    size_t moe_act_n = 0;
+    float* moe_y = nullptr;
+    size_t moe_y_n = 0;
 };
 std::mutex g_scratch_mu;
 std::map<int, Scratch> g_scratch;
@@ -1023,6 +1030,83 @@ dec_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k, 
     r.idx = idx_out;
     r.w = w_out;
     CUDA_TRY(moe_route_launch(r, T, reinterpret_cast<cudaStream_t>(stream), false));
+    return DEC_OK;
+}
+
+dec_status moe_experts(const void* x, const int32_t* idx, const float* w, int32_t T, int32_t h, int32_t E,
+                       int32_t k, int32_t I, const void* Wgu, const void* Wd, float* out, dec_stream_t stream) {
+    g_err.clear();
+    if (!x || !idx || !w || !Wgu || !Wd || !out) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
+    if (T <= 0 || h <= 0 || E <= 0 || k <= 0 || k > E || I <= 0) return fail(DEC_ERR_INVALID_ARG, "bad T / h / E / k / I");
+    if (E > 256 || k > 16) return fail(DEC_ERR_UNSUPPORTED, "E <= 256 and k <= 16");
+    if (h % 8 != 0 || I % 8 != 0) return fail(DEC_ERR_UNSUPPORTED, "h and I must be multiples of 8");
+    const int nb = grouped_nb_for(T);
+    const int cap = device_smem_cap();
+    if (!grouped_fits(nb, h, cap) || !grouped_fits(nb, I, cap))
+        return fail(DEC_ERR_UNSUPPORTED, "rows too long for shared memory");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    Scratch& S = g_scratch[dev];
+    size_t one = 0;
+    if (!S.err) CUDA_TRY(grow(&S.err, &one, 1, true));
+    const size_t tk = (size_t)T * k;
+    CUDA_TRY(grow(&S.moe_i, &S.moe_i_n, 6 * tk + 1, false));
+    CUDA_TRY(grow(&S.moe_act, &S.moe_act_n, tk * I, false));
+    CUDA_TRY(grow(&S.moe_y, &S.moe_y_n, tk * h, false));
+    int32_t* perm = S.moe_i;
+    int32_t* inv = perm + tk;
+    int32_t* groups = inv + tk;
+    int32_t* n_groups = groups + 4 * tk;
+    MoePermArgs p{};
+    p.idx = idx;
+    p.n = T;
+    p.k = k;
+    p.E = E;
+    p.nb = nb;
+    p.perm_tok = perm;
+    p.inv = inv;
+    p.groups = groups;
+    p.n_groups = n_groups;
+    CUDA_TRY(moe_permute_launch(p, st, false));
+    GroupedGemvArgs g{};
+    g.W = static_cast<const uint16_t*>(Wgu);
+    g.wstride = (size_t)2 * I * h;
+    g.M = 2 * I;
+    g.K = h;
+    g.E = E;
+    g.groups = groups;
+    g.n_groups = n_groups;
+    g.x = static_cast<const uint16_t*>(x);
+    g.x_map = perm;
+    g.ldx = h;
+    g.act = S.moe_act;
+    g.ldact = I;
+    g.err = S.err;
+    g.smem_cap = cap;
+    const int sms = device_sms();
+    CUDA_TRY(grouped_gemv_launch(g, nb, true, st, sms, false));
+    g.W = static_cast<const uint16_t*>(Wd);
+    g.wstride = (size_t)h * I;
+    g.M = h;
+    g.K = I;
+    g.x = S.moe_act;
+    g.x_map = nullptr;
+    g.ldx = I;
+    g.act = nullptr;
+    g.y = S.moe_y;
+    g.ldy = h;
+    CUDA_TRY(grouped_gemv_launch(g, nb, false, st, sms, false));
+    CUDA_TRY(cudaMemsetAsync(out, 0, (size_t)T * h * sizeof(float), st));
+    MoeCombineArgs m{};
+    m.x = out;
+    m.y = S.moe_y;
+    m.w = w;
+    m.inv = inv;
+    m.k = k;
+    m.h = h;
+    CUDA_TRY(moe_combine_launch(m, T, st, false));
     return DEC_OK;
 }
 

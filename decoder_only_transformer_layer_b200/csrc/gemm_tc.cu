@@ -679,6 +679,11 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
 
 }  // namespace
 
+// Row-major bf16 [rows][K] read in 128B-swizzled boxes of 64 columns x box_rows rows.
+cudaError_t tmap_bf16_rows(CUtensorMap* tm, const uint16_t* base, int rows, int K, int box_rows) {
+    return encode_2d(tm, base, rows, K, box_rows);
+}
+
 // Column tile: the whole batch up to 128 tokens; 256 beyond (more work per operand byte
 // once the product is compute-bound).
 int gemm_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }

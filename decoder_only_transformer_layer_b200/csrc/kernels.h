@@ -68,6 +68,9 @@ cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16
 size_t gemm_ws_floats(int num_sms);
 int gemm_cnt_needed(int M, int N);
 cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl);
+// Tensor map over a row-major bf16 [rows][K] matrix, read in 128B-swizzled boxes of 64
+// columns x box_rows rows (host; fails on a base or stride the TMA unit cannot take).
+cudaError_t tmap_bf16_rows(CUtensorMap* tm, const uint16_t* base, int rows, int K, int box_rows);
 
 // ----------------------------------------------------------------- attention
 
@@ -201,6 +204,7 @@ struct GroupedGemvArgs {
     const uint16_t* W;    // expert 0 weights [M][K]; expert e at W + e * wstride
     size_t wstride;
     int M, K;
+    int E;                // experts in W (the tensor-core path reads W as [E*M][K])
     const int32_t* groups;
     const int32_t* n_groups;
     const uint16_t* x;    // token rows (bf16), row of slot p = x_map ? x_map[p] : p
@@ -214,6 +218,7 @@ struct GroupedGemvArgs {
     int smem_cap;
 };
 int grouped_nb_for(int n);
+bool grouped_uses_mma(int nb, int M, int K, size_t wstride, int smem_cap);
 bool grouped_fits(int nb, int K, int smem_cap);
 cudaError_t grouped_gemv_launch(const GroupedGemvArgs& a, int nb, bool swiglu, cudaStream_t st, int num_sms,
                                 bool pdl);

@@ -7,16 +7,19 @@
 //
 // B200 design: the tokens of a step or prefill chunk are permuted by expert (counts,
 // offsets, a deterministic token list per expert), split into groups of at most NB tokens,
-// and every (group, 4-row weight block) pair is one work item of a grouped weight-streaming
-// GEMV: each expert's weights stream once per group through the same bulk-copy ring as the
-// dense GEMV (8 KB row copies), the group's token rows sit in shared memory, and the
-// epilogue writes SiLU(gate)*up (bf16) or the projection (fp32) per (token, expert) slot.
+// and each expert's weights stream once per group. Groups of up to 4 tokens run a grouped
+// weight-streaming GEMV on the CUDA cores (work item = group x 4-row weight block, the same
+// bulk-copy ring as the dense GEMV); groups of 8 run on the tensor pipe (work item = group
+// x 128-row block, TMA boxes, mma.sync with the 8 tokens as the n dimension). Either way
+// the group's token rows sit in shared memory and the epilogue writes SiLU(gate)*up (bf16)
+// or the projection (fp32) per (token, expert) slot.
 // A combine kernel adds the weighted slots and the gated shared expert to the residual in
 // a fixed order (routed experts in top-k order, then the shared expert).
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace dec {
 
@@ -114,44 +117,68 @@ __global__ void __launch_bounds__(32) moe_route_kernel(MoeRouteArgs a) {
 
 // ------------------------------------------------------------------ permutation by expert
 
-// One CTA: counts per expert, offsets, per-expert token lists in (token, slot) order,
-// the inverse map, and the groups of at most nb tokens (expert order) for the grouped GEMV.
+// One CTA, thread e owns expert e: counts per expert, offsets, per-expert token lists in
+// (token, slot) order, the inverse map, and the groups of at most nb tokens (expert order)
+// for the grouped GEMV. The routing table passes through shared memory in tiles, so each
+// thread's scan is a run of broadcast reads.
+constexpr int kPermTile = 2048;
+
 __global__ void __launch_bounds__(256) moe_permute_kernel(MoePermArgs a) {
-    __shared__ int cnt[256], off[256], goff[256];
+    __shared__ int off[256], goff[256];
+    __shared__ int sidx[kPermTile];
     pdl_trigger();
     pdl_wait();
     const int tid = threadIdx.x;
     const int total = a.n * a.k;
-    for (int e = tid; e < a.E; e += 256) {
-        int c = 0;
-        for (int i = 0; i < total; ++i) c += a.idx[i] == e;
-        cnt[e] = c;
+    const bool mine = tid < a.E;
+    int cnt = 0;
+    for (int base = 0; base < total; base += kPermTile) {
+        const int m = min(kPermTile, total - base);
+        __syncthreads();
+        for (int i = tid; i < m; i += 256) sidx[i] = a.idx[base + i];
+        __syncthreads();
+        if (mine)
+            for (int i = 0; i < m; ++i) cnt += sidx[i] == tid;
     }
+    if (mine) off[tid] = cnt;
     __syncthreads();
     if (tid == 0) {
         int o = 0, g = 0;
         for (int e = 0; e < a.E; ++e) {
+            const int c = off[e];
             off[e] = o;
             goff[e] = g;
-            o += cnt[e];
-            g += (cnt[e] + a.nb - 1) / a.nb;
+            o += c;
+            g += (c + a.nb - 1) / a.nb;
         }
         *a.n_groups = g;
     }
     __syncthreads();
-    for (int e = tid; e < a.E; e += 256) {
-        int p = off[e];
-        for (int i = 0; i < total; ++i)
-            if (a.idx[i] == e) {
-                a.perm_tok[p] = i / a.k;
-                a.inv[i] = p;
-                ++p;
-            }
+    int p = mine ? off[tid] : 0;
+    for (int base = 0; base < total; base += kPermTile) {
+        const int m = min(kPermTile, total - base);
+        __syncthreads();
+        for (int i = tid; i < m; i += 256) {
+            const int e = a.idx[base + i];
+            sidx[i] = e;
+            if (e < 0 || e >= a.E) a.inv[base + i] = -1;  // dropped: the combine skips it
+        }
+        __syncthreads();
+        if (mine)
+            for (int i = 0; i < m; ++i)
+                if (sidx[i] == tid) {
+                    a.perm_tok[p] = (base + i) / a.k;
+                    a.inv[base + i] = p;
+                    ++p;
+                }
+    }
+    if (mine) {
+        const int e = tid, o = off[e];
         int g = goff[e];
-        for (int s = 0; s < cnt[e]; s += a.nb, ++g) {
+        for (int s = 0; s < cnt; s += a.nb, ++g) {
             a.groups[g * 4 + 0] = e;
-            a.groups[g * 4 + 1] = off[e] + s;
-            a.groups[g * 4 + 2] = min(a.nb, cnt[e] - s);
+            a.groups[g * 4 + 1] = o + s;
+            a.groups[g * 4 + 2] = min(a.nb, cnt - s);
             a.groups[g * 4 + 3] = 0;
         }
     }
@@ -339,6 +366,177 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(GroupedGemvAr
     }
 }
 
+// ------------------------------------------------------------------ grouped GEMM on the tensor pipe
+
+// Groups of up to 8 tokens: the CUDA-core GEMV above converts every token element once per
+// weight row and becomes ALU-bound, so here each group's token rows are the n = 8 operand
+// of mma.sync m16n8k16 (bf16 in, fp32 accumulate). A work item is (group, 128-row weight
+// block); the TMA unit streams the block in 128B-swizzled boxes of 64 columns x 128 rows,
+// and consumer warp w owns rows 16w .. 16w+15 of the block over the whole K, so no partial
+// sums cross warps. Token rows sit in shared memory with a 16-byte pad per row, which
+// makes the ldmatrix reads of both operands free of bank conflicts.
+constexpr int kTcRows = 128;
+constexpr int kTcK = 64;
+constexpr uint32_t kTcBox = kTcRows * kTcK * 2;  // 16 KB
+constexpr int kTcMaxStages = 8;
+constexpr int kTcTok = 8;
+
+struct TcLayout {
+    int kp, stages;  // padded token row (elements); operand ring depth
+    uint32_t xs_off, ring_off, total;
+};
+
+__host__ __device__ inline TcLayout make_tc_layout(int K, int smem_cap) {
+    TcLayout L;
+    L.kp = ((K + kTcK - 1) / kTcK) * kTcK + 8;
+    L.xs_off = 2 * kTcMaxStages * 8;
+    L.ring_off = (L.xs_off + (uint32_t)kTcTok * L.kp * 2 + 1023) & ~1023u;
+    int st = (int)(((long long)smem_cap - 1024 - (long long)L.ring_off) / (long long)kTcBox);
+    L.stages = st > kTcMaxStages ? kTcMaxStages : st;
+    L.total = L.ring_off + (uint32_t)(L.stages > 0 ? L.stages : 0) * kTcBox + 1024;  // + base alignment
+    return L;
+}
+
+template <int SWIGLU>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_mma_kernel(const __grid_constant__ CUtensorMap tmW, GroupedGemvArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // swizzle atoms: 1 KB
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const TcLayout L = make_tc_layout(a.K, a.smem_cap);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kTcMaxStages;
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
+    uint8_t* ring = smem + L.ring_off;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < L.stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_trigger();
+    pdl_wait();  // the groups come from the previous kernel
+
+    const int nrb = a.M / kTcRows;
+    const int nkb = (a.K + kTcK - 1) / kTcK;
+    const int items = *a.n_groups * nrb;
+    const int i0 = (int)((int64_t)blockIdx.x * items / gridDim.x);
+    const int i1 = (int)((int64_t)(blockIdx.x + 1) * items / gridDim.x);
+
+    if (warp == kWarps) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            int s = 0;
+            uint32_t ph = 0;
+            for (int it = i0; it < i1; ++it) {
+                const int g = it / nrb, rb = it % nrb;
+                const int row = a.groups[g * 4] * a.M + rb * kTcRows;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, a.err)) return;
+                    mbar_arrive_expect_tx(&full[s], kTcBox);  // columns past K arrive zero-filled
+                    tma_load_2d_hint(ring + (size_t)s * kTcBox, &tmW, kb * kTcK, row, &full[s], pol);
+                    if (++s == L.stages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+        }
+        return;
+    }
+
+    // ldmatrix lane roles. A (x4): matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15) of the warp's
+    // 16 rows; B (x4): token rows 0-7 at k offsets 0, 8, 16, 24 (two k16 steps).
+    const int mi = lane >> 3, ri = lane & 7;
+    const int a_row = warp * 16 + ri + ((mi & 1) << 3);
+    const uint32_t a_row_off = (uint32_t)a_row * 128;
+    const int a_sw = a_row & 7;
+    const int a_chunk = mi >> 1;
+    const uint16_t* b_base = xs + (size_t)ri * L.kp + mi * 8;
+    const int g4 = lane >> 2, t4 = lane & 3;
+
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    int cur_g = -1, c = 0, p0 = 0;
+    for (int it = i0; it < i1; ++it) {
+        const int g = it / nrb, rb = it % nrb;
+        if (g != cur_g) {  // the group's token rows, zero past the c tokens and past K
+            cur_g = g;
+            p0 = a.groups[g * 4 + 1];
+            c = a.groups[g * 4 + 2];
+            consumer_sync();
+            const int kw = L.kp - 8;
+            for (int b = 0; b < kTcTok; ++b) {
+                uint16_t* xrow = xs + (size_t)b * L.kp;
+                const uint16_t* xr = nullptr;
+                if (b < c) xr = a.x + (size_t)(a.x_map ? a.x_map[p0 + b] : p0 + b) * a.ldx;
+                for (int k = threadIdx.x * 8; k < kw; k += kConsumers * 8)
+                    *reinterpret_cast<uint4*>(xrow + k) =
+                        (xr && k < a.K) ? *reinterpret_cast<const uint4*>(xr + k) : make_uint4(0, 0, 0, 0);
+            }
+            consumer_sync();
+        }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int kb = 0; kb < nkb; ++kb) {
+            if (ok && !mbar_wait_bounded(&full[s], ph, a.err)) ok = false;
+            if (ok) {
+                const uint8_t* stage = ring + (size_t)s * kTcBox + a_row_off;
+                const uint16_t* bk = b_base + kb * kTcK;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t bf[4];
+                    ldsm_x4(bf, bk + h2 * 32);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int chunk = (h2 * 2 + j) * 2 + a_chunk;
+                        uint32_t af[4];
+                        ldsm_x4(af, stage + ((chunk ^ a_sw) << 4));
+                        mma_bf16_16816(acc, af, bf + 2 * j);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            if (++s == L.stages) {
+                s = 0;
+                ph ^= 1;
+            }
+        }
+        // acc: rows r0 = 16w + g4 and r0 + 8 of the block, tokens 2*t4 and 2*t4 + 1.
+        const int r0 = rb * kTcRows + warp * 16 + g4;
+        const int tok = 2 * t4;
+        if (!SWIGLU) {
+            if (ok) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int tq = tok + (q & 1), rq = r0 + ((q >> 1) << 3);
+                    if (tq < c) a.y[(size_t)(p0 + tq) * a.ldy + rq] = acc[q];
+                }
+            }
+        } else {
+            // gate rows are even, up rows odd: the up partner of lane l sits in lane l + 4
+            float up[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) up[q] = __shfl_down_sync(0xffffffffu, acc[q], 4);
+            if (ok && (g4 & 1) == 0) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int tq = tok + (q & 1), rq = r0 + ((q >> 1) << 3);
+                    if (tq < c) {
+                        const float gv = acc[q];
+                        const float sg = gv * (1.0f / (1.0f + expf(-gv)));
+                        a.act[(size_t)(p0 + tq) * a.ldact + (rq >> 1)] = f2bf(sg * up[q]);
+                    }
+                }
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ combine
 
 // x[t][i] += (sum_j w[t][j] * y[inv[t*k+j]][i]) + sgate[t] * ys[t][i]
@@ -355,7 +553,8 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(MoeCombineArgs a) {
     const float sg = a.sgate ? a.sgate[t] : 1.f;
     for (int i = threadIdx.x; i < a.h; i += 256) {
         float routed = 0.f;
-        for (int j = 0; j < a.k && j < 16; ++j) routed += wt[j] * a.y[(size_t)slot[j] * a.h + i];
+        for (int j = 0; j < a.k && j < 16; ++j)
+            if (slot[j] >= 0) routed += wt[j] * a.y[(size_t)slot[j] * a.h + i];
         const float shared = a.ys ? sg * a.ys[(size_t)t * a.h + i] : 0.f;
         a.x[(size_t)t * a.h + i] += routed + shared;
     }
@@ -369,6 +568,28 @@ cudaError_t launch_grouped_nb(const GroupedGemvArgs& a, cudaStream_t st, int num
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)L.total);
     if (e != cudaSuccess) return e;
     return launch_ex(kern, dim3(num_sms), dim3(kThreads), L.total, st, pdl, a);
+}
+
+template <int SW>
+cudaError_t launch_grouped_mma(const GroupedGemvArgs& a, cudaStream_t st, int num_sms, bool pdl) {
+    const TcLayout L = make_tc_layout(a.K, a.smem_cap);
+    CUtensorMap tm;
+    cudaError_t e = tmap_bf16_rows(&tm, a.W, a.E * a.M, a.K, kTcRows);
+    if (e != cudaSuccess) return e;
+    auto kern = grouped_mma_kernel<SW>;
+    e = ensure_smem(reinterpret_cast<const void*>(kern), (int)L.total);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L.total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, tm, a);
 }
 
 }  // namespace
@@ -390,9 +611,19 @@ bool grouped_fits(int nb, int K, int smem_cap) {
     return make_layout(nb, K, smem_cap).stages >= 3;
 }
 
+// Groups of 8 tokens go to the tensor pipe when the weights tile into 128-row blocks that
+// stay inside one expert and the TMA unit can read them as one [E*M][K] matrix.
+bool grouped_uses_mma(int nb, int M, int K, size_t wstride, int smem_cap) {
+    return nb == kTcTok && M % kTcRows == 0 && K % 8 == 0 && wstride == (size_t)M * K &&
+           make_tc_layout(K, smem_cap).stages >= 3;
+}
+
 cudaError_t grouped_gemv_launch(const GroupedGemvArgs& a, int nb, bool swiglu, cudaStream_t st, int num_sms,
                                 bool pdl) {
     if (swiglu && a.M % kRows != 0) return cudaErrorInvalidValue;
+    if (grouped_uses_mma(nb, a.M, a.K, a.wstride, a.smem_cap) && a.E > 0 &&
+        (reinterpret_cast<uintptr_t>(a.W) & 15) == 0)
+        return swiglu ? launch_grouped_mma<1>(a, st, num_sms, pdl) : launch_grouped_mma<0>(a, st, num_sms, pdl);
 #define DEC_G(NB_)                                                                                   \
     case NB_:                                                                                        \
         return swiglu ? launch_grouped_nb<NB_, 1>(a, st, num_sms, pdl) : launch_grouped_nb<NB_, 0>(a, st, num_sms, pdl);

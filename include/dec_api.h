@@ -198,6 +198,24 @@ dec_status gqa_decode_attn_noalloc(const void* q, const void* k_new, const void*
 dec_status moe_route_topk(const float* logits, int32_t T, int32_t E, int32_t k, int32_t renorm, int32_t* idx_out,
                           float* w_out, dec_stream_t stream);
 
+/* Routed experts of the MoE FFN for T token rows whose routing is given (ANEDVD
+ * moeExpertAccum; frink decoder.rs expert loop; cortiq MoeFfn):
+ *   out[t] = sum_j w[t][j] * SwiGLU_{idx[t][j]}(x[t]),
+ *   SwiGLU_e(x) = Wd_e . bf16(SiLU(Wg_e . x) * (Wu_e . x)),
+ * summed in top-k order. The tokens are permuted by expert and each expert's weights
+ * stream once per group of at most 8 of its tokens (the same kernels as the MoE layer).
+ *   x     device bf16 [T][h]
+ *   idx   device int32 [T][k]; an entry outside [0, E) contributes nothing
+ *   w     device fp32 [T][k]
+ *   Wgu   device bf16 [E][2I][h]: gate row i of expert e at row 2i, up row i at 2i+1
+ *   Wd    device bf16 [E][h][I]
+ *   out   device fp32 [T][h], overwritten; stream-ordered, the call does not synchronise.
+ * Errors: NULL pointer, T/h/E/k/I <= 0 or k > E -> INVALID_ARG; E > 256, k > 16, h or I
+ * not a multiple of 8, or rows too long for shared memory -> UNSUPPORTED. Scratch
+ * buffers are kept per device and grow on demand; calls must be serialised. */
+dec_status moe_experts(const void* x, const int32_t* idx, const float* w, int32_t T, int32_t h, int32_t E,
+                       int32_t k, int32_t I, const void* Wgu, const void* Wd, float* out, dec_stream_t stream);
+
 /* Weight-streaming projection y[b][n] = sum_k W[n][k] x[b][k] (ANEDVD 1x1 conv
  * kernels; every projection of the layer). W device bf16 [N][K]; x device bf16
  * [B][K]; y device fp32 [B][N]. K % 8 == 0. B <= 8 streams W once through the

@@ -32,6 +32,7 @@ def test_validation_errors_need_no_gpu():
     lib = dec.lib()
     assert lib.moe_route_topk(None, 4, 60, 4, 0, None, None, None) == 1
     assert lib.weight_gemv(None, None, 1, 8, 8, None, None) == 1
+    assert lib.moe_experts(None, None, None, 4, 256, 8, 2, 128, None, None, None, None) == 1
     assert b"NULL" in lib.dec_last_error()
     h = C.c_void_p()
     assert lib.dec_init(None, None, None, C.byref(h)) == 1

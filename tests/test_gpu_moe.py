@@ -148,3 +148,83 @@ def test_qwen_moe_shape_batch64_decode_sampled():
     for b in sample:
         assert_parity(got[b], ref[b][0], what=f"qwen-moe B=64 seq {b}")
         assert np.array_equal(routes[:, b, :], ref[b][1])
+
+
+# (T, E, k, h, I): T = 1 and 3 run the CUDA-core grouped GEMV (groups of 1 and 4 tokens);
+# from T = 5 on, groups of 8 go to the tensor pipe wherever the weight rows tile into
+# 128-row blocks (2I = 256, h = 256 / 2048 / 2816), else the CUDA-core kernel (2I = 192, 272);
+# K tails of 96 and 136 columns; T * k = 2800 crosses the permutation's shared-memory tile.
+EXPERT_CASES = [(1, 8, 2, 256, 96), (3, 8, 2, 256, 128), (8, 16, 4, 256, 128), (40, 8, 2, 256, 136),
+                (64, 60, 4, 2048, 1408), (700, 16, 4, 256, 96), (33, 8, 8, 256, 128)]
+
+
+def _experts_case(T, E, k, h, I, seed):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    w = rng.uniform(0.05, 1.0, (T, k)).astype(np.float32)
+    x = synth.bf16_normal((T, h), seed, 1, 0.0, 1.0)
+    Wg = synth.bf16_normal((E, I, h), seed, 2, 0.0, h ** -0.5)  # unit-scale gate and up
+    Wu = synth.bf16_normal((E, I, h), seed, 3, 0.0, h ** -0.5)
+    Wd = synth.bf16_normal((E, h, I), seed, 4, 0.0, I ** -0.5)
+    return idx, w, x, Wg, Wu, Wd
+
+
+def _experts_ref(rows, idx, w, x, Wg, Wu, Wd):
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = np.zeros((len(rows), x.shape[1]))
+    for i, t in enumerate(rows):
+        for j, e in enumerate(idx[t]):
+            if 0 <= e < Wg.shape[0]:
+                ref[i] += float(w[t, j]) * oracle.swiglu(xf[t], Wg[e], Wu[e], Wd[e])
+    return ref
+
+
+def _experts_run(idx, w, x, Wg, Wu, Wd):
+    import torch
+    from _util import to_dev_bf16
+    E, I, h = Wg.shape
+    Wgu = np.stack([Wg, Wu], axis=2).reshape(E, 2 * I, h)  # gate row i at 2i, up row i at 2i + 1
+    out = torch.full((x.shape[0], h), float("nan"), device="cuda")
+    dec.moe_experts(to_dev_bf16(x, torch), torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda(),
+                    to_dev_bf16(Wgu, torch), to_dev_bf16(Wd, torch), out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,E,k,h,I", EXPERT_CASES)
+def test_moe_experts_standalone_matches_oracle(T, E, k, h, I):
+    idx, w, x, Wg, Wu, Wd = _experts_case(T, E, k, h, I, 5000 + T)
+    got = _experts_run(idx, w, x, Wg, Wu, Wd)
+    rows = list(range(T)) if T <= 64 and h * I <= 2048 * 128 else sorted({0, 1, T // 3, T // 2, T - 2, T - 1})
+    if T > 64:
+        rows = sorted(set(rows) | set(range(0, T, 37)))
+    ref = _experts_ref(rows, idx, w, x, Wg, Wu, Wd)
+    d, r = assert_parity(got[rows], ref, what=f"moe_experts T={T} E={E} k={k} h={h} I={I}")
+    # fp32 accumulation; the bf16 rounding of SiLU(g)*u may land one ulp apart on a few elements
+    assert r <= 2e-3, f"kernel-level bar: rel={r:.2e}"
+
+
+def test_moe_experts_drops_out_of_range_entries():
+    T, E, k, h, I = 24, 8, 2, 256, 128
+    idx, w, x, Wg, Wu, Wd = _experts_case(T, E, k, h, I, 5100)
+    idx[3, 1] = -1
+    idx[10, 0] = E
+    idx[17, :] = E + 5
+    got = _experts_run(idx, w, x, Wg, Wu, Wd)
+    ref = _experts_ref(range(T), idx, w, x, Wg, Wu, Wd)
+    assert_parity(got, ref, what="moe_experts with dropped entries")
+    assert np.all(got[17] == 0.0)
+
+
+def test_tiny_moe_tensor_core_expert_blocks():
+    # 2I = 256 and h = 256 tile into 128-row blocks: prefill chunks of 32 tokens (groups of 8)
+    # run both expert projections on the tensor pipe inside the model
+    cfg = tiny_moe(expert_inter=128, prefill_chunk=32)
+    w = synth.make_weights(cfg)
+    toks, greedy, lg, routes, m = run_gated(cfg, w, 70, 2, seed0=1700)
+    d = dec.Decoder(cfg, w)
+    assert_parity(d.prefill_logits(0, toks, 0), lg[0], what="moe tensor-core prefill")
+    assert d.last_argmax(1)[0] == oracle.argmax(lg[0])
+    for s, t in enumerate(greedy):
+        assert_parity(d.step_logits([t], [70 + s])[0], lg[s + 1], what=f"moe tensor-core step {s}")
+    d.close()
