@@ -356,6 +356,8 @@ def run_workload(args, torch, dec):
     base = getattr(configs, spec["model"])
     B, ctx = spec["B"], spec["ctx"]
     cfg = dict(base, max_batch=B, max_context=ctx + W + K + 8, prefill_chunk=128)
+    if args.layers:  # profiling only: fewer layers of the same shape
+        cfg = configs.with_layers(cfg, args.layers)
     w = make_device_weights(cfg, torch)
     d = dec.Decoder(cfg, w)
     del w
@@ -420,7 +422,7 @@ def run_workload(args, torch, dec):
                 steps=K, warmup=W, ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None,
                 dtype="bf16", data="synthetic",
                 config=dict(workload=f"{spec['model'].lower()} shape, batch {B}, context {ctx}", global_batch=B,
-                            seq_len=ctx, l2="inputs larger than L2"),
+                            seq_len=ctx, layers=cfg["layers"], l2="inputs larger than L2"),
                 step_roofline=dict(bytes_per_step=step_bytes, achieved_gbs=round(gbs, 1),
                                    frac=round(gbs / P["hbm"], 4), peak=P["hbm"], unit="GB/s", peak_source=P["src"]),
                 clocks=clocks, **extra)

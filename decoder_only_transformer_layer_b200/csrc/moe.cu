@@ -117,68 +117,98 @@ __global__ void __launch_bounds__(32) moe_route_kernel(MoeRouteArgs a) {
 
 // ------------------------------------------------------------------ permutation by expert
 
-// One CTA, thread e owns expert e: counts per expert, offsets, per-expert token lists in
-// (token, slot) order, the inverse map, and the groups of at most nb tokens (expert order)
-// for the grouped GEMV. The routing table passes through shared memory in tiles, so each
-// thread's scan is a run of broadcast reads.
-constexpr int kPermTile = 2048;
+// One CTA: counts per expert, offsets, per-expert token lists in (token, slot) order, the
+// inverse map, and the groups of at most nb tokens (expert order) for the grouped
+// projections. Warp w owns a contiguous range of routing slots: it counts them into its
+// own histogram, the histograms are scanned over warps (per expert) and over experts
+// (warp shuffles), and each warp then places its slots 32 at a time, ranking lanes that
+// share an expert by lane order, so every expert's list keeps slot order.
+constexpr int kPermWarps = 8;
 
-__global__ void __launch_bounds__(256) moe_permute_kernel(MoePermArgs a) {
-    __shared__ int off[256], goff[256];
-    __shared__ int sidx[kPermTile];
+__global__ void __launch_bounds__(kPermWarps * 32) moe_permute_kernel(MoePermArgs a) {
+    __shared__ int hist[kPermWarps][256];  // counts, then each warp's next position per expert
+    __shared__ int cnt[256], off[256], goff[256];
     pdl_trigger();
     pdl_wait();
-    const int tid = threadIdx.x;
-    const int total = a.n * a.k;
-    const bool mine = tid < a.E;
-    int cnt = 0;
-    for (int base = 0; base < total; base += kPermTile) {
-        const int m = min(kPermTile, total - base);
-        __syncthreads();
-        for (int i = tid; i < m; i += 256) sidx[i] = a.idx[base + i];
-        __syncthreads();
-        if (mine)
-            for (int i = 0; i < m; ++i) cnt += sidx[i] == tid;
-    }
-    if (mine) off[tid] = cnt;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int total = a.n * a.k, E = a.E;
+    int* hflat = &hist[0][0];
+    for (int i = tid; i < kPermWarps * 256; i += kPermWarps * 32) hflat[i] = 0;
     __syncthreads();
-    if (tid == 0) {
-        int o = 0, g = 0;
-        for (int e = 0; e < a.E; ++e) {
-            const int c = off[e];
-            off[e] = o;
-            goff[e] = g;
-            o += c;
-            g += (c + a.nb - 1) / a.nb;
-        }
-        *a.n_groups = g;
+    const int r0 = (int)((int64_t)total * warp / kPermWarps);
+    const int r1 = (int)((int64_t)total * (warp + 1) / kPermWarps);
+    for (int i = r0 + lane; i < r1; i += 32) {
+        const int e = a.idx[i];
+        if (e >= 0 && e < E)
+            atomicAdd(&hist[warp][e], 1);
+        else
+            a.inv[i] = -1;  // dropped: the combine skips it
     }
     __syncthreads();
-    int p = mine ? off[tid] : 0;
-    for (int base = 0; base < total; base += kPermTile) {
-        const int m = min(kPermTile, total - base);
-        __syncthreads();
-        for (int i = tid; i < m; i += 256) {
-            const int e = a.idx[base + i];
-            sidx[i] = e;
-            if (e < 0 || e >= a.E) a.inv[base + i] = -1;  // dropped: the combine skips it
-        }
-        __syncthreads();
-        if (mine)
-            for (int i = 0; i < m; ++i)
-                if (sidx[i] == tid) {
-                    a.perm_tok[p] = (base + i) / a.k;
-                    a.inv[base + i] = p;
-                    ++p;
-                }
+    {  // thread e: count of expert e and the exclusive prefix of its histogram over warps
+        int c = 0;
+        if (tid < E)
+            for (int w = 0; w < kPermWarps; ++w) {
+                const int h = hist[w][tid];
+                hist[w][tid] = c;
+                c += h;
+            }
+        cnt[tid] = tid < E ? c : 0;
     }
-    if (mine) {
-        const int e = tid, o = off[e];
+    __syncthreads();
+    if (warp == 0) {  // exclusive scans over the 256 experts, 8 per lane: slot and group offsets
+        int lc[8], lg[8], s = 0, gs = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            lc[j] = cnt[lane * 8 + j];
+            lg[j] = (lc[j] + a.nb - 1) / a.nb;
+            s += lc[j];
+            gs += lg[j];
+        }
+        int si = s, gi = gs;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int t1 = __shfl_up_sync(0xffffffffu, si, d);
+            const int t2 = __shfl_up_sync(0xffffffffu, gi, d);
+            if (lane >= d) {
+                si += t1;
+                gi += t2;
+            }
+        }
+        int o = si - s, g = gi - gs;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            off[lane * 8 + j] = o;
+            goff[lane * 8 + j] = g;
+            o += lc[j];
+            g += lg[j];
+        }
+        if (lane == 31) *a.n_groups = gi;
+    }
+    __syncthreads();
+    for (int i = tid; i < kPermWarps * 256; i += kPermWarps * 32) hflat[i] += off[i & 255];
+    __syncthreads();
+    for (int b0 = r0; b0 < r1; b0 += 32) {
+        const int i = b0 + lane;
+        const int e = i < r1 ? a.idx[i] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned m = __match_any_sync(0xffffffffu, valid ? e : 1024 + lane);
+        if (valid) {
+            const int p = hist[warp][e] + __popc(m & ((1u << lane) - 1u));
+            a.perm_tok[p] = i / a.k;
+            a.inv[i] = p;
+        }
+        __syncwarp();
+        if (valid && lane == 31 - __clz(m)) hist[warp][e] += __popc(m);
+        __syncwarp();
+    }
+    if (tid < E) {
+        const int e = tid, o = off[e], c = cnt[e];
         int g = goff[e];
-        for (int s = 0; s < cnt; s += a.nb, ++g) {
+        for (int s = 0; s < c; s += a.nb, ++g) {
             a.groups[g * 4 + 0] = e;
             a.groups[g * 4 + 1] = o + s;
-            a.groups[g * 4 + 2] = min(a.nb, cnt - s);
+            a.groups[g * 4 + 2] = min(a.nb, c - s);
             a.groups[g * 4 + 3] = 0;
         }
     }
