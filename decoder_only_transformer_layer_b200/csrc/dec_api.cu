@@ -559,6 +559,13 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
         dec_free(c);
         return st_;
     };
+    if (k.n_experts > 0) {  // the largest token group (8) must fit the grouped projections' shared memory
+        const int nbmax = grouped_nb_for(c->max_tok);
+        if (!grouped_fits(nbmax, h, c->smem_cap) || !grouped_fits(nbmax, k.expert_inter, c->smem_cap)) {
+            fail(DEC_ERR_UNSUPPORTED, "hidden / expert_inter too long for the grouped expert projections");
+            return cleanup(DEC_ERR_UNSUPPORTED);
+        }
+    }
 #define INIT_TRY(expr)                                                                         \
     do {                                                                                       \
         cudaError_t e_ = (expr);                                                               \

@@ -110,7 +110,12 @@ typedef struct dec_ctx dec_ctx;
  * weights into library-owned device memory (fused gate/up), allocate the paged
  * KV pool, the block table and the workspace. Like ANEDVD Engine.init, but the
  * caller's weight buffers may be freed as soon as this returns (the copies are
- * complete: the call synchronises `stream`). */
+ * complete: the call synchronises `stream`).
+ * Errors: NULL cfg / w / out, or a non-positive size -> INVALID_ARG; a shape the kernels
+ * do not handle (more than 16 query heads per kv head, head_dim other than 64 / 128,
+ * hidden or an FFN width not a multiple of
+ * 8, page_size other than 16, more than 256 experts or top_k above 16, MoE rows too long
+ * for the grouped projections' shared memory) -> UNSUPPORTED; device memory -> OOM. */
 dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t stream, dec_ctx** out);
 
 /* Release everything dec_init allocated (ANEDVD Engine.deinit). NULL is a no-op. */
