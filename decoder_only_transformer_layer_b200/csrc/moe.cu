@@ -7,15 +7,18 @@
 //
 // B200 design: the tokens of a step or prefill chunk are permuted by expert (counts,
 // offsets, a deterministic token list per expert), split into groups of at most NB tokens,
-// and each expert's weights stream once per group. Groups of up to 4 tokens run a grouped
+// and each expert's weights stream once per group. Where an expert's weight rows tile into
+// 128-row blocks, every group runs on the tensor pipe (work item = group x 128-row block,
+// TMA boxes, mma.sync with the group's tokens as the n dimension of 8); otherwise a grouped
 // weight-streaming GEMV on the CUDA cores (work item = group x 4-row weight block, the same
-// bulk-copy ring as the dense GEMV); groups of 8 run on the tensor pipe (work item = group
-// x 128-row block, TMA boxes, mma.sync with the 8 tokens as the n dimension). Either way
+// bulk-copy ring as the dense GEMV). Either way
 // the group's token rows sit in shared memory and the epilogue writes SiLU(gate)*up (bf16)
 // or the projection (fp32) per (token, expert) slot.
 // A combine kernel adds the weighted slots and the gated shared expert to the residual in
 // a fixed order (routed experts in top-k order, then the shared expert).
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -399,8 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(GroupedGemvAr
 // ------------------------------------------------------------------ grouped GEMM on the tensor pipe
 
 // Groups of up to 8 tokens: the CUDA-core GEMV above converts every token element once per
-// weight row and becomes ALU-bound, so here each group's token rows are the n = 8 operand
-// of mma.sync m16n8k16 (bf16 in, fp32 accumulate). A work item is (group, 128-row weight
+// weight row and becomes ALU-bound with 8 tokens (and streams small 4-row items with 1), so
+// here each group's token rows are the n = 8 operand of mma.sync m16n8k16 (bf16 in, fp32
+// accumulate; token rows past the group's count are zero). A work item is (group, 128-row weight
 // block); the TMA unit streams the block in 128B-swizzled boxes of 64 columns x 128 rows,
 // and consumer warp w owns rows 16w .. 16w+15 of the block over the whole K, so no partial
 // sums cross warps. Token rows sit in shared memory with a 16-byte pad per row, which
@@ -581,7 +585,7 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(MoeCombineArgs a) {
         wt[j] = a.w[(size_t)t * a.k + j];
     }
     const float sg = a.sgate ? a.sgate[t] : 1.f;
-    for (int i = threadIdx.x; i < a.h; i += 256) {
+    for (int i = blockIdx.y * 256 + threadIdx.x; i < a.h; i += 256 * gridDim.y) {
         float routed = 0.f;
         for (int j = 0; j < a.k && j < 16; ++j)
             if (slot[j] >= 0) routed += wt[j] * a.y[(size_t)slot[j] * a.h + i];
@@ -641,10 +645,11 @@ bool grouped_fits(int nb, int K, int smem_cap) {
     return make_layout(nb, K, smem_cap).stages >= 3;
 }
 
-// Groups of 8 tokens go to the tensor pipe when the weights tile into 128-row blocks that
-// stay inside one expert and the TMA unit can read them as one [E*M][K] matrix.
+// Groups (of any size up to 8 tokens) go to the tensor pipe when the weights tile into
+// 128-row blocks that stay inside one expert and the TMA unit can read them as one
+// [E*M][K] matrix.
 bool grouped_uses_mma(int nb, int M, int K, size_t wstride, int smem_cap) {
-    return nb == kTcTok && M % kTcRows == 0 && K % 8 == 0 && wstride == (size_t)M * K &&
+    return nb >= 1 && nb <= kTcTok && M % kTcRows == 0 && K % 8 == 0 && wstride == (size_t)M * K &&
            make_tc_layout(K, smem_cap).stages >= 3;
 }
 
@@ -669,7 +674,10 @@ cudaError_t grouped_gemv_launch(const GroupedGemvArgs& a, int nb, bool swiglu, c
 
 cudaError_t moe_combine_launch(const MoeCombineArgs& a, int n, cudaStream_t st, bool pdl) {
     if (a.k > 16) return cudaErrorInvalidValue;
-    return launch_ex(moe_combine_kernel, dim3(n), dim3(256), 0, st, pdl, a);
+    // few tokens: split each row over CTAs, so the combine is not one CTA's serial walk of h
+    const int cols = (a.h + 255) / 256;
+    const int gy = std::min(cols, std::max(1, 1024 / std::max(n, 1)));
+    return launch_ex(moe_combine_kernel, dim3(n, gy), dim3(256), 0, st, pdl, a);
 }
 
 }  // namespace dec

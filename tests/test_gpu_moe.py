@@ -150,11 +150,12 @@ def test_qwen_moe_shape_batch64_decode_sampled():
         assert np.array_equal(routes[:, b, :], ref[b][1])
 
 
-# (T, E, k, h, I): T = 1, 2 and 3 run the CUDA-core grouped GEMV (groups of 1, 2 and 4 tokens);
-# from T = 5 on, groups of 8 go to the tensor pipe wherever the weight rows tile into
-# 128-row blocks (2I = 256, h = 256 / 2048 / 2816), else the CUDA-core kernel (2I = 192, 272);
-# K tails of 96 and 136 columns; T * k = 2800 crosses the permutation's shared-memory tile.
+# (T, E, k, h, I): groups of 1, 2, 4 (T = 1, 2, 3) and 8 tokens (T >= 5) run on the tensor
+# pipe wherever the projection's rows tile into 128-row blocks (2I = 256; h = 256 / 2048),
+# else on the CUDA-core grouped GEMV (2I = 192, 272; h = 200): both kernels at every group
+# size; K tails of 96, 136 and 200 columns; T * k = 2800 crosses the permutation's tile.
 EXPERT_CASES = [(1, 8, 2, 256, 96), (2, 8, 2, 256, 96), (3, 8, 2, 256, 128), (5, 4, 2, 256, 128),
+                (2, 8, 2, 200, 96), (3, 8, 2, 200, 128), (9, 8, 2, 200, 128),
                 (8, 16, 4, 256, 128), (40, 8, 2, 256, 136),
                 (64, 60, 4, 2048, 1408), (700, 16, 4, 256, 96), (33, 8, 8, 256, 128)]
 
