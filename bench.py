@@ -427,8 +427,40 @@ def run_workload(args, torch, dec):
                                    frac=round(gbs / P["hbm"], 4), peak=P["hbm"], unit="GB/s", peak_source=P["src"]),
                 clocks=clocks, **extra)
     print(json.dumps(line))
+    if args.breakdown:  # 4 more steps; the context has room for 8 past the timed ones
+        def one_step():
+            d.step(toks, pos)
+            pos[:] += 1
+        kernel_breakdown(torch, one_step, 4, f"{name} (B={B}, ctx {ctx}, {cfg['layers']} layers)")
     d.close()
     return 0
+
+
+def kernel_breakdown(torch, step, n, title):
+    """Per-kernel share of `n` more steps, from the torch profiler's device activity. Kernels
+    overlap under programmatic dependent launch, so each one is charged the time from the
+    end of everything before it to its own end (its exclusive share of the critical path)."""
+    import collections
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        for _ in range(n):
+            step()
+        torch.cuda.synchronize()
+    ev = sorted((e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA),
+                key=lambda e: e.time_range.start)
+    agg = collections.defaultdict(lambda: [0, 0.0])
+    last = None
+    for e in ev:
+        name = e.name.replace("(anonymous namespace)::", "").replace("void ", "").split("(")[0][-60:]
+        agg[name][0] += 1
+        agg[name][1] += max(0.0, e.time_range.end - (e.time_range.start if last is None else max(last, e.time_range.start)))
+        last = e.time_range.end if last is None else max(last, e.time_range.end)
+    total = sum(v[1] for v in agg.values())
+    print(f"kernel breakdown, {title}: {total / n:.0f} us per step (exclusive shares)", file=sys.stderr)
+    for name, (c, t) in sorted(agg.items(), key=lambda x: -x[1][1]):
+        print(f"  {name:60s} {c // n:4d}/step {t / c:9.2f} us/launch {t / n:9.1f} us/step {100 * t / total:5.1f}%",
+              file=sys.stderr)
 
 
 def run_gqa_sweep(args, torch, dec, P):
@@ -485,6 +517,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling only; not a bench number)")
+    ap.add_argument("--breakdown", action="store_true",
+                    help="decode workloads: after the timed region, per-kernel exclusive times of a few more "
+                         "steps (torch profiler) on stderr; the JSON line is unchanged")
     ap.add_argument("--workload", default="llama3-8b", choices=["llama3-8b"] + sorted(WORKLOADS),
                     help="llama3-8b: the headline line (prefill 4096 + batch-1 decode); others: one extra line each")
     args = ap.parse_args()
