@@ -268,6 +268,9 @@ WORKLOADS = {
     "tiny": dict(model="TINY", B=1, ctx=16, prefill=16),
     # standalone decode attention
     "gqa-sweep": dict(),
+    # standalone weight-streaming GEMV on the gate/up matrix of the Llama-3-8B shape (the
+    # default line's roofline kernel, launched the way its `achieved` figure is timed)
+    "gemv-gate-up": dict(),
     # 4096-token prefill of the Llama-3-8B shape with longer chunks: the projections become
     # compute-bound GEMMs (the chunk-128 line is HBM-bound)
     "llama3-8b-prefill-c512": dict(prefill_chunk=512),
@@ -350,6 +353,17 @@ def run_workload(args, torch, dec):
     W, K = max(3, args.warmup), max(1, args.steps)
     if name == "gqa-sweep":
         return run_gqa_sweep(args, torch, dec, P)
+    if name == "gemv-gate-up":
+        N, Kd = 2 * configs.LLAMA3_8B["ffn_inter"], configs.LLAMA3_8B["hidden"]
+        ms, byt = time_gemv(dec, torch, N, Kd, reps=K)
+        gbs = byt / (ms * 1e-3) / 1e9
+        print(json.dumps(dict(metric=f"weight-streaming GEMV GB/s ([{N}][{Kd}] bf16, batch 1)", value=round(gbs, 1),
+                              unit="GB/s", n_gpus=1, steps=K, warmup=3, ms_per_step=ms, higher_is_better=True,
+                              scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+                              config=dict(workload=f"gemv [{N}][{Kd}] x [1][{Kd}]", l2="rotating weights > L2"),
+                              roofline=dict(bound="hbm", achieved=round(gbs, 1), peak=P["hbm"], unit="GB/s",
+                                            frac=round(gbs / P["hbm"], 4), peak_source=P["src"]))))
+        return 0
     if "prefill_chunk" in WORKLOADS[name]:
         return run_prefill_workload(args, torch, dec, P)
     spec = WORKLOADS[name]
