@@ -3,7 +3,6 @@
 The roofline `traffic` figure comes from a committed ncu summary and is only valid for the
 kernel source it was captured on; the peaks come from the measured file or the stated
 fallback. Both rules are exercised on a scratch copy of the files they read."""
-import json
 import os
 import shutil
 
