@@ -79,6 +79,7 @@ def _declare(L):
     L.orc_bf16.argtypes = [C.c_double]
     L.orc_matvec.argtypes = [_P, C.c_int64, C.c_int64, _P, _P]
     L.orc_rmsnorm.argtypes = [_P, _P, C.c_int, C.c_double, _P]
+    L.orc_head_rmsnorm.argtypes = [_P, C.c_int, C.c_int, _P, C.c_double]
     L.orc_rope.argtypes = [_P, C.c_int, C.c_int, C.c_int64, C.c_double]
     L.orc_attend.argtypes = [_P, _P, _P, C.c_int64, C.c_int, C.c_int64, C.c_double, _P]
     L.orc_route_topk.argtypes = [_P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
@@ -130,6 +131,15 @@ def rmsnorm(x, g, eps) -> np.ndarray:
     out = np.empty_like(x)
     lib().orc_rmsnorm(_p(x), _p(g), x.size, float(eps), _p(out))
     return out
+
+
+def head_rmsnorm(v: np.ndarray, g, eps) -> np.ndarray:
+    """QK-norm of v [heads][d]: each head normalised by its own mean square, times g [d]."""
+    v = np.array(v, dtype=np.float64, order="C")
+    heads, d = v.shape
+    g = _c(g, np.float32)
+    lib().orc_head_rmsnorm(_p(v), heads, d, _p(g), float(eps))
+    return v
 
 
 def rope(v: np.ndarray, pos: int, base: float) -> np.ndarray:

@@ -25,7 +25,7 @@
  * elements; each element is summed by one thread in index order, so results
  * do not depend on the thread count.
  *
- * Readings taken where the pages are silent (each listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - RoPE pairing is half-split: element i pairs with i + d/2, angle
  *     pos * base^(-2i/d) ("rope" vs "ropeAdjacent" in ANEDVD; inv_freq from
  *     (head_dim, base) in cortiq).
@@ -88,6 +88,12 @@ void orc_rmsnorm(const double* x, const float* g, int n, double eps, double* out
     for (int i = 0; i < n; ++i) acc += x[i] * x[i];
     double inv = 1.0 / sqrt(acc / (double)n + eps);
     for (int i = 0; i < n; ++i) out[i] = x[i] * inv * (double)g[i];
+}
+
+/* QK-norm (ANEDVD applyHeadNorm): each d-wide head of v [heads][d] is normalised by
+ * its own mean square and scaled by the [d] gain g, in place. */
+void orc_head_rmsnorm(double* v, int heads, int d, const float* g, double eps) {
+    for (int hh = 0; hh < heads; ++hh) orc_rmsnorm(v + (int64_t)hh * d, g, d, eps, v + (int64_t)hh * d);
 }
 
 /* Rotate every head of v ([heads][d]) to position pos, half-split pairing. */
@@ -307,10 +313,10 @@ static void layer_forward(orc_model* m, int li, int seq, int64_t pos, double* x)
     double* q = qkv;
     double* k = qkv + qd;
     double* v = qkv + qd + kvd;
-    /* 3. optional per-head QK-norm (applyHeadNorm) */
+    /* 3. optional per-head QK-norm (applyHeadNorm): q heads with q_norm, k heads with k_norm */
     if (c->qk_norm) {
-        for (int hh = 0; hh < nq; ++hh) orc_rmsnorm(q + (int64_t)hh * d, L->q_norm, d, c->eps, q + (int64_t)hh * d);
-        for (int hh = 0; hh < nkv; ++hh) orc_rmsnorm(k + (int64_t)hh * d, L->k_norm, d, c->eps, k + (int64_t)hh * d);
+        orc_head_rmsnorm(q, nq, d, L->q_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->k_norm, c->eps);
     }
     /* 4. RoPE on q and k at pos */
     orc_rope(q, nq, d, pos, c->rope_base);

@@ -53,6 +53,7 @@ typedef struct orc_model orc_model;
 double orc_bf16(double v);
 void orc_matvec(const uint16_t* W, int64_t N, int64_t K, const double* x, double* y);
 void orc_rmsnorm(const double* x, const float* g, int n, double eps, double* out);
+void orc_head_rmsnorm(double* v, int heads, int d, const float* g, double eps);
 void orc_rope(double* v, int heads, int d, int64_t pos, double base);
 void orc_attend(const double* q, const uint16_t* K, const uint16_t* V, int64_t stride, int d, int64_t n,
                 double scale, double* out);

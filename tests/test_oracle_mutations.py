@@ -37,6 +37,44 @@ MUTATIONS = {
     "qkv_bias_dropped": ("qkv[r] += (double)L->bqkv[r];", "qkv[r] += 0.0;"),
     "cache_row_off_by_one": ("uint16_t* krow = kslot(m, m->kc, seq, li, pos);",
                              "uint16_t* krow = kslot(m, m->kc, seq, li, pos + 1 < m->c.max_ctx ? pos + 1 : pos);"),
+    "qk_norm_after_rope": ("""    if (c->qk_norm) {
+        orc_head_rmsnorm(q, nq, d, L->q_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->k_norm, c->eps);
+    }
+    /* 4. RoPE on q and k at pos */
+    orc_rope(q, nq, d, pos, c->rope_base);
+    orc_rope(k, nkv, d, pos, c->rope_base);""", """    orc_rope(q, nq, d, pos, c->rope_base);
+    orc_rope(k, nkv, d, pos, c->rope_base);
+    if (c->qk_norm) {
+        orc_head_rmsnorm(q, nq, d, L->q_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->k_norm, c->eps);
+    }"""),
+    "qk_norm_gains_swapped": ("""        orc_head_rmsnorm(q, nq, d, L->q_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->k_norm, c->eps);""", """        orc_head_rmsnorm(q, nq, d, L->k_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->q_norm, c->eps);"""),
+    "qk_norm_whole_vector": ("""    for (int hh = 0; hh < heads; ++hh) orc_rmsnorm(v + (int64_t)hh * d, g, d, eps, v + (int64_t)hh * d);""",
+                             """    double acc = 0.0;
+    for (int64_t i = 0; i < (int64_t)heads * d; ++i) acc += v[i] * v[i];
+    double inv = 1.0 / sqrt(acc / ((double)heads * d) + eps);
+    for (int64_t i = 0; i < (int64_t)heads * d; ++i) v[i] = v[i] * inv * (double)g[i % d];"""),
+    "qk_norm_bias_after_norm": ("""    if (c->qkv_bias && L->bqkv)
+        for (int64_t r = 0; r < rows; ++r) qkv[r] += (double)L->bqkv[r];
+    double* q = qkv;
+    double* k = qkv + qd;
+    double* v = qkv + qd + kvd;
+    /* 3. optional per-head QK-norm (applyHeadNorm): q heads with q_norm, k heads with k_norm */
+    if (c->qk_norm) {
+        orc_head_rmsnorm(q, nq, d, L->q_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->k_norm, c->eps);
+    }""", """    double* q = qkv;
+    double* k = qkv + qd;
+    double* v = qkv + qd + kvd;
+    if (c->qk_norm) {
+        orc_head_rmsnorm(q, nq, d, L->q_norm, c->eps);
+        orc_head_rmsnorm(k, nkv, d, L->k_norm, c->eps);
+    }
+    if (c->qkv_bias && L->bqkv)
+        for (int64_t r = 0; r < rows; ++r) qkv[r] += (double)L->bqkv[r];"""),
     "tied_head_ignored": ("const uint16_t* head = c->tied ? m->w.embed : m->w.lm_head;",
                           "const uint16_t* head = m->w.embed;"),
 }

@@ -135,6 +135,99 @@ def test_rope_dot_product_depends_only_on_relative_position():
         assert math.isclose(got, ref, rel_tol=1e-9, abs_tol=1e-10)
 
 
+# ------------------------------------------------------------------ QK-norm (ANEDVD applyHeadNorm)
+
+def test_head_rmsnorm_normalises_each_head_by_its_own_mean_square():
+    # Heads of very different scale: with unit gains every head comes out with RMS
+    # sqrt(ms / (ms + eps)) of its OWN mean square ms; one statistic over the whole
+    # vector would leave the heads' scale ratio in place.
+    rng = np.random.default_rng(40)
+    d = 16
+    v = rng.standard_normal((3, d)) * np.array([[0.05], [1.0], [40.0]])
+    out = oracle.head_rmsnorm(v, np.ones(d, np.float32), 1e-5)
+    for h in range(3):
+        ms = np.mean(v[h] ** 2)
+        assert math.isclose(np.sqrt(np.mean(out[h] ** 2)), math.sqrt(ms / (ms + 1e-5)), rel_tol=1e-13)
+        assert np.allclose(out[h], v[h] / math.sqrt(ms + 1e-5), rtol=1e-14)
+
+
+def test_head_rmsnorm_gain_is_per_element_of_the_head():
+    rng = np.random.default_rng(41)
+    d = 8
+    v = rng.standard_normal((2, d))
+    g = np.arange(1, d + 1, dtype=np.float32)
+    plain = oracle.head_rmsnorm(v, np.ones(d, np.float32), 1e-5)
+    assert np.allclose(oracle.head_rmsnorm(v, g, 1e-5), plain * g[None, :].astype(np.float64), rtol=1e-14)
+
+
+def _qk_cfg(**over):
+    return dict(configs.COMMON, name="qk", hidden=32, layers=1, n_q_heads=2, n_kv_heads=2, head_dim=8,
+                ffn_inter=16, vocab=12, max_context=8, qk_norm=1, **over)
+
+
+def test_qk_norm_keys_in_the_cache_have_unit_rms_per_head():
+    # Unit gains, no bias, position 0 (RoPE is the identity there): every cached key head is
+    # the bf16 rounding of a unit-RMS vector, even with the second head's projection rows
+    # scaled by 64 (a whole-vector norm would leave them 64x apart).
+    cfg = _qk_cfg()
+    w = synth.make_weights(cfg, seed=42)
+    lw = w["layers"][0]
+    d, nq, nkv = 8, 2, 2
+    wq = f(lw["wqkv"])
+    wq[nq * d + d: nq * d + 2 * d] *= 64.0     # k rows of kv head 1 (exact: a power of two)
+    lw["wqkv"] = bits(wq)
+    lw["q_norm"] = np.ones(d, np.float32)
+    lw["k_norm"] = np.ones(d, np.float32)
+    m = oracle.Model(cfg, w)
+    m.forward(0, 5, 0, want_logits=False)
+    k, _ = m.kv_read(0, 0, 0, 1)
+    kh = f(k[0]).reshape(nkv, d)
+    rms = np.sqrt(np.mean(kh ** 2, axis=1))
+    assert np.all(np.abs(rms - 1.0) < 2 ** -7), rms
+
+
+def test_qk_norm_applies_to_the_biased_projection():
+    # With the key projection rows zero, k = bias; the norm must see the bias (added before
+    # the norm), so each cached key head is bf16(b_h / sqrt(mean(b_h^2) + eps) * g_k) at p = 0.
+    cfg = _qk_cfg(qkv_bias=1)
+    w = synth.make_weights(cfg, seed=43)
+    lw = w["layers"][0]
+    d, nq, nkv = 8, 2, 2
+    wq = f(lw["wqkv"])
+    wq[nq * d: nq * d + nkv * d] = 0.0
+    lw["wqkv"] = bits(wq)
+    m = oracle.Model(cfg, w)
+    m.forward(0, 3, 0, want_logits=False)
+    k, _ = m.kv_read(0, 0, 0, 1)
+    b = lw["bqkv"][nq * d: nq * d + nkv * d].astype(np.float64).reshape(nkv, d)
+    g = lw["k_norm"].astype(np.float64)
+    want = b / np.sqrt(np.mean(b * b, axis=1, keepdims=True) + cfg["rms_eps"]) * g[None, :]
+    assert np.array_equal(f(k[0]), torch_bf16(want.reshape(-1)))
+
+
+def test_qk_norm_comes_before_rope():
+    # At p > 0 the cached key is bf16(rope(norm(k))): with a non-uniform gain, normalising
+    # after the rotation applies the gain in the rotated frame and gives other values.
+    cfg = _qk_cfg()
+    w = synth.make_weights(cfg, seed=44)
+    lw = w["layers"][0]
+    d, nq, nkv = 8, 2, 2
+    m = oracle.Model(cfg, w)
+    toks = [4, 9, 2]
+    m.prefill(0, toks, 0)
+    k, _ = m.kv_read(0, 0, 0, 3)
+    for p, t in enumerate(toks):
+        x = f(w["embed"][t])
+        xn = torch_bf16(x / np.sqrt(np.mean(x * x) + cfg["rms_eps"]) * lw["attn_norm"].astype(np.float64))
+        kraw = (f(lw["wqkv"])[nq * d: nq * d + nkv * d] @ xn).reshape(nkv, d)
+        kn = kraw / np.sqrt(np.mean(kraw ** 2, axis=1, keepdims=True) + cfg["rms_eps"]) \
+            * lw["k_norm"].astype(np.float64)[None, :]
+        ang = p * cfg["rope_base"] ** (-np.arange(0, d, 2) / d)
+        a, bb = kn[:, : d // 2], kn[:, d // 2:]
+        rot = np.concatenate([a * np.cos(ang) - bb * np.sin(ang), a * np.sin(ang) + bb * np.cos(ang)], 1)
+        assert np.allclose(f(k[p]), torch_bf16(rot.reshape(-1)), rtol=0, atol=1e-12), p
+
+
 # ------------------------------------------------------------------ attention
 
 def test_attention_single_key_returns_that_value():
@@ -470,6 +563,10 @@ def _textbook_forward(cfg, w, toks):
         q = qkv[:, : nq * d].reshape(T, nq, d)
         k = qkv[:, nq * d: nq * d + nkv * d].reshape(T, nkv, d)
         v = qkv[:, nq * d + nkv * d:].reshape(T, nkv, d)
+        if cfg.get("qk_norm"):
+            def head_norm(M, g):
+                return M / np.sqrt(np.mean(M * M, axis=-1, keepdims=True) + eps) * g.astype(np.float64)
+            q, k = head_norm(q, lw["q_norm"]), head_norm(k, lw["k_norm"])
         q, k, v = torch_bf16(rope(q)), torch_bf16(rope(k)), torch_bf16(v)
         o = _brute_force_causal(q, k, v, nq, nkv, 1 / math.sqrt(d))
         X = X + torch_bf16(o.reshape(T, nq * d)) @ f(lw["wo"]).T
@@ -485,12 +582,19 @@ def _textbook_forward(cfg, w, toks):
     return (xf @ f(head).T)[0]
 
 
-@pytest.mark.parametrize("variant", ["dense", "tied_bias", "moe"])
+@pytest.mark.parametrize("variant", ["dense", "tied_bias", "qknorm", "qknorm_bias", "moe", "moe_qknorm_bias"])
 def test_oracle_matches_whole_sequence_matrix_form(variant):
     if variant == "dense":
         cfg = _small_dense()
     elif variant == "tied_bias":
         cfg = _small_dense(tied=1, qkv_bias=1, rope_base=500000.0)
+    elif variant == "qknorm":
+        cfg = _small_dense(qk_norm=1)
+    elif variant == "qknorm_bias":
+        cfg = _small_dense(qk_norm=1, qkv_bias=1)
+    elif variant == "moe_qknorm_bias":
+        cfg = dict(_moe_cfg(E=6, k=2), hidden=32, layers=2, n_q_heads=4, n_kv_heads=2, head_dim=8,
+                   qkv_bias=1, qk_norm=1, vocab=48, max_context=16)
     else:
         cfg = dict(_moe_cfg(E=6, k=2), hidden=32, layers=2, n_q_heads=4, n_kv_heads=4, head_dim=8,
                    qkv_bias=1, vocab=48, max_context=16)
