@@ -55,16 +55,23 @@ class Config(C.Structure):
         "hidden", "layers", "nq", "nkv", "d", "inter", "vocab",
         "tied", "qkv_bias", "qk_norm",
         "n_experts", "top_k", "expert_inter", "shared_inter", "shared_gate", "norm_topk",
-        "max_ctx")] + [("eps", C.c_double), ("rope_base", C.c_double)]
+        "max_ctx")] + [("eps", C.c_double), ("rope_base", C.c_double)] + \
+        [(n, C.c_int32) for n in ("sliding_window", "swa_pattern", "sandwich", "q8")] + \
+        [("attn_softcap", C.c_double), ("final_softcap", C.c_double)]
 
 
 class Weights(C.Structure):
-    _fields_ = [("embed", C.c_void_p), ("lm_head", C.c_void_p), ("final_norm", C.c_void_p)]
+    _fields_ = [("embed", C.c_void_p), ("lm_head", C.c_void_p), ("final_norm", C.c_void_p),
+                ("lm_head_q", C.c_void_p), ("lm_head_s", C.c_void_p)]
 
 
 _LAYER_FIELDS = ("attn_norm", "ffn_norm", "wqkv", "bqkv", "q_norm", "k_norm", "wo",
                  "w_gate", "w_up", "w_down", "w_router", "e_gate", "e_up", "e_down",
-                 "s_gate", "s_up", "s_down", "s_gate_vec")
+                 "s_gate", "s_up", "s_down", "s_gate_vec", "post_attn_norm", "post_ffn_norm",
+                 "wqkv_q", "wqkv_s", "wo_q", "wo_s", "w_gate_q", "w_gate_s", "w_up_q", "w_up_s",
+                 "w_down_q", "w_down_s")
+# projections that q8_row models hold as int8 [rows][cols] + fp32 row scales
+Q8_MATS = ("wqkv", "wo", "w_gate", "w_up", "w_down")
 
 
 class Layer(C.Structure):
@@ -82,6 +89,10 @@ def _declare(L):
     L.orc_head_rmsnorm.argtypes = [_P, C.c_int, C.c_int, _P, C.c_double]
     L.orc_rope.argtypes = [_P, C.c_int, C.c_int, C.c_int64, C.c_double]
     L.orc_attend.argtypes = [_P, _P, _P, C.c_int64, C.c_int, C.c_int64, C.c_double, _P]
+    L.orc_attend_window.argtypes = [_P, _P, _P, C.c_int64, C.c_int, C.c_int64, C.c_int64, C.c_double, C.c_double,
+                                    _P]
+    L.orc_matvec_q8.argtypes = [_P, _P, C.c_int64, C.c_int64, _P, _P]
+    L.orc_layer_window.argtypes = [C.POINTER(Config), C.c_int]
     L.orc_route_topk.argtypes = [_P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
     L.orc_swiglu.argtypes = [_P, _P, _P, _P, C.c_int, C.c_int, _P]
     L.orc_moe_ffn.argtypes = [C.POINTER(Config), C.POINTER(Layer), _P, _P, _P, _P, _P]
@@ -160,6 +171,31 @@ def attend(q, K, V, scale) -> np.ndarray:
     return out
 
 
+def attend_window(q, K, V, scale, first=0, softcap=0.0) -> np.ndarray:
+    """One head over rows first .. n-1 of K/V (bf16 bits [n][d]), optional logit softcap."""
+    q = _c(q, np.float64)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    out = np.empty(q.size, np.float64)
+    lib().orc_attend_window(_p(q), _p(K), _p(V), K.shape[1], q.size, int(first), K.shape[0], float(scale),
+                            float(softcap), _p(out))
+    return out
+
+
+def matvec_q8(Q, S, x) -> np.ndarray:
+    """q8_row matrix (int8 [N][K], fp32 scales [N]) times x [K]."""
+    Q = _c(Q, np.int8)
+    S = _c(S, np.float32)
+    x = _c(x, np.float64)
+    y = np.empty(Q.shape[0], np.float64)
+    lib().orc_matvec_q8(_p(Q), _p(S), Q.shape[0], Q.shape[1], _p(x), _p(y))
+    return y
+
+
+def layer_window(cfg: dict, layer: int) -> int:
+    return lib().orc_layer_window(C.byref(_make_config(cfg, 1)), int(layer))
+
+
 def route_topk(logits, k, renorm):
     logits = _c(logits, np.float64)
     idx = np.empty(k, np.int32)
@@ -213,7 +249,8 @@ def gemv_rows(W, x) -> np.ndarray:
 
 # ----------------------------------------------------------------- model
 
-_F32_FIELDS = ("attn_norm", "ffn_norm", "bqkv", "q_norm", "k_norm", "s_gate_vec")
+_F32_FIELDS = ("attn_norm", "ffn_norm", "bqkv", "q_norm", "k_norm", "s_gate_vec", "post_attn_norm",
+               "post_ffn_norm")
 
 
 def _make_config(cfg: dict, max_ctx: int) -> Config:
@@ -227,14 +264,26 @@ def _make_config(cfg: dict, max_ctx: int) -> Config:
     c.shared_gate, c.norm_topk = cfg.get("shared_gate", 0), cfg.get("norm_topk", 0)
     c.max_ctx = int(max_ctx)
     c.eps, c.rope_base = float(cfg["rms_eps"]), float(cfg["rope_base"])
+    c.sliding_window, c.swa_pattern = cfg.get("sliding_window", 0), cfg.get("swa_pattern", 0)
+    c.sandwich, c.q8 = cfg.get("sandwich", 0), int(cfg.get("weight_format", 0) == 1)
+    c.attn_softcap, c.final_softcap = float(cfg.get("attn_softcap", 0.0)), float(cfg.get("final_softcap", 0.0))
     return c
 
 
-def _fill_layer(dst: Layer, lw: dict, keep: list) -> None:
+def _fill_layer(dst: Layer, lw: dict, keep: list, q8: bool = False) -> None:
+    """Point a Layer at the arrays of a synth layer dict. In a q8_row model the projection
+    entries (Q8_MATS) are int8 and their row scales sit under '<name>_scale'."""
     for f in _LAYER_FIELDS:
-        a = lw.get(f)
-        if a is None:
-            setattr(dst, f, None)
+        setattr(dst, f, None)
+    for f, a in lw.items():
+        if a is None or f.endswith("_scale") or f not in _LAYER_FIELDS:
+            continue
+        if q8 and f in Q8_MATS:
+            qa = np.ascontiguousarray(a, dtype=np.int8)
+            sa = np.ascontiguousarray(lw[f + "_scale"], dtype=np.float32)
+            keep += [qa, sa]
+            setattr(dst, f + "_q", qa.ctypes.data)
+            setattr(dst, f + "_s", sa.ctypes.data)
             continue
         a = np.ascontiguousarray(a, dtype=np.float32 if f in _F32_FIELDS else np.uint16)
         keep.append(a)
@@ -246,7 +295,7 @@ def moe_ffn(cfg: dict, lw: dict, xn):
     keep = []
     c = _make_config(cfg, 1)
     L = Layer()
-    _fill_layer(L, lw, keep)
+    _fill_layer(L, lw, keep, cfg.get("weight_format", 0) == 1)
     xn = _c(xn, np.float64)
     k = max(1, cfg.get("top_k", 0))
     out = np.empty(cfg["hidden"], np.float64)
@@ -281,13 +330,18 @@ class Model:
             keep.append(a)
             return a.ctypes.data
 
+        q8 = cfg.get("weight_format", 0) == 1
         w = Weights()
         w.embed = ptr(weights["embed"], np.uint16)
-        w.lm_head = ptr(weights.get("lm_head"), np.uint16)
+        if q8 and weights.get("lm_head") is not None:
+            w.lm_head_q = ptr(weights["lm_head"], np.int8)
+            w.lm_head_s = ptr(weights["lm_head_scale"], np.float32)
+        else:
+            w.lm_head = ptr(weights.get("lm_head"), np.uint16)
         w.final_norm = ptr(weights["final_norm"], np.float32)
         layers = (Layer * cfg["layers"])()
         for i, lw in enumerate(weights["layers"]):
-            _fill_layer(layers[i], lw, keep)
+            _fill_layer(layers[i], lw, keep, q8)
         self._keep = _Keep(keep)
         self._c = c
         self.n_seqs = n_seqs

@@ -34,6 +34,19 @@
  *     index first on ties, optional renormalisation of the k weights.
  *   - MoE output joins the residual as (routed + shared).
  *   - Greedy argmax picks the lowest index on ties.
+ *   - Sliding window W: the query at position p attends keys p-W+1 .. p (the
+ *     last W positions, itself included); a layer l is windowed when
+ *     (l + 1) % max(pattern, 1) != 0 (cortiq layer_is_local / layer_window;
+ *     ANEDVD passes `.window` to attentionDecode for sliding layers).
+ *   - Attention logit softcap c: each scaled score s becomes c * tanh(s / c)
+ *     before the softmax (ANEDVD `.logit_softcap`); the final logit softcap
+ *     maps every logit the same way after the LM head (ANEDVD runHead).
+ *   - Sandwich norms: the o_proj output and the dense FFN output are each
+ *     RMS-normalised with their own gain before they join the residual
+ *     (ANEDVD forward: post_attn / post_ffw through rmsnormFlat), no rounding.
+ *   - q8_row weights: an int8 matrix with one fp32 scale per row stands for
+ *     the matrix W[n][k] = scale[n] * q[n][k], dequantised exactly in fp64
+ *     (cortiq's q8_row_parts of the projections).
  */
 #include "oracle.h"
 
@@ -82,6 +95,18 @@ void orc_matvec(const uint16_t* W, int64_t N, int64_t K, const double* x, double
     }
 }
 
+/* q8_row: y[n] = sum_k (S[n] * Q[n][k]) * x[k], the int8 row dequantised exactly. */
+void orc_matvec_q8(const int8_t* Q, const float* S, int64_t N, int64_t K, const double* x, double* y) {
+#pragma omp parallel for schedule(static) if (N * K > 65536)
+    for (int64_t n = 0; n < N; ++n) {
+        const int8_t* q = Q + n * K;
+        const double sc = (double)S[n];
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += (sc * (double)q[k]) * x[k];
+        y[n] = acc;
+    }
+}
+
 /* out = x * (1 / sqrt(mean(x^2) + eps)) * g, unrounded (rmsnormColumn / rmsnormFlat). */
 void orc_rmsnorm(const double* x, const float* g, int n, double eps, double* out) {
     double acc = 0.0;
@@ -112,32 +137,48 @@ void orc_rope(double* v, int heads, int d, int64_t pos, double base) {
     }
 }
 
-/* One query head against n cached rows of one kv head:
- * out = sum_j softmax_j(q . K_j * scale) V_j, max subtracted, sums in j order.
+/* One query head against cached rows first .. n-1 of one kv head:
+ * s_j = q . K_j * scale, then c * tanh(s_j / c) when softcap c > 0;
+ * out = sum_j softmax_j(s) V_j, max subtracted, sums in j order.
  * K, V rows are bf16 with row stride `stride` elements. */
-void orc_attend(const double* q, const uint16_t* K, const uint16_t* V, int64_t stride, int d, int64_t n,
-                double scale, double* out) {
+void orc_attend_window(const double* q, const uint16_t* K, const uint16_t* V, int64_t stride, int d, int64_t first,
+                       int64_t n, double scale, double softcap, double* out) {
     double* s = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
     double m = -INFINITY;
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = first; j < n; ++j) {
         const uint16_t* k = K + j * stride;
         double acc = 0.0;
         for (int i = 0; i < d; ++i) acc += q[i] * bf(k[i]);
         s[j] = acc * scale;
+        if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);
         if (s[j] > m) m = s[j];
     }
     double den = 0.0;
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = first; j < n; ++j) {
         s[j] = exp(s[j] - m);
         den += s[j];
     }
     for (int i = 0; i < d; ++i) out[i] = 0.0;
-    for (int64_t j = 0; j < n; ++j) {
+    for (int64_t j = first; j < n; ++j) {
         const uint16_t* v = V + j * stride;
         for (int i = 0; i < d; ++i) out[i] += s[j] * bf(v[i]);
     }
     for (int i = 0; i < d; ++i) out[i] /= den;
     free(s);
+}
+
+/* Full causal attention over rows 0 .. n-1, no softcap. */
+void orc_attend(const double* q, const uint16_t* K, const uint16_t* V, int64_t stride, int d, int64_t n,
+                double scale, double* out) {
+    orc_attend_window(q, K, V, stride, d, 0, n, scale, 0.0, out);
+}
+
+/* Attention window of layer `layer`: sliding_window on local layers, 0 (whole context) on
+ * global ones; every max(swa_pattern, 1)-th layer is global. */
+int orc_layer_window(const orc_config* c, int layer) {
+    if (c->sliding_window <= 0) return 0;
+    const int pattern = c->swa_pattern > 1 ? c->swa_pattern : 1;
+    return (layer + 1) % pattern != 0 ? c->sliding_window : 0;
 }
 
 /* Softmax over all E logits, then the k most probable experts (lower index first on
@@ -186,17 +227,33 @@ void orc_route_topk(const double* logits, int E, int k, int renorm, int32_t* idx
 static double silu(double z) { return z * (1.0 / (1.0 + exp(-z))); }
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* y = W x with W either bf16 (W) or q8_row (Q, S). */
+static void matvec_w(const uint16_t* W, const int8_t* Q, const float* S, int64_t N, int64_t K, const double* x,
+                     double* y) {
+    if (Q)
+        orc_matvec_q8(Q, S, N, K, x, y);
+    else
+        orc_matvec(W, N, K, x, y);
+}
+
+/* SwiGLU with each of the three matrices bf16 or q8_row. */
+static void swiglu_w(const double* x, const uint16_t* Wg, const int8_t* Qg, const float* Sg, const uint16_t* Wu,
+                     const int8_t* Qu, const float* Su, const uint16_t* Wd, const int8_t* Qd, const float* Sd, int I,
+                     int h, double* out) {
+    double* g = (double*)malloc(sizeof(double) * (size_t)I);
+    double* u = (double*)malloc(sizeof(double) * (size_t)I);
+    matvec_w(Wg, Qg, Sg, I, h, x, g);
+    matvec_w(Wu, Qu, Su, I, h, x, u);
+    for (int i = 0; i < I; ++i) g[i] = orc_bf16(silu(g[i]) * u[i]);
+    matvec_w(Wd, Qd, Sd, h, I, g, out);
+    free(g);
+    free(u);
+}
+
 /* out = Wd * R4(silu(Wg x) * (Wu x)); Wg, Wu [I][h], Wd [h][I]. */
 void orc_swiglu(const double* x, const uint16_t* Wg, const uint16_t* Wu, const uint16_t* Wd, int I, int h,
                 double* out) {
-    double* g = (double*)malloc(sizeof(double) * (size_t)I);
-    double* u = (double*)malloc(sizeof(double) * (size_t)I);
-    orc_matvec(Wg, I, h, x, g);
-    orc_matvec(Wu, I, h, x, u);
-    for (int i = 0; i < I; ++i) g[i] = orc_bf16(silu(g[i]) * u[i]);
-    orc_matvec(Wd, h, I, g, out);
-    free(g);
-    free(u);
+    swiglu_w(x, Wg, NULL, NULL, Wu, NULL, NULL, Wd, NULL, NULL, I, h, out);
 }
 
 /* MoE FFN on one normalised (R1) input row xn [h]:
@@ -307,7 +364,7 @@ static void layer_forward(orc_model* m, int li, int seq, int64_t pos, double* x)
     orc_rmsnorm(x, L->attn_norm, h, c->eps, xn);
     for (int i = 0; i < h; ++i) xn[i] = orc_bf16(xn[i]);
     /* 2. fused QKV projection (+ bias before any norm or rotation) */
-    orc_matvec(L->wqkv, rows, h, xn, qkv);
+    matvec_w(L->wqkv, L->wqkv_q, L->wqkv_s, rows, h, xn, qkv);
     if (c->qkv_bias && L->bqkv)
         for (int64_t r = 0; r < rows; ++r) qkv[r] += (double)L->bqkv[r];
     double* q = qkv;
@@ -329,27 +386,33 @@ static void layer_forward(orc_model* m, int li, int seq, int64_t pos, double* x)
         krow[i] = to_bits(orc_bf16(k[i]));
         vrow[i] = to_bits(orc_bf16(v[i]));
     }
-    /* 6. causal GQA attention over rows 0..pos, scale 1/sqrt(d); R3 */
+    /* 6. causal GQA attention over rows 0..pos (the last `window` of them on a windowed
+     *    layer), scale 1/sqrt(d), optional logit softcap; R3 */
     const int group = nq / nkv;
     const double scale = 1.0 / sqrt((double)d);
     const uint16_t* K0 = kslot(m, m->kc, seq, li, 0);
     const uint16_t* V0 = kslot(m, m->vc, seq, li, 0);
+    const int64_t window = orc_layer_window(c, li);
+    const int64_t first = window > 0 && pos + 1 > window ? pos + 1 - window : 0;
 #pragma omp parallel for schedule(static) if (pos > 256)
     for (int hh = 0; hh < nq; ++hh) {
         int g = hh / group;
-        orc_attend(q + (int64_t)hh * d, K0 + (int64_t)g * d, V0 + (int64_t)g * d, kvd, d, pos + 1, scale,
-                   o + (int64_t)hh * d);
+        orc_attend_window(q + (int64_t)hh * d, K0 + (int64_t)g * d, V0 + (int64_t)g * d, kvd, d, first, pos + 1,
+                          scale, c->attn_softcap, o + (int64_t)hh * d);
     }
     for (int64_t i = 0; i < qd; ++i) o[i] = orc_bf16(o[i]);
-    /* 7. o_proj and residual */
-    orc_matvec(L->wo, h, qd, o, t);
+    /* 7. o_proj (sandwich: RMS-normalised with post_attn_norm) and residual */
+    matvec_w(L->wo, L->wo_q, L->wo_s, h, qd, o, t);
+    if (c->sandwich) orc_rmsnorm(t, L->post_attn_norm, h, c->eps, t);
     for (int i = 0; i < h; ++i) x[i] += t[i];
     /* 8. FFN-input RMSNorm, R1 */
     orc_rmsnorm(x, L->ffn_norm, h, c->eps, xn);
     for (int i = 0; i < h; ++i) xn[i] = orc_bf16(xn[i]);
     if (c->n_experts <= 0) {
-        /* 9. dense SwiGLU */
-        orc_swiglu(xn, L->w_gate, L->w_up, L->w_down, c->inter, h, t);
+        /* 9. dense SwiGLU (sandwich: RMS-normalised with post_ffn_norm) */
+        swiglu_w(xn, L->w_gate, L->w_gate_q, L->w_gate_s, L->w_up, L->w_up_q, L->w_up_s, L->w_down, L->w_down_q,
+                 L->w_down_s, c->inter, h, t);
+        if (c->sandwich) orc_rmsnorm(t, L->post_ffn_norm, h, c->eps, t);
         for (int i = 0; i < h; ++i) x[i] += t[i];
     } else {
         /* 10. MoE: router softmax, top-k, weighted routed experts, gated shared expert */
@@ -376,12 +439,14 @@ int orc_forward(orc_model* m, int seq, int32_t token, int64_t pos, double* logit
     for (int i = 0; i < h; ++i) x[i] = bf(m->w.embed[(int64_t)token * h + i]);
     for (int li = 0; li < c->layers; ++li) layer_forward(m, li, seq, pos, x);
     memcpy(m->hidden, x, sizeof(double) * (size_t)h);
-    /* final RMSNorm (R1) and LM head */
+    /* final RMSNorm (R1), LM head, optional final logit softcap */
     if (logits) {
         orc_rmsnorm(x, m->w.final_norm, h, c->eps, xn);
         for (int i = 0; i < h; ++i) xn[i] = orc_bf16(xn[i]);
         const uint16_t* head = c->tied ? m->w.embed : m->w.lm_head;
-        orc_matvec(head, c->vocab, h, xn, logits);
+        matvec_w(head, c->tied ? NULL : m->w.lm_head_q, m->w.lm_head_s, c->vocab, h, xn, logits);
+        if (c->final_softcap > 0.0)
+            for (int64_t v = 0; v < c->vocab; ++v) logits[v] = c->final_softcap * tanh(logits[v] / c->final_softcap);
     }
     free(x);
     free(xn);

@@ -19,12 +19,20 @@ typedef struct orc_config {
     int32_t n_experts, top_k, expert_inter, shared_inter, shared_gate, norm_topk;
     int32_t max_ctx;
     double eps, rope_base;
+    /* sliding-window attention: layer l attends the last `sliding_window` positions when
+     * (l + 1) % max(swa_pattern, 1) != 0 (0 = no window on any layer) */
+    int32_t sliding_window, swa_pattern;
+    int32_t sandwich; /* 1: post-attention and post-FFN RMSNorm before each residual add */
+    int32_t q8;       /* 1: projections and LM head are int8 with one fp32 scale per row */
+    double attn_softcap, final_softcap; /* 0 = off */
 } orc_config;
 
 typedef struct orc_weights {
     const uint16_t* embed;     /* bf16 [V][h] */
     const uint16_t* lm_head;   /* bf16 [V][h], unused when tied */
     const float* final_norm;   /* [h] */
+    const int8_t* lm_head_q;   /* q8: int8 [V][h] (untied head only) */
+    const float* lm_head_s;    /* q8: fp32 [V] row scales */
 } orc_weights;
 
 typedef struct orc_layer {
@@ -46,6 +54,19 @@ typedef struct orc_layer {
     const uint16_t* s_up;      /* bf16 [Is][h] */
     const uint16_t* s_down;    /* bf16 [h][Is] */
     const float* s_gate_vec;   /* [h] or NULL */
+    const float* post_attn_norm; /* sandwich: [h] */
+    const float* post_ffn_norm;  /* sandwich: [h] */
+    /* q8: the projections as int8 [rows][cols] with fp32 row scales [rows] */
+    const int8_t* wqkv_q;
+    const float* wqkv_s;
+    const int8_t* wo_q;
+    const float* wo_s;
+    const int8_t* w_gate_q;
+    const float* w_gate_s;
+    const int8_t* w_up_q;
+    const float* w_up_s;
+    const int8_t* w_down_q;
+    const float* w_down_s;
 } orc_layer;
 
 typedef struct orc_model orc_model;
@@ -57,6 +78,10 @@ void orc_head_rmsnorm(double* v, int heads, int d, const float* g, double eps);
 void orc_rope(double* v, int heads, int d, int64_t pos, double base);
 void orc_attend(const double* q, const uint16_t* K, const uint16_t* V, int64_t stride, int d, int64_t n,
                 double scale, double* out);
+void orc_attend_window(const double* q, const uint16_t* K, const uint16_t* V, int64_t stride, int d, int64_t first,
+                       int64_t n, double scale, double softcap, double* out);
+void orc_matvec_q8(const int8_t* Q, const float* S, int64_t N, int64_t K, const double* x, double* y);
+int orc_layer_window(const orc_config* c, int layer);
 void orc_route_topk(const double* logits, int E, int k, int renorm, int32_t* idx, double* w, double* gap);
 void orc_swiglu(const double* x, const uint16_t* Wg, const uint16_t* Wu, const uint16_t* Wd, int I, int h,
                 double* out);

@@ -12,8 +12,14 @@ Recipe (seed 0 unless stated):
   * prompts: uniform ids in [0, V) from seed 1000 + k
   * synthetic KV fills: N(0, 1) -> bf16 from seed 2000
 
-Stream ids: 1 embed, 2 lm_head, 3 final_norm; layer l uses 1000 + 100 l + slot
-(slots below); expert e of layer l uses 10_000_000 + 10_000 l + 10 e + {0 gate, 1 up, 2 down}.
+  * post-attention / post-FFN norm gains (sandwich norms): 1 + N(0, 0.1), like the other gains
+  * q8_row models (weight_format 1): each projection and the untied LM head as int8 values
+    nearbyint(32 z) clamped to [-127, 127], and one fp32 scale per row, the bf16 value of
+    (0.02 / 32)(1 + 0.1 z'): entries of about N(0, 0.02) like the bf16 weights
+
+Stream ids: 1 embed, 2 lm_head, 3 final_norm, 4 lm_head row scales; layer l uses
+1000 + 100 l + slot (slots below; a q8_row scale uses its matrix's slot + 50); expert e of
+layer l uses 10_000_000 + 10_000 l + 10 e + {0 gate, 1 up, 2 down}.
 """
 from __future__ import annotations
 
@@ -35,8 +41,11 @@ WEIGHT_STD = 0.02
 GAIN_STD = 0.1
 
 SLOTS = dict(attn_norm=0, ffn_norm=1, wqkv=2, bqkv=3, q_norm=4, k_norm=5, wo=6, w_gate=7, w_up=8,
-             w_down=9, w_router=10, s_gate=11, s_up=12, s_down=13, s_gate_vec=14)
-GAINS = ("attn_norm", "ffn_norm", "q_norm", "k_norm")
+             w_down=9, w_router=10, s_gate=11, s_up=12, s_down=13, s_gate_vec=14, post_attn_norm=15,
+             post_ffn_norm=16)
+GAINS = ("attn_norm", "ffn_norm", "q_norm", "k_norm", "post_attn_norm", "post_ffn_norm")
+Q8_MATS = ("wqkv", "wo", "w_gate", "w_up", "w_down")
+Q8_STD = 32.0  # int8 values ~ N(0, 32^2); scales ~ WEIGHT_STD / Q8_STD
 VECTORS = ("bqkv", "s_gate_vec")
 
 
@@ -79,6 +88,7 @@ def lib():
         L.syn_fill_tokens.argtypes = [C.c_void_p, C.c_int64, C.c_uint64, C.c_uint64, C.c_int32]
         L.syn_fill_normal_f64.argtypes = [C.c_void_p, C.c_int64, C.c_uint64, C.c_uint64]
         L.syn_fill_uniform_f64.argtypes = [C.c_void_p, C.c_int64, C.c_uint64, C.c_uint64]
+        L.syn_fill_i8.argtypes = [C.c_void_p, C.c_int64, C.c_uint64, C.c_uint64, C.c_double]
         _lib = L
     return _lib
 
@@ -107,6 +117,20 @@ def bf16_normal_f32(n: int, seed: int, tid: int, mean: float = 0.0, std: float =
     out = np.empty(n, np.float32)
     lib().syn_fill_bf16_as_f32(out.ctypes.data, n, seed, tid, mean, std)
     return out
+
+
+def int8_normal(shape, seed: int, tid: int, std: float = Q8_STD) -> np.ndarray:
+    """int8 values nearbyint(std * N(0,1)) clamped to [-127, 127], one stream per (seed, tid)."""
+    out = np.empty(shape, np.int8)
+    lib().syn_fill_i8(out.ctypes.data, out.size, seed, tid, std)
+    return out
+
+
+def q8_rows(shape, seed: int, tid: int, scale_tid: int):
+    """A synthetic q8_row matrix: (int8 values [rows][cols], fp32 row scales [rows])."""
+    q = int8_normal(shape, seed, tid)
+    s = bf16_normal_f32(shape[0], seed, scale_tid, WEIGHT_STD / Q8_STD, 0.1 * WEIGHT_STD / Q8_STD)
+    return q, s
 
 
 def tokens(n: int, vocab: int, seed: int, tid: int = 0) -> np.ndarray:
@@ -153,7 +177,9 @@ def tensor_shapes(cfg: dict) -> dict:
     s = dict(attn_norm=(h,), ffn_norm=(h,), wqkv=(qkv, h), wo=(h, nq * d),
              bqkv=(qkv,) if cfg.get("qkv_bias") else None,
              q_norm=(d,) if cfg.get("qk_norm") else None,
-             k_norm=(d,) if cfg.get("qk_norm") else None)
+             k_norm=(d,) if cfg.get("qk_norm") else None,
+             post_attn_norm=(h,) if cfg.get("sandwich") else None,
+             post_ffn_norm=(h,) if cfg.get("sandwich") else None)
     if cfg.get("n_experts", 0) > 0:
         E, Ie, Is = cfg["n_experts"], cfg["expert_inter"], cfg.get("shared_inter", 0)
         s.update(w_router=(E, h), e_gate=(E, Ie, h), e_up=(E, Ie, h), e_down=(E, h, Ie),
@@ -168,9 +194,13 @@ def tensor_shapes(cfg: dict) -> dict:
 
 def make_layer(cfg: dict, layer: int, seed: int = 0) -> dict:
     out = {}
+    q8 = cfg.get("weight_format", 0) == 1
     for name, shape in tensor_shapes(cfg).items():
         if shape is None:
             out[name] = None
+        elif q8 and name in Q8_MATS:
+            tid = layer_tid(layer, name)
+            out[name], out[name + "_scale"] = q8_rows(shape, seed, tid, tid + 50)
         elif name in ("e_gate", "e_up", "e_down"):
             part = ("e_gate", "e_up", "e_down").index(name)
             arr = np.empty(shape, np.uint16)
@@ -193,6 +223,8 @@ def make_weights(cfg: dict, seed: int = 0) -> dict:
     w = dict(embed=bf16_normal((V, h), seed, 1, 0.0, WEIGHT_STD),
              lm_head=None if cfg.get("tied") else bf16_normal((V, h), seed, 2, 0.0, WEIGHT_STD),
              final_norm=bf16_normal_f32(h, seed, 3, 1.0, GAIN_STD))
+    if cfg.get("weight_format", 0) == 1 and not cfg.get("tied"):
+        w["lm_head"], w["lm_head_scale"] = q8_rows((V, h), seed, 2, 4)
     w["layers"] = [make_layer(cfg, l, seed) for l in range(cfg["layers"])]
     return w
 

@@ -8,7 +8,8 @@ no top-k renormalisation.
 
 COMMON = dict(qkv_bias=0, qk_norm=0, tied=0, n_experts=0, top_k=0, expert_inter=0,
               shared_inter=0, shared_gate=0, norm_topk=0, rms_eps=1e-5, rope_base=10000.0,
-              page_size=16, prefill_chunk=128, max_batch=1)
+              page_size=16, prefill_chunk=128, max_batch=1, sliding_window=0, swa_pattern=0,
+              attn_softcap=0.0, final_softcap=0.0, sandwich=0, weight_format=0)
 
 # Tiny dense decoder: 16-token prompt then 8 greedy decode steps, batch 1.
 TINY = dict(COMMON, name="tiny-dense", hidden=256, layers=2, n_q_heads=4, n_kv_heads=2, head_dim=64,

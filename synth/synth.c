@@ -19,6 +19,9 @@
  *
  * Uniform integers in [0, V): R(K, n) mod V.
  *
+ * int8 values (synthetic q8_row weight rows): nearbyint(std * z) clamped to
+ * [-127, 127], z a normal of the same stream definition.
+ *
  * The device twin of these functions lives in synth_fill.cu and follows the
  * same definitions; tests compare the two.
  */
@@ -101,4 +104,16 @@ void syn_fill_normal_f64(double* out, int64_t n, uint64_t seed, uint64_t id) {
 void syn_fill_uniform_f64(double* out, int64_t n, uint64_t seed, uint64_t id) {
     uint64_t key = syn_stream_key(seed, id);
     for (int64_t i = 0; i < n; ++i) out[i] = (double)(syn_raw(key, (uint64_t)i) >> 11) * 0x1.0p-53;
+}
+
+/* out[i] = clamp(nearbyint(std * z_i), -127, 127) as int8; z from stream (seed, id). */
+void syn_fill_i8(int8_t* out, int64_t n, uint64_t seed, uint64_t id, double std) {
+    uint64_t key = syn_stream_key(seed, id);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double v = nearbyint(std * syn_normal(key, (uint64_t)i));
+        if (v > 127.0) v = 127.0;
+        if (v < -127.0) v = -127.0;
+        out[i] = (int8_t)v;
+    }
 }

@@ -19,9 +19,9 @@ MUTATIONS = {
                               "            x[i + half] = x0 * s + x1 * c;",
                               "double x0 = x[2 * i], x1 = x[2 * i + 1];\n            x[2 * i] = x0 * c - x1 * s;\n"
                               "            x[2 * i + 1] = x0 * s + x1 * c;"),
-    "causal_drops_current_token": ("d, pos + 1, scale,", "d, pos, scale,"),
-    "gqa_interleaved_mapping": ("        int g = hh / group;\n        orc_attend(q + (int64_t)hh * d, K0",
-                                "        int g = hh % nkv;\n        orc_attend(q + (int64_t)hh * d, K0"),
+    "causal_drops_current_token": ("d, first, pos + 1,", "d, first, pos,"),
+    "gqa_interleaved_mapping": ("        int g = hh / group;\n        orc_attend_window(q + (int64_t)hh * d, K0",
+                                "        int g = hh % nkv;\n        orc_attend_window(q + (int64_t)hh * d, K0"),
     "rmsnorm_no_eps": ("acc / (double)n + eps", "acc / (double)n"),
     "attention_no_scale": ("s[j] = acc * scale;", "s[j] = acc;"),
     "silu_is_sigmoid": ("return z * (1.0 / (1.0 + exp(-z)));", "return (1.0 / (1.0 + exp(-z)));"),
@@ -32,8 +32,8 @@ MUTATIONS = {
     "renorm_ignored": ("w[r] = renorm ? p[order[r]] / sum : p[order[r]];", "w[r] = p[order[r]];"),
     "shared_gate_no_sigmoid": ("sc = sigmoid(gdot);", "sc = gdot;"),
     "tie_break_higher_index": ("(best < 0 || p[e] > p[best])", "(best < 0 || p[e] >= p[best])"),
-    "residual_dropped": ("    orc_matvec(L->wo, h, qd, o, t);\n    for (int i = 0; i < h; ++i) x[i] += t[i];",
-                         "    orc_matvec(L->wo, h, qd, o, t);\n    for (int i = 0; i < h; ++i) x[i] = t[i];"),
+    "residual_dropped": ("post_attn_norm, h, c->eps, t);\n    for (int i = 0; i < h; ++i) x[i] += t[i];",
+                         "post_attn_norm, h, c->eps, t);\n    for (int i = 0; i < h; ++i) x[i] = t[i];"),
     "qkv_bias_dropped": ("qkv[r] += (double)L->bqkv[r];", "qkv[r] += 0.0;"),
     "cache_row_off_by_one": ("uint16_t* krow = kslot(m, m->kc, seq, li, pos);",
                              "uint16_t* krow = kslot(m, m->kc, seq, li, pos + 1 < m->c.max_ctx ? pos + 1 : pos);"),
@@ -75,6 +75,19 @@ MUTATIONS = {
     }
     if (c->qkv_bias && L->bqkv)
         for (int64_t r = 0; r < rows; ++r) qkv[r] += (double)L->bqkv[r];"""),
+    "window_one_key_too_many": ("pos + 1 > window ? pos + 1 - window : 0;", "pos + 1 > window ? pos - window : 0;"),
+    "window_schedule_inverted": ("(layer + 1) % pattern != 0 ? c->sliding_window : 0",
+                                 "(layer + 1) % pattern == 0 ? c->sliding_window : 0"),
+    "softcap_before_scale": ("""        s[j] = acc * scale;
+        if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);""",
+                             """        s[j] = (softcap > 0.0 ? softcap * tanh(acc / softcap) : acc) * scale;"""),
+    "softcap_ignored": ("        if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);\n", ""),
+    "sandwich_post_attn_dropped": ("    if (c->sandwich) orc_rmsnorm(t, L->post_attn_norm, h, c->eps, t);\n", ""),
+    "sandwich_ffn_uses_attn_gain": ("orc_rmsnorm(t, L->post_ffn_norm,", "orc_rmsnorm(t, L->post_attn_norm,"),
+    "final_softcap_dropped": ("logits[v] = c->final_softcap * tanh(logits[v] / c->final_softcap);",
+                              "logits[v] = logits[v];"),
+    "q8_scale_ignored": ("acc += (sc * (double)q[k]) * x[k];", "acc += ((double)q[k]) * x[k];"),
+    "q8_first_row_scale": ("const double sc = (double)S[n];", "const double sc = (double)S[0];"),
     "tied_head_ignored": ("const uint16_t* head = c->tied ? m->w.embed : m->w.lm_head;",
                           "const uint16_t* head = m->w.embed;"),
 }

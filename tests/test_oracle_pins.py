@@ -247,15 +247,20 @@ def test_attention_equal_scores_average_values():
     assert np.allclose(out, f(V).mean(axis=0), rtol=1e-14, atol=1e-15)
 
 
-def _brute_force_causal(Q, K, V, nq, nkv, scale):
+def _brute_force_causal(Q, K, V, nq, nkv, scale, window=0, softcap=0.0):
     """Textbook masked-matrix attention for T queries at positions 0..T-1:
-    O_h = softmax(mask(Q_h K_g^T * scale)) V_g, g = h // (nq // nkv)."""
+    O_h = softmax(mask(cap(Q_h K_g^T * scale))) V_g, g = h // (nq // nkv); the mask hides
+    later keys and, with a window W, keys W or more positions back."""
     T, d = Q.shape[0], Q.shape[2]
     out = np.zeros((T, nq, d))
     mask = np.triu(np.ones((T, T), bool), 1)
+    if window:
+        mask |= np.tril(np.ones((T, T), bool), -window)
     for h in range(nq):
         g = h // (nq // nkv)
         S = Q[:, h, :] @ K[:, g, :].T * scale
+        if softcap:
+            S = softcap * np.tanh(S / softcap)
         S[mask] = -np.inf
         P = np.exp(S - S.max(axis=1, keepdims=True))
         P /= P.sum(axis=1, keepdims=True)
@@ -487,11 +492,151 @@ def test_shared_expert_gate_changes_logits_like_the_pages_fixture():
     assert np.max(np.abs(gated - ungated)) > g["min_abs_difference_between_runs"]
 
 
+# ------------------------------------------------------------------ sliding window, softcaps, sandwich, q8_row
+
+def test_layer_window_schedule_every_pattern_th_layer_is_global():
+    base = _small_dense(layers=6, sliding_window=4)
+    assert [oracle.layer_window(dict(base, swa_pattern=3), l) for l in range(6)] == [4, 4, 0, 4, 4, 0]
+    assert [oracle.layer_window(dict(base, swa_pattern=2), l) for l in range(6)] == [4, 0, 4, 0, 4, 0]
+    assert [oracle.layer_window(dict(base, swa_pattern=7), l) for l in range(6)] == [4] * 6
+    assert [oracle.layer_window(dict(base, swa_pattern=1), l) for l in range(6)] == [0] * 6
+    assert [oracle.layer_window(dict(base, swa_pattern=0), l) for l in range(6)] == [0] * 6
+    assert [oracle.layer_window(dict(base, sliding_window=0, swa_pattern=3), l) for l in range(6)] == [0] * 6
+
+
+def test_window_of_one_returns_the_current_value_and_a_wide_window_changes_nothing():
+    rng = np.random.default_rng(60)
+    n, d = 9, 16
+    q = rng.standard_normal(d)
+    K, V = rnd_bf16_bits((n, d), 61), rnd_bf16_bits((n, d), 62)
+    assert np.array_equal(oracle.attend_window(q, K, V, 0.25, first=n - 1), f(V[n - 1]))
+    full = oracle.attend(q, K, V, 0.25)
+    assert np.array_equal(oracle.attend_window(q, K, V, 0.25, first=0), full)
+    # a window of 3 is the plain softmax over the last 3 keys only
+    s = np.array([q @ f(K[j]) * 0.25 for j in range(n - 3, n)])
+    p = np.exp(s - s.max())
+    want = (p[:, None] * f(V[n - 3:])).sum(0) / p.sum()
+    assert np.allclose(oracle.attend_window(q, K, V, 0.25, first=n - 3), want, rtol=1e-13, atol=1e-15)
+
+
+def test_attention_softcap_two_keys_closed_form():
+    # q . k_0 = 3 and q . k_1 = -1 at scale 1; a cap of 2 turns them into 2 tanh(1.5) and
+    # 2 tanh(-0.5), so key 0 weighs 1 / (1 + e^(2 tanh(-0.5) - 2 tanh(1.5)))
+    q = np.array([1.0, 0.0])
+    K = bits(np.array([[3.0, 0.0], [-1.0, 0.0]]))
+    V = bits(np.array([[1.0, 0.0], [0.0, 1.0]]))
+    got = oracle.attend_window(q, K, V, 1.0, softcap=2.0)
+    w0 = 1.0 / (1.0 + math.exp(2 * math.tanh(-0.5) - 2 * math.tanh(1.5)))
+    assert np.allclose(got, [w0, 1.0 - w0], rtol=1e-14)
+    # uncapped, the weight is the logistic of the raw score difference
+    w0_raw = 1.0 / (1.0 + math.exp(-4.0))
+    assert np.allclose(oracle.attend_window(q, K, V, 1.0), [w0_raw, 1 - w0_raw], rtol=1e-14)
+    # the cap acts on the scaled score: scale 0.5 with cap 2 is tanh of q.k / 4
+    got = oracle.attend_window(q, K, V, 0.5, softcap=2.0)
+    w0 = 1.0 / (1.0 + math.exp(2 * math.tanh(-0.25) - 2 * math.tanh(0.75)))
+    assert np.allclose(got, [w0, 1.0 - w0], rtol=1e-14)
+
+
+def test_final_softcap_maps_the_uncapped_logits():
+    cfg = _small_dense()
+    w = synth.make_weights(cfg, seed=63)
+    toks = synth.tokens(6, cfg["vocab"], 1003)
+    raw = oracle.Model(cfg, w).prefill(0, toks, 0)
+    capped = oracle.Model(dict(cfg, final_softcap=0.25), w).prefill(0, toks, 0)
+    assert np.all(np.abs(capped) < 0.25)
+    assert np.allclose(capped, 0.25 * np.tanh(raw / 0.25), rtol=1e-14, atol=1e-16)
+
+
+def test_sandwich_with_zero_post_gains_leaves_only_the_embedding():
+    # zero post-norm gains cancel every attention and FFN contribution: the residual stays
+    # the embedding row, and the logits are the head applied to its final norm
+    cfg = _small_dense(sandwich=1)
+    w = synth.make_weights(cfg, seed=64)
+    for lw in w["layers"]:
+        lw["post_attn_norm"] = np.zeros(cfg["hidden"], np.float32)
+        lw["post_ffn_norm"] = np.zeros(cfg["hidden"], np.float32)
+    m = oracle.Model(cfg, w)
+    got = m.forward(0, 11, 0)
+    x = f(w["embed"][11])
+    assert np.array_equal(m.last_hidden(), x)
+    xn = torch_bf16(x / np.sqrt(np.mean(x * x) + cfg["rms_eps"]) * w["final_norm"].astype(np.float64))
+    assert np.allclose(got, f(w["lm_head"]) @ xn, rtol=1e-13, atol=1e-15)
+
+
+def test_sandwich_post_attention_norm_closed_form_at_position_zero():
+    # At p = 0 attention returns the single cached value row, so with a zero post-FFN gain the
+    # layer adds exactly rmsnorm(Wo bf16(v)) * g_post to the embedding, v = Wv xn.
+    cfg = dict(_small_dense(sandwich=1), layers=1, n_kv_heads=4)
+    w = synth.make_weights(cfg, seed=65)
+    lw = w["layers"][0]
+    lw["post_ffn_norm"] = np.zeros(cfg["hidden"], np.float32)
+    m = oracle.Model(cfg, w)
+    m.forward(0, 4, 0)
+    h, qd, eps = cfg["hidden"], cfg["n_q_heads"] * cfg["head_dim"], cfg["rms_eps"]
+    x = f(w["embed"][4])
+    xn = torch_bf16(x / np.sqrt(np.mean(x * x) + eps) * lw["attn_norm"].astype(np.float64))
+    v = torch_bf16(f(lw["wqkv"])[2 * qd:] @ xn)      # nkv == nq: v has the width of o
+    y = f(lw["wo"]) @ v
+    want = x + y / np.sqrt(np.mean(y * y) + eps) * lw["post_attn_norm"].astype(np.float64)
+    assert np.allclose(m.last_hidden(), want, rtol=1e-12, atol=1e-14)
+
+
+def test_q8_matvec_equals_exact_rational_sum():
+    rng = np.random.default_rng(66)
+    N, K = 5, 37
+    Q = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    S = bits_to_fp32_bf16(rng.uniform(1e-4, 1e-3, N))
+    x = f(rnd_bf16_bits(K, 67))
+    got = oracle.matvec_q8(Q, S, x)
+    for n in range(N):
+        exact = Fraction(float(S[n])) * sum(Fraction(int(Q[n, k])) * Fraction(float(x[k])) for k in range(K))
+        assert abs(Fraction(float(got[n])) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
+    # rows: row n uses scale n only
+    e = np.zeros(K)
+    e[3] = 1.0
+    assert np.array_equal(oracle.matvec_q8(Q, S, e), Q[:, 3].astype(np.float64) * S.astype(np.float64))
+
+
+def bits_to_fp32_bf16(v):
+    return f(bits(torch_bf16(v))).astype(np.float32)
+
+
+def test_q8_with_power_of_two_scales_is_the_bf16_model():
+    # scale 2^-9 times an int8 value is an exact bf16 number: the q8_row model must equal
+    # the bf16 model holding those values, bit for bit
+    cfg = _small_dense(weight_format=1)
+    wq = synth.make_weights(cfg, seed=68)
+    wb = synth.make_weights(dict(cfg, weight_format=0), seed=68)
+    for lq, lb in zip(wq["layers"], wb["layers"]):
+        for name in synth.Q8_MATS:
+            lq[name + "_scale"] = np.full(lq[name].shape[0], 2.0 ** -9, np.float32)
+            lb[name] = bits(lq[name].astype(np.float64) * 2.0 ** -9)
+    wq["lm_head_scale"] = np.full(cfg["vocab"], 2.0 ** -9, np.float32)
+    wb["lm_head"] = bits(wq["lm_head"].astype(np.float64) * 2.0 ** -9)
+    toks = synth.tokens(7, cfg["vocab"], 1004)
+    a = oracle.Model(cfg, wq).prefill(0, toks, 0)
+    b = oracle.Model(dict(cfg, weight_format=0), wb).prefill(0, toks, 0)
+    assert np.array_equal(a, b)
+
+
+def test_q8_scales_change_the_result_row_by_row():
+    cfg = _small_dense(weight_format=1)
+    w = synth.make_weights(cfg, seed=69)
+    toks = synth.tokens(5, cfg["vocab"], 1005)
+    a = oracle.Model(cfg, w).prefill(0, toks, 0)
+    w["lm_head_scale"] = w["lm_head_scale"].copy()
+    w["lm_head_scale"][7] *= 2
+    b = oracle.Model(cfg, w).prefill(0, toks, 0)
+    assert b[7] == 2 * a[7] and np.array_equal(np.delete(a, 7), np.delete(b, 7))
+
+
 # ------------------------------------------------------------------ whole stack
 
 def _small_dense(**over):
-    return dict(configs.COMMON, name="small", hidden=48, layers=2, n_q_heads=4, n_kv_heads=2, head_dim=16,
-                ffn_inter=96, vocab=80, max_context=24, **over)
+    cfg = dict(configs.COMMON, name="small", hidden=48, layers=2, n_q_heads=4, n_kv_heads=2, head_dim=16,
+               ffn_inter=96, vocab=80, max_context=24)
+    cfg.update(over)
+    return cfg
 
 
 def test_prefill_equals_sequential_decode_bit_exact():
@@ -555,9 +700,22 @@ def _textbook_forward(cfg, w, toks):
         a, b = M[..., : d // 2], M[..., d // 2:]
         return np.concatenate([a * cos[:, None] - b * sin[:, None], a * sin[:, None] + b * cos[:, None]], -1)
 
-    for lw in w["layers"]:
+    q8 = cfg.get("weight_format", 0) == 1
+
+    def mat(lw, name):  # the layer's matrix as fp64 values (a q8_row matrix dequantised)
+        if q8 and name in synth.Q8_MATS:
+            return lw[name].astype(np.float64) * lw[name + "_scale"].astype(np.float64)[:, None]
+        return f(lw[name])
+
+    def post(Y, g):  # sandwich norm: RMS-normalised, not rounded
+        return Y / np.sqrt(np.mean(Y * Y, axis=1, keepdims=True) + eps) * g.astype(np.float64)
+
+    for li, lw in enumerate(w["layers"]):
+        W_l = 0
+        if cfg.get("sliding_window", 0) and (li + 1) % max(cfg.get("swa_pattern", 0), 1) != 0:
+            W_l = cfg["sliding_window"]
         xn = norm(X, lw["attn_norm"])
-        qkv = xn @ f(lw["wqkv"]).T
+        qkv = xn @ mat(lw, "wqkv").T
         if cfg.get("qkv_bias"):
             qkv = qkv + lw["bqkv"].astype(np.float64)
         q = qkv[:, : nq * d].reshape(T, nq, d)
@@ -568,24 +726,46 @@ def _textbook_forward(cfg, w, toks):
                 return M / np.sqrt(np.mean(M * M, axis=-1, keepdims=True) + eps) * g.astype(np.float64)
             q, k = head_norm(q, lw["q_norm"]), head_norm(k, lw["k_norm"])
         q, k, v = torch_bf16(rope(q)), torch_bf16(rope(k)), torch_bf16(v)
-        o = _brute_force_causal(q, k, v, nq, nkv, 1 / math.sqrt(d))
-        X = X + torch_bf16(o.reshape(T, nq * d)) @ f(lw["wo"]).T
+        o = _brute_force_causal(q, k, v, nq, nkv, 1 / math.sqrt(d), W_l, cfg.get("attn_softcap", 0.0))
+        ao = torch_bf16(o.reshape(T, nq * d)) @ mat(lw, "wo").T
+        X = X + (post(ao, lw["post_attn_norm"]) if cfg.get("sandwich") else ao)
         xn = norm(X, lw["ffn_norm"])
         if cfg.get("n_experts", 0):
             ffn = np.stack([oracle.moe_ffn(cfg, lw, xn[t])[0] for t in range(T)])
         else:
-            g, u = xn @ f(lw["w_gate"]).T, xn @ f(lw["w_up"]).T
-            ffn = torch_bf16(g / (1 + np.exp(-g)) * u) @ f(lw["w_down"]).T
+            g, u = xn @ mat(lw, "w_gate").T, xn @ mat(lw, "w_up").T
+            ffn = torch_bf16(g / (1 + np.exp(-g)) * u) @ mat(lw, "w_down").T
+            if cfg.get("sandwich"):
+                ffn = post(ffn, lw["post_ffn_norm"])
         X = X + ffn
     xf = norm(X[-1:], w["final_norm"])
-    head = w["embed"] if cfg.get("tied") else w["lm_head"]
-    return (xf @ f(head).T)[0]
+    if cfg.get("tied"):
+        head = f(w["embed"])
+    elif q8:
+        head = w["lm_head"].astype(np.float64) * w["lm_head_scale"].astype(np.float64)[:, None]
+    else:
+        head = f(w["lm_head"])
+    logits = (xf @ head.T)[0]
+    cap = cfg.get("final_softcap", 0.0)
+    return cap * np.tanh(logits / cap) if cap else logits
 
 
-@pytest.mark.parametrize("variant", ["dense", "tied_bias", "qknorm", "qknorm_bias", "moe", "moe_qknorm_bias"])
+@pytest.mark.parametrize("variant", ["dense", "tied_bias", "qknorm", "qknorm_bias", "moe", "moe_qknorm_bias",
+                                     "swa_softcaps_sandwich", "swa_every_layer", "q8", "q8_swa_sandwich"])
 def test_oracle_matches_whole_sequence_matrix_form(variant):
     if variant == "dense":
         cfg = _small_dense()
+    elif variant == "swa_softcaps_sandwich":
+        # layers 0 and 2 windowed (3 keys), layer 1 global; scores capped at 0.9 (the scores
+        # of this model reach a few units, so the cap bends them); logits capped at 0.5
+        cfg = dict(_small_dense(qk_norm=1), layers=3, sliding_window=3, swa_pattern=2, attn_softcap=0.9,
+                   final_softcap=0.5, sandwich=1)
+    elif variant == "swa_every_layer":
+        cfg = _small_dense(sliding_window=4, swa_pattern=5, attn_softcap=2.0)
+    elif variant == "q8":
+        cfg = _small_dense(weight_format=1)
+    elif variant == "q8_swa_sandwich":
+        cfg = _small_dense(weight_format=1, sliding_window=2, swa_pattern=2, sandwich=1, final_softcap=3.0)
     elif variant == "tied_bias":
         cfg = _small_dense(tied=1, qkv_bias=1, rope_base=500000.0)
     elif variant == "qknorm":
@@ -599,7 +779,10 @@ def test_oracle_matches_whole_sequence_matrix_form(variant):
         cfg = dict(_moe_cfg(E=6, k=2), hidden=32, layers=2, n_q_heads=4, n_kv_heads=4, head_dim=8,
                    qkv_bias=1, vocab=48, max_context=16)
     w = synth.make_weights(cfg, seed=14)
-    toks = synth.tokens(9, cfg["vocab"], 1002)
+    # The matrix form sums in another order (fp64 differences ~1e-16). A value that close to
+    # a bf16 rounding boundary rounds the other way and moves the logits by ~1e-4: prompt
+    # 1002 meets one such value in the q8 + window + sandwich model, so that model uses 1003.
+    toks = synth.tokens(9, cfg["vocab"], 1003 if variant == "q8_swa_sandwich" else 1002)
     got = oracle.Model(cfg, w).prefill(0, toks, 0)
     want = _textbook_forward(cfg, w, toks)
     assert np.allclose(got, want, rtol=1e-9, atol=1e-11)
