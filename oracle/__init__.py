@@ -95,6 +95,7 @@ def _declare(L):
     L.orc_layer_window.argtypes = [C.POINTER(Config), C.c_int]
     L.orc_route_topk.argtypes = [_P, C.c_int, C.c_int, C.c_int, _P, _P, _P]
     L.orc_swiglu.argtypes = [_P, _P, _P, _P, C.c_int, C.c_int, _P]
+    L.orc_swiglu_act.argtypes = [_P, _P, _P, C.c_int, C.c_int, _P]
     L.orc_moe_ffn.argtypes = [C.POINTER(Config), C.POINTER(Layer), _P, _P, _P, _P, _P]
     L.orc_create.restype = _P
     L.orc_create.argtypes = [C.POINTER(Config), C.POINTER(Weights), C.POINTER(Layer), C.c_int]
@@ -210,6 +211,15 @@ def swiglu(x, Wg, Wu, Wd) -> np.ndarray:
     Wg, Wu, Wd = (_c(a, np.uint16) for a in (Wg, Wu, Wd))
     out = np.empty(Wd.shape[0], np.float64)
     lib().orc_swiglu(_p(x), _p(Wg), _p(Wu), _p(Wd), Wg.shape[0], Wg.shape[1], _p(out))
+    return out
+
+
+def swiglu_act(x, Wg, Wu) -> np.ndarray:
+    """The SwiGLU activation R4(silu(Wg x) * (Wu x)) [I] (before the down projection)."""
+    x = _c(x, np.float64)
+    Wg, Wu = _c(Wg, np.uint16), _c(Wu, np.uint16)
+    out = np.empty(Wg.shape[0], np.float64)
+    lib().orc_swiglu_act(_p(x), _p(Wg), _p(Wu), Wg.shape[0], Wg.shape[1], _p(out))
     return out
 
 

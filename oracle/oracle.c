@@ -236,17 +236,30 @@ static void matvec_w(const uint16_t* W, const int8_t* Q, const float* S, int64_t
         orc_matvec(W, N, K, x, y);
 }
 
+/* The SwiGLU activation a = R4(silu(Wg x) * (Wu x)) [I]; u is scratch [I]. */
+static void swiglu_act_w(const double* x, const uint16_t* Wg, const int8_t* Qg, const float* Sg, const uint16_t* Wu,
+                         const int8_t* Qu, const float* Su, int I, int h, double* g, double* u) {
+    matvec_w(Wg, Qg, Sg, I, h, x, g);
+    matvec_w(Wu, Qu, Su, I, h, x, u);
+    for (int i = 0; i < I; ++i) g[i] = orc_bf16(silu(g[i]) * u[i]);
+}
+
 /* SwiGLU with each of the three matrices bf16 or q8_row. */
 static void swiglu_w(const double* x, const uint16_t* Wg, const int8_t* Qg, const float* Sg, const uint16_t* Wu,
                      const int8_t* Qu, const float* Su, const uint16_t* Wd, const int8_t* Qd, const float* Sd, int I,
                      int h, double* out) {
     double* g = (double*)malloc(sizeof(double) * (size_t)I);
     double* u = (double*)malloc(sizeof(double) * (size_t)I);
-    matvec_w(Wg, Qg, Sg, I, h, x, g);
-    matvec_w(Wu, Qu, Su, I, h, x, u);
-    for (int i = 0; i < I; ++i) g[i] = orc_bf16(silu(g[i]) * u[i]);
+    swiglu_act_w(x, Wg, Qg, Sg, Wu, Qu, Su, I, h, g, u);
     matvec_w(Wd, Qd, Sd, h, I, g, out);
     free(g);
+    free(u);
+}
+
+/* The activation alone: act = R4(silu(Wg x) * (Wu x)); Wg, Wu [I][h]. */
+void orc_swiglu_act(const double* x, const uint16_t* Wg, const uint16_t* Wu, int I, int h, double* act) {
+    double* u = (double*)malloc(sizeof(double) * (size_t)I);
+    swiglu_act_w(x, Wg, NULL, NULL, Wu, NULL, NULL, I, h, act, u);
     free(u);
 }
 

@@ -85,6 +85,7 @@ int orc_layer_window(const orc_config* c, int layer);
 void orc_route_topk(const double* logits, int E, int k, int renorm, int32_t* idx, double* w, double* gap);
 void orc_swiglu(const double* x, const uint16_t* Wg, const uint16_t* Wu, const uint16_t* Wd, int I, int h,
                 double* out);
+void orc_swiglu_act(const double* x, const uint16_t* Wg, const uint16_t* Wu, int I, int h, double* act);
 
 void orc_moe_ffn(const orc_config* c, const orc_layer* L, const double* xn, double* out, int32_t* idx, double* w,
                  double* gap);

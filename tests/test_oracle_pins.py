@@ -350,6 +350,20 @@ def test_swiglu_zero_gate_or_zero_up_gives_zero():
     assert not oracle.swiglu(x, W, Z, Wd).any()
 
 
+def test_swiglu_is_the_down_projection_of_its_activation():
+    rng = np.random.default_rng(70)
+    h, I = 24, 40
+    x = f(rnd_bf16_bits(h, 71))
+    Wg, Wu = rnd_bf16_bits((I, h), 72, 0.3), rnd_bf16_bits((I, h), 73, 0.3)
+    Wd = rnd_bf16_bits((h, I), 74, 0.3)
+    act = oracle.swiglu_act(x, Wg, Wu)
+    assert np.array_equal(act, torch_bf16(act))  # R4: bf16 values
+    assert np.allclose(oracle.swiglu(x, Wg, Wu, Wd), f(Wd) @ act, rtol=1e-13, atol=1e-15)
+    z = f(Wg) @ x
+    u = f(Wu) @ x
+    assert np.allclose(act, torch_bf16(z / (1 + np.exp(-z)) * u), rtol=0, atol=1e-12)
+
+
 def test_swiglu_gate_and_up_are_not_swapped():
     # silu is not symmetric: silu(g) * u != silu(u) * g in general.
     h, I = 8, 4
