@@ -85,22 +85,34 @@ def measured_traffic():
 
 
 def layer_bytes(cfg):
+    """Projection weight bytes of one layer: bf16, or q8_row (1 byte per weight + a 4-byte scale
+    per row)."""
     h, d, nq, nkv, I = cfg["hidden"], cfg["head_dim"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["ffn_inter"]
-    qkv = (nq * d + 2 * nkv * d) * h
-    return 2 * (qkv + h * nq * d + 3 * I * h)
+    qkv_rows = nq * d + 2 * nkv * d
+    params = qkv_rows * h + h * nq * d + 3 * I * h
+    if cfg.get("weight_format", 0) == 1:
+        return params + 4 * (qkv_rows + h + 2 * I + h)
+    return 2 * params
 
 
 def step_bytes(cfg, B, ctx_list):
     """Algorithmic bytes of one decode step: every weight once + each sequence's KV once."""
     L, h, V = cfg["layers"], cfg["hidden"], cfg["vocab"]
     kv_row = 2 * cfg["n_kv_heads"] * cfg["head_dim"] * 2  # k + v, bf16
-    weights = L * layer_bytes(cfg) + V * h * 2 + L * 2 * h * 4 + h * 4
+    head = V * h + 4 * V if cfg.get("weight_format", 0) == 1 else V * h * 2
+    weights = L * layer_bytes(cfg) + head + L * 2 * h * 4 + h * 4
     kv = sum(L * c * kv_row for c in ctx_list)
     return weights, kv
 
 
+def prefill_weight_bytes(cfg):
+    """Weight bytes the tensor-core GEMMs read per chunk (bf16: q8_row models keep their
+    integers in bf16 for the tensor pipe)."""
+    return cfg["layers"] * layer_bytes(dict(cfg, weight_format=0))
+
+
 def gemm_flops_per_token(cfg):
-    return 2 * (layer_bytes(cfg) // 2 * cfg["layers"])
+    return 2 * (layer_bytes(dict(cfg, weight_format=0)) // 2 * cfg["layers"])
 
 
 def attn_flops_prefill(cfg, T):
@@ -162,14 +174,27 @@ def make_device_weights(cfg, torch, seed=0):
         keep.append(t)
         return t
 
+    q8 = cfg.get("weight_format", 0) == 1
+
+    def q8mat(shape, tid, scale_tid):
+        t = torch.empty(shape, dtype=torch.int8, device="cuda")
+        assert dl.syn_dev_fill_i8(t.data_ptr(), t.numel(), seed, tid, synth.Q8_STD, st) == 0
+        keep.append(t)
+        return t, vec(shape[0], scale_tid, synth.WEIGHT_STD / synth.Q8_STD, 0.1 * synth.WEIGHT_STD / synth.Q8_STD)
+
     h, V = cfg["hidden"], cfg["vocab"]
     w = dict(embed=mat((V, h), 1), lm_head=None if cfg.get("tied") else mat((V, h), 2),
              final_norm=vec(h, 3, 1.0, synth.GAIN_STD), layers=[])
+    if q8 and not cfg.get("tied"):
+        w["lm_head"], w["lm_head_scale"] = q8mat((V, h), 2, 4)
     for l in range(cfg["layers"]):
         lw = {}
         for name, shape in synth.tensor_shapes(cfg).items():
             if shape is None:
                 lw[name] = None
+            elif q8 and name in synth.Q8_MATS:
+                tid = synth.layer_tid(l, name)
+                lw[name], lw[name + "_scale"] = q8mat(shape, tid, tid + 50)
             elif name in synth.GAINS:
                 lw[name] = vec(shape[0], synth.layer_tid(l, name), 1.0, synth.GAIN_STD)
             elif name in synth.VECTORS:
@@ -189,26 +214,46 @@ def make_device_weights(cfg, torch, seed=0):
     return w
 
 
-def time_gemv(dec, torch, N, K, reps=20):
-    """Average device time of the weight-streaming GEMV on one [N][K] matrix at B=1 (CUDA events
-    on the launching stream); the inputs rotate over buffers larger than L2."""
-    nbuf = max(2, int(math.ceil(300e6 / (N * K * 2))))
-    Ws = [torch.empty((N, K), dtype=torch.bfloat16, device="cuda").normal_(0, 0.02) for _ in range(nbuf)]
-    x = torch.randn((1, K), device="cuda").to(torch.bfloat16)
-    y = torch.empty((1, N), device="cuda")
+def _time_launches(torch, call, nbuf, reps):
+    """Average device time of `reps` launches of call(i) (CUDA events on the launching stream)."""
     for i in range(3):
-        dec.weight_gemv(Ws[i % nbuf], x, y)
+        call(i % nbuf)
     s = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(s)
     for i in range(reps):
-        dec.weight_gemv(Ws[i % nbuf], x, y)
+        call(i % nbuf)
     e1.record(s)
     e1.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+    return e0.elapsed_time(e1) / reps
+
+
+def time_gate_up(dec, torch, I, K, reps=20):
+    """The decode step's dominant launch, alone: gemv_kernel<1, SWIGLU> with its fused RMSNorm
+    prologue (ffn_gate_up) on the interleaved [2I][K] gate/up matrix at B = 1; the weights rotate
+    over copies larger than L2. Returns (ms, algorithmic bytes per launch)."""
+    nbuf = max(2, int(math.ceil(300e6 / (2 * I * K * 2))))
+    Ws = [torch.empty((2 * I, K), dtype=torch.bfloat16, device="cuda").normal_(0, 0.02) for _ in range(nbuf)]
+    x = torch.randn((1, K), device="cuda") * 3
+    g = torch.ones(K, device="cuda")
+    act = torch.empty((1, I), dtype=torch.bfloat16, device="cuda")
+    ms = _time_launches(torch, lambda i: dec.ffn_gate_up(Ws[i], x, g, 1e-5, act), nbuf, reps)
     del Ws
-    return ms, N * K * 2 + K * 2 + N * 4
+    return ms, 2 * I * K * 2 + K * 4 + K * 4 + I * 2
+
+
+def time_gemv_q8(dec, torch, N, K, reps=20):
+    """The q8_row GEMV (weight_gemv_q8, store epilogue) on one int8 [N][K] matrix at B = 1 on
+    rotating copies larger than L2. Returns (ms, algorithmic bytes per launch)."""
+    nbuf = max(2, int(math.ceil(300e6 / (N * K))))
+    Ws = [torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda") for _ in range(nbuf)]
+    sc = torch.full((N,), 0.02 / 32, device="cuda")
+    x = torch.randn((1, K), device="cuda").to(torch.bfloat16)
+    y = torch.empty((1, N), device="cuda")
+    ms = _time_launches(torch, lambda i: dec.weight_gemv_q8(Ws[i], sc, x, y), nbuf, reps)
+    del Ws
+    return ms, N * K + N * 4 + K * 2 + N * 4
 
 
 def cpu_oracle_sample(cfg, ctx):
@@ -271,6 +316,11 @@ WORKLOADS = {
     # standalone weight-streaming GEMV on the gate/up matrix of the Llama-3-8B shape (the
     # default line's roofline kernel, launched the way its `achieved` figure is timed)
     "gemv-gate-up": dict(),
+    # the headline decode line with q8_row weights (int8 rows, fp32 row scales)
+    "llama3-8b-q8": dict(),
+    # the CPU oracle's own throughput on the tiny, SmolLM2-135M and Qwen1.5-MoE shapes (B = 1),
+    # on this host's cores: a baseline, not the target
+    "oracle-baselines": dict(),
     # 4096-token prefill of the Llama-3-8B shape with longer chunks: the projections become
     # compute-bound GEMMs (the chunk-128 line is HBM-bound)
     "llama3-8b-prefill-c512": dict(prefill_chunk=512),
@@ -347,23 +397,69 @@ def run_prefill_workload(args, torch, dec, P):
     return 0
 
 
+def run_oracle_baselines(args):
+    """The fp64 oracle as it stands, timed on this host: prefill tok/s and batch-1 decode tok/s
+    of the tiny, SmolLM2-135M and Qwen1.5-MoE-A2.7B shapes. Prefill is timed on a 128-token
+    sample for SmolLM2 (every token costs the same weights; attention grows slowly at these
+    lengths); decode at the workload's context over a synthetic cache."""
+    import oracle
+    rows = []
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    for name, cfg, n_prompt, ctx in (("tiny", dict(configs.TINY), 16, 16),
+                                     ("smollm2-135m", dict(configs.SMOLLM2_135M, max_context=1040), 128, 1024),
+                                     ("qwen1.5-moe-a2.7b", dict(configs.QWEN15_MOE_A27B, max_context=2056), 0, 2048)):
+        w = synth.make_weights(cfg)
+        m = oracle.Model(cfg, w)
+        row = dict(model=name)
+        if n_prompt:
+            toks = synth.tokens(n_prompt, cfg["vocab"], 1000)
+            t0 = time.perf_counter()
+            m.prefill(0, toks, 0)
+            row["prefill_tok_s"] = round(n_prompt / (time.perf_counter() - t0), 2)
+            row["prefill_tokens"] = n_prompt
+        kvd = cfg["n_kv_heads"] * cfg["head_dim"]
+        if ctx > n_prompt:
+            for l in range(cfg["layers"]):
+                k, v = synth.kv_fill(ctx, kvd, 2000, l)
+                m.kv_write(0, l, 0, k, v)
+        steps = 3
+        t0 = time.perf_counter()
+        for s in range(steps):
+            m.forward(0, 1 + s, ctx + s)
+        row["decode_tok_s"] = round(steps / (time.perf_counter() - t0), 3)
+        row["decode_ctx"] = ctx
+        rows.append(row)
+        m.close()
+        del w
+    print(json.dumps(dict(metric="CPU oracle tok/s (fp64, batch 1)", value=rows[-1]["decode_tok_s"], unit="tok/s",
+                          n_gpus=0, steps=3, warmup=0, higher_is_better=True, dtype="f64", data="synthetic",
+                          cpu_baseline=dict(kind="oracle", cores=threads), points=rows)))
+    return 0
+
+
 def run_workload(args, torch, dec):
     name = args.workload
+    if name == "oracle-baselines":
+        return run_oracle_baselines(args)
     P = peaks()
     W, K = max(3, args.warmup), max(1, args.steps)
     if name == "gqa-sweep":
         return run_gqa_sweep(args, torch, dec, P)
     if name == "gemv-gate-up":
-        N, Kd = 2 * configs.LLAMA3_8B["ffn_inter"], configs.LLAMA3_8B["hidden"]
-        ms, byt = time_gemv(dec, torch, N, Kd, reps=K)
+        I, Kd = configs.LLAMA3_8B["ffn_inter"], configs.LLAMA3_8B["hidden"]
+        ms, byt = time_gate_up(dec, torch, I, Kd, reps=K)
         gbs = byt / (ms * 1e-3) / 1e9
-        print(json.dumps(dict(metric=f"weight-streaming GEMV GB/s ([{N}][{Kd}] bf16, batch 1)", value=round(gbs, 1),
-                              unit="GB/s", n_gpus=1, steps=K, warmup=3, ms_per_step=ms, higher_is_better=True,
-                              scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-                              config=dict(workload=f"gemv [{N}][{Kd}] x [1][{Kd}]", l2="rotating weights > L2"),
+        print(json.dumps(dict(metric=f"fused norm + gate/up + SiLU GEMV GB/s ([{2 * I}][{Kd}] bf16, batch 1)",
+                              value=round(gbs, 1), unit="GB/s", n_gpus=1, steps=K, warmup=3, ms_per_step=ms,
+                              higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+                              data="synthetic",
+                              config=dict(workload=f"ffn_gate_up [{2 * I}][{Kd}] x [1][{Kd}]",
+                                          l2="rotating weights > L2"),
                               roofline=dict(bound="hbm", achieved=round(gbs, 1), peak=P["hbm"], unit="GB/s",
                                             frac=round(gbs / P["hbm"], 4), peak_source=P["src"]))))
         return 0
+    if name == "llama3-8b-q8":
+        return run_headline(args, torch, dec, q8=True)
     if "prefill_chunk" in WORKLOADS[name]:
         return run_prefill_workload(args, torch, dec, P)
     spec = WORKLOADS[name]
@@ -530,6 +626,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-c4096", action="store_true", help="skip the one-chunk 4096-token prefill sub-object")
     ap.add_argument("--layers", type=int, default=0, help="fewer layers (profiling only; not a bench number)")
     ap.add_argument("--breakdown", action="store_true",
                     help="decode workloads: after the timed region, per-kernel exclusive times of a few more "
@@ -541,17 +638,51 @@ def main():
         return run_reference(args)
 
     import torch
-    import torch.distributed as dist
 
     import decoder_only_transformer_layer_b200 as dec
 
     if args.workload != "llama3-8b":
         return run_workload(args, torch, dec)
+    return run_headline(args, torch, dec)
 
+
+def time_prefill_c4096(torch, dec, weights, P, runs=2):
+    """The 4096-token prefill in ONE chunk of 4096 (same weights): every projection is a
+    compute-bound tcgen05 GEMM, the configuration where the tensor-core target applies."""
+    cfg = dict(configs.LLAMA3_8B, max_context=PROMPT + 8, max_batch=1, prefill_chunk=PROMPT)
+    d = dec.Decoder(cfg, weights)
+    stream = torch.cuda.current_stream()
+    prompt = synth.tokens(PROMPT, cfg["vocab"], 1000)
+    d.prefill(0, prompt, 0)  # warm-up
+    d.reset(0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(runs):
+        torch.cuda.synchronize()
+        e0.record(stream)
+        d.prefill(0, prompt, 0)
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+        d.reset(0)
+    d.close()
+    ms = statistics.mean(times)
+    flops = gemm_flops_per_token(cfg) * PROMPT + attn_flops_prefill(cfg, PROMPT)
+    tf = flops / (ms * 1e-3) / 1e12
+    return dict(tokens=PROMPT, chunk=PROMPT, ms=round(ms, 2), tok_s=round(PROMPT / (ms * 1e-3), 1),
+                tflops=round(tf, 1), tc_frac_sustained=round(tf / P["tc_sus"], 4),
+                tc_frac_burst=round(tf / P["tc"], 4), tc_peak_sustained=P["tc_sus"], tc_peak_burst=P["tc"],
+                bar_uses="sustained: 64 GEMM launches back to back for tens of ms under the power cap")
+
+
+def run_headline(args, torch, dec, q8=False):
+    """Llama-3-8B shape: 4096-token prefill (chunk 128), then batch-1 greedy decode at context
+    4096+. With q8 the projections and the LM head are q8_row (int8 rows, fp32 row scales)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
+    import torch.distributed as dist
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
@@ -563,12 +694,15 @@ def main():
     W = max(3, args.warmup)
     K = max(1, args.steps)
     e2e_steps = min(K, 16)
-    cfg = dict(configs.LLAMA3_8B, max_context=PROMPT + W + K + e2e_steps + 8, max_batch=1, prefill_chunk=128)
+    cfg = dict(configs.LLAMA3_8B, max_context=PROMPT + W + K + e2e_steps + 16, max_batch=1, prefill_chunk=128,
+               weight_format=1 if q8 else 0)
     if args.layers:
         cfg = configs.with_layers(cfg, args.layers)
     weights = make_device_weights(cfg, torch)
     d = dec.Decoder(cfg, weights)
-    del weights
+    if q8 or args.layers or args.no_c4096:
+        del weights
+        weights = None
     torch.cuda.empty_cache()
     stream = torch.cuda.current_stream()
     prompt = synth.tokens(PROMPT, cfg["vocab"], 1000)
@@ -622,11 +756,35 @@ def main():
     e2e_s = (time.perf_counter() - t0) / e2e_steps
     if world > 1:
         (e2e_s,) = max_over_ranks([e2e_s], "cuda")
+    if args.breakdown and rank == 0:  # after every timed region: per-kernel shares
+        state = dict(tok=tok, pos=pos)
 
-    # ---- dominant kernel alone: weight-streaming GEMV on the fused gate/up matrix
+        def one_step():
+            d.step([state["tok"]], [state["pos"]])
+            state["pos"] += 1
+        kernel_breakdown(torch, one_step, 4, f"decode b=1 ({cfg['layers']} layers)")
+        d.reset(0)
+        kernel_breakdown(torch, lambda: d.prefill(0, prompt, 0), 1, f"prefill {PROMPT} tokens, chunk 128")
+    d.close()
+
+    # ---- dominant kernel alone: the decode step's gate/up launch
     P = peaks()
-    gemv_ms, gemv_bytes = time_gemv(dec, torch, 2 * cfg["ffn_inter"], cfg["hidden"])
-    gemv_gbs = gemv_bytes / (gemv_ms * 1e-3) / 1e9
+    I, Kd = cfg["ffn_inter"], cfg["hidden"]
+    if q8:
+        k_ms, k_bytes = time_gemv_q8(dec, torch, 2 * I, Kd)
+        k_name = f"gemv_kernel<1,STORE,q8> (weight_gemv_q8) on int8 [{2 * I}][{Kd}] + row scales"
+    else:
+        k_ms, k_bytes = time_gate_up(dec, torch, I, Kd)
+        k_name = (f"gemv_kernel<1,SWIGLU> with the fused RMSNorm prologue (ffn_gate_up: the decode step's "
+                  f"gate/up launch) on [{2 * I}][{Kd}] bf16")
+    k_gbs = k_bytes / (k_ms * 1e-3) / 1e9
+
+    # ---- the same prompt prefilled in one 4096-token chunk (tensor-core bound GEMMs)
+    c4096 = None
+    if weights is not None:
+        torch.cuda.synchronize()
+        c4096 = time_prefill_c4096(torch, dec, weights, P)
+        del weights
 
     wbytes, kvbytes = step_bytes(cfg, 1, ctx_list)
     step_gbs = (wbytes + kvbytes / K) / (ms_step * 1e-3) / 1e9
@@ -634,22 +792,25 @@ def main():
     pf_tok_s = replica_throughput(PROMPT, world, prefill_ms)
     pf_flops = gemm_flops_per_token(cfg) * PROMPT + attn_flops_prefill(cfg, PROMPT)
     pf_tflops = pf_flops / (prefill_ms * 1e-3) / 1e12
-    chunk_hbm_floor_ms = (PROMPT / 128) * (cfg["layers"] * layer_bytes(cfg)) / (P["hbm"] * 1e9) * 1e3
+    chunk_hbm_floor_ms = (PROMPT / 128) * prefill_weight_bytes(cfg) / (P["hbm"] * 1e9) * 1e3
     launches_per_step = 1 + 5 * cfg["layers"] + 2
 
     cpu_b = None
-    if rank == 0 and not args.no_cpu_baseline and not args.layers:
+    if rank == 0 and not args.no_cpu_baseline and not args.layers and not q8:
         cpu_b = cpu_oracle_sample(dict(configs.LLAMA3_8B), PROMPT)
     if rank == 0:
+        metric = METRIC if not q8 else "decode tok/s + % HBM roofline (8B-shape, b=1, q8_row weights)"
         line = dict(
-            metric=METRIC, value=value, unit="tok/s", n_gpus=world, steps=K, warmup=W, ms_per_step=ms_step,
-            higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-            config=main_config(world, cfg["layers"]),
-            roofline=dict(bound="hbm", achieved=round(gemv_gbs, 1), peak=P["hbm"], unit="GB/s",
-                          frac=round(gemv_gbs / P["hbm"], 4), traffic=measured_traffic(),
-                          traffic_unit="bytes per launch (ncu dram read+write)",
-                          kernel=f"gemv_kernel<1,SWIGLU-shaped> on [{2 * cfg['ffn_inter']}][{cfg['hidden']}] bf16",
-                          peak_source=P["src"]),
+            metric=metric, value=value, unit="tok/s", n_gpus=world, steps=K, warmup=W, ms_per_step=ms_step,
+            higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16" if not q8 else "int8xbf16",
+            data="synthetic",
+            config=main_config(world, cfg["layers"]) if not q8 else dict(
+                main_config(world, cfg["layers"]), workload="llama3-8b-shape, q8_row projections and LM head, "
+                                                            "decode b=1 at context 4096 after a 4096-token prefill"),
+            roofline=dict(bound="hbm", achieved=round(k_gbs, 1), peak=P["hbm"], unit="GB/s",
+                          frac=round(k_gbs / P["hbm"], 4), traffic=None if q8 else measured_traffic(),
+                          traffic_unit="bytes per launch (ncu dram read+write)", kernel=k_name,
+                          algorithmic_bytes=k_bytes, launch_us=round(k_ms * 1e3, 2), peak_source=P["src"]),
             step_roofline=dict(bytes_per_step=wbytes + kvbytes / K, achieved_gbs=round(step_gbs, 1),
                                frac=round(step_gbs / P["hbm"], 4), peak=P["hbm"], unit="GB/s"),
             prefill=dict(tokens=PROMPT, chunk=128, ms=round(prefill_ms, 2), tok_s=round(pf_tok_s, 1),
@@ -659,8 +820,9 @@ def main():
             cpu_baseline=cpu_b,
             e2e=dict(value=world / e2e_s, unit="tok/s", h2d_bytes_per_step=8, d2h_bytes_per_step=4 * cfg["vocab"]),
             gpu_launches=launches_per_step * K, clocks=clocks)
+        if c4096:
+            line["prefill_c4096"] = c4096
         print(json.dumps(line))
-    d.close()
     if world > 1:
         dist.destroy_process_group()
     return 0

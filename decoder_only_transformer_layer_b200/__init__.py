@@ -14,7 +14,8 @@ import numpy as np
 
 from ._build import LIB, build, stale  # noqa: F401
 
-__all__ = ["lib", "Decoder", "DecError", "gqa_decode_attn", "moe_route_topk", "moe_experts", "weight_gemv", "STATUS"]
+__all__ = ["lib", "Decoder", "DecError", "gqa_decode_attn", "moe_route_topk", "moe_experts", "weight_gemv",
+           "weight_gemv_q8", "ffn_gate_up", "check_standalone", "STATUS"]
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "CONTEXT_OVERFLOW", 3: "PAGES_EXHAUSTED", 4: "OOM", 5: "CUDA",
           6: "TIMEOUT", 7: "UNSUPPORTED"}
@@ -32,11 +33,16 @@ class Config(C.Structure):
         "hidden", "layers", "n_q_heads", "n_kv_heads", "head_dim", "ffn_inter", "vocab",
         "tied_embeddings", "qkv_bias", "qk_norm", "n_experts", "top_k", "expert_inter", "shared_inter",
         "shared_gate", "norm_topk_prob")] + [("rms_eps", C.c_float), ("rope_base", C.c_float)] + \
-        [(n, C.c_int32) for n in ("max_batch", "max_context", "page_size", "prefill_chunk", "n_pages")]
+        [(n, C.c_int32) for n in ("max_batch", "max_context", "page_size", "prefill_chunk", "n_pages",
+                                  "sliding_window", "swa_pattern")] + \
+        [("attn_softcap", C.c_float), ("final_softcap", C.c_float), ("sandwich_norms", C.c_int32),
+         ("weight_format", C.c_int32)]
 
 
 LAYER_FIELDS = ("attn_norm", "ffn_norm", "wqkv", "bqkv", "q_norm", "k_norm", "wo", "w_gate", "w_up", "w_down",
-                "w_router", "e_gate", "e_up", "e_down", "s_gate", "s_up", "s_down", "s_gate_vec")
+                "w_router", "e_gate", "e_up", "e_down", "s_gate", "s_up", "s_down", "s_gate_vec",
+                "post_attn_norm", "post_ffn_norm", "wqkv_scale", "wo_scale", "w_gate_scale", "w_up_scale",
+                "w_down_scale")
 
 
 class LayerWeights(C.Structure):
@@ -45,7 +51,7 @@ class LayerWeights(C.Structure):
 
 class Weights(C.Structure):
     _fields_ = [("embed", C.c_void_p), ("lm_head", C.c_void_p), ("final_norm", C.c_void_p),
-                ("layers", C.POINTER(LayerWeights))]
+                ("layers", C.POINTER(LayerWeights)), ("lm_head_scale", C.c_void_p)]
 
 
 _P = C.c_void_p
@@ -77,10 +83,19 @@ def lib():
         L.gqa_decode_attn_noalloc.argtypes = L.gqa_decode_attn.argtypes
         L.moe_route_topk.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
         L.weight_gemv.argtypes = [_P, _P, _I, _I, _I, _P, _P]
+        L.weight_gemv_q8.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+        L.ffn_gate_up.argtypes = [_P, _P, _P, C.c_float, _I, _I, _I, _P, _P]
         L.moe_experts.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]
+        L.dec_check.argtypes = [_P]
+        L.dec_verify.argtypes = [_P, _I, _P, _I, _I, _P]
+        L.dec_truncate.argtypes = [_P, _I, _I]
+        L.dec_check_standalone.argtypes = [_P]
+        L.dec_test_fail_alloc.argtypes = [_I]
+        L.dec_test_gemm_wait.argtypes = [_I, C.c_int64]
         for f in ("dec_init", "dec_free", "dec_reset", "dec_prefill", "dec_step", "dec_last_argmax", "dec_kv_read",
                   "dec_kv_write", "dec_last_routes", "dec_last_hidden", "dec_seq_len", "gqa_decode_attn",
-                  "gqa_decode_attn_noalloc", "moe_route_topk", "moe_experts", "weight_gemv"):
+                  "gqa_decode_attn_noalloc", "moe_route_topk", "moe_experts", "weight_gemv", "dec_check",
+                  "dec_check_standalone", "dec_test_fail_alloc", "dec_test_gemm_wait", "dec_verify", "dec_truncate", "weight_gemv_q8", "ffn_gate_up"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -124,6 +139,9 @@ def make_config(cfg: dict) -> Config:
     c.max_batch, c.max_context = cfg.get("max_batch", 1), cfg["max_context"]
     c.page_size, c.prefill_chunk = cfg.get("page_size", 16), cfg.get("prefill_chunk", 128)
     c.n_pages = cfg.get("n_pages", 0)
+    c.sliding_window, c.swa_pattern = cfg.get("sliding_window", 0), cfg.get("swa_pattern", 0)
+    c.attn_softcap, c.final_softcap = cfg.get("attn_softcap", 0.0), cfg.get("final_softcap", 0.0)
+    c.sandwich_norms, c.weight_format = cfg.get("sandwich", 0), cfg.get("weight_format", 0)
     return c
 
 
@@ -148,6 +166,7 @@ class Decoder:
         w.lm_head = _ptr(weights.get("lm_head"))
         w.final_norm = _ptr(weights["final_norm"])
         w.layers = layers
+        w.lm_head_scale = _ptr(weights.get("lm_head_scale"))
         h = _P()
         _check(lib().dec_init(C.byref(self._cfg_c), C.byref(w), self.stream, C.byref(h)))
         self.h = h
@@ -188,10 +207,28 @@ class Decoder:
         self.step(tokens, pos, out)
         return out
 
+    def verify(self, seq: int, tokens, pos0: int, logits_out=None):
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        _check(lib().dec_verify(self.h, seq, toks.ctypes.data if toks.size else None, toks.size, pos0,
+                                _ptr(logits_out)))
+        return logits_out
+
+    def verify_logits(self, seq: int, tokens, pos0: int) -> np.ndarray:
+        out = np.empty((len(tokens), self.cfg["vocab"]), np.float32)
+        self.verify(seq, tokens, pos0, out)
+        return out
+
+    def truncate(self, seq: int, length: int):
+        _check(lib().dec_truncate(self.h, seq, length))
+
     def last_argmax(self, B: int) -> np.ndarray:
         out = np.empty(B, np.int32)
         _check(lib().dec_last_argmax(self.h, out.ctypes.data, B))
         return out
+
+    def check(self):
+        """Synchronise and raise DecError(TIMEOUT) if a device wait of an earlier call ran out."""
+        _check(lib().dec_check(self.h))
 
     def reset(self, seq: int = -1):
         _check(lib().dec_reset(self.h, seq))
@@ -276,3 +313,37 @@ def weight_gemv(W, x, y, stream=None):
     B = x.shape[0]
     _check(lib().weight_gemv(_ptr(W), _ptr(x), B, N, K, _ptr(y), _stream(stream)))
     return y
+
+
+def ffn_gate_up(Wgu, x, gain, eps, act, stream=None):
+    """Device tensors: Wgu bf16 [2I][K] (gate row i at 2i, up row i at 2i+1); x fp32 [B][K];
+    gain fp32 [K]; act bf16 [B][I] = bf16(SiLU(gate . xn) * (up . xn)), xn the RMS-normed x."""
+    I2, K = Wgu.shape
+    B = x.shape[0]
+    _check(lib().ffn_gate_up(_ptr(Wgu), _ptr(x), _ptr(gain), float(eps), B, I2 // 2, K, _ptr(act), _stream(stream)))
+    return act
+
+
+def weight_gemv_q8(Wq, scale, x, y, stream=None):
+    """Device tensors: Wq int8 [N][K]; scale fp32 [N]; x bf16 [B][K]; y fp32 [B][N]."""
+    N, K = Wq.shape
+    B = x.shape[0]
+    _check(lib().weight_gemv_q8(_ptr(Wq), _ptr(scale), _ptr(x), B, N, K, _ptr(y), _stream(stream)))
+    return y
+
+
+def check_standalone(stream=None):
+    """Synchronise `stream`; raise DecError(TIMEOUT) if a bounded device wait of a standalone
+    call on the current device ran out since the last check."""
+    _check(lib().dec_check_standalone(_stream(stream)))
+
+
+def test_fail_alloc(n: int):
+    """Test hook: the n-th device allocation of the library from now on fails (0 = off)."""
+    _check(lib().dec_test_fail_alloc(int(n)))
+
+
+def test_gemm_wait(extra_pieces: int, limit_cycles: int):
+    """Test hook: later tensor-core GEMM launches wait for pieces that never arrive and give
+    up after limit_cycles; (0, 0) restores normal operation."""
+    _check(lib().dec_test_gemm_wait(int(extra_pieces), int(limit_cycles)))

@@ -4,7 +4,9 @@
 // cpu.attentionPrefill; frink_models decoder.rs: gqa_attention / the CUDA
 // gqa_decode kernel; cortiq_engine pipeline.rs: attn_scale = 1/sqrt(head_dim)):
 //   q head h reads kv head g = h / (nq / nkv); the query at position p attends
-//   cache rows 0..p; o = sum_j softmax_j(q . k_j * scale) v_j.
+//   cache rows 0..p; o = sum_j softmax_j(q . k_j * scale) v_j. Optionally (ANEDVD's
+//   attentionDecode options .window and .logit_softcap; cortiq's per-layer window)
+//   only rows p-W+1..p are attended, and each scaled score s becomes c tanh(s / c).
 // Before attention q and the new k get an optional per-head RMSNorm (QK-norm)
 // and RoPE (half-split pairs (i, i + d/2), angle p * base^(-2i/d), evaluated in
 // fp64), and are rounded to bf16; k and v enter the cache once, at row p.
@@ -37,6 +39,13 @@ constexpr int kPage = 16;
 constexpr int kRing = 3;  // pages in flight per warp in the decode kernel
 constexpr int kDecodeMaxSplits = 16;  // context splits of one (sequence, kv head): one cluster
 constexpr float kLog2e = 1.4426950408889634f;
+
+// A raw q.k product -> the softmax argument in log2 units: times scale, then the logit
+// softcap c tanh(s / c) when c > 0.
+DEC_DEVINL float score_log2(float raw, float scale, float softcap) {
+    const float s = raw * scale;
+    return (softcap > 0.f ? softcap * tanhf(s / softcap) : s) * kLog2e;
+}
 
 // A warp transforms one head vector of D fp32 values: optional RMSNorm with weight
 // nw, optional RoPE at position pos, rounding to bf16. Lane l holds elements
@@ -73,6 +82,58 @@ DEC_DEVINL void head_transform(const float* vals_in, bool in_bf16, const uint16_
             } else {
                 rope_cs(pos, lane + 32 * m, D, base, &c, &s);
             }
+            const float x0 = v[m], x1 = v[m + E / 2];
+            v[m] = x0 * c - x1 * s;
+            v[m + E / 2] = x0 * s + x1 * c;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < E; ++m) dst[lane + 32 * m] = f2bf(v[m]);
+}
+
+// Per-position constants of head_transform, read before the grid-dependency wait (they do
+// not depend on the previous kernel): this lane's (cos, sin) pairs and norm gains.
+template <int D>
+struct HeadRegs {
+    float2 cs[D / 64];
+    float qn[D / 32], kn[D / 32];
+};
+
+template <int D>
+DEC_DEVINL void load_head_regs(HeadRegs<D>& r, const float2* tab, const float* qn, const float* kn) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int m = 0; m < D / 64; ++m) r.cs[m] = tab ? tab[lane + 32 * m] : make_float2(1.f, 0.f);
+#pragma unroll
+    for (int m = 0; m < D / 32; ++m) {
+        r.qn[m] = qn ? qn[lane + 32 * m] : 1.f;
+        r.kn[m] = kn ? kn[lane + 32 * m] : 1.f;
+    }
+}
+
+// head_transform with the norm gains (nw, or null for none) and the angles held in
+// registers: the same arithmetic in the same order.
+template <int D>
+DEC_DEVINL void head_transform_regs(const float* vals_in, const float* nw, bool norm, float eps, bool rope,
+                                    const float2* cs, uint16_t* dst) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+    float v[E];
+#pragma unroll
+    for (int m = 0; m < E; ++m) v[m] = vals_in[lane + 32 * m];
+    if (norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int m = 0; m < E; ++m) ss = fmaf(v[m], v[m], ss);
+        ss = warp_sum(ss);
+        const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+#pragma unroll
+        for (int m = 0; m < E; ++m) v[m] = v[m] * inv * nw[m];
+    }
+    if (rope) {
+#pragma unroll
+        for (int m = 0; m < E / 2; ++m) {
+            const float c = cs[m].x, s = cs[m].y;
             const float x0 = v[m], x1 = v[m + E / 2];
             v[m] = x0 * c - x1 * s;
             v[m + E / 2] = x0 * s + x1 * c;
@@ -186,51 +247,77 @@ DEC_DEVINL void load_page_warp(const uint16_t* kpool, const uint16_t* vpool, int
 
 // ================================================================== decode
 
-template <int D>
-__global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
+// Page ring depth per warp: 8-warp CTAs (split contexts, few pages each) keep 2 pages in
+// flight per warp, 4-warp CTAs (one CTA per sequence and kv head, many pages) keep 3.
+template <int NW>
+constexpr int kDecRing = NW >= 8 ? 2 : kRing;
+
+template <int D, int NW>
+__global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) {
     constexpr int LD = D + 8;
     constexpr int PAGE = kPage * LD;
     constexpr int LDR = D + 4;  // receive rows: o[D], m, l, 2 pad (16-byte aligned)
+    constexpr int RING = kDecRing<NW>;
+    constexpr int NT = NW * 32;
     __shared__ __align__(16) uint16_t qs[16 * LD];
     __shared__ __align__(16) uint16_t newkv[2][D];  // the appended k and v rows (bf16)
-    __shared__ float wm[4][16], wl[4][16];
+    __shared__ float wm[NW][16], wl[NW][16];
     extern __shared__ __align__(16) uint8_t dyn[];
-    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [4 warps][kRing][K,V][16][LD]
-    float* wo = reinterpret_cast<float*>(dyn);           // [4][16][D] after the page loop
-    float* recv = wo + 4 * 16 * D;                       // [rows owned][splits][LDR]
+    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [NW warps][RING][K,V][16][LD]
+    float* wo = reinterpret_cast<float*>(dyn);           // [NW][16][D] after the page loop
+    float* recv = wo + NW * 16 * D;                      // [rows owned][splits][LDR]
 
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z, S = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
     const int G = a.nq / a.nkv;
     // Without a scratch buffer the splits of one (sequence, kv head) form a cluster and
-    // merge in distributed shared memory; mark this CTA as running before any other CTA
-    // of the cluster writes into its shared memory.
+    // merge in distributed shared memory. The partials land in a receive area that overlaps
+    // the page rings, so a CTA arrives on the cluster barrier only once its page loop is
+    // done, and nobody writes into another CTA's shared memory before every CTA has arrived.
     const bool cl = S > 1 && a.part == nullptr;
-    if (cl) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     __shared__ int ticket_s;
 
     // ---- independent of the previous kernel: positions, block table and the cache pages
     // (the row being appended is patched in after it is written, below)
     const int p = a.pos[b];
     const int n = p + 1;
+    const int kf = a.window > 0 && n > a.window ? n - a.window : 0;  // first attended key
     const int np = (n + kPage - 1) / kPage;
-    const int pps = (np + S - 1) / S;
-    const int pg0 = s * pps, pg1 = min(np, pg0 + pps);
+    const int pf = kf / kPage;  // first page with an attended key
+    const int pps = (np - pf + S - 1) / S;
+    const int pg0 = pf + s * pps, pg1 = min(np, pg0 + pps);
     const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
     const bool has_last = pg0 < pg1 && pg1 == np;
     const float sl2 = a.scale * kLog2e;
-    // this warp's pages: pg0 + warp + 4 i, i < cnt; the first kRing are fetched now
-    uint16_t* wbuf = kvbuf + (size_t)warp * kRing * 2 * PAGE;
-    const int cnt = pg0 + warp < pg1 ? (pg1 - pg0 - warp + 3) / 4 : 0;
+    // this warp's pages: pg0 + warp + NW i, i < cnt; the first RING are fetched now. Lane j
+    // holds the block-table entry of page i = base + j and of page i = base + 32 + j, so a
+    // refill never waits on a block-table load (the next 32 are fetched 32 pages ahead).
+    uint16_t* wbuf = kvbuf + (size_t)warp * RING * 2 * PAGE;
+    const int cnt = pg0 + warp < pg1 ? (pg1 - pg0 - warp + NW - 1) / NW : 0;
+    int bt_base = 0;
+    int bt_cur = lane < cnt ? bt[pg0 + warp + NW * lane] : 0;
+    int bt_next = lane + 32 < cnt ? bt[pg0 + warp + NW * (lane + 32)] : 0;
+    auto page_entry = [&](int i) {  // warp-collective; i grows by one per call
+        if (i >= bt_base + 32) {
+            bt_base += 32;
+            bt_cur = bt_next;
+            bt_next = lane + bt_base + 32 < cnt ? bt[pg0 + warp + NW * (lane + bt_base + 32)] : 0;
+        }
+        return __shfl_sync(0xffffffffu, bt_cur, i - bt_base);
+    };
     int issued = 0;
-    for (; issued < cnt && issued < kRing; ++issued) {
+    for (; issued < cnt && issued < RING; ++issued) {
         uint16_t* slot = wbuf + (size_t)issued * 2 * PAGE;
-        load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg0 + warp + 4 * issued], a.nkv, g, slot, slot + PAGE);
+        load_page_warp<D, LD>(a.k_pool, a.v_pool, page_entry(issued), a.nkv, g, slot, slot + PAGE);
     }
+    // the model path's angles and QK-norm gains do not depend on the previous kernel either
+    const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
+    HeadRegs<D> hr;
+    const bool regs = a.qkv != nullptr && (tab != nullptr || !a.rope);
+    if (regs) load_head_regs<D>(hr, a.rope ? tab : nullptr, a.q_norm, a.k_norm);
 
     pdl_trigger();
     pdl_wait();
-    const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
     const bool have_new = a.qkv != nullptr || a.k_new != nullptr;
     const size_t off_p = has_last ? (((size_t)bt[p / kPage] * a.nkv + g) * kPage + (p % kPage)) * D : 0;
 
@@ -242,11 +329,14 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
 
     if (pg0 < pg1) {
         // ---- q tile of the group (rows >= G are zero); the split holding row p appends it
-        for (int r = warp; r < 16; r += 4) {
+        for (int r = warp; r < 16; r += NW) {
             uint16_t* dst = qs + r * LD;
             if (r < G) {
                 const int h = g * G + r;
-                if (a.qkv)
+                if (regs)
+                    head_transform_regs<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)h * D, hr.qn, a.q_norm != nullptr,
+                                           a.eps, a.rope, hr.cs, dst);
+                else if (a.qkv)
                     head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)h * D, false, nullptr, a.q_norm, a.eps,
                                       a.rope, p, a.rope_base, dst, tab);
                 else
@@ -260,7 +350,10 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             // the new row: k gets QK-norm and RoPE, v is only rounded; staged in shared
             // memory (patched into the page fetched before it existed) and appended to the cache
             if (warp == 0) {
-                if (a.qkv)
+                if (regs)
+                    head_transform_regs<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + g) * D, hr.kn,
+                                           a.k_norm != nullptr, a.eps, a.rope, hr.cs, newkv[0]);
+                else if (a.qkv)
                     head_transform<D>(a.qkv + (size_t)b * a.ld_qkv + (size_t)(a.nq + g) * D, false, nullptr, a.k_norm,
                                       a.eps, a.rope, p, a.rope_base, newkv[0], tab);
                 else
@@ -284,10 +377,10 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
         uint32_t qf[D / 16][4];
         load_q_frags<D, LD>(qs, qf);
 
-        // each warp streams its pages through a kRing-page cp.async ring; a slot is refilled
+        // each warp streams its pages through a RING-page cp.async ring; a slot is refilled
         // as soon as its page has been used
         for (int i = 0; i < cnt; ++i) {
-            const int pg = pg0 + warp + 4 * i;
+            const int pg = pg0 + warp + NW * i;
             switch (issued - i - 1) {  // groups that may stay in flight
                 case 0: cp_async_wait<0>(); break;
                 case 1: cp_async_wait<1>(); break;
@@ -295,7 +388,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
                 default: cp_async_wait<3>(); break;
             }
             __syncwarp();
-            uint16_t* kd = wbuf + (size_t)(i % kRing) * 2 * PAGE;
+            uint16_t* kd = wbuf + (size_t)(i % RING) * 2 * PAGE;
             if (pg == np - 1 && has_last && have_new) {
                 // the page was fetched before row p existed: copy the staged row in
                 uint16_t* row = kd + (lane < 16 ? 0 : PAGE) + (p % kPage) * LD;
@@ -305,12 +398,24 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             }
             float sc[2][4];
             qk_page<D, LD>(qf, kd, sc);
+            // the softcap test stays outside the loops: the plain path carries no tanh at all
+            if (a.softcap > 0.f) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sc[nt][c] = score_log2(sc[nt][c], a.scale, a.softcap);
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sc[nt][c] *= sl2;
+            }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const int key = pg * kPage + nt * 8 + 2 * t4 + (c & 1);
-                    sc[nt][c] = key < n ? sc[nt][c] * sl2 : -INFINITY;
+                    if (!(key < n && key >= kf)) sc[nt][c] = -INFINITY;
                 }
             float corr[2];
             softmax_page(sc, m, l, corr);
@@ -324,7 +429,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
             pv_page<D, LD>(sc, kd + PAGE, o);
             __syncwarp();
             if (issued < cnt) {
-                load_page_warp<D, LD>(a.k_pool, a.v_pool, bt[pg0 + warp + 4 * issued], a.nkv, g, kd, kd + PAGE);
+                load_page_warp<D, LD>(a.k_pool, a.v_pool, page_entry(issued), a.nkv, g, kd, kd + PAGE);
                 ++issued;
             }
         }
@@ -338,6 +443,9 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     // ---- merge the 4 warps of the CTA through shared memory (a CTA without pages
     // contributes m = -inf, l = 0, o = 0)
     __syncthreads();  // page buffers are free
+    // this CTA no longer reads its page rings: the other CTAs of the cluster may write
+    // their partials into them once everyone has arrived (release: the reads come first)
+    if (cl) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     if (t4 == 0) {
         wm[warp][gr] = m[0];
         wm[warp][gr + 8] = m[1];
@@ -357,16 +465,17 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     // Split partial of row r: o (relative to M) and M, L. In a cluster, row r is finished
     // by CTA r % S, which receives every split's partial of it in slot [r / S][s];
     // otherwise the partials go to the scratch and the last CTA of (b, g) merges them.
-    if (cl) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA is running
-    for (int idx = tid; idx < G * (D / 4); idx += 128) {
+    // every CTA of the cluster is past its page loop (and still running)
+    if (cl) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    for (int idx = tid; idx < G * (D / 4); idx += NT) {
         const int r = idx / (D / 4), c = (idx % (D / 4)) * 4;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][r]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w][r]);
         float L = 0.f;
         float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < NW; ++w) {
             if (wm[w][r] == -INFINITY) continue;
             const float f = exp2f(wm[w][r] - M);
             L += f * wl[w][r];
@@ -404,22 +513,29 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     if (cl) {
         cluster_sync();  // all partials have arrived
         // rows r = s, s + S, ...: weighted sum over the splits in split order
+        // (unrolled to the cluster bound: the split weights are computed once per row, and
+        // the loads of every split are in flight together)
         for (int r = s; r < G; r += S) {
             const float* rv = recv + (size_t)(r / S) * S * LDR;
+            float mz[kDecodeMaxSplits], wz[kDecodeMaxSplits];
             float M = -INFINITY;
-            for (int z = 0; z < S; ++z) M = fmaxf(M, rv[(size_t)z * LDR + D]);
+#pragma unroll
+            for (int z = 0; z < kDecodeMaxSplits; ++z) {
+                mz[z] = z < S ? rv[(size_t)z * LDR + D] : -INFINITY;
+                M = fmaxf(M, mz[z]);
+            }
             float L = 0.f;
-            for (int z = 0; z < S; ++z) {
-                const float mz = rv[(size_t)z * LDR + D];
-                if (mz != -INFINITY) L += exp2f(mz - M) * rv[(size_t)z * LDR + D + 1];
+#pragma unroll
+            for (int z = 0; z < kDecodeMaxSplits; ++z) {
+                wz[z] = mz[z] != -INFINITY ? exp2f(mz[z] - M) : 0.f;
+                if (mz[z] != -INFINITY) L += wz[z] * rv[(size_t)z * LDR + D + 1];
             }
             const float invL = 1.0f / L;
-            for (int c = tid; c < D; c += 128) {
+            for (int c = tid; c < D; c += NT) {
                 float O = 0.f;
-                for (int z = 0; z < S; ++z) {
-                    const float mz = rv[(size_t)z * LDR + D];
-                    if (mz != -INFINITY) O += exp2f(mz - M) * rv[(size_t)z * LDR + c];
-                }
+#pragma unroll
+                for (int z = 0; z < kDecodeMaxSplits; ++z)
+                    if (mz[z] != -INFINITY) O += wz[z] * rv[(size_t)z * LDR + c];
                 a.out[(size_t)b * a.nq * D + (size_t)(g * G + r) * D + c] = f2bf(O * invL);
             }
         }
@@ -435,7 +551,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     __threadfence();
     // weights of each split: f_z = exp2(m_z - M) / sum_z exp2(m_z - M) l_z (one warp per head)
     float* fz = reinterpret_cast<float*>(kvbuf);  // [G][splits]
-    for (int r = warp; r < G; r += 4) {
+    for (int r = warp; r < G; r += NW) {
         const float* pp = a.part + ((size_t)b * a.nq + g * G + r) * S * (D + 2);
         float M = -INFINITY;
         for (int z = lane; z < S; z += 32) M = fmaxf(M, __ldcg(pp + (size_t)z * (D + 2) + D));
@@ -453,7 +569,7 @@ __global__ void __launch_bounds__(128) attn_decode_kernel(AttnDecodeArgs a) {
     }
     __syncthreads();
     // weighted sum over splits in split order; loads of one split are coalesced across threads
-    for (int idx = tid; idx < G * D; idx += 128) {
+    for (int idx = tid; idx < G * D; idx += NT) {
         const int r = idx / D, c = idx % D;
         const int h = g * G + r;
         const float* pp = a.part + ((size_t)b * a.nq + h) * S * (D + 2) + c;
@@ -625,9 +741,13 @@ __global__ void __launch_bounds__(128, 3) attn_prefill_kernel(AttnPrefillArgs a)
     const int rbase = qb * kPrefRows;
     const int t_last = min(a.T - 1, (rbase + kPrefRows - 1) / G);
     const int n_cta = a.pos0 + t_last + 1;  // keys any row of this CTA may see
+    const int W = a.window;
+    // with a window, the first key any row of this CTA may see (its first row's window start)
+    const int kf_cta = W > 0 ? max(0, a.pos0 + rbase / G - W + 1) : 0;
     const int nblk = (n_cta + kPrefKeys - 1) / kPrefKeys;
-    const int bps = (nblk + S - 1) / S;
-    const int blk0 = s * bps, blk1 = min(nblk, blk0 + bps);
+    const int bf = kf_cta / kPrefKeys;
+    const int bps = (nblk - bf + S - 1) / S;
+    const int blk0 = bf + s * bps, blk1 = min(nblk, blk0 + bps);
 
     // this thread's rows (g and g + 8 of the warp's 16) and their last visible key
     const int r0 = rbase + warp * 16;
@@ -637,6 +757,10 @@ __global__ void __launch_bounds__(128, 3) attn_prefill_kernel(AttnPrefillArgs a)
     const int lim_b = rb < R ? a.pos0 + rb / G : -1;
     const int warp_hi = r0 < R ? a.pos0 + min(R - 1, r0 + 15) / G : -1;  // largest limit of the warp
     const int warp_lo = r0 + 15 < R ? a.pos0 + r0 / G : -1;              // smallest (-1: padding rows)
+    // with a window: keys below wlo_min are outside every row's window, keys from wlo_max on
+    // inside every row's window
+    const int wlo_min = W > 0 && r0 < R ? a.pos0 + r0 / G - W + 1 : 0;
+    const int wlo_max = W > 0 ? warp_hi - W + 1 : 0;
 
     // Q fragments straight from global memory (A layout of m16n8k16)
     uint32_t qf[D / 16][4];
@@ -694,22 +818,32 @@ __global__ void __launch_bounds__(128, 3) attn_prefill_kernel(AttnPrefillArgs a)
         }
         __syncthreads();
         const int k0 = blk * kPrefKeys;
-        if (k0 <= warp_hi) {  // else every key of the block is masked for this warp's rows
+        // else every key of the block is masked for this warp's rows (past the causal edge,
+        // or before every row's window)
+        if (k0 <= warp_hi && k0 + kPrefKeys - 1 >= wlo_min) {
             float sc[8][4];
             qk_block<D, LD>(qf, kb + buf * kPrefKeys * LD, sc);
-            if (k0 + kPrefKeys - 1 > warp_lo) {  // the causal edge (or padding rows) cross the block
+            if (a.softcap > 0.f) {
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int key = k0 + nt * 8 + 2 * t4 + (c & 1);
-                        sc[nt][c] = key <= (c < 2 ? lim_a : lim_b) ? sc[nt][c] * sl2 : -INFINITY;
-                    }
+                    for (int c = 0; c < 4; ++c) sc[nt][c] = score_log2(sc[nt][c], a.scale, a.softcap);
             } else {
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) sc[nt][c] *= sl2;
+            }
+            // the causal edge (or padding rows), or a window start, crosses the block
+            if (k0 + kPrefKeys - 1 > warp_lo || (W > 0 && k0 < wlo_max)) {
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int key = k0 + nt * 8 + 2 * t4 + (c & 1);
+                        const int lim = c < 2 ? lim_a : lim_b;
+                        if (key > lim || (W > 0 && key <= lim - W)) sc[nt][c] = -INFINITY;
+                    }
             }
             float corr[2];
             softmax_block(sc, m, l, corr);
@@ -821,32 +955,32 @@ int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms, bool cluster) {
     return s;
 }
 
-template <int D>
+template <int D, int NW>
 size_t decode_smem(int G, int splits) {
-    const size_t ring = (size_t)4 * kRing * 2 * kPage * (D + 8) * 2;  // page rings of 4 warps
+    const size_t ring = (size_t)NW * kDecRing<NW> * 2 * kPage * (D + 8) * 2;  // page rings of NW warps
     const size_t rows_owned = (size_t)(G + splits - 1) / splits;
-    const size_t merge = (size_t)4 * 16 * D * 4 + rows_owned * splits * (D + 4) * 4;  // warp partials + receive
+    const size_t merge = (size_t)NW * 16 * D * 4 + rows_owned * splits * (D + 4) * 4;  // warp partials + receive
     return ring > merge ? ring : merge;
 }
 
-template <int D>
-cudaError_t decode_launch_d(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
+template <int D, int NW>
+cudaError_t decode_launch_dw(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
     const int G = a.nq / a.nkv;
-    const size_t smem = decode_smem<D>(G, a.splits);
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<D>), (int)smem);
+    const size_t smem = decode_smem<D, NW>(G, a.splits);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<D, NW>), (int)smem);
     if (e != cudaSuccess) return e;
     const bool cl = a.splits > 1 && a.part == nullptr;
     if (cl && a.splits > 8) {
         static std::once_flag once;
         static cudaError_t ce = cudaSuccess;
         std::call_once(once, [] {
-            ce = cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            ce = cudaFuncSetAttribute(attn_decode_kernel<D, NW>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         });
         if (ce != cudaSuccess) return ce;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.splits, a.nkv, a.B);
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(NW * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -865,13 +999,20 @@ cudaError_t decode_launch_d(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) 
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, attn_decode_kernel<D>, a);
+    return cudaLaunchKernelEx(&cfg, attn_decode_kernel<D, NW>, a);
+}
+
+// 4 warps with 3-page rings. (8 warps with 2-page rings, all of a split's pages in flight at
+// once, measured slower at batch 1: 20.8 against 11-13 us per launch of the Llama-3-8B shape.)
+template <int D>
+cudaError_t decode_launch_d(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
+    return decode_launch_dw<D, 4>(a, st, pdl);
 }
 
 cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
     if (a.splits < 1 || a.nkv <= 0 || a.nq % a.nkv != 0 || a.nq / a.nkv > 16) return cudaErrorInvalidValue;
     if (a.splits > 1 && a.part == nullptr && a.splits > kDecodeMaxSplits) return cudaErrorInvalidValue;
-    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64>(a.nq / a.nkv, a.splits)) return cudaErrorInvalidValue;
+    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64, 4>(a.nq / a.nkv, a.splits)) return cudaErrorInvalidValue;
     if (a.d == 128) return decode_launch_d<128>(a, st, pdl);
     if (a.d == 64) return decode_launch_d<64>(a, st, pdl);
     return cudaErrorInvalidValue;

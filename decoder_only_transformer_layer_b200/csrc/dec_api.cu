@@ -14,6 +14,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <string>
@@ -25,6 +26,10 @@
 using namespace dec;
 
 namespace {
+
+// Positions one dec_verify call may forward (the pages' multi-position verify checks up
+// to a handful of draft tokens).
+constexpr int kMaxVerify = 8;
 
 thread_local std::string g_err;
 
@@ -40,9 +45,20 @@ dec_status fail(dec_status s, const std::string& msg) {
             return fail(DEC_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_));      \
     } while (0)
 
+// Test hook (dec_test_fail_alloc): the n-th device allocation from now on fails as if the
+// device were out of memory; 0 = off.
+std::atomic<long> g_fail_alloc_in{0};
+
 template <typename T>
 cudaError_t dmalloc(T** p, size_t count) {
     if (count == 0) count = 1;
+    long n = g_fail_alloc_in.load();
+    while (n > 0 && !g_fail_alloc_in.compare_exchange_weak(n, n - 1)) {
+    }
+    if (n == 1) {
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+    }
     return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
 }
 
@@ -60,6 +76,11 @@ struct LayerDev {
     uint16_t *wqkv = nullptr, *wo = nullptr, *wgu = nullptr, *wdown = nullptr;
     uint16_t *wrouter = nullptr, *egu = nullptr, *edown = nullptr, *sgu = nullptr, *sdown = nullptr;
     float* sgate_vec = nullptr;
+    float *post_attn_norm = nullptr, *post_ffn_norm = nullptr;  // sandwich norms
+    // q8_row models: the int8 projections (gate/up rows interleaved like wgu) and their row
+    // scales; wqkv / wo / wgu / wdown then hold the same integers as bf16 (tensor-core path)
+    int8_t *qkv_q = nullptr, *wo_q = nullptr, *gu_q = nullptr, *down_q = nullptr;
+    float *qkv_s = nullptr, *wo_s = nullptr, *gu_s = nullptr, *down_s = nullptr;
     uint16_t *k_pool = nullptr, *v_pool = nullptr;
 };
 
@@ -73,9 +94,11 @@ struct dec_ctx {
     bool bridge = false;            // caller gave the legacy default stream: own stream + events
     cudaEvent_t ev_in = nullptr, ev_out = nullptr;
     int qd = 0, kvd = 0, qkv_rows = 0, max_pages = 0, n_pages = 0;
-    int max_tok = 0;  // rows of the per-step buffers: max(max_batch, prefill_chunk)
+    int max_tok = 0;  // rows of the per-step buffers: max(max_batch, prefill_chunk, kMaxVerify)
     std::vector<LayerDev> L;
     uint16_t *embed = nullptr, *head = nullptr;
+    int8_t* head_q = nullptr;  // q8_row LM head and its row scales
+    float* head_s = nullptr;
     float* final_norm = nullptr;
     // paging
     std::vector<int> free_pages;
@@ -88,20 +111,28 @@ struct dec_ctx {
     unsigned long long* d_amax = nullptr;  // packed greedy argmax, 32 words per row
     float2* rope_tab = nullptr;            // [max_context][d/2] (cos, sin): fp64 on the host, stored fp32
     float *x = nullptr, *qkv = nullptr, *logits = nullptr;
+    float* ysub = nullptr;  // sandwich norms: a sublayer's output [max_tok][h] before its norm
     uint16_t *xn = nullptr, *qrot = nullptr, *attn = nullptr, *act = nullptr;
     float* gemm_ws = nullptr;  // tensor-core GEMM: pieces of tiles shared between CTAs
     int* gemm_cnt = nullptr;   // and their arrival counters (zero between launches)
     int gemm_cnt_n = 0;
-    int* d_err = nullptr;
-    int32_t* h_stage = nullptr;  // pinned: tokens, positions, block rows
-    int32_t* h_prompt = nullptr; // pinned [max_context]: one prefill's tokens
+    int* d_err = nullptr;        // set by a device wait that ran out (cleared by dec_check)
+    // Host-to-device staging: two pinned slots used in turn, each fenced by an event
+    // recorded after the copies that read it, so a call never waits for the device
+    // unless the slot it needs is still being copied from (two calls back).
+    int32_t* h_stage[2] = {nullptr, nullptr};
+    cudaEvent_t ev_stage[2] = {nullptr, nullptr};
+    int stage_next = 0;
+    size_t stage_ints = 0;
+    float** d_ldst = nullptr;    // device slot: where the head stores the logits (null: nowhere)
     int32_t* d_prompt = nullptr; // [max_context]
-    int* h_err = nullptr;
+    int* h_err = nullptr;        // pinned copy of d_err for the synchronising paths
     int act_cols = 0;
     // MoE step buffers (rows: max_tok tokens, or max_tok * top_k (token, expert) slots)
     float *moe_logits = nullptr, *moe_w = nullptr, *moe_sgate = nullptr, *moe_y = nullptr, *moe_ys = nullptr;
     int32_t *moe_routes = nullptr, *moe_perm = nullptr, *moe_inv = nullptr, *moe_groups = nullptr, *moe_ngroups = nullptr;
     uint16_t* moe_act = nullptr;
+    int head_rows = 0;  // rows of the logits / argmax buffers: max(max_batch, kMaxVerify)
     std::map<int, cudaGraphExec_t> graphs;
     int last_rows = 0;
     bool last_was_step = false;
@@ -131,7 +162,22 @@ dec_status check_config(const dec_config* c) {
         return fail(DEC_ERR_UNSUPPORTED, "ffn_inter must be a positive multiple of 8");
     }
     if (!(c->rms_eps > 0.f)) return fail(DEC_ERR_INVALID_ARG, "rms_eps must be positive");
+    if (c->sliding_window < 0 || c->swa_pattern < 0 || !(c->attn_softcap >= 0.f) || !(c->final_softcap >= 0.f))
+        return fail(DEC_ERR_INVALID_ARG, "sliding_window, swa_pattern and the softcaps must be >= 0");
+    if (c->sandwich_norms && c->n_experts > 0)
+        return fail(DEC_ERR_UNSUPPORTED, "sandwich norms are built for the dense FFN only");
+    if (c->weight_format != 0 && c->weight_format != 1) return fail(DEC_ERR_UNSUPPORTED, "weight_format must be 0 or 1");
+    if (c->weight_format == 1 && (c->n_experts > 0 || c->tied_embeddings))
+        return fail(DEC_ERR_UNSUPPORTED, "q8_row weights are built for dense models with an untied LM head");
     return DEC_OK;
+}
+
+// Attention window of layer li (0 = the whole context): every max(swa_pattern, 1)-th layer
+// is global (cortiq layer_is_local).
+int layer_window(const dec_config& k, int li) {
+    if (k.sliding_window <= 0) return 0;
+    const int pattern = k.swa_pattern > 1 ? k.swa_pattern : 1;
+    return (li + 1) % pattern != 0 ? k.sliding_window : 0;
 }
 
 cudaError_t copy_in(void* dst, const void* src, size_t bytes, cudaStream_t st) {
@@ -139,30 +185,40 @@ cudaError_t copy_in(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, st);
 }
 
-// Interleave rows of gate [rows][h] and up [rows][h] into dst [2*rows][h]: row 2j = gate j, 2j+1 = up j.
-cudaError_t interleave_in(uint16_t* dst, const void* gate, const void* up, size_t rows, int h, cudaStream_t st) {
+// Interleave rows of gate [rows][rb bytes] and up into dst [2*rows]: row 2j = gate j, 2j+1 = up j.
+cudaError_t interleave_rows_in(void* dst, const void* gate, const void* up, size_t rows, size_t rb, cudaStream_t st) {
     if (!gate || !up) return cudaErrorInvalidValue;
-    const size_t rb = (size_t)h * 2;
     cudaError_t e = cudaMemcpy2DAsync(dst, 2 * rb, gate, rb, rb, rows, cudaMemcpyDefault, st);
     if (e != cudaSuccess) return e;
     return cudaMemcpy2DAsync(reinterpret_cast<uint8_t*>(dst) + rb, 2 * rb, up, rb, rb, rows, cudaMemcpyDefault, st);
 }
 
+cudaError_t interleave_in(uint16_t* dst, const void* gate, const void* up, size_t rows, int h, cudaStream_t st) {
+    return interleave_rows_in(dst, gate, up, rows, (size_t)h * 2, st);
+}
+
 // ----------------------------------------------------------------- projections
 
-// y = W x for `n` token rows: GEMV when n is small, tcgen05 GEMM otherwise.
+// y = W x for `n` token rows: GEMV when n is small, tcgen05 GEMM otherwise. A q8_row
+// projection also carries its int8 rows Q and row scales S (the GEMV streams Q; the GEMM
+// multiplies W, the same integers in bf16, and scales each row in its epilogue).
 struct Proj {
     const uint16_t* W;
     int M, K;
+    const int8_t* Q = nullptr;
+    const float* S = nullptr;
 };
 
 dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, const float* xr, const float* g,
                     const uint16_t* xb, float* y, int ldy, const float* bias, uint16_t* act, int ldact,
-                    cudaStream_t st, unsigned long long* amax = nullptr) {
+                    cudaStream_t st, unsigned long long* amax = nullptr, float* const* y_ptr = nullptr,
+                    float softcap = 0.f) {
     const int cap = c->smem_cap;
-    if (n <= 8 && gemv_fits(n, p.K, cap)) {
+    if (n <= 8 && gemv_fits(n, p.K, cap, p.Q != nullptr)) {
         GemvArgs a{};
         a.W = p.W;
+        a.Wq = p.Q;
+        a.wscale = p.S;
         a.N = p.M;
         a.K = p.K;
         a.B = n;
@@ -172,11 +228,13 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
         a.eps = c->c.rms_eps;
         a.ldx = p.K;
         a.y = y;
+        a.y_ptr = y_ptr;
         a.ldy = ldy;
         a.bias = bias;
         a.act = act;
         a.ldact = ldact;
         a.amax = amax;
+        a.softcap = softcap;
         a.err = c->d_err;
         a.smem_cap = cap;
         const int ge = epi == GEMM_STORE ? GEMV_STORE : epi == GEMM_RESID ? GEMV_RESID : GEMV_SWIGLU;
@@ -193,11 +251,14 @@ dec_status run_proj(dec_ctx* c, const Proj& p, int n, int epi, bool fused_norm, 
     GemmArgs a{};
     a.epi = epi;
     a.y = y;
+    a.y_ptr = y_ptr;
     a.ldy = ldy;
     a.bias = bias;
+    a.rscale = p.Q ? p.S : nullptr;
     a.act = act;
     a.ldact = ldact;
     a.amax = amax;
+    a.softcap = softcap;
     a.cnt = c->gemm_cnt;
     a.err = c->d_err;
     if (gemm_cnt_needed(p.M, n) > c->gemm_cnt_n) return fail(DEC_ERR_UNSUPPORTED, "GEMM tile counters too small");
@@ -302,8 +363,8 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
     for (int li = 0; li < k.layers; ++li) {
         LayerDev& L = c->L[li];
         // attention input norm + fused QKV (+bias)
-        dec_status s = run_proj(c, {L.wqkv, c->qkv_rows, h}, n, GEMM_STORE, true, c->x, L.attn_norm, nullptr, c->qkv,
-                                c->qkv_rows, L.bqkv, nullptr, 0, st);
+        dec_status s = run_proj(c, {L.wqkv, c->qkv_rows, h, L.qkv_q, L.qkv_s}, n, GEMM_STORE, true, c->x,
+                                L.attn_norm, nullptr, c->qkv, c->qkv_rows, L.bqkv, nullptr, 0, st);
         if (s != DEC_OK) return s;
         if (decode) {
             AttnDecodeArgs a{};
@@ -325,8 +386,11 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
             a.nkv = k.n_kv_heads;
             a.d = d;
             a.scale = scale;
-            // context splits merged inside a cluster: no scratch, chosen per batch size
-            a.splits = attn_decode_splits(n, k.n_kv_heads, k.max_context, c->num_sms, true);
+            a.window = layer_window(k, li);
+            a.softcap = k.attn_softcap;
+            // context splits merged inside a cluster: no scratch, chosen per batch size and span
+            const int span = a.window > 0 ? std::min(a.window, k.max_context) : k.max_context;
+            a.splits = attn_decode_splits(n, k.n_kv_heads, span, c->num_sms, true);
             a.part = nullptr;
             a.counters = nullptr;
             a.out = c->attn;
@@ -362,38 +426,59 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
             a.nkv = k.n_kv_heads;
             a.d = d;
             a.scale = scale;
-            a.splits = attn_prefill_splits(n, k.n_q_heads, k.n_kv_heads, pos0 + n, c->num_sms);
+            a.window = layer_window(k, li);
+            a.softcap = k.attn_softcap;
+            a.splits = attn_prefill_splits(n, k.n_q_heads, k.n_kv_heads, attn_prefill_span(pos0, n, a.window),
+                                           c->num_sms);
             a.out = c->attn;
             a.err = c->d_err;
             CUDA_TRY(attn_prefill_launch(a, st, true));
         }
-        // o_proj + residual
-        s = run_proj(c, {L.wo, h, c->qd}, n, GEMM_RESID, false, nullptr, nullptr, c->attn, c->x, h, nullptr, nullptr,
-                     0, st);
-        if (s != DEC_OK) return s;
+        // o_proj + residual (sandwich: the output is RMS-normalised with its own gain first)
+        if (k.sandwich_norms) {
+            s = run_proj(c, {L.wo, h, c->qd, L.wo_q, L.wo_s}, n, GEMM_STORE, false, nullptr, nullptr, c->attn, c->ysub,
+                         h, nullptr, nullptr, 0, st);
+            if (s != DEC_OK) return s;
+            CUDA_TRY(add_rmsnorm_launch(c->x, c->ysub, L.post_attn_norm, n, h, k.rms_eps, st, true));
+        } else {
+            s = run_proj(c, {L.wo, h, c->qd, L.wo_q, L.wo_s}, n, GEMM_RESID, false, nullptr, nullptr, c->attn, c->x, h,
+                         nullptr, nullptr, 0, st);
+            if (s != DEC_OK) return s;
+        }
         if (k.n_experts > 0) {
             s = moe_ffn(c, li, n, st);
             if (s != DEC_OK) return s;
             continue;
         }
         // FFN: norm + fused gate/up + SiLU, then down + residual
-        s = run_proj(c, {L.wgu, 2 * k.ffn_inter, h}, n, GEMM_SWIGLU, true, c->x, L.ffn_norm, nullptr, nullptr, 0,
-                     nullptr, c->act, c->act_cols, st);
+        s = run_proj(c, {L.wgu, 2 * k.ffn_inter, h, L.gu_q, L.gu_s}, n, GEMM_SWIGLU, true, c->x, L.ffn_norm, nullptr,
+                     nullptr, 0, nullptr, c->act, c->act_cols, st);
         if (s != DEC_OK) return s;
-        s = run_proj(c, {L.wdown, h, k.ffn_inter}, n, GEMM_RESID, false, nullptr, nullptr, c->act, c->x, h, nullptr,
-                     nullptr, 0, st);
-        if (s != DEC_OK) return s;
+        if (k.sandwich_norms) {
+            s = run_proj(c, {L.wdown, h, k.ffn_inter, L.down_q, L.down_s}, n, GEMM_STORE, false, nullptr, nullptr,
+                         c->act, c->ysub, h, nullptr, nullptr, 0, st);
+            if (s != DEC_OK) return s;
+            CUDA_TRY(add_rmsnorm_launch(c->x, c->ysub, L.post_ffn_norm, n, h, k.rms_eps, st, true));
+        } else {
+            s = run_proj(c, {L.wdown, h, k.ffn_inter, L.down_q, L.down_s}, n, GEMM_RESID, false, nullptr, nullptr,
+                         c->act, c->x, h, nullptr, nullptr, 0, st);
+            if (s != DEC_OK) return s;
+        }
     }
     return DEC_OK;
 }
 
-// Final norm + LM head for `n` rows starting at residual row `row0` -> c->logits [n][V];
-// the greedy token of each row is folded into the head's epilogue (packed argmax words).
-dec_status head(dec_ctx* c, int row0, int n, cudaStream_t st) {
+// Final norm + LM head for `n` rows starting at residual row `row0`. The logits [n][V] go
+// to `y`, or, when y_ptr is given, to the device address it holds (read when the head
+// runs, so one captured graph serves every destination); a null destination stores
+// nothing. The greedy token of each row is folded into the head's epilogue (packed
+// argmax words) either way.
+dec_status head(dec_ctx* c, int row0, int n, cudaStream_t st, float* y, float* const* y_ptr) {
     const dec_config& k = c->c;
     CUDA_TRY(cudaMemsetAsync(c->d_amax, 0, sizeof(unsigned long long) * 32 * (size_t)n, st));
-    return run_proj(c, {c->head, k.vocab, k.hidden}, n, GEMM_STORE, true, c->x + (size_t)row0 * k.hidden,
-                    c->final_norm, nullptr, c->logits, k.vocab, nullptr, nullptr, 0, st, c->d_amax);
+    return run_proj(c, {c->head, k.vocab, k.hidden, c->head_q, c->head_s}, n, GEMM_STORE, true,
+                    c->x + (size_t)row0 * k.hidden,
+                    c->final_norm, nullptr, y, k.vocab, nullptr, nullptr, 0, st, c->d_amax, y_ptr, k.final_softcap);
 }
 
 dec_status ensure_pages(dec_ctx* c, int seq, int upto) {
@@ -410,27 +495,86 @@ dec_status ensure_pages(dec_ctx* c, int seq, int upto) {
     return DEC_OK;
 }
 
-dec_status upload_bt_row(dec_ctx* c, int seq, cudaStream_t st) {
-    int32_t* stg = c->h_stage + 2 * c->max_tok;
-    memcpy(stg, &c->h_bt[(size_t)seq * c->max_pages], sizeof(int32_t) * c->max_pages);
-    CUDA_TRY(cudaMemcpyAsync(c->d_bt + (size_t)seq * c->max_pages, stg, sizeof(int32_t) * c->max_pages,
-                             cudaMemcpyHostToDevice, st));
-    // the staging area is reused by the next call: make the copy complete first
-    CUDA_TRY(cudaStreamSynchronize(st));
+// One staging slot, in int32 words: tokens [max_tok] | positions [max_tok] | logits
+// destination (one 8-byte pointer) | block-table rows [max_batch][max_pages] | prompt
+// tokens [max_context].
+struct StageLayout {
+    size_t tok, pos, dst, bt, prompt, total;
+};
+
+StageLayout stage_layout(const dec_ctx* c) {
+    StageLayout L;
+    L.tok = 0;
+    L.pos = L.tok + (size_t)c->max_tok;
+    L.dst = (L.pos + (size_t)c->max_tok + 1) & ~(size_t)1;  // 8-byte aligned
+    L.bt = L.dst + 2;
+    L.prompt = L.bt + (size_t)c->c.max_batch * c->max_pages;
+    L.total = L.prompt + (size_t)c->c.max_context;
+    return L;
+}
+
+// The next staging slot. Its previous use was two calls ago; the event recorded after
+// that use's copies has normally completed long since, so this rarely waits.
+dec_status stage_acquire(dec_ctx* c, int32_t** slot, int* which) {
+    const int i = c->stage_next;
+    CUDA_TRY(cudaEventSynchronize(c->ev_stage[i]));
+    c->stage_next ^= 1;
+    *slot = c->h_stage[i];
+    *which = i;
     return DEC_OK;
 }
 
-dec_status deliver_logits(dec_ctx* c, float* out, int rows, cudaStream_t st) {
-    if (!out) return DEC_OK;
-    const size_t bytes = (size_t)rows * c->c.vocab * sizeof(float);
-    if (is_host_ptr(out)) {
-        CUDA_TRY(cudaMemcpyAsync(out, c->logits, bytes, cudaMemcpyDeviceToHost, st));
-        CUDA_TRY(cudaStreamSynchronize(st));
-        if (*c->h_err) return fail(DEC_ERR_TIMEOUT, "a device wait ran out of time");
-    } else {
-        CUDA_TRY(cudaMemcpyAsync(out, c->logits, bytes, cudaMemcpyDeviceToDevice, st));
-    }
+// Fence the slot: recorded on `st` right after the copies that read it.
+dec_status stage_release(dec_ctx* c, int which, cudaStream_t st) {
+    CUDA_TRY(cudaEventRecord(c->ev_stage[which], st));
     return DEC_OK;
+}
+
+// Copy the block-table rows of sequences [s0, s1) through the staging slot.
+dec_status stage_bt_rows(dec_ctx* c, int32_t* slot, int s0, int s1, cudaStream_t st) {
+    const StageLayout L = stage_layout(c);
+    const size_t off = (size_t)s0 * c->max_pages, n = (size_t)(s1 - s0) * c->max_pages;
+    memcpy(slot + L.bt + off, &c->h_bt[off], sizeof(int32_t) * n);
+    CUDA_TRY(cudaMemcpyAsync(c->d_bt + off, slot + L.bt + off, sizeof(int32_t) * n, cudaMemcpyHostToDevice, st));
+    return DEC_OK;
+}
+
+// After the stream has been synchronised: report a device wait that ran out (the error
+// word a kernel sets when one of its bounded waits gives up) as DEC_ERR_TIMEOUT, and make
+// the context usable again: clear the word and zero the GEMM tile counters that an
+// abandoned reduction can leave behind.
+dec_status take_device_error(dec_ctx* c, cudaStream_t st) {
+    if (!*c->h_err) return DEC_OK;
+    *c->h_err = 0;
+    CUDA_TRY(cudaMemsetAsync(c->d_err, 0, sizeof(int), st));
+    CUDA_TRY(cudaMemsetAsync(c->gemm_cnt, 0, sizeof(int) * (size_t)c->gemm_cnt_n, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return fail(DEC_ERR_TIMEOUT,
+                "a bounded device wait ran out (this call or an earlier one on this context); the context "
+                "has been reset for further calls");
+}
+
+// Synchronise and check the error word (the synchronising entry points).
+dec_status sync_and_check(dec_ctx* c, cudaStream_t st) {
+    CUDA_TRY(cudaMemcpyAsync(c->h_err, c->d_err, sizeof(int), cudaMemcpyDeviceToHost, st));
+    CUDA_TRY(cudaStreamSynchronize(st));
+    return take_device_error(c, st);
+}
+
+// Where the head should store the logits for a caller's logits_out: its own buffer for a
+// device pointer, the context's buffer for a host pointer (copied out afterwards), nowhere
+// for NULL.
+float* logits_target(dec_ctx* c, float* out, bool* host) {
+    *host = out && is_host_ptr(out);
+    if (!out) return nullptr;
+    return *host ? c->logits : out;
+}
+
+// Host logits: copy them out, synchronise and check the error word.
+dec_status finish_host_logits(dec_ctx* c, float* out, int rows, cudaStream_t st) {
+    const size_t bytes = (size_t)rows * c->c.vocab * sizeof(float);
+    CUDA_TRY(cudaMemcpyAsync(out, c->logits, bytes, cudaMemcpyDeviceToHost, st));
+    return sync_and_check(c, st);
 }
 
 // Order the context's stream after the caller's legacy-stream work, and back.
@@ -524,6 +668,19 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     if (s != DEC_OK) return s;
     if (!w || !w->embed || !w->final_norm || !w->layers) return fail(DEC_ERR_INVALID_ARG, "weights missing");
     if (!cfg->tied_embeddings && !w->lm_head) return fail(DEC_ERR_INVALID_ARG, "lm_head missing (untied)");
+    if (cfg->weight_format == 1) {
+        bool ok = w->lm_head_scale != nullptr;
+        for (int li = 0; li < cfg->layers && ok; ++li) {
+            const dec_layer_weights& l = w->layers[li];
+            ok = l.wqkv_scale && l.wo_scale && l.w_gate_scale && l.w_up_scale && l.w_down_scale;
+        }
+        if (!ok) return fail(DEC_ERR_INVALID_ARG, "q8_row weights need every row-scale array");
+    }
+    if (cfg->sandwich_norms) {
+        for (int li = 0; li < cfg->layers; ++li)
+            if (!w->layers[li].post_attn_norm || !w->layers[li].post_ffn_norm)
+                return fail(DEC_ERR_INVALID_ARG, "sandwich norms need post_attn_norm and post_ffn_norm");
+    }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     dec_ctx* c = new dec_ctx();
     c->c = *cfg;
@@ -553,7 +710,7 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     c->qkv_rows = c->qd + 2 * c->kvd;
     c->max_pages = (k.max_context + 15) / 16;
     c->n_pages = k.n_pages > 0 ? k.n_pages : k.max_batch * c->max_pages;
-    c->max_tok = std::max(k.max_batch, k.prefill_chunk);
+    c->max_tok = std::max({k.max_batch, k.prefill_chunk, kMaxVerify});
     c->act_cols = std::max(k.ffn_inter, k.shared_inter);
     auto cleanup = [&](dec_status st_) {
         dec_free(c);
@@ -566,6 +723,19 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
             return cleanup(DEC_ERR_UNSUPPORTED);
         }
     }
+    const bool q8 = k.weight_format == 1;
+    // q8_row: int8 copy Q and row scales S of a [rows][cols] projection, plus the same
+    // integers as bf16 in W for the tensor-core path (exact: every int8 is a bf16 value)
+    auto load_q8 = [&](int8_t** Q, float** S, uint16_t** W, const void* src, const float* src_s, size_t rows,
+                       size_t cols) -> cudaError_t {
+        cudaError_t e = dmalloc(Q, rows * cols);
+        if (e == cudaSuccess) e = copy_in(*Q, src, rows * cols, st);
+        if (e == cudaSuccess) e = dmalloc(S, rows);
+        if (e == cudaSuccess) e = copy_in(*S, src_s, rows * 4, st);
+        if (e == cudaSuccess) e = dmalloc(W, rows * cols);
+        if (e == cudaSuccess) e = widen_i8_launch(*Q, *W, rows * cols, st);
+        return e;
+    };
 #define INIT_TRY(expr)                                                                         \
     do {                                                                                       \
         cudaError_t e_ = (expr);                                                               \
@@ -583,6 +753,8 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(copy_in(c->embed, w->embed, V * h * 2, st));
     if (k.tied_embeddings) {
         c->head = c->embed;
+    } else if (q8) {
+        INIT_TRY(load_q8(&c->head_q, &c->head_s, &c->head, w->lm_head, w->lm_head_scale, V, h));
     } else {
         INIT_TRY(dmalloc(&c->head, V * h));
         INIT_TRY(copy_in(c->head, w->lm_head, V * h * 2, st));
@@ -598,8 +770,12 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
         INIT_TRY(copy_in(L.attn_norm, s_.attn_norm, (size_t)h * 4, st));
         INIT_TRY(dmalloc(&L.ffn_norm, h));
         INIT_TRY(copy_in(L.ffn_norm, s_.ffn_norm, (size_t)h * 4, st));
-        INIT_TRY(dmalloc(&L.wqkv, (size_t)c->qkv_rows * h));
-        INIT_TRY(copy_in(L.wqkv, s_.wqkv, (size_t)c->qkv_rows * h * 2, st));
+        if (q8) {
+            INIT_TRY(load_q8(&L.qkv_q, &L.qkv_s, &L.wqkv, s_.wqkv, s_.wqkv_scale, c->qkv_rows, h));
+        } else {
+            INIT_TRY(dmalloc(&L.wqkv, (size_t)c->qkv_rows * h));
+            INIT_TRY(copy_in(L.wqkv, s_.wqkv, (size_t)c->qkv_rows * h * 2, st));
+        }
         if (k.qkv_bias) {
             INIT_TRY(dmalloc(&L.bqkv, c->qkv_rows));
             INIT_TRY(copy_in(L.bqkv, s_.bqkv, (size_t)c->qkv_rows * 4, st));
@@ -610,8 +786,18 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
             INIT_TRY(dmalloc(&L.k_norm, d));
             INIT_TRY(copy_in(L.k_norm, s_.k_norm, (size_t)d * 4, st));
         }
-        INIT_TRY(dmalloc(&L.wo, (size_t)h * c->qd));
-        INIT_TRY(copy_in(L.wo, s_.wo, (size_t)h * c->qd * 2, st));
+        if (k.sandwich_norms) {
+            INIT_TRY(dmalloc(&L.post_attn_norm, h));
+            INIT_TRY(copy_in(L.post_attn_norm, s_.post_attn_norm, (size_t)h * 4, st));
+            INIT_TRY(dmalloc(&L.post_ffn_norm, h));
+            INIT_TRY(copy_in(L.post_ffn_norm, s_.post_ffn_norm, (size_t)h * 4, st));
+        }
+        if (q8) {
+            INIT_TRY(load_q8(&L.wo_q, &L.wo_s, &L.wo, s_.wo, s_.wo_scale, h, c->qd));
+        } else {
+            INIT_TRY(dmalloc(&L.wo, (size_t)h * c->qd));
+            INIT_TRY(copy_in(L.wo, s_.wo, (size_t)h * c->qd * 2, st));
+        }
         if (k.n_experts > 0) {
             const size_t E = k.n_experts, Ie = k.expert_inter, Is = k.shared_inter;
             INIT_TRY(dmalloc(&L.wrouter, E * h));
@@ -630,6 +816,15 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
                     INIT_TRY(copy_in(L.sgate_vec, s_.s_gate_vec, (size_t)h * 4, st));
                 }
             }
+        } else if (q8) {
+            const size_t I = k.ffn_inter;
+            INIT_TRY(dmalloc(&L.gu_q, 2 * I * h));
+            INIT_TRY(interleave_rows_in(L.gu_q, s_.w_gate, s_.w_up, I, (size_t)h, st));
+            INIT_TRY(dmalloc(&L.gu_s, 2 * I));
+            INIT_TRY(interleave_rows_in(L.gu_s, s_.w_gate_scale, s_.w_up_scale, I, 4, st));
+            INIT_TRY(dmalloc(&L.wgu, 2 * I * h));
+            INIT_TRY(widen_i8_launch(L.gu_q, L.wgu, 2 * I * h, st));
+            INIT_TRY(load_q8(&L.down_q, &L.down_s, &L.wdown, s_.w_down, s_.w_down_scale, h, I));
         } else {
             INIT_TRY(dmalloc(&L.wgu, (size_t)2 * k.ffn_inter * h));
             INIT_TRY(interleave_in(L.wgu, s_.w_gate, s_.w_up, (size_t)k.ffn_inter, h, st));
@@ -656,7 +851,8 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     INIT_TRY(dmalloc(&c->d_tok, T));
     INIT_TRY(dmalloc(&c->d_prompt, (size_t)k.max_context));
     INIT_TRY(dmalloc(&c->d_pos, T));
-    INIT_TRY(dmalloc(&c->d_amax, (size_t)32 * k.max_batch));
+    c->head_rows = std::max(k.max_batch, kMaxVerify);  // decode rows, or the positions of one verify
+    INIT_TRY(dmalloc(&c->d_amax, (size_t)32 * c->head_rows));
     {
         const int qkv_rows = k.n_q_heads * d + 2 * k.n_kv_heads * d;
         const int m_max = std::max({k.vocab, qkv_rows, k.hidden, 2 * k.ffn_inter, 2 * k.shared_inter, k.n_experts});
@@ -678,8 +874,9 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
         INIT_TRY(cudaMemcpy(c->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice));
     }
     INIT_TRY(dmalloc(&c->x, (size_t)T * h));
+    if (k.sandwich_norms) INIT_TRY(dmalloc(&c->ysub, (size_t)T * h));
     INIT_TRY(dmalloc(&c->qkv, (size_t)T * c->qkv_rows));
-    INIT_TRY(dmalloc(&c->logits, (size_t)k.max_batch * V));
+    INIT_TRY(dmalloc(&c->logits, (size_t)c->head_rows * V));
     INIT_TRY(dmalloc(&c->xn, (size_t)T * std::max(h, c->qd)));
     INIT_TRY(dmalloc(&c->qrot, (size_t)T * c->qd));
     INIT_TRY(dmalloc(&c->attn, (size_t)T * c->qd));
@@ -701,8 +898,13 @@ dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t st
     }
     INIT_TRY(dmalloc(&c->d_err, 1));
     INIT_TRY(cudaMemsetAsync(c->d_err, 0, 4, st));
-    INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_stage), sizeof(int32_t) * (2 * T + c->max_pages + 16)));
-    INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_prompt), sizeof(int32_t) * (size_t)k.max_context));
+    c->stage_ints = stage_layout(c).total;
+    for (int i = 0; i < 2; ++i) {
+        INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_stage[i]), sizeof(int32_t) * c->stage_ints));
+        INIT_TRY(cudaEventCreateWithFlags(&c->ev_stage[i], cudaEventDisableTiming));
+    }
+    INIT_TRY(dmalloc(&c->d_ldst, 1));
+    INIT_TRY(cudaMemsetAsync(c->d_ldst, 0, sizeof(float*), st));
     INIT_TRY(cudaMallocHost(reinterpret_cast<void**>(&c->h_err), sizeof(int)));
     *c->h_err = 0;
 
@@ -731,10 +933,22 @@ dec_status dec_free(dec_ctx* c) {
         cudaFree(L.sgu);
         cudaFree(L.sdown);
         cudaFree(L.sgate_vec);
+        cudaFree(L.post_attn_norm);
+        cudaFree(L.post_ffn_norm);
+        cudaFree(L.qkv_q);
+        cudaFree(L.qkv_s);
+        cudaFree(L.wo_q);
+        cudaFree(L.wo_s);
+        cudaFree(L.gu_q);
+        cudaFree(L.gu_s);
+        cudaFree(L.down_q);
+        cudaFree(L.down_s);
         cudaFree(L.k_pool);
         cudaFree(L.v_pool);
     }
     if (c->head != c->embed) cudaFree(c->head);
+    cudaFree(c->head_q);
+    cudaFree(c->head_s);
     cudaFree(c->embed);
     cudaFree(c->final_norm);
     cudaFree(c->d_bt);
@@ -744,6 +958,7 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->d_amax);
     cudaFree(c->rope_tab);
     cudaFree(c->x);
+    cudaFree(c->ysub);
     cudaFree(c->qkv);
     cudaFree(c->logits);
     cudaFree(c->xn);
@@ -764,8 +979,12 @@ dec_status dec_free(dec_ctx* c) {
     cudaFree(c->moe_y);
     cudaFree(c->moe_ys);
     cudaFree(c->d_err);
-    if (c->h_stage) cudaFreeHost(c->h_stage);
-    if (c->h_prompt) cudaFreeHost(c->h_prompt);
+    cudaFree(c->d_ldst);
+    for (int i = 0; i < 2; ++i) {
+        if (c->ev_stage[i]) cudaEventSynchronize(c->ev_stage[i]);
+        if (c->h_stage[i]) cudaFreeHost(c->h_stage[i]);
+        if (c->ev_stage[i]) cudaEventDestroy(c->ev_stage[i]);
+    }
     if (c->h_err) cudaFreeHost(c->h_err);
     if (c->bridge) {
         if (c->stream) cudaStreamDestroy(c->stream);
@@ -809,14 +1028,21 @@ dec_status dec_prefill(dec_ctx* c, int32_t seq, const int32_t* tokens, int32_t T
     if (s != DEC_OK) return s;
     cudaStream_t st = c->stream;
     Scope scope(c);
-    s = upload_bt_row(c, seq, st);
+    // the sequence's block-table row and all the prompt tokens in one staging slot, then the
+    // chunks back to back with no host wait between them
+    int32_t* slot = nullptr;
+    int which = 0;
+    s = stage_acquire(c, &slot, &which);
+    if (s != DEC_OK) return s;
+    const StageLayout SL = stage_layout(c);
+    s = stage_bt_rows(c, slot, seq, seq + 1, st);
+    if (s != DEC_OK) return s;
+    memcpy(slot + SL.prompt, tokens, sizeof(int32_t) * T);
+    CUDA_TRY(cudaMemcpyAsync(c->d_prompt, slot + SL.prompt, sizeof(int32_t) * T, cudaMemcpyHostToDevice, st));
+    s = stage_release(c, which, st);
     if (s != DEC_OK) return s;
     const int C = k.prefill_chunk;
     int last_rows = 0;
-    // all the tokens in one copy (the pinned buffer is reused only after this call has
-    // synchronised), then the chunks back to back with no host wait between them
-    memcpy(c->h_prompt, tokens, sizeof(int32_t) * T);
-    CUDA_TRY(cudaMemcpyAsync(c->d_prompt, c->h_prompt, sizeof(int32_t) * T, cudaMemcpyHostToDevice, st));
     for (int done = 0; done < T; done += C) {
         const int n = std::min(C, T - done);
         CUDA_TRY(embed_launch(c->embed, c->d_prompt + done, n, k.hidden, c->x, st, false));
@@ -824,12 +1050,13 @@ dec_status dec_prefill(dec_ctx* c, int32_t seq, const int32_t* tokens, int32_t T
         if (s != DEC_OK) return s;
         last_rows = n;
     }
-    s = head(c, last_rows - 1, 1, st);
+    bool host = false;
+    float* dst = logits_target(c, logits_out, &host);
+    s = head(c, last_rows - 1, 1, st, dst, nullptr);
     if (s != DEC_OK) return s;
     c->seq_len[seq] = pos0 + T;
     c->last_rows = 1;
-    CUDA_TRY(cudaMemcpyAsync(c->h_err, c->d_err, 4, cudaMemcpyDeviceToHost, st));
-    return deliver_logits(c, logits_out, 1, st);
+    return host ? finish_host_logits(c, logits_out, 1, st) : DEC_OK;
 }
 
 dec_status dec_step(dec_ctx* c, const int32_t* tokens, const int32_t* pos, int32_t B, float* logits_out) {
@@ -845,31 +1072,47 @@ dec_status dec_step(dec_ctx* c, const int32_t* tokens, const int32_t* pos, int32
     }
     cudaStream_t st = c->stream;
     Scope scope(c);
-    bool bt_dirty = false;
+    int dirty_lo = B, dirty_hi = -1;
     for (int b = 0; b < B; ++b) {
         const size_t before = c->seq_pages[b].size();
         dec_status s = ensure_pages(c, b, pos[b] + 1);
         if (s != DEC_OK) return s;
-        if (c->seq_pages[b].size() != before) bt_dirty = true;
+        if (c->seq_pages[b].size() != before) {
+            dirty_lo = std::min(dirty_lo, b);
+            dirty_hi = std::max(dirty_hi, b);
+        }
     }
-    int32_t* stg = c->h_stage;
-    memcpy(stg, tokens, sizeof(int32_t) * B);
-    memcpy(stg + c->max_tok, pos, sizeof(int32_t) * B);
-    CUDA_TRY(cudaMemcpyAsync(c->d_tok, stg, sizeof(int32_t) * B, cudaMemcpyHostToDevice, st));
-    CUDA_TRY(cudaMemcpyAsync(c->d_pos, stg + c->max_tok, sizeof(int32_t) * B, cudaMemcpyHostToDevice, st));
-    if (bt_dirty)
-        CUDA_TRY(cudaMemcpyAsync(c->d_bt, c->h_bt.data(), sizeof(int32_t) * (size_t)B * c->max_pages,
-                                 cudaMemcpyHostToDevice, st));
+    bool host = false;
+    float* dst = logits_target(c, logits_out, &host);
+    // tokens, positions, the logits destination and any block-table rows that gained a
+    // page, through one staging slot (no host wait: the slot is fenced by its event)
+    int32_t* slot = nullptr;
+    int which = 0;
+    dec_status s = stage_acquire(c, &slot, &which);
+    if (s != DEC_OK) return s;
+    const StageLayout SL = stage_layout(c);
+    memcpy(slot + SL.tok, tokens, sizeof(int32_t) * B);
+    memcpy(slot + SL.pos, pos, sizeof(int32_t) * B);
+    memcpy(slot + SL.dst, &dst, sizeof(float*));
+    CUDA_TRY(cudaMemcpyAsync(c->d_tok, slot + SL.tok, sizeof(int32_t) * B, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(c->d_pos, slot + SL.pos, sizeof(int32_t) * B, cudaMemcpyHostToDevice, st));
+    CUDA_TRY(cudaMemcpyAsync(c->d_ldst, slot + SL.dst, sizeof(float*), cudaMemcpyHostToDevice, st));
+    if (dirty_hi >= 0) {
+        s = stage_bt_rows(c, slot, dirty_lo, dirty_hi + 1, st);
+        if (s != DEC_OK) return s;
+    }
+    s = stage_release(c, which, st);
+    if (s != DEC_OK) return s;
 
     auto it = c->graphs.find(B);
     if (it == c->graphs.end()) {
         cudaGraph_t g = nullptr;
         CUDA_TRY(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
-        dec_status s = DEC_OK;
+        s = DEC_OK;
         if (embed_launch(c->embed, c->d_tok, B, k.hidden, c->x, st, false) != cudaSuccess)
             s = fail(DEC_ERR_CUDA, "embed launch failed");
         if (s == DEC_OK) s = forward_layers(c, B, true, 0, 0, st);
-        if (s == DEC_OK) s = head(c, 0, B, st);
+        if (s == DEC_OK) s = head(c, 0, B, st, nullptr, c->d_ldst);
         cudaError_t e = cudaStreamEndCapture(st, &g);
         if (s != DEC_OK) {
             if (g) cudaGraphDestroy(g);
@@ -885,12 +1128,72 @@ dec_status dec_step(dec_ctx* c, const int32_t* tokens, const int32_t* pos, int32
     CUDA_TRY(cudaGraphLaunch(it->second, st));
     for (int b = 0; b < B; ++b) c->seq_len[b] = pos[b] + 1;
     c->last_rows = B;
-    CUDA_TRY(cudaMemcpyAsync(c->h_err, c->d_err, 4, cudaMemcpyDeviceToHost, st));
-    dec_status s = deliver_logits(c, logits_out, B, st);
+    return host ? finish_host_logits(c, logits_out, B, st) : DEC_OK;
+}
+
+dec_status dec_verify(dec_ctx* c, int32_t seq, const int32_t* tokens, int32_t N, int32_t pos0, float* logits_out) {
+    g_err.clear();
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    const dec_config& k = c->c;
+    if (seq < 0 || seq >= k.max_batch) return fail(DEC_ERR_INVALID_ARG, "seq out of range");
+    if (N <= 0 || !tokens) return fail(DEC_ERR_INVALID_ARG, "no tokens");
+    if (N > kMaxVerify) return fail(DEC_ERR_INVALID_ARG, "more than 8 positions");
+    if (pos0 < 0 || (int64_t)pos0 + N > k.max_context) return fail(DEC_ERR_CONTEXT_OVERFLOW, "pos0 + N > max_context");
+    if (pos0 != c->seq_len[seq]) return fail(DEC_ERR_INVALID_ARG, "pos0 must equal the sequence length");
+    for (int i = 0; i < N; ++i)
+        if (tokens[i] < 0 || tokens[i] >= k.vocab) return fail(DEC_ERR_INVALID_ARG, "token id out of range");
+    dec_status s = ensure_pages(c, seq, pos0 + N);
     if (s != DEC_OK) return s;
-    // the pinned staging area is reused by the next call
-    if (!logits_out || !is_host_ptr(logits_out)) CUDA_TRY(cudaStreamSynchronize(st));
+    cudaStream_t st = c->stream;
+    Scope scope(c);
+    int32_t* slot = nullptr;
+    int which = 0;
+    s = stage_acquire(c, &slot, &which);
+    if (s != DEC_OK) return s;
+    const StageLayout SL = stage_layout(c);
+    s = stage_bt_rows(c, slot, seq, seq + 1, st);
+    if (s != DEC_OK) return s;
+    memcpy(slot + SL.prompt, tokens, sizeof(int32_t) * N);
+    CUDA_TRY(cudaMemcpyAsync(c->d_prompt, slot + SL.prompt, sizeof(int32_t) * N, cudaMemcpyHostToDevice, st));
+    s = stage_release(c, which, st);
+    if (s != DEC_OK) return s;
+    // the N positions as one chunk: every projection streams its weights once for all of
+    // them (the GEMV takes up to 8 columns); chunk-causal attention over the cache
+    CUDA_TRY(embed_launch(c->embed, c->d_prompt, N, k.hidden, c->x, st, false));
+    s = forward_layers(c, N, false, seq, pos0, st);
+    if (s != DEC_OK) return s;
+    bool host = false;
+    float* dst = logits_target(c, logits_out, &host);
+    s = head(c, 0, N, st, dst, nullptr);
+    if (s != DEC_OK) return s;
+    c->seq_len[seq] = pos0 + N;
+    c->last_rows = N;
+    return host ? finish_host_logits(c, logits_out, N, st) : DEC_OK;
+}
+
+dec_status dec_truncate(dec_ctx* c, int32_t seq, int32_t len) {
+    g_err.clear();
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    if (seq < 0 || seq >= c->c.max_batch) return fail(DEC_ERR_INVALID_ARG, "seq out of range");
+    if (len < 0 || len > c->seq_len[seq]) return fail(DEC_ERR_INVALID_ARG, "len must be in [0, sequence length]");
+    // pages wholly past the new length go back to the pool; rows past it in the last kept
+    // page are stale and are overwritten before anything reads them (a query at position p
+    // reads rows 0..p only)
+    std::vector<int>& pg = c->seq_pages[seq];
+    const size_t keep = (size_t)(len + 15) / 16;
+    while (pg.size() > keep) {
+        c->free_pages.push_back(pg.back());
+        pg.pop_back();
+    }
+    c->seq_len[seq] = len;
     return DEC_OK;
+}
+
+dec_status dec_check(dec_ctx* c) {
+    if (!c) return fail(DEC_ERR_INVALID_ARG, "ctx is NULL");
+    g_err.clear();
+    Scope scope(c);
+    return sync_and_check(c, c->stream);
 }
 
 dec_status dec_last_argmax(dec_ctx* c, int32_t* out, int32_t B) {
@@ -899,7 +1202,8 @@ dec_status dec_last_argmax(dec_ctx* c, int32_t* out, int32_t B) {
     std::vector<unsigned long long> w((size_t)32 * B);
     CUDA_TRY(cudaMemcpyAsync(w.data(), c->d_amax, sizeof(unsigned long long) * 32 * B, cudaMemcpyDeviceToHost,
                              c->stream));
-    CUDA_TRY(cudaStreamSynchronize(c->stream));
+    dec_status s = sync_and_check(c, c->stream);
+    if (s != DEC_OK) return s;
     for (int b = 0; b < B; ++b) out[b] = argmax_unpack(w[(size_t)32 * b]);
     return DEC_OK;
 }
@@ -913,7 +1217,13 @@ dec_status dec_kv_write(dec_ctx* c, int32_t seq, int32_t layer, int32_t pos0, in
     dec_status s = ensure_pages(c, seq, pos0 + n);
     if (s != DEC_OK) return s;
     cudaStream_t st = c->stream;
-    s = upload_bt_row(c, seq, st);
+    int32_t* slot = nullptr;
+    int which = 0;
+    s = stage_acquire(c, &slot, &which);
+    if (s != DEC_OK) return s;
+    s = stage_bt_rows(c, slot, seq, seq + 1, st);
+    if (s != DEC_OK) return s;
+    s = stage_release(c, which, st);
     if (s != DEC_OK) return s;
     const size_t bytes = (size_t)n * c->kvd * 2;
     uint16_t *dk = nullptr, *dv = nullptr;
@@ -1157,6 +1467,101 @@ dec_status weight_gemv(const void* W, const void* x, int32_t B, int32_t N, int32
     a.cnt = S.cnt;
     a.err = S.err;
     CUDA_TRY(gemm_launch(plan, a, st, false));
+    return DEC_OK;
+}
+
+dec_status ffn_gate_up(const void* Wgu, const float* x, const float* gain, float eps, int32_t B, int32_t I, int32_t K,
+                       void* act, dec_stream_t stream) {
+    g_err.clear();
+    if (!Wgu || !x || !gain || !act) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
+    if (B <= 0 || I <= 0 || K <= 0 || !(eps > 0.f)) return fail(DEC_ERR_INVALID_ARG, "B, I, K, eps must be positive");
+    if (K % 8 != 0 || I % 2 != 0) return fail(DEC_ERR_UNSUPPORTED, "K must be a multiple of 8 and I even");
+    const int cap = device_smem_cap();
+    if (B > 8 || !gemv_fits(B, K, cap)) return fail(DEC_ERR_UNSUPPORTED, "B * K too large for the GEMV");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    Scratch& S = g_scratch[dev];
+    size_t one = 0;
+    if (!S.err) CUDA_TRY(grow(&S.err, &one, 1, true));
+    // the decode step's launch: RMSNorm prologue, interleaved gate/up rows, SiLU(g) * u epilogue
+    GemvArgs a{};
+    a.W = static_cast<const uint16_t*>(Wgu);
+    a.N = 2 * I;
+    a.K = K;
+    a.B = B;
+    a.xr = x;
+    a.g = gain;
+    a.eps = eps;
+    a.ldx = K;
+    a.act = static_cast<uint16_t*>(act);
+    a.ldact = I;
+    a.err = S.err;
+    a.smem_cap = cap;
+    CUDA_TRY(gemv_launch(a, GEMV_SWIGLU, st, device_sms(), false));
+    return DEC_OK;
+}
+
+dec_status weight_gemv_q8(const void* Wq, const float* scale, const void* x, int32_t B, int32_t N, int32_t K, float* y,
+                          dec_stream_t stream) {
+    g_err.clear();
+    if (!Wq || !scale || !x || !y) return fail(DEC_ERR_INVALID_ARG, "NULL pointer");
+    if (B <= 0 || N <= 0 || K <= 0) return fail(DEC_ERR_INVALID_ARG, "B, N, K must be positive");
+    if (K % 16 != 0) return fail(DEC_ERR_UNSUPPORTED, "K must be a multiple of 16");
+    const int cap = device_smem_cap();
+    if (B > 8 || !gemv_fits(B, K, cap, true)) return fail(DEC_ERR_UNSUPPORTED, "B * K too large for the q8 GEMV");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    Scratch& S = g_scratch[dev];
+    size_t one = 0;
+    if (!S.err) CUDA_TRY(grow(&S.err, &one, 1, true));
+    GemvArgs a{};
+    a.Wq = static_cast<const int8_t*>(Wq);
+    a.wscale = scale;
+    a.N = N;
+    a.K = K;
+    a.B = B;
+    a.xb = static_cast<const uint16_t*>(x);
+    a.ldx = K;
+    a.y = y;
+    a.ldy = N;
+    a.err = S.err;
+    a.smem_cap = cap;
+    CUDA_TRY(gemv_launch(a, GEMV_STORE, st, device_sms(), false));
+    return DEC_OK;
+}
+
+dec_status dec_check_standalone(dec_stream_t stream) {
+    g_err.clear();
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    CUDA_TRY(cudaStreamSynchronize(st));
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    auto it = g_scratch.find(dev);
+    if (it == g_scratch.end() || !it->second.err) return DEC_OK;
+    Scratch& S = it->second;
+    int e = 0;
+    CUDA_TRY(cudaMemcpy(&e, S.err, sizeof(int), cudaMemcpyDeviceToHost));
+    if (!e) return DEC_OK;
+    // clear the word and the GEMM tile counters an abandoned reduction can leave behind
+    CUDA_TRY(cudaMemset(S.err, 0, sizeof(int)));
+    if (S.cnt) CUDA_TRY(cudaMemset(S.cnt, 0, sizeof(int) * S.cnt_n));
+    CUDA_TRY(cudaDeviceSynchronize());
+    return fail(DEC_ERR_TIMEOUT, "a bounded device wait of a standalone call ran out; its output is not valid");
+}
+
+dec_status dec_test_fail_alloc(int32_t n) {
+    g_fail_alloc_in.store(n > 0 ? n : 0);
+    return DEC_OK;
+}
+
+dec_status dec_test_gemm_wait(int32_t extra_pieces, int64_t limit_cycles) {
+    if (extra_pieces < 0 || limit_cycles < 0) return fail(DEC_ERR_INVALID_ARG, "negative argument");
+    gemm_set_test_wait(extra_pieces, limit_cycles);
     return DEC_OK;
 }
 

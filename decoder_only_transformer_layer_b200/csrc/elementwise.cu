@@ -3,6 +3,8 @@
 //    embed scale 1;
 //  * RMSNorm of fp32 residual rows to bf16 (ANEDVD rmsnormColumn / rmsnormChunk:
 //    x * (1/sqrt(mean(x^2) + eps)) * w, written in the device input precision);
+//  * the sandwich norm's residual add (ANEDVD Engine.forward: the o_proj and FFN outputs
+//    pass through rmsnormFlat with their own gains before joining the residual), fp32;
 //  * moving cache rows between the paged pool and dense arrays (test hooks).
 // The greedy argmax is folded into the LM-head epilogues (gemv.cu, gemm_tc.cu) and the
 // MoE routing lives in moe.cu.
@@ -92,8 +94,67 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
     }
 }
 
+struct AddNormArgs {
+    float* x;        // [T][h] residual, updated
+    const float* y;  // [T][h] sublayer output
+    const float* g;
+    int h;
+    float eps;
+};
+
+// x[t] += y[t] * (1 / sqrt(mean(y[t]^2) + eps)) * g, one CTA per row, all in fp32.
+__global__ void __launch_bounds__(256) add_rmsnorm_kernel(AddNormArgs a) {
+    __shared__ float red[8];
+    pdl_trigger();
+    pdl_wait();
+    const int t = blockIdx.x;
+    const float* y = a.y + (size_t)t * a.h;
+    float ss = 0.f;
+    for (int i = threadIdx.x * 4; i < a.h; i += 256 * 4) {
+        const float4 v = *reinterpret_cast<const float4*>(y + i);
+        ss = fmaf(v.x, v.x, ss);
+        ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss);
+        ss = fmaf(v.w, v.w, ss);
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const float inv = 1.0f / sqrtf(tot / (float)a.h + a.eps);
+    float* x = a.x + (size_t)t * a.h;
+    for (int i = threadIdx.x * 4; i < a.h; i += 256 * 4) {
+        const float4 v = *reinterpret_cast<const float4*>(y + i);
+        const float4 g = *reinterpret_cast<const float4*>(a.g + i);
+        float4 r = *reinterpret_cast<const float4*>(x + i);
+        r.x += v.x * inv * g.x;
+        r.y += v.y * inv * g.y;
+        r.z += v.z * inv * g.z;
+        r.w += v.w * inv * g.w;
+        *reinterpret_cast<float4*>(x + i) = r;
+    }
+}
+
+// out[i] = bf16(q[i]): every int8 value is exactly a bf16 value (at most 8 significant bits).
+__global__ void widen_i8_kernel(const int8_t* q, uint16_t* out, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        out[i] = f2bf((float)q[i]);
+}
 
 }  // namespace
+
+cudaError_t widen_i8_launch(const int8_t* q, uint16_t* out, size_t n, cudaStream_t st) {
+    widen_i8_kernel<<<1184, 256, 0, st>>>(q, out, n);
+    return cudaGetLastError();
+}
+
+cudaError_t add_rmsnorm_launch(float* x, const float* y, const float* g, int T, int h, float eps, cudaStream_t st,
+                               bool pdl) {
+    AddNormArgs a{x, y, g, h, eps};
+    return launch_ex(add_rmsnorm_kernel, dim3(T), dim3(256), 0, st, pdl, a);
+}
 
 cudaError_t embed_launch(const uint16_t* E, const int32_t* tok, int B, int h, float* x, cudaStream_t st, bool pdl) {
     EmbedArgs a{E, tok, h, x};

@@ -24,7 +24,8 @@
 //    so one tile's epilogue overlaps the next tile's main loop;
 //  * warps 0-3 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
 //    32w..32w+31 = weight rows) and apply the epilogue: store (+bias, + greedy
-//    argmax), residual add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
+//    argmax; the destination may be read from device memory, and a null one stores
+//    nothing), residual add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -57,12 +58,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16() {
     return idesc_bf16_mn<BM, BN>();
 }
 
-// Apply the epilogue to the 16 values v[j] of (row, t0 + j). All lanes of the warp call
+// The STORE value: the optional final logit softcap c tanh(v / c).
+DEC_DEVINL float store_value(const GemmArgs& a, float v) {
+    return a.softcap > 0.f ? a.softcap * tanhf(v / a.softcap) : v;
+}
+
+// Apply the epilogue EPI to the 16 values v[j] of (row, t0 + j). All lanes of the warp call
 // it together (the SwiGLU pairing uses a shuffle). Every global load of a chunk is issued
 // before any store, so the 16 accesses overlap instead of waiting on one another.
-DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v)[16]) {
+template <int EPI>
+DEC_DEVINL void epilogue16_t(const GemmArgs& a, int row, int t0, const float (&v_in)[16]) {
     const bool row_ok = row < a.M;
-    if (a.epi == GEMM_SWIGLU) {
+    float v[16];
+    const float rs = (a.rscale && row_ok) ? a.rscale[row] : 1.f;  // q8_row: the row's scale
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = v_in[j] * rs;
+    if constexpr (EPI == GEMM_SWIGLU) {
         // rows 2i (gate) and 2i+1 (up) sit in adjacent lanes; the even lane finishes the
         // even tokens and the odd lane the odd ones, so every lane evaluates 8 SiLUs
         const bool odd = (threadIdx.x & 1) != 0;
@@ -77,10 +88,8 @@ DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v)[
                 a.act[(size_t)t * a.ldact + (row >> 1)] = f2bf(sg * u);
             }
         }
-        return;
-    }
-    if (!row_ok) return;
-    if (a.epi == GEMM_RESID) {
+    } else if constexpr (EPI == GEMM_RESID) {
+        if (!row_ok) return;
         float old[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) old[j] = t0 + j < a.N ? a.y[(size_t)(t0 + j) * a.ldy + row] : 0.f;
@@ -88,11 +97,31 @@ DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v)[
         for (int j = 0; j < 16; ++j)
             if (t0 + j < a.N) a.y[(size_t)(t0 + j) * a.ldy + row] = old[j] + v[j];
     } else {
+        if (!row_ok) return;
+        float* const y = a.y_ptr ? *a.y_ptr : a.y;  // null: only the greedy argmax is kept
+        if (!y) return;
         const float bias = a.bias ? a.bias[row] : 0.f;
+        // the softcap test stays outside the loop: the plain path carries no tanh at all
+        if (a.softcap > 0.f) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (t0 + j < a.N) a.y[(size_t)(t0 + j) * a.ldy + row] = v[j] + bias;
+            for (int j = 0; j < 16; ++j)
+                if (t0 + j < a.N) y[(size_t)(t0 + j) * a.ldy + row] = store_value(a, v[j] + bias);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (t0 + j < a.N) y[(size_t)(t0 + j) * a.ldy + row] = v[j] + bias;
+        }
     }
+}
+
+// The same with the epilogue chosen at run time (the persistent stream-K kernel).
+DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v_in)[16]) {
+    if (a.epi == GEMM_SWIGLU)
+        epilogue16_t<GEMM_SWIGLU>(a, row, t0, v_in);
+    else if (a.epi == GEMM_RESID)
+        epilogue16_t<GEMM_RESID>(a, row, t0, v_in);
+    else
+        epilogue16_t<GEMM_STORE>(a, row, t0, v_in);
 }
 
 // Greedy argmax of the STORE epilogue: warp maximum of the packed (value, row) words of
@@ -100,9 +129,18 @@ DEC_DEVINL void epilogue16(const GemmArgs& a, int row, int t0, const float (&v)[
 DEC_DEVINL void argmax16(const GemmArgs& a, int row, int t0, const float (&v)[16]) {
     const int lane = threadIdx.x & 31;
     const float bias = (a.bias && row < a.M) ? a.bias[row] : 0.f;
+    const float rs = (a.rscale && row < a.M) ? a.rscale[row] : 1.f;
+    float o[16];
+    if (a.softcap > 0.f) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j] = store_value(a, v[j] * rs + bias);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j] = v[j] * rs + bias;
+    }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-        unsigned long long w = (row < a.M && t0 + j < a.N) ? argmax_pack(v[j] + bias, row) : 0ull;
+        unsigned long long w = (row < a.M && t0 + j < a.N) ? argmax_pack(o[j], row) : 0ull;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const unsigned long long u = __shfl_xor_sync(0xffffffffu, w, o);
@@ -226,13 +264,16 @@ DEC_DEVINL int ld_acquire_gpu(const int* p) {
 }
 
 // Whether every piece of a shared tile has been published (tile counter >= P), waiting
-// for it (bounded: on time-out sets the error flag and returns false).
+// for it (bounded: on time-out sets the error flag and returns false). It is only called
+// once the CTA's own operand loads and MMAs have all completed and before it issues any
+// reduction load, so a CTA that gives up here leaves nothing in flight.
 DEC_DEVINL bool tile_ready(const GemmArgs& a, int tile, int P, volatile int* flag_s) {
     if (threadIdx.x == 0) {
         int r = 1;
         const long long st = clock64();
-        while (ld_acquire_gpu(&a.cnt[tile]) < P) {
-            if (clock64() - st > (1ll << 31)) {
+        const long long limit = a.wait_limit > 0 ? a.wait_limit : (1ll << 31);
+        while (ld_acquire_gpu(&a.cnt[tile]) < P + a.wait_extra) {
+            if (clock64() - st > limit) {
                 atomicExch(a.err, 1);
                 r = 0;
                 break;
@@ -615,6 +656,183 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+// ----------------------------------------------------------------- cluster split-K
+//
+// Products with one column tile (N <= 128: prefill chunks, decode batches) and few 128-row
+// tiles (the QKV, o_proj and down projections) split each tile's k blocks over the S <= 8
+// CTAs of one thread-block cluster. Every CTA streams 1/S of the tile's weights into its
+// own TMEM accumulator. The partial tiles are then summed inside the cluster through
+// distributed shared memory: CTA r owns a 32-row-aligned slice of the tile, receives every
+// CTA's partial of that slice, sums them in rank order (deterministic) and applies the
+// epilogue. There is no global round trip and no wait on CTAs outside the cluster.
+//
+// The receive area reuses the operand ring, so no CTA writes into another before every
+// CTA of the cluster has passed its accumulator barrier (all its loads consumed, all its
+// MMAs complete); every CTA executes the same two cluster barriers on every path.
+
+constexpr int kMaxSplitK = 8;
+
+// Rows of the tile each owner CTA finishes: a multiple of 32 (one warp's lanes).
+__host__ __device__ constexpr int splitk_rows(int S) { return 32 * ((4 + S - 1) / S); }
+
+template <int BN>
+__host__ __device__ constexpr size_t splitk_recv_bytes(int S) {
+    return (size_t)S * splitk_rows(S) * (BN + 4) * 4;
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs a,
+                       int S) {
+    using C = Cfg<BN>;
+    constexpr int LDR = BN + 4;  // receive rows padded by 16 bytes: conflict-free 16-byte stores
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* accf = empty + C::STAGES;  // the accumulator is complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+    float* recv = reinterpret_cast<float*>(smem);  // [S][rows per owner][LDR], over the drained ring
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)cluster_rank();
+    const int tile = blockIdx.x / S;
+    const int m0 = tile * BM;
+    const int nkb = (a.K + BK - 1) / BK;
+    const int kb0 = (int)((long long)nkb * rank / S), kb1 = (int)((long long)nkb * (rank + 1) / S);
+    const int iters = kb1 - kb0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(BN)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_trigger();
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer (each weight block
+            // is read once: evict-first)
+            const uint64_t pol = policy_evict_first();
+            const int pre = iters < C::STAGES ? iters : C::STAGES;
+            for (int i = 0; i < pre; ++i) {  // weights do not depend on the previous kernel
+                mbar_arrive_expect_tx(&full[i], C::STAGE);
+                tma_load_2d_hint(smem + i * C::STAGE, &tmA, (kb0 + i) * BK, m0, &full[i], pol);
+            }
+            pdl_wait();
+            for (int i = 0; i < pre; ++i) tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmB, (kb0 + i) * BK, 0, &full[i]);
+            for (int i = pre; i < iters; ++i) {
+                const int s = i % C::STAGES;
+                const uint32_t u = (uint32_t)(i / C::STAGES);
+                if (!mbar_wait_bounded(&empty[s], (u & 1u) ^ 1u, a.err)) break;
+                mbar_arrive_expect_tx(&full[s], C::STAGE);
+                tma_load_2d_hint(smem + s * C::STAGE, &tmA, (kb0 + i) * BK, m0, &full[s], pol);
+                tma_load_2d(smem + s * C::STAGE + C::A_BYTES, &tmB, (kb0 + i) * BK, 0, &full[s]);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        pdl_wait();
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_bf16<BN>();
+            const uint32_t sbase = smem_u32(smem);
+            for (int i = 0; i < iters; ++i) {
+                const int s = i % C::STAGES;
+                const uint32_t u = (uint32_t)(i / C::STAGES);
+                if (!mbar_wait_bounded(&full[s], u & 1u, a.err)) break;
+                tc_fence_after();
+                const uint32_t abase = sbase + s * C::STAGE, bbase = abase + C::A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    tc_mma(tmem, sdesc_sw128(abase + kk * 32), sdesc_sw128(bbase + kk * 32), idesc,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&empty[s]);
+            }
+            tc_commit(accf);
+        }
+        __syncwarp();
+    } else {
+        pdl_wait();
+        mbar_wait_bounded(accf, 0, a.err);  // on a time-out the partial is garbage, the flag is set
+        tc_fence_after();
+    }
+    // every CTA of the cluster has its accumulator: the operand rings are free to receive
+    cluster_sync();
+
+    const int RS = splitk_rows(S);
+    if (warp < 4) {
+        // push this CTA's partial of every row to the row's owner (lane = TMEM lane = row)
+        const int row = warp * 32 + lane;
+        const int owner = (warp * 32) / RS;  // a warp's 32 rows belong to one owner
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t dst = smem_u32(recv + ((size_t)rank * RS + (row - owner * RS)) * LDR);
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t r[32];
+            if (iters > 0) {
+                tmem_ld16_issue(tmem + lane_off + (uint32_t)c0, r);
+                tmem_ld16_issue(tmem + lane_off + (uint32_t)c0 + 16, r + 16);
+                tmem_ld_wait32(r);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) r[q] = 0u;
+            }
+#pragma unroll
+            for (int q = 0; q < 32; q += 4) dsmem_st4(dst + (c0 + q) * 4, owner, r[q], r[q + 1], r[q + 2], r[q + 3]);
+        }
+    }
+    cluster_sync();  // every partial has landed; from here on only local shared memory is read
+
+    if (warp < 4) {
+        // the owner sums its rows' partials in rank order and applies the epilogue:
+        // units of (32 rows, 16 columns), lane = row
+        const int my0 = rank * RS, my1 = min(BM, my0 + RS);
+        const int groups = my1 > my0 ? (my1 - my0) / 32 : 0;
+        for (int u = warp; u < groups * (BN / 16); u += 4) {
+            const int gi = u / (BN / 16), c0 = (u % (BN / 16)) * 16;
+            const int lr = gi * 32 + lane;
+            float acc[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+            for (int z = 0; z < S; ++z) {
+                const float4* src = reinterpret_cast<const float4*>(recv + ((size_t)z * RS + lr) * LDR + c0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 v = src[q];
+                    acc[4 * q] += v.x;
+                    acc[4 * q + 1] += v.y;
+                    acc[4 * q + 2] += v.z;
+                    acc[4 * q + 3] += v.w;
+                }
+            }
+            const int row = m0 + my0 + lr;
+            epilogue16_t<EPI>(a, row, c0, acc);
+            if constexpr (EPI == GEMM_STORE) {
+                if (a.amax) argmax16(a, row, c0, acc);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN) : "memory");
+    }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -677,6 +895,45 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, p.tmW, a);
 }
 
+template <int BN, int EPI>
+cudaError_t launch_splitk(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, bool pdl) {
+    using C = Cfg<BN>;
+    const int smem = C::SMEM;  // the receive area fits the operand ring (checked by the planner)
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(gemm_splitk_kernel<BN, EPI>), smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = (p.M + BM - 1) / BM;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles * p.splitk);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    attr[na].id = cudaLaunchAttributeClusterDimension;  // the S splits of a tile: one cluster
+    attr[na].val.clusterDim.x = p.splitk;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, gemm_splitk_kernel<BN, EPI>, p.tmA, p.tmB, a, p.splitk);
+}
+
+template <int EPI>
+cudaError_t launch_splitk_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, bool pdl) {
+    switch (p.bn) {
+        case 32: return launch_splitk<32, EPI>(p, a, st, pdl);
+        case 64: return launch_splitk<64, EPI>(p, a, st, pdl);
+        case 128: return launch_splitk<128, EPI>(p, a, st, pdl);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
 
 // Row-major bf16 [rows][K] read in 128B-swizzled boxes of 64 columns x box_rows rows.
@@ -687,6 +944,69 @@ cudaError_t tmap_bf16_rows(CUtensorMap* tm, const uint16_t* base, int rows, int 
 // Column tile: the whole batch up to 128 tokens; 256 beyond (more work per operand byte
 // once the product is compute-bound).
 int gemm_bn(int N) { return N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256; }
+
+namespace {
+// How many clusters of S CTAs of gemm_splitk_kernel<BN> the device holds at once (GPCs hold
+// whole clusters, so this can be below SMs / S). Cached per device, column tile and S.
+template <int BN>
+int splitk_resident(int S) {
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, int> known;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = known.find(std::make_pair(dev, S));
+    if (it != known.end()) return it->second;
+    int n = 0;
+    if (ensure_smem(reinterpret_cast<const void*>(gemm_splitk_kernel<BN, GEMM_STORE>), Cfg<BN>::SMEM) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(S * 8);
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = Cfg<BN>::SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_splitk_kernel<BN, GEMM_STORE>, &cfg) != cudaSuccess) {
+            n = 0;               // the stream-K kernel runs instead
+            cudaGetLastError();  // and the refused query leaves no error behind
+        }
+    }
+    known[std::make_pair(dev, S)] = n;
+    return n;
+}
+
+template <int BN>
+int splitk_pick(int tiles, int nkb, int num_sms) {
+    int S = num_sms / tiles;
+    if (S > kMaxSplitK) S = kMaxSplitK;
+    if (S > nkb / 4) S = nkb / 4;
+    for (; S >= 2; --S) {
+        if (tiles * S * 2 < num_sms) return 0;  // the clusters would leave most SMs idle
+        if (splitk_recv_bytes<BN>(S) > Cfg<BN>::STAGES * (size_t)Cfg<BN>::STAGE) continue;
+        if (splitk_resident<BN>(S) >= tiles) return S;  // one wave: every cluster resident at once
+    }
+    return 0;
+}
+}  // namespace
+
+// Cluster split-K for one column tile (N <= 128) when the 128-row tiles are too few to
+// fill the SMs: the largest S <= min(8, SMs / tiles, k blocks / 4) CTAs per tile whose
+// clusters are all resident at once and still cover at least half of the SMs; 0 = use the
+// persistent stream-K kernel.
+int gemm_splitk(int M, int N, int K, int num_sms) {
+    if (N > 128) return 0;
+    const int tiles = (M + BM - 1) / BM;
+    const int nkb = (K + BK - 1) / BK;
+    switch (gemm_bn(N)) {
+        case 32: return splitk_pick<32>(tiles, nkb, num_sms);
+        case 64: return splitk_pick<64>(tiles, nkb, num_sms);
+        default: return splitk_pick<128>(tiles, nkb, num_sms);
+    }
+}
 
 // One persistent CTA per SM, each with at least 8 k blocks of work.
 int gemm_ctas(int M, int N, int K, int num_sms) {
@@ -710,6 +1030,7 @@ cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16
     p->K = K;
     p->bn = gemm_bn(N);
     p->nc = gemm_ctas(M, N, K, num_sms);
+    p->splitk = gemm_splitk(M, N, K, num_sms);
     p->ws = ws;
     cudaError_t e = encode_2d(&p->tmA, A, M, K, BM);
     if (e != cudaSuccess) return e;
@@ -718,11 +1039,31 @@ cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16
     return encode_ws(&p->tmW, ws, 2 * p->nc, p->bn);
 }
 
+namespace {
+int g_test_extra = 0;
+long long g_test_limit = 0;
+}  // namespace
+
+void gemm_set_test_wait(int extra_pieces, long long limit_cycles) {
+    g_test_extra = extra_pieces > 0 ? extra_pieces : 0;
+    g_test_limit = limit_cycles > 0 ? limit_cycles : 0;
+}
+
 cudaError_t gemm_launch(const GemmPlan& p, GemmArgs a, cudaStream_t st, bool pdl) {
+    a.wait_extra = g_test_extra;
+    a.wait_limit = g_test_limit;
     a.M = p.M;
     a.N = p.N;
     a.K = p.K;
     a.ws = const_cast<float*>(p.ws);
+    if (p.splitk >= 2) {
+        switch (a.epi) {
+            case GEMM_STORE: return launch_splitk_bn<GEMM_STORE>(p, a, st, pdl);
+            case GEMM_RESID: return launch_splitk_bn<GEMM_RESID>(p, a, st, pdl);
+            case GEMM_SWIGLU: return launch_splitk_bn<GEMM_SWIGLU>(p, a, st, pdl);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (!a.cnt) return cudaErrorInvalidValue;
     switch (p.bn) {
         case 32: return launch_bn<32>(p, a, st, pdl);

@@ -14,6 +14,8 @@ enum GemvEpi { GEMV_STORE = 0, GEMV_RESID = 1, GEMV_SWIGLU = 2 };
 
 struct GemvArgs {
     const uint16_t* W;  // [N][K]
+    const int8_t* Wq;   // q8_row weights [N][K] (used instead of W when set), with
+    const float* wscale;  // one fp32 scale per row: W[n][k] = wscale[n] * Wq[n][k]
     int N, K;
     int B, nb;          // active columns; nb = compiled column count (set by the launcher)
     const uint16_t* xb; // bf16 input [B][ldx], or
@@ -22,17 +24,20 @@ struct GemvArgs {
     float eps;
     int ldx;
     float* y;           // STORE: y[b*ldy+n] = acc (+bias); RESID: y[b*ldy+n] += acc
+    float* const* y_ptr;  // STORE: when set, the destination is *y_ptr, read on the device
+                          // (a null *y_ptr stores nothing: only the greedy argmax is kept)
     int ldy;
     const float* bias;
     uint16_t* act;      // SWIGLU: act[b*ldact + n/2] = bf16(silu(acc[even]) * acc[odd])
     int ldact;
     unsigned long long* amax;  // STORE: per column, packed greedy argmax of y (null = off)
+    float softcap;      // STORE: > 0 stores (and takes the argmax of) softcap * tanh(v / softcap)
     int* err;
     int smem_cap;
 };
 
 int gemv_nb_for(int B);
-bool gemv_fits(int B, int K, int smem_cap);
+bool gemv_fits(int B, int K, int smem_cap, bool q8 = false);
 cudaError_t gemv_launch(GemvArgs a, int epi, cudaStream_t st, int num_sms, bool pdl);
 
 // ----------------------------------------------------------------- tcgen05 GEMM (prefill, large batch)
@@ -45,21 +50,35 @@ struct GemmPlan {
     CUtensorMap tmW;  // stream-K pieces (fp32 workspace), box 32 rows x BN
     const float* ws;
     int M, N, K, bn, nc;  // nc: persistent CTAs (stream-K ranges)
+    int splitk;           // >= 2: cluster split-K with this many CTAs per tile (N <= 128, few tiles)
 };
 
 struct GemmArgs {
     int M, N, K;      // D[M][N] = A[M][K] . B[N][K]^T, stored transposed: y[n][m]
     int epi;
     float* y;
+    float* const* y_ptr;  // STORE: as GemvArgs::y_ptr
     int ldy;
     const float* bias;
+    const float* rscale;  // per weight row: the product is scaled by rscale[m] first (null = 1);
+                          // q8_row weights run as their exact bf16 integer values times it
     uint16_t* act;
     int ldact;
     unsigned long long* amax;  // STORE: per token, packed greedy argmax of y (null = off)
+    float softcap;    // STORE: as GemvArgs::softcap
     float* ws;        // set from the plan: fp32 pieces of tiles shared between CTAs
     int* cnt;         // gemm_cnt_needed(M, N) zeroed tile counters (left zeroed)
     int* err;
+    int wait_extra;   // set by the launcher from gemm_set_test_wait (0 in normal use)
+    long long wait_limit;
 };
+
+// Test hook: the stream-K reduction wait of later GEMM launches waits for `extra_pieces`
+// more pieces than a tile has (so it cannot be satisfied) and gives up after `limit_cycles`
+// (0 = the normal limit). A CTA leaves that wait with every operand load and MMA of its
+// own completed and no reduction load issued, so it exits cleanly; the tile counters it
+// leaves behind must be zeroed by the host before the next launch.
+void gemm_set_test_wait(int extra_pieces, long long limit_cycles);
 
 // Build the tensor maps for one GEMM shape (host; encodes the A, B and workspace
 // addresses). ws holds gemm_ws_floats(num_sms) floats.
@@ -94,6 +113,8 @@ struct AttnDecodeArgs {
     const int32_t* pos;     // [B]
     int B, nq, nkv, d;
     float scale;
+    int window;             // > 0: the query at p attends keys p-window+1 .. p only
+    float softcap;          // > 0: each scaled score s becomes softcap * tanh(s / softcap)
     int splits;
     float* part;            // [B][nq][splits][d+2], or null: the splits merge inside a cluster (<= 16)
     int* counters;          // [B][nkv] (with part)
@@ -126,12 +147,20 @@ struct AttnPrefillArgs {
     const int32_t* block_row;
     int T, pos0, nq, nkv, d;
     float scale;
+    int window;         // as AttnDecodeArgs
+    float softcap;
     int splits;         // key splits (1..8): the split CTAs of a row block form one cluster
     uint16_t* out;      // [T][nq*d]
     int* err;
 };
 cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl);
 int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms);
+// Keys a prefill chunk's rows may see: the whole causal prefix, or with a window the last
+// window + T - 1 positions (sizes the key splits).
+inline int attn_prefill_span(int pos0, int T, int window) {
+    const int n = pos0 + T;
+    return window > 0 && window + T - 1 < n ? window + T - 1 : n;
+}
 
 // Greedy argmax as one 64-bit word per row: high half an order-preserving key of the
 // fp32 value, low half ~index (so on equal values the lowest index is the largest word).
@@ -149,6 +178,11 @@ __host__ __device__ inline int argmax_unpack(unsigned long long w) { return (int
 cudaError_t embed_launch(const uint16_t* E, const int32_t* tok, int B, int h, float* x, cudaStream_t st, bool pdl);
 cudaError_t rmsnorm_launch(const float* x, const float* g, int T, int h, float eps, uint16_t* out, cudaStream_t st,
                            bool pdl);
+// out[i] = bf16(q[i]) for n int8 values (exact: every int8 is a bf16 value).
+cudaError_t widen_i8_launch(const int8_t* q, uint16_t* out, size_t n, cudaStream_t st);
+// Sandwich norm: x[t] += y[t] * rsqrt(mean(y[t]^2) + eps) * g for T rows of h (fp32).
+cudaError_t add_rmsnorm_launch(float* x, const float* y, const float* g, int T, int h, float eps, cudaStream_t st,
+                               bool pdl);
 
 }  // namespace dec
 

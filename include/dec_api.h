@@ -22,8 +22,15 @@
  *     unless the status is DEC_ERR_CUDA; dec_last_error() gives a message
  *     (thread-local, valid until the next call on the same thread).
  *   - Work is enqueued on the caller's stream and is not synchronised unless
- *     a host output buffer is given (documented per call).
+ *     a host output buffer is given (documented per call). Host inputs are copied
+ *     through pinned staging memory before the call returns, so the caller may reuse
+ *     its buffers at once.
  *   - A stream argument of 0 means the legacy default stream.
+ *   - Device waits are bounded. A kernel whose wait runs out sets an error word and
+ *     returns (nothing traps). The word is reported as DEC_ERR_TIMEOUT by the next call
+ *     that synchronises (a host logits buffer, dec_last_argmax, dec_check; for the
+ *     standalone calls dec_check_standalone), which also clears it; the output of the
+ *     failed call is not valid.
  */
 #ifndef DEC_API_H
 #define DEC_API_H
@@ -72,6 +79,18 @@ typedef struct dec_config {
     int32_t page_size;       /* KV page size in tokens: 16 */
     int32_t prefill_chunk;   /* tokens per prefill chunk (layer-major within a chunk) */
     int32_t n_pages;         /* KV pages in the pool; 0 = max_batch * ceil(max_context / page_size) */
+    /* Sliding-window attention (ANEDVD attentionDecode .window; cortiq layer_window): layer l
+     * is windowed when sliding_window > 0 and (l + 1) % max(swa_pattern, 1) != 0, and its
+     * query at position p then attends positions p - sliding_window + 1 .. p only. */
+    int32_t sliding_window;
+    int32_t swa_pattern;
+    float attn_softcap;      /* > 0: each scaled attention score s becomes c * tanh(s / c) */
+    float final_softcap;     /* > 0: each logit v becomes c * tanh(v / c) (ANEDVD runHead) */
+    int32_t sandwich_norms;  /* 1: the o_proj and the dense FFN outputs are RMS-normalised with
+                                post_attn_norm / post_ffn_norm before each residual add */
+    int32_t weight_format;   /* 0: bf16 projections; 1: q8_row: the QKV, o, gate, up and down
+                                projections and the untied LM head are int8 [rows][cols] with one
+                                fp32 scale per row, W[n][k] = scale[n] * q[n][k] (dense models) */
 } dec_config;
 
 /* One layer's weights. Pointers may be host or device memory; they are read
@@ -95,6 +114,15 @@ typedef struct dec_layer_weights {
     const void* s_up;        /* bf16 [Is][h] */
     const void* s_down;      /* bf16 [h][Is] */
     const float* s_gate_vec; /* [h] or NULL */
+    const float* post_attn_norm; /* sandwich_norms: [h] */
+    const float* post_ffn_norm;  /* sandwich_norms: [h] */
+    /* weight_format 1: the row scales of wqkv, wo, w_gate, w_up, w_down (whose pointers then
+     * hold int8 values, same shapes) */
+    const float* wqkv_scale;     /* [nq*d + 2*nkv*d] */
+    const float* wo_scale;       /* [h] */
+    const float* w_gate_scale;   /* [I] */
+    const float* w_up_scale;     /* [I] */
+    const float* w_down_scale;   /* [h] */
 } dec_layer_weights;
 
 typedef struct dec_weights {
@@ -102,6 +130,7 @@ typedef struct dec_weights {
     const void* lm_head;              /* bf16 [V][h]; ignored when tied_embeddings */
     const float* final_norm;          /* [h] */
     const dec_layer_weights* layers;  /* host array of L entries */
+    const float* lm_head_scale;       /* weight_format 1: [V] row scales of the int8 lm_head */
 } dec_weights;
 
 typedef struct dec_ctx dec_ctx;
@@ -115,7 +144,8 @@ typedef struct dec_ctx dec_ctx;
  * do not handle (more than 16 query heads per kv head, head_dim other than 64 / 128,
  * hidden or an FFN width not a multiple of
  * 8, page_size other than 16, more than 256 experts or top_k above 16, MoE rows too long
- * for the grouped projections' shared memory) -> UNSUPPORTED; device memory -> OOM. */
+ * for the grouped projections' shared memory, sandwich norms or q8_row weights with MoE,
+ * q8_row with tied embeddings) -> UNSUPPORTED; device memory -> OOM. */
 dec_status dec_init(const dec_config* cfg, const dec_weights* w, dec_stream_t stream, dec_ctx** out);
 
 /* Release everything dec_init allocated (ANEDVD Engine.deinit). NULL is a no-op. */
@@ -130,8 +160,12 @@ dec_status dec_reset(dec_ctx* ctx, int32_t seq);
  * cfg.prefill_chunk tokens; every token's k and v enter the cache once.
  *   tokens     host int32 [T], each in [0, V)
  *   pos0       must equal the sequence's current length (each token enters once)
- *   logits_out fp32 [V]: logits of the last token; device pointer (stream-ordered) or
- *              host pointer (the call synchronises before returning); may be NULL.
+ *   logits_out fp32 [V]: logits of the last token. A device pointer is written by the
+ *              LM head directly (stream-ordered, no synchronisation); a host pointer
+ *              makes the call synchronise before returning; NULL stores no logits (the
+ *              greedy token is still kept for dec_last_argmax).
+ * Stream-ordered: with a device or NULL logits_out the call returns without waiting for
+ * the device.
  * Errors: T <= 0 or a bad token -> INVALID_ARG; pos0 + T > max_context ->
  * CONTEXT_OVERFLOW (exact fit allowed); no free page -> PAGES_EXHAUSTED. */
 dec_status dec_prefill(dec_ctx* ctx, int32_t seq, const int32_t* tokens, int32_t T, int32_t pos0,
@@ -141,13 +175,48 @@ dec_status dec_prefill(dec_ctx* ctx, int32_t seq, const int32_t* tokens, int32_t
  * MultiSeqKv): token tokens[b] at position pos[b] of sequence b.
  *   tokens, pos host int32 [B]; pos[b] must equal sequence b's current length and be
  *               < max_context (else CONTEXT_OVERFLOW).
- *   logits_out  fp32 [B][V], device or host pointer as in dec_prefill; may be NULL.
- * The whole step is replayed from a CUDA graph captured on the first call for each B. */
+ *   logits_out  fp32 [B][V], device or host pointer as in dec_prefill. NULL is the
+ *               greedy-only step: the LM head stores no logits at all and keeps only
+ *               each row's argmax (read with dec_last_argmax), as the pages' folded
+ *               head downloads the argmax instead of the full-vocabulary logits
+ *               (frink_models decoder.rs FoldedLmHead).
+ * The whole step is replayed from a CUDA graph captured on the first call for each B;
+ * the logits destination is read by the head on the device, so the same graph serves
+ * device, host and NULL outputs. With a device or NULL logits_out the call returns
+ * without waiting for the device. */
 dec_status dec_step(dec_ctx* ctx, const int32_t* tokens, const int32_t* pos, int32_t B, float* logits_out);
 
-/* Greedy tokens of the last dec_step / dec_prefill: argmax over each logits row,
- * lowest index on ties. out: host int32 [B] (B = rows of the last call). Synchronises. */
+/* Multi-position verify (cortiq_engine pipeline.rs forward_pair: several positions of one
+ * sequence share one pass over the weights, as speculative decoding's check of draft
+ * tokens needs): forward tokens[0..N-1] of sequence `seq` at positions pos0 .. pos0+N-1
+ * and return the logits of every position. Equal to N dec_step calls on that sequence,
+ * but each projection streams its weights once for all N positions.
+ *   tokens     host int32 [N], 1 <= N <= 8, each in [0, V)
+ *   pos0       must equal the sequence's current length; the N rows enter the cache
+ *   logits_out fp32 [N][V] (row i = position pos0 + i), device, host or NULL as in dec_prefill
+ * dec_last_argmax(ctx, out, N) then gives the greedy token of every position. Reject
+ * draft tokens with dec_truncate.
+ * Errors: N outside [1, 8], a bad token or pos0 -> INVALID_ARG; pos0 + N > max_context ->
+ * CONTEXT_OVERFLOW; no free page -> PAGES_EXHAUSTED. */
+dec_status dec_verify(dec_ctx* ctx, int32_t seq, const int32_t* tokens, int32_t N, int32_t pos0,
+                      float* logits_out);
+
+/* Roll sequence `seq` back to its first `len` positions (cortiq_engine pipeline.rs
+ * truncate_last: the KV rows of rejected draft tokens are dropped). Pages past the new
+ * length return to the pool. Host-side only: nothing is launched and nothing waits.
+ * Errors: len < 0 or len > the current length -> INVALID_ARG. */
+dec_status dec_truncate(dec_ctx* ctx, int32_t seq, int32_t len);
+
+/* Greedy tokens of the last dec_step / dec_prefill / dec_verify: argmax over each logits row,
+ * lowest index on ties. out: host int32 [B] (B = rows of the last call). Synchronises;
+ * returns DEC_ERR_TIMEOUT if a device wait of an earlier call ran out. */
 dec_status dec_last_argmax(dec_ctx* ctx, int32_t* out, int32_t B);
+
+/* Synchronise the context's stream and report whether a bounded device wait of any
+ * earlier call on this context ran out (DEC_ERR_TIMEOUT; the outputs of the failing call
+ * are not valid). Clears the error word and the tile counters an abandoned GEMM
+ * reduction leaves behind, so later calls run normally. */
+dec_status dec_check(dec_ctx* ctx);
 
 /* ---------------------------------------------------------------- standalone hot-path calls */
 
@@ -228,7 +297,46 @@ dec_status moe_experts(const void* x, const int32_t* idx, const float* w, int32_
 dec_status weight_gemv(const void* W, const void* x, int32_t B, int32_t N, int32_t K, float* y,
                        dec_stream_t stream);
 
+/* Synchronise `stream` and report whether a bounded device wait of a standalone call
+ * (weight_gemv, weight_gemv_q8, moe_experts) on the current device ran out since the last check:
+ * DEC_ERR_TIMEOUT, and the word and the GEMM tile counters are cleared. */
+dec_status dec_check_standalone(dec_stream_t stream);
+
+/* The front half of the dense SwiGLU FFN in one weight-streaming pass, as the decode step runs
+ * it (ANEDVD engine.zig: rmsnormColumn, then the fused gate/up/SiLU program of
+ * makeFusedFfnKernel): for each of B rows,
+ *   xn = bf16(x * (1 / sqrt(mean(x^2) + eps)) * gain),
+ *   act[i] = bf16(SiLU(Wgu[2i] . xn) * (Wgu[2i+1] . xn)),  SiLU(z) = z / (1 + e^-z).
+ *   Wgu  device bf16 [2I][K]: gate row i at 2i, up row i at 2i+1
+ *   x    device fp32 [B][K] (the residual stream); gain device fp32 [K]
+ *   act  device bf16 [B][I]
+ * B <= 8. Errors: NULL pointer or a non-positive size -> INVALID_ARG; K not a multiple of 8,
+ * I odd, B > 8 or B * K beyond shared memory -> UNSUPPORTED. Stream-ordered. */
+dec_status ffn_gate_up(const void* Wgu, const float* x, const float* gain, float eps, int32_t B, int32_t I, int32_t K,
+                       void* act, dec_stream_t stream);
+
+/* q8_row weight-streaming projection (cortiq_engine pipeline.rs q8_row_parts: int8 rows with
+ * one fp32 scale per row): y[b][n] = scale[n] * sum_k Wq[n][k] x[b][k], the row's exactly
+ * dequantised dot product, accumulated in fp32. Each weight byte is read once.
+ *   Wq device int8 [N][K]; scale device fp32 [N]; x device bf16 [B][K]; y device fp32 [B][N]
+ * Errors: NULL pointer or a non-positive size -> INVALID_ARG; K not a multiple of 16, B > 8
+ * or B * K beyond the kernel's shared memory -> UNSUPPORTED. Stream-ordered; a device wait
+ * that runs out is reported by dec_check_standalone. */
+dec_status weight_gemv_q8(const void* Wq, const float* scale, const void* x, int32_t B, int32_t N, int32_t K,
+                          float* y, dec_stream_t stream);
+
 /* ---------------------------------------------------------------- test hooks */
+
+/* The n-th device allocation made by the library from now on fails as if the device
+ * were out of memory (n = 0 turns this off). Process-wide; for testing the OOM paths. */
+dec_status dec_test_fail_alloc(int32_t n);
+
+/* The stream-K reduction wait of tensor-core GEMM launches made after this call waits
+ * for `extra_pieces` more partial tiles than exist, giving up after `limit_cycles` SM
+ * clock cycles (0 = the normal limit of about 1 s). (0, 0) restores normal operation.
+ * Process-wide; a dec_step graph keeps the setting it was captured with. For testing the
+ * DEC_ERR_TIMEOUT path: a CTA leaves that wait with all its loads and MMAs complete. */
+dec_status dec_test_gemm_wait(int32_t extra_pieces, int64_t limit_cycles);
 
 /* Copy cache rows [pos0, pos0+n) of layer `layer` of sequence `seq` to / from host
  * buffers bf16 [n][nkv*d] (k and v). dec_kv_write also extends the sequence's length

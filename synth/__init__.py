@@ -100,6 +100,8 @@ def dev_lib():
         for f in (L.syn_dev_fill_bf16, L.syn_dev_fill_bf16_as_f32):
             f.restype = C.c_int
             f.argtypes = [C.c_void_p, C.c_int64, C.c_uint64, C.c_uint64, C.c_double, C.c_double, C.c_void_p]
+        L.syn_dev_fill_i8.restype = C.c_int
+        L.syn_dev_fill_i8.argtypes = [C.c_void_p, C.c_int64, C.c_uint64, C.c_uint64, C.c_double, C.c_void_p]
         _dev = L
     return _dev
 

@@ -59,9 +59,27 @@ __global__ void fill_bf16_as_f32_kernel(float* out, int64_t n, uint64_t key, dou
         out[i] = __uint_as_float((uint32_t)round_bf16(mean + std * normal(key, (uint64_t)i)) << 16);
 }
 
+__global__ void fill_i8_kernel(int8_t* out, int64_t n, uint64_t key, double std) {
+    int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        double v = rint(std * normal(key, (uint64_t)i));
+        v = v > 127.0 ? 127.0 : (v < -127.0 ? -127.0 : v);
+        out[i] = (int8_t)v;
+    }
+}
+
 }  // namespace
 
 extern "C" {
+
+// out (device, int8 [n]) = clamp(nearbyint(std * z_i), -127, 127) for stream (seed, id).
+int syn_dev_fill_i8(void* out, int64_t n, uint64_t seed, uint64_t id, double std, cudaStream_t stream) {
+    if (n <= 0) return 0;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 148 * 32) blocks = 148 * 32;
+    fill_i8_kernel<<<blocks, 256, 0, stream>>>((int8_t*)out, n, stream_key(seed, id), std);
+    return (int)cudaGetLastError();
+}
 
 // out (device, bf16 bits [n]) = bf16(mean + std * z_i) for stream (seed, id). Returns cudaError_t.
 int syn_dev_fill_bf16(void* out, int64_t n, uint64_t seed, uint64_t id, double mean, double std,

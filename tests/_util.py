@@ -68,3 +68,25 @@ def gather_paged(pool, bt, ctx):
             n = rows.stop - rows.start
             out[b, rows] = pool[bt[b, j], :, :n].transpose(1, 0, 2)
     return out
+
+
+def perturb_inputs(weights):
+    """The same weights with every embedding value moved by one bf16 ulp (its lowest mantissa
+    bit flipped). fp32 accumulation makes a fraction of a percent of the bf16 roundings at every
+    rounding point of every layer land one ulp from the fp64 oracle's; this input change is of
+    the same order, so the oracle's response to it measures the noise floor of the problem."""
+    out = dict(weights)
+    out["embed"] = weights["embed"] ^ np.uint16(1)
+    return out
+
+
+def assert_within_conditioning(got, ref, ref_perturbed, factor=2.0, what=""):
+    """Parity where the fixed bar is tighter than the problem's conditioning (a deep
+    random-init stack moves its logits by percents when its inputs move by one bf16 ulp).
+    Pass if the fixed bar holds, or if the error is within `factor` times the oracle's own
+    response to the one-ulp input change on the same input."""
+    d, r = max_err(got, ref)
+    floor = float(np.max(np.abs(np.asarray(ref, np.float64) - np.asarray(ref_perturbed, np.float64))))
+    ok = (d <= ABS_TOL and r <= REL_TOL) or d <= factor * floor
+    assert ok, f"{what}: max|d|={d:.3e} rel={r:.3e}; one-ulp input floor {floor:.3e} (x{factor})"
+    return d, floor

@@ -38,6 +38,10 @@ def test_validation_errors_need_no_gpu():
     assert lib.dec_init(None, None, None, C.byref(h)) == 1
     assert lib.dec_prefill(None, 0, None, 0, 0, None) == 1
     assert lib.dec_step(None, None, None, 1, None) == 1
+    assert lib.dec_check(None) == 1
+    assert lib.dec_test_gemm_wait(-1, 0) == 1
+    assert lib.dec_test_gemm_wait(0, 0) == 0
+    assert lib.dec_test_fail_alloc(0) == 0
 
 
 def test_config_struct_matches_header():

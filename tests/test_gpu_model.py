@@ -198,3 +198,19 @@ def test_bad_arguments_are_refused_before_any_launch():
     d.reset(0)
     d.prefill(1, [1], 0)  # pages returned by reset are reused
     assert d.seq_len(1) == 1 and d.seq_len(0) == 0
+
+
+def test_decode_splits_of_unequal_length_merge_correctly():
+    # SmolLM2 shape at context 1024..1039: the batch-1 decode attention runs 9 context splits
+    # per kv head as one thread-block cluster, 8 of 8 pages and the last of 1 page. The short
+    # split finishes first and pushes its partial into the other CTAs' shared memory; that
+    # must wait until they are done with the page rings the receive area overlaps.
+    cfg = configs.with_layers(configs.SMOLLM2_135M, 3, max_context=1040)
+    w = synth.make_weights(cfg)
+    toks, greedy, ref, m = gated_run(cfg, w, 1024, 14, seq_seed=1900)
+    d = dec.Decoder(cfg, w)
+    assert_parity(d.prefill_logits(0, toks, 0), ref[0], what="prefill 1024")
+    for s, t in enumerate(greedy):
+        got = d.step_logits([t], [1024 + s])[0]
+        assert_parity(got, ref[s + 1], what=f"step {s} at position {1024 + s}")
+    d.close()
