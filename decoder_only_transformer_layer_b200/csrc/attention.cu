@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(128) rope_append_kernel(RopeAppendArgs a) {
     const int slot = p % kPage;
     const int nh = a.nq + 2 * a.nkv;
     const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
-    for (int hh = warp; hh < nh; hh += 4) {
+    for (int hh = blockIdx.y * 4 + warp; hh < nh; hh += 4 * gridDim.y) {
         if (hh < a.nq) {
             head_transform<D>(row + (size_t)hh * D, false, nullptr, a.q_norm, a.eps, true, p, a.rope_base,
                               a.q_out + ((size_t)t * a.nq + hh) * D, tab);
@@ -1020,8 +1020,11 @@ cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pd
 
 cudaError_t rope_append_launch(const RopeAppendArgs& a, cudaStream_t st, bool pdl) {
     if (a.T <= 0) return cudaSuccess;
-    if (a.d == 128) return launch_ex(rope_append_kernel<128>, dim3(a.T), dim3(128), 0, st, pdl, a);
-    if (a.d == 64) return launch_ex(rope_append_kernel<64>, dim3(a.T), dim3(128), 0, st, pdl, a);
+    // one (token, 4 heads) per CTA: each warp transforms one head, so a head costs one memory
+    // round trip instead of a warp walking a dozen heads one after another
+    const dim3 grid(a.T, (a.nq + 2 * a.nkv + 3) / 4);
+    if (a.d == 128) return launch_ex(rope_append_kernel<128>, grid, dim3(128), 0, st, pdl, a);
+    if (a.d == 64) return launch_ex(rope_append_kernel<64>, grid, dim3(128), 0, st, pdl, a);
     return cudaErrorInvalidValue;
 }
 

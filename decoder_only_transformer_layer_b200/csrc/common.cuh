@@ -186,6 +186,27 @@ DEC_DEVINL void dsmem_st2f(uint32_t saddr, int rank, float a, float b) {
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(a), "f"(b) : "memory");
 }
 
+// Bulk copy (DMA engine) of `bytes` from this CTA's shared memory to shared memory of
+// another CTA of the cluster: `dst` and `bar` are cluster addresses (dsmem_map), the bytes
+// complete as transactions on the destination's mbarrier. 16-byte aligned, size a multiple
+// of 16. The source must stay untouched (and its CTA alive) until the destination has
+// seen the bytes arrive.
+DEC_DEVINL void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst),
+                 "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (bulk
+// copies, TMA stores) issued after the next barrier.
+DEC_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// SiLU(g) = g / (1 + e^-g) with the hardware exponential and approximate divide (a few ulp
+// of fp32; the products it feeds are rounded to bf16). For g far below zero e^-g is +inf
+// and the quotient is -0.
+DEC_DEVINL float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
 // ----------------------------------------------------------------- RoPE angle
 
 // cos/sin of pos * base^(-2i/d), evaluated in fp64 and rounded to fp32.

@@ -62,35 +62,76 @@ struct NormArgs {
     uint16_t* out;
 };
 
+// Rows up to 256 threads x 4 floats x kNormU are held in registers: every load of a row is
+// issued before the first use (one memory round trip per row instead of one per piece), and
+// the gains, which do not depend on the previous kernel, are loaded before waiting on it.
+// Thread tid sums the squares of pieces tid, tid + 256, ... in that order on either path.
+constexpr int kNormU = 8;
+
 __global__ void __launch_bounds__(256) rmsnorm_kernel(NormArgs a) {
     __shared__ float red[8];
+    const int t = blockIdx.x, tid = threadIdx.x;
+    const bool held = a.h <= 256 * 4 * kNormU;
+    float4 gv[kNormU], xv[kNormU];
+    if (held) {
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u)
+            if ((u * 256 + tid) * 4 < a.h) gv[u] = *reinterpret_cast<const float4*>(a.g + (u * 256 + tid) * 4);
+    }
     pdl_trigger();
     pdl_wait();
-    const int t = blockIdx.x;
     const float* x = a.x + (size_t)t * a.h;
     float ss = 0.f;
-    for (int i = threadIdx.x * 4; i < a.h; i += 256 * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(x + i);
-        ss = fmaf(v.x, v.x, ss);
-        ss = fmaf(v.y, v.y, ss);
-        ss = fmaf(v.z, v.z, ss);
-        ss = fmaf(v.w, v.w, ss);
+    if (held) {
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u)
+            if ((u * 256 + tid) * 4 < a.h) xv[u] = *reinterpret_cast<const float4*>(x + (u * 256 + tid) * 4);
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            if ((u * 256 + tid) * 4 < a.h) {
+                ss = fmaf(xv[u].x, xv[u].x, ss);
+                ss = fmaf(xv[u].y, xv[u].y, ss);
+                ss = fmaf(xv[u].z, xv[u].z, ss);
+                ss = fmaf(xv[u].w, xv[u].w, ss);
+            }
+        }
+    } else {
+        for (int i = tid * 4; i < a.h; i += 256 * 4) {
+            const float4 v = *reinterpret_cast<const float4*>(x + i);
+            ss = fmaf(v.x, v.x, ss);
+            ss = fmaf(v.y, v.y, ss);
+            ss = fmaf(v.z, v.z, ss);
+            ss = fmaf(v.w, v.w, ss);
+        }
     }
     ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) tot += red[w];
     const float inv = 1.0f / sqrtf(tot / (float)a.h + a.eps);
     uint16_t* o = a.out + (size_t)t * a.h;
-    for (int i = threadIdx.x * 4; i < a.h; i += 256 * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(x + i);
-        const float4 g = *reinterpret_cast<const float4*>(a.g + i);
-        uint2 r;
-        r.x = pack_bf2(v.x * inv * g.x, v.y * inv * g.y);
-        r.y = pack_bf2(v.z * inv * g.z, v.w * inv * g.w);
-        *reinterpret_cast<uint2*>(o + i) = r;
+    if (held) {
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            const int i = (u * 256 + tid) * 4;
+            if (i < a.h) {
+                uint2 r;
+                r.x = pack_bf2(xv[u].x * inv * gv[u].x, xv[u].y * inv * gv[u].y);
+                r.y = pack_bf2(xv[u].z * inv * gv[u].z, xv[u].w * inv * gv[u].w);
+                *reinterpret_cast<uint2*>(o + i) = r;
+            }
+        }
+    } else {
+        for (int i = tid * 4; i < a.h; i += 256 * 4) {
+            const float4 v = *reinterpret_cast<const float4*>(x + i);
+            const float4 g = *reinterpret_cast<const float4*>(a.g + i);
+            uint2 r;
+            r.x = pack_bf2(v.x * inv * g.x, v.y * inv * g.y);
+            r.y = pack_bf2(v.z * inv * g.z, v.w * inv * g.w);
+            *reinterpret_cast<uint2*>(o + i) = r;
+        }
     }
 }
 
@@ -102,38 +143,80 @@ struct AddNormArgs {
     float eps;
 };
 
-// x[t] += y[t] * (1 / sqrt(mean(y[t]^2) + eps)) * g, one CTA per row, all in fp32.
+// x[t] += y[t] * (1 / sqrt(mean(y[t]^2) + eps)) * g, one CTA per row, all in fp32 (rows held
+// in registers as in rmsnorm_kernel).
 __global__ void __launch_bounds__(256) add_rmsnorm_kernel(AddNormArgs a) {
     __shared__ float red[8];
+    const int t = blockIdx.x, tid = threadIdx.x;
+    const bool held = a.h <= 256 * 4 * kNormU;
+    float4 gv[kNormU], yv[kNormU], xv[kNormU];
+    if (held) {
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u)
+            if ((u * 256 + tid) * 4 < a.h) gv[u] = *reinterpret_cast<const float4*>(a.g + (u * 256 + tid) * 4);
+    }
     pdl_trigger();
     pdl_wait();
-    const int t = blockIdx.x;
     const float* y = a.y + (size_t)t * a.h;
+    float* x = a.x + (size_t)t * a.h;
     float ss = 0.f;
-    for (int i = threadIdx.x * 4; i < a.h; i += 256 * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(y + i);
-        ss = fmaf(v.x, v.x, ss);
-        ss = fmaf(v.y, v.y, ss);
-        ss = fmaf(v.z, v.z, ss);
-        ss = fmaf(v.w, v.w, ss);
+    if (held) {
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            if ((u * 256 + tid) * 4 < a.h) {
+                yv[u] = *reinterpret_cast<const float4*>(y + (u * 256 + tid) * 4);
+                xv[u] = *reinterpret_cast<const float4*>(x + (u * 256 + tid) * 4);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            if ((u * 256 + tid) * 4 < a.h) {
+                ss = fmaf(yv[u].x, yv[u].x, ss);
+                ss = fmaf(yv[u].y, yv[u].y, ss);
+                ss = fmaf(yv[u].z, yv[u].z, ss);
+                ss = fmaf(yv[u].w, yv[u].w, ss);
+            }
+        }
+    } else {
+        for (int i = tid * 4; i < a.h; i += 256 * 4) {
+            const float4 v = *reinterpret_cast<const float4*>(y + i);
+            ss = fmaf(v.x, v.x, ss);
+            ss = fmaf(v.y, v.y, ss);
+            ss = fmaf(v.z, v.z, ss);
+            ss = fmaf(v.w, v.w, ss);
+        }
     }
     ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) tot += red[w];
     const float inv = 1.0f / sqrtf(tot / (float)a.h + a.eps);
-    float* x = a.x + (size_t)t * a.h;
-    for (int i = threadIdx.x * 4; i < a.h; i += 256 * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(y + i);
-        const float4 g = *reinterpret_cast<const float4*>(a.g + i);
-        float4 r = *reinterpret_cast<const float4*>(x + i);
-        r.x += v.x * inv * g.x;
-        r.y += v.y * inv * g.y;
-        r.z += v.z * inv * g.z;
-        r.w += v.w * inv * g.w;
-        *reinterpret_cast<float4*>(x + i) = r;
+    if (held) {
+#pragma unroll
+        for (int u = 0; u < kNormU; ++u) {
+            const int i = (u * 256 + tid) * 4;
+            if (i < a.h) {
+                float4 r = xv[u];
+                r.x += yv[u].x * inv * gv[u].x;
+                r.y += yv[u].y * inv * gv[u].y;
+                r.z += yv[u].z * inv * gv[u].z;
+                r.w += yv[u].w * inv * gv[u].w;
+                *reinterpret_cast<float4*>(x + i) = r;
+            }
+        }
+    } else {
+        for (int i = tid * 4; i < a.h; i += 256 * 4) {
+            const float4 v = *reinterpret_cast<const float4*>(y + i);
+            const float4 g = *reinterpret_cast<const float4*>(a.g + i);
+            float4 r = *reinterpret_cast<const float4*>(x + i);
+            r.x += v.x * inv * g.x;
+            r.y += v.y * inv * g.y;
+            r.z += v.z * inv * g.z;
+            r.w += v.w * inv * g.w;
+            *reinterpret_cast<float4*>(x + i) = r;
+        }
     }
 }
 

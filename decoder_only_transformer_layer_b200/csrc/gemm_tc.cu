@@ -84,32 +84,46 @@ DEC_DEVINL void epilogue16_t(const GemmArgs& a, int row, int t0, const float (&v
             const float g = odd ? other : own, u = odd ? own : other;
             const int t = t0 + 2 * jj + (odd ? 1 : 0);
             if (row_ok && t < a.N) {
-                const float sg = g * (1.0f / (1.0f + expf(-g)));
+                const float sg = silu_f(g);
                 a.act[(size_t)t * a.ldact + (row >> 1)] = f2bf(sg * u);
             }
         }
     } else if constexpr (EPI == GEMM_RESID) {
         if (!row_ok) return;
+        float* yr = a.y + (size_t)t0 * a.ldy + row;
+        const size_t ld = a.ldy;
         float old[16];
+        if (t0 + 16 <= a.N) {  // a whole chunk: no per-token test
 #pragma unroll
-        for (int j = 0; j < 16; ++j) old[j] = t0 + j < a.N ? a.y[(size_t)(t0 + j) * a.ldy + row] : 0.f;
+            for (int j = 0; j < 16; ++j) old[j] = yr[j * ld];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (t0 + j < a.N) a.y[(size_t)(t0 + j) * a.ldy + row] = old[j] + v[j];
+            for (int j = 0; j < 16; ++j) yr[j * ld] = old[j] + v[j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) old[j] = t0 + j < a.N ? yr[j * ld] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (t0 + j < a.N) yr[j * ld] = old[j] + v[j];
+        }
     } else {
         if (!row_ok) return;
         float* const y = a.y_ptr ? *a.y_ptr : a.y;  // null: only the greedy argmax is kept
         if (!y) return;
         const float bias = a.bias ? a.bias[row] : 0.f;
+        float* yr = y + (size_t)t0 * a.ldy + row;
+        const size_t ld = a.ldy;
         // the softcap test stays outside the loop: the plain path carries no tanh at all
         if (a.softcap > 0.f) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                if (t0 + j < a.N) y[(size_t)(t0 + j) * a.ldy + row] = store_value(a, v[j] + bias);
+                if (t0 + j < a.N) yr[j * ld] = store_value(a, v[j] + bias);
+        } else if (t0 + 16 <= a.N) {  // a whole chunk: no per-token test
+#pragma unroll
+            for (int j = 0; j < 16; ++j) yr[j * ld] = v[j] + bias;
         } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                if (t0 + j < a.N) y[(size_t)(t0 + j) * a.ldy + row] = v[j] + bias;
+                if (t0 + j < a.N) yr[j * ld] = v[j] + bias;
         }
     }
 }
@@ -477,6 +491,11 @@ __global__ void __launch_bounds__(192, 1)
     int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);  // reduction wait timed out
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmW);
+    }
     const Work w = make_work(a, BN);
     const int c = blockIdx.x;
     const Range rg = cta_range(w, c);
@@ -661,14 +680,17 @@ __global__ void __launch_bounds__(192, 1)
 // Products with one column tile (N <= 128: prefill chunks, decode batches) and few 128-row
 // tiles (the QKV, o_proj and down projections) split each tile's k blocks over the S <= 8
 // CTAs of one thread-block cluster. Every CTA streams 1/S of the tile's weights into its
-// own TMEM accumulator. The partial tiles are then summed inside the cluster through
-// distributed shared memory: CTA r owns a 32-row-aligned slice of the tile, receives every
-// CTA's partial of that slice, sums them in rank order (deterministic) and applies the
-// epilogue. There is no global round trip and no wait on CTAs outside the cluster.
+// own TMEM accumulator. The partial tiles are then summed inside the cluster: each CTA
+// writes its partial into its own shared memory, and once every CTA of the cluster is past
+// its MMAs (one cluster barrier) the DMA engine copies each 32-row-aligned slice to the CTA
+// that owns it (cp.async.bulk shared::cta -> shared::cluster, completing on the owner's
+// mbarrier). The owner sums the S partials of its rows in rank order (deterministic) and
+// applies the epilogue. There is no global round trip and no wait on CTAs outside the
+// cluster; a last cluster barrier keeps every CTA (the copies' sources) alive until the
+// owners have their bytes.
 //
-// The receive area reuses the operand ring, so no CTA writes into another before every
-// CTA of the cluster has passed its accumulator barrier (all its loads consumed, all its
-// MMAs complete); every CTA executes the same two cluster barriers on every path.
+// Shared memory after the main loop (it overlays the drained operand ring):
+// [recv: S slots x rows per owner x LDR floats][stage: BM x LDR floats], LDR = BN + 4.
 
 constexpr int kMaxSplitK = 8;
 
@@ -680,6 +702,26 @@ __host__ __device__ constexpr size_t splitk_recv_bytes(int S) {
     return (size_t)S * splitk_rows(S) * (BN + 4) * 4;
 }
 
+// The largest receive area over every S <= kMaxSplitK, then this CTA's own partial.
+template <int BN>
+__host__ __device__ constexpr size_t splitk_exchange_bytes() {
+    size_t m = 0;
+    for (int S = 2; S <= kMaxSplitK; ++S) m = splitk_recv_bytes<BN>(S) > m ? splitk_recv_bytes<BN>(S) : m;
+    return m + (size_t)BM * (BN + 4) * 4;
+}
+
+template <int BN>
+__host__ __device__ constexpr size_t splitk_body_bytes() {
+    return (size_t)Cfg<BN>::STAGES * Cfg<BN>::STAGE > splitk_exchange_bytes<BN>()
+               ? (size_t)Cfg<BN>::STAGES * Cfg<BN>::STAGE
+               : splitk_exchange_bytes<BN>();
+}
+
+template <int BN>
+__host__ __device__ constexpr int splitk_smem() {
+    return (int)splitk_body_bytes<BN>() + 1024 + 256;
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs a,
@@ -688,11 +730,13 @@ __global__ void __launch_bounds__(192, 1)
     constexpr int LDR = BN + 4;  // receive rows padded by 16 bytes: conflict-free 16-byte stores
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + splitk_body_bytes<BN>());
     uint64_t* empty = full + C::STAGES;
     uint64_t* accf = empty + C::STAGES;  // the accumulator is complete
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+    uint64_t* recvb = accf + 1;          // the other CTAs' slices of this CTA's rows have landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recvb + 1);
     float* recv = reinterpret_cast<float*>(smem);  // [S][rows per owner][LDR], over the drained ring
+    float* stage = recv + splitk_recv_bytes<BN>(S) / 4;  // [BM][LDR]: this CTA's partial
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_rank();
@@ -701,13 +745,24 @@ __global__ void __launch_bounds__(192, 1)
     const int nkb = (a.K + BK - 1) / BK;
     const int kb0 = (int)((long long)nkb * rank / S), kb1 = (int)((long long)nkb * (rank + 1) / S);
     const int iters = kb1 - kb0;
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
 
+    const int RS = splitk_rows(S);
+    const int my0 = rank * RS, my1 = min(BM, my0 + RS);  // the rows this CTA finishes
+    const uint32_t slice_bytes = (uint32_t)RS * LDR * 4;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
+        mbar_init(recvb, 1);
+        // the S - 1 other CTAs each send (my1 - my0) rows; armed before the first cluster
+        // barrier, so no byte can arrive before the count
+        if (my1 > my0) mbar_arrive_expect_tx(recvb, (uint32_t)(S - 1) * (my1 - my0) * LDR * 4);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -770,16 +825,11 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait_bounded(accf, 0, a.err);  // on a time-out the partial is garbage, the flag is set
         tc_fence_after();
     }
-    // every CTA of the cluster has its accumulator: the operand rings are free to receive
-    cluster_sync();
-
-    const int RS = splitk_rows(S);
     if (warp < 4) {
-        // push this CTA's partial of every row to the row's owner (lane = TMEM lane = row)
+        // this CTA's partial into its own (drained) ring: lane = TMEM lane = row
         const int row = warp * 32 + lane;
-        const int owner = (warp * 32) / RS;  // a warp's 32 rows belong to one owner
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t dst = smem_u32(recv + ((size_t)rank * RS + (row - owner * RS)) * LDR);
+        float* dst = stage + (size_t)row * LDR;
         for (int c0 = 0; c0 < BN; c0 += 32) {
             uint32_t r[32];
             if (iters > 0) {
@@ -791,24 +841,39 @@ __global__ void __launch_bounds__(192, 1)
                 for (int q = 0; q < 32; ++q) r[q] = 0u;
             }
 #pragma unroll
-            for (int q = 0; q < 32; q += 4) dsmem_st4(dst + (c0 + q) * 4, owner, r[q], r[q + 1], r[q + 2], r[q + 3]);
+            for (int q = 0; q < 32; q += 4)
+                *reinterpret_cast<uint4*>(dst + c0 + q) = make_uint4(r[q], r[q + 1], r[q + 2], r[q + 3]);
+        }
+        fence_proxy_async_smem();  // the copies below read these writes through the async proxy
+    }
+    // every CTA of the cluster has its accumulator (its ring is free to receive) and its
+    // partial staged
+    cluster_sync();
+
+    if (threadIdx.x == 0) {
+        // one DMA copy per other owner: my partial of its rows into its slot [rank]
+        for (int o = 0; o < S; ++o) {
+            const int o0 = o * RS, o1 = min(BM, o0 + RS);
+            if (o == rank || o1 <= o0) continue;
+            const uint32_t dst = dsmem_map(smem_u32(recv) + (uint32_t)rank * slice_bytes, o);
+            bulk_s2cluster(dst, stage + (size_t)o0 * LDR, (uint32_t)(o1 - o0) * LDR * 4, dsmem_map(smem_u32(recvb), o));
         }
     }
-    cluster_sync();  // every partial has landed; from here on only local shared memory is read
 
-    if (warp < 4) {
+    if (warp < 4 && my1 > my0) {
         // the owner sums its rows' partials in rank order and applies the epilogue:
         // units of (32 rows, 16 columns), lane = row
-        const int my0 = rank * RS, my1 = min(BM, my0 + RS);
-        const int groups = my1 > my0 ? (my1 - my0) / 32 : 0;
-        for (int u = warp; u < groups * (BN / 16); u += 4) {
+        const bool got = mbar_wait_bounded(recvb, 0, a.err);
+        const int groups = (my1 - my0) / 32;
+        for (int u = warp; got && u < groups * (BN / 16); u += 4) {
             const int gi = u / (BN / 16), c0 = (u % (BN / 16)) * 16;
             const int lr = gi * 32 + lane;
             float acc[16];
 #pragma unroll
             for (int q = 0; q < 16; ++q) acc[q] = 0.f;
             for (int z = 0; z < S; ++z) {
-                const float4* src = reinterpret_cast<const float4*>(recv + ((size_t)z * RS + lr) * LDR + c0);
+                const float* zrow = z == rank ? stage + (size_t)(my0 + lr) * LDR : recv + ((size_t)z * RS + lr) * LDR;
+                const float4* src = reinterpret_cast<const float4*>(zrow + c0);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float4 v = src[q];
@@ -825,6 +890,9 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     }
+    // the copies out of this CTA's shared memory have landed at their owners (each owner
+    // arrives here only after its barrier completed): only now may any CTA exit
+    cluster_sync();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -897,8 +965,7 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
 
 template <int BN, int EPI>
 cudaError_t launch_splitk(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, bool pdl) {
-    using C = Cfg<BN>;
-    const int smem = C::SMEM;  // the receive area fits the operand ring (checked by the planner)
+    const int smem = splitk_smem<BN>();
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(gemm_splitk_kernel<BN, EPI>), smem);
     if (e != cudaSuccess) return e;
     const int tiles = (p.M + BM - 1) / BM;
@@ -958,11 +1025,12 @@ int splitk_resident(int S) {
     auto it = known.find(std::make_pair(dev, S));
     if (it != known.end()) return it->second;
     int n = 0;
-    if (ensure_smem(reinterpret_cast<const void*>(gemm_splitk_kernel<BN, GEMM_STORE>), Cfg<BN>::SMEM) == cudaSuccess) {
+    if (ensure_smem(reinterpret_cast<const void*>(gemm_splitk_kernel<BN, GEMM_STORE>), splitk_smem<BN>()) ==
+        cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(S * 8);
         cfg.blockDim = dim3(192);
-        cfg.dynamicSmemBytes = Cfg<BN>::SMEM;
+        cfg.dynamicSmemBytes = splitk_smem<BN>();
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = S;
@@ -986,7 +1054,6 @@ int splitk_pick(int tiles, int nkb, int num_sms) {
     if (S > nkb / 4) S = nkb / 4;
     for (; S >= 2; --S) {
         if (tiles * S * 2 < num_sms) return 0;  // the clusters would leave most SMs idle
-        if (splitk_recv_bytes<BN>(S) > Cfg<BN>::STAGES * (size_t)Cfg<BN>::STAGE) continue;
         if (splitk_resident<BN>(S) >= tiles) return S;  // one wave: every cluster resident at once
     }
     return 0;

@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvArgs a) {
 #pragma unroll
                         for (int w = 0; w < kWarps; ++w) u += rd[w * 64 + tid + NB];
                         u *= a.wscale[row + 1];
-                        const float sg = v * (1.0f / (1.0f + expf(-v)));
+                        const float sg = silu_f(v);
                         a.act[(size_t)b * a.ldact + (row >> 1)] = f2bf(sg * u);
                     }
                 }
@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvArgs a) {
                 if ((r_in & 1) == 0 && half == 0 && valid && ok && lane < a.B) {
                     const float g = rd[warp * 16 + lane] + rd[(warp + 1) * 16 + lane];
                     const float u = rd[(warp + 2) * 16 + lane] + rd[(warp + 3) * 16 + lane];
-                    const float sg = g * (1.0f / (1.0f + expf(-g)));
+                    const float sg = silu_f(g);
                     a.act[(size_t)lane * a.ldact + (row >> 1)] = f2bf(sg * u);
                 }
             }

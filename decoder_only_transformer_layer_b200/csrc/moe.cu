@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(GroupedGemvAr
         } else if ((r_in & 1) == 0 && half == 0 && valid && ok && lane < c) {
             const float gv = red[warp * 16 + lane] + red[(warp + 1) * 16 + lane];
             const float uv = red[(warp + 2) * 16 + lane] + red[(warp + 3) * 16 + lane];
-            const float sg = gv * (1.0f / (1.0f + expf(-gv)));
+            const float sg = silu_f(gv);
             a.act[(size_t)(p0 + lane) * a.ldact + (row >> 1)] = f2bf(sg * uv);
         }
         consumer_sync();
@@ -442,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* empty = full + kTcMaxStages;
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs_off);
     uint8_t* ring = smem + L.ring_off;
+    if (threadIdx.x == 0) prefetch_tmap(&tmW);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < L.stages; ++s) {
@@ -562,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int tq = tok + (q & 1), rq = r0 + ((q >> 1) << 3);
                     if (tq < c) {
                         const float gv = acc[q];
-                        const float sg = gv * (1.0f / (1.0f + expf(-gv)));
+                        const float sg = silu_f(gv);
                         a.act[(size_t)(p0 + tq) * a.ldact + (rq >> 1)] = f2bf(sg * up[q]);
                     }
                 }

@@ -29,6 +29,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_mn() {
            | ((uint32_t)(M >> 4) << 24); // M
 }
 
+// Fetch a tensor map (a kernel parameter) into the descriptor cache ahead of its first use.
+DEC_DEVINL void prefetch_tmap(const void* tm) { asm volatile("prefetch.tensormap [%0];" ::"l"(tm) : "memory"); }
+
 DEC_DEVINL void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
