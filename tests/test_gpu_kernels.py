@@ -101,6 +101,14 @@ def test_gqa_decode_small_ragged(rope, new):
             assert np.array_equal(kg[b, :p], ko[b, :p])
 
 
+@pytest.mark.parametrize("nq,nkv,d,pos", [(16, 16, 128, [300]), (16, 16, 128, [2046]), (16, 1, 64, [300, 999]),
+                                          (8, 1, 128, [513]), (4, 2, 128, [1500, 7])])
+def test_gqa_decode_group_sizes(nq, nkv, d, pos):
+    # groups of 1 (Qwen1.5-MoE shape), 2, 8 and 16 query heads per kv head, over 1 to 16 splits
+    got, ref, _ = _attn_case(len(pos), nq, nkv, d, pos, 1, 1, 13)
+    _check_attn(got, ref, f"G={nq // nkv} d={d} pos={pos}", rope=True)
+
+
 def test_gqa_decode_head_dim_64_group_3():
     got, ref, _ = _attn_case(2, 9, 3, 64, [40, 1000], 1, 1, 12)
     _check_attn(got, ref, "d=64 G=3", rope=True)

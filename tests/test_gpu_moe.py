@@ -1,6 +1,9 @@
 """MoE layers through the C ABI against the CPU oracle: router top-k indices must match
-bit-exactly (inputs reseeded until every checked routing decision is at least 1e-3 away
-from a tie), logits within the parity bar, greedy tokens exact."""
+bit-exactly, logits within the parity bar, greedy tokens exact. Inputs are reseeded until
+every checked routing decision is at least 1e-3 away from a tie and, past the first layer,
+is also left in place when every embedding value moves by one bf16 ulp: fp32 accumulation
+lands some bf16 roundings of each layer one ulp from the fp64 oracle's, and a decision that
+noise of that size moves is not determined by the arithmetic."""
 import numpy as np
 import pytest
 
@@ -8,7 +11,7 @@ import oracle
 import synth
 from synth import configs
 import decoder_only_transformer_layer_b200 as dec
-from _util import assert_parity
+from _util import assert_parity, perturb_inputs
 
 pytestmark = pytest.mark.gpu
 MARGIN = 1e-3
@@ -27,15 +30,26 @@ def top_gap(v):
     return s[-1] - s[-2]
 
 
+def stable(a, b):
+    """The oracle's decisions (routes per layer, greedy token) and those of the one-ulp
+    perturbed oracle agree."""
+    (lga, rta), (lgb, rtb) = a, b
+    return np.array_equal(rta[0], rtb[0]) and oracle.argmax(lga) == oracle.argmax(lgb)
+
+
 def run_gated(cfg, w, n_prompt, n_steps, seed0=1100, tries=60):
     """Oracle prefill + teacher-forced decode; every step's logit gap and every decode
-    step's router gaps must clear the margin. Returns prompt, greedy tokens, logits, routes."""
+    step's router gaps must clear the margin, and the one-ulp perturbed oracle must make the
+    same decisions. Returns prompt, greedy tokens, logits, routes."""
+    wp = perturb_inputs(w)
     for t in range(tries):
         toks = synth.tokens(n_prompt, cfg["vocab"], seed0 + t)
-        m = oracle.Model(cfg, w)
+        m, mp = oracle.Model(cfg, w), oracle.Model(cfg, wp)
         lg = [m.prefill(0, toks, 0)]
         routes = [m.last_routes()]
-        ok = top_gap(lg[0]) >= MARGIN and routes[0][2].min() >= MARGIN
+        pl = mp.prefill(0, toks, 0)
+        ok = top_gap(lg[0]) >= MARGIN and routes[0][2].min() >= MARGIN and stable((lg[0], routes[0]),
+                                                                                  (pl, mp.last_routes()))
         greedy = []
         for s in range(n_steps):
             if not ok:
@@ -44,9 +58,13 @@ def run_gated(cfg, w, n_prompt, n_steps, seed0=1100, tries=60):
             greedy.append(tok)
             lg.append(m.forward(0, tok, n_prompt + s))
             routes.append(m.last_routes())
-            ok = top_gap(lg[-1]) >= MARGIN and routes[-1][2].min() >= MARGIN
+            pl = mp.forward(0, tok, n_prompt + s)
+            ok = top_gap(lg[-1]) >= MARGIN and routes[-1][2].min() >= MARGIN and stable((lg[-1], routes[-1]),
+                                                                                        (pl, mp.last_routes()))
+        mp.close()
         if ok:
             return toks, greedy, lg, routes, m
+        m.close()
     pytest.fail("no prompt seed cleared the margins")
 
 
@@ -89,16 +107,21 @@ def test_qwen_moe_shape_batch1_decode():
     kvd = cfg["n_kv_heads"] * cfg["head_dim"]
     ctx = 300
     fills = [synth.kv_fill(ctx, kvd, 2000, l) for l in range(cfg["layers"])]
+    wp = perturb_inputs(w)
     for attempt in range(40):
         toks = synth.tokens(3, cfg["vocab"], 1300 + attempt)
-        m = oracle.Model(cfg, w)
+        m, mp = oracle.Model(cfg, w), oracle.Model(cfg, wp)
         for l, (k, v) in enumerate(fills):
             m.kv_write(0, l, 0, k, v)
+            mp.kv_write(0, l, 0, k, v)
         lgs, rts, ok = [], [], True
         for s, t in enumerate(toks):
             lgs.append(m.forward(0, int(t), ctx + s))
             rts.append(m.last_routes())
-            ok = ok and rts[-1][2].min() >= MARGIN and top_gap(lgs[-1]) >= MARGIN
+            pl = mp.forward(0, int(t), ctx + s)
+            ok = ok and rts[-1][2].min() >= MARGIN and top_gap(lgs[-1]) >= MARGIN and stable(
+                (lgs[-1], rts[-1]), (pl, mp.last_routes()))
+        mp.close()
         if ok:
             break
     else:
@@ -123,16 +146,21 @@ def test_qwen_moe_shape_batch64_decode_sampled():
     sample = (0, 9, 23, 40, 51, 63)
     toks = synth.tokens(B, cfg["vocab"], 1400)
     ref = {}
+    wp = perturb_inputs(w)
     for b in sample:  # reseed the sampled sequences' tokens until their routing clears the margin
         for attempt in range(40):
             tok = int(synth.tokens(1, cfg["vocab"], 1500 + 100 * b + attempt)[0])
-            m = oracle.Model(cfg, w)
+            m, mp = oracle.Model(cfg, w), oracle.Model(cfg, wp)
             for l in range(cfg["layers"]):
                 k, v = synth.kv_fill(lens[b], kvd, 2000, 100 * b + l)
                 m.kv_write(0, l, 0, k, v)
+                mp.kv_write(0, l, 0, k, v)
             lg = m.forward(0, tok, lens[b])
             rt = m.last_routes()
-            if rt[2].min() >= MARGIN:
+            ok = rt[2].min() >= MARGIN and stable((lg, rt), (mp.forward(0, tok, lens[b]), mp.last_routes()))
+            m.close()
+            mp.close()
+            if ok:
                 toks[b] = tok
                 ref[b] = (lg, rt[0])
                 break
