@@ -202,6 +202,23 @@ DEC_DEVINL void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, ui
 // copies, TMA stores) issued after the next barrier.
 DEC_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Packed fp32x2 arithmetic (sm_100): d = a * b + c and d = a + b on both halves.
+DEC_DEVINL float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+          "l"(*reinterpret_cast<unsigned long long*>(&c)));
+    return *reinterpret_cast<float2*>(&d);
+}
+DEC_DEVINL float2 fadd2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+    return *reinterpret_cast<float2*>(&d);
+}
+
 // SiLU(g) = g / (1 + e^-g) with the hardware exponential and approximate divide (a few ulp
 // of fp32; the products it feeds are rounded to bf16). For g far below zero e^-g is +inf
 // and the quotient is -0.

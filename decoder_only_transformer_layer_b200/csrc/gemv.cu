@@ -67,6 +67,13 @@ __host__ __device__ inline Layout make_layout(int nb, int K, int smem_cap, bool 
     const int kcmax = q8 ? kKCq : kKC;
     L.kc = K < kcmax ? K : kcmax;
     L.stage_bytes = (uint32_t)rows_per_stage(nb, q8) * L.kc * (q8 ? 1 : 2);
+    // shorter stages when fewer than 4 of them would fit (long rows, several input columns)
+    const uint32_t fixed = (((uint32_t)(2 * kMaxStages * 8) + (uint32_t)(2 * kWarps * 64 + 64) * 4 + 127) & ~127u) +
+                           (((uint32_t)nb * K * 2 + 127) & ~127u);
+    while (L.kc > 1024 && L.kc % 16 == 0 && (int)fixed + 4 * (int)L.stage_bytes > smem_cap) {
+        L.kc /= 2;
+        L.stage_bytes /= 2;
+    }
     const uint32_t bars = 2 * kMaxStages * 8;
     L.red_off = bars;  // two [kWarps][64] float areas (q8 alternates them) + 64 floats scratch
     const uint32_t red = (uint32_t)(2 * kWarps * 64 + 64) * 4;
@@ -96,23 +103,6 @@ DEC_DEVINL float dot8(uint4 w, uint4 x, float acc) {
 __device__ __noinline__ float softcap_apply(float o, float c) { return c * tanhf(o / c); }
 
 DEC_DEVINL void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
-
-// Packed fp32x2 arithmetic (sm_100): d = a * b + c and d = a + b on both halves.
-DEC_DEVINL float2 ffma2(float2 a, float2 b, float2 c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;"
-        : "=l"(d)
-        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
-          "l"(*reinterpret_cast<unsigned long long*>(&c)));
-    return *reinterpret_cast<float2*>(&d);
-}
-DEC_DEVINL float2 fadd2(float2 a, float2 b) {
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;"
-        : "=l"(d)
-        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
-    return *reinterpret_cast<float2*>(&d);
-}
 
 // The four int8 values of w as exact fp32 values: byte i of w ^ 0x80808080 (q + 128) goes
 // into the mantissa of 2^23, and 2^23 + 128 is subtracted.
