@@ -1075,6 +1075,7 @@ cudaError_t prefill_launch_d(const AttnPrefillArgs& a, cudaStream_t st, bool pdl
 
 cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl) {
     if (a.T <= 0) return cudaSuccess;
+    if (attn_prefill_tc_ok(a)) return attn_prefill_tc_launch(a, st, pdl);
     if (a.splits < 1 || a.splits > kPrefMaxSplits) return cudaErrorInvalidValue;
     if (a.d == 128) return prefill_launch_d<128>(a, st, pdl);
     if (a.d == 64) return prefill_launch_d<64>(a, st, pdl);

@@ -1,0 +1,560 @@
+// Causal GQA attention of a prefill chunk on the tensor cores (tcgen05, TMEM accumulators).
+//
+// The chunk's rows are (token, head) pairs of one kv head's group: a CTA owns 128 of them
+// (128 / G tokens x the G query heads that share the kv head), so every key and value it
+// loads serves all G heads. Per 128-key block of the paged cache:
+//   S = Q K^T          tcgen05.mma M=128 N=128 K=16 (x 8 over d = 128), fp32 in TMEM
+//   P = exp2(S' - m)   4 softmax warps, thread = row = TMEM lane; S' is the scaled (or
+//                      softcapped) score in log2 units; P written to shared memory as two
+//                      bf16 terms P_hi + P_lo (16 significant bits: a single bf16 P moved
+//                      the Llama-3-8B-shape logits by ~0.6%, past the parity bar)
+//   O += P V           tcgen05.mma M=128 N=64 K=16 (x 8 over keys, x 2 halves of d, x 2 terms)
+// with S double-buffered in TMEM, so the scores of block j + 1 are computed while the
+// softmax warps work on block j. The running maximum m is moved, and O and l rescaled,
+// only when a row's maximum grows by more than 2^8 (P <= 2^8 never overflows, and O / l
+// is unchanged by the choice of m), so O stays in TMEM untouched almost always.
+// Keys past a row's position (or before its window) are masked per element; blocks before
+// every row's window are skipped.
+// With S > 1 key splits (short chunks would otherwise fill few SMs) the S CTAs of a row
+// block form a cluster, each taking a contiguous run of key blocks. Each stages its rows'
+// unnormalised O with their m and l in its own drained ring; after one cluster barrier the
+// DMA engine copies every owner's rows (128 / S of them) into the owner's receive slots
+// (cp.async.bulk shared::cta -> shared::cluster, completing on the owner's mbarrier), and
+// the owner merges the S partials in split order (deterministic).
+//
+// Operand layouts in shared memory (all 128-byte swizzled, 1024-byte aligned):
+//   Q  [2 d-halves][128 rows][64 d]   A of S, K-major      (TMA 3-D box {64, G, 128/G})
+//   K  [2 d-halves][128 keys][64 d]   B of S, K-major      (TMA box {64, 16} per page)
+//   V  [2 d-halves][128 keys][64 d]   B of O, MN-major (d contiguous)
+//   P  [2 key-halves][128 rows][64 keys]  A of O, K-major  (written by the softmax warps)
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace dec {
+
+namespace {
+
+constexpr int kTcRows = 128;  // (token, head) rows per CTA: the MMA's M
+constexpr int kTcKeys = 128;  // keys per block: N of S, K of O
+constexpr int kTcPage = 16;
+constexpr float kTcLog2e = 1.4426950408889634f;
+constexpr float kTcRescale = 8.0f;  // log2 units
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = 32768;         // 2 stages of [K 32 KB][V 32 KB]
+constexpr uint32_t kStageKV = 65536;
+constexpr uint32_t kOffP = kOffKV + 2 * kStageKV;  // P as two bf16 terms: hi, then lo
+constexpr uint32_t kOffPlo = kOffP + 32768;
+constexpr uint32_t kOffBar = kOffPlo + 32768;
+// after the last block: [stage: 128 rows][LDR] this CTA's partial, then [recv: S][128 / S][LDR]
+constexpr int kLdr = 132;  // O[128], m, l, 2 pad: 16-byte rows, conflict-free
+constexpr uint32_t kOffStage = kOffKV;
+constexpr uint32_t kOffRecv = kOffKV + kTcRows * kLdr * 4;
+constexpr uint32_t kTcSmem = kOffBar + 256 + 1024;  // + alignment slack
+
+// Shared-memory descriptor of a 128-byte-swizzled operand whose 128-byte rows run along K
+// with the MN dimension contiguous inside a row (MN-major, one 64-element atom along MN):
+// both byte offsets are the stride between 8-row groups along K.
+DEC_DEVINL uint64_t sdesc_sw128_mn(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)(1024 >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// kind::f16 instruction descriptor: bf16 A (K-major) and B (MN-major when b_mn), fp32 D.
+template <int M, int N, bool B_MN>
+__host__ __device__ constexpr uint32_t idesc_tc() {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (B_MN ? (1u << 16) : 0u) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+DEC_DEVINL void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+DEC_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+DEC_DEVINL void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// The softcapped score c tanh(raw scale / c) in log2 units, out of line so the uncapped
+// path never evaluates the tanh.
+__device__ __noinline__ float capped_score(float raw, float scale, float c) {
+    return c * tanhf(raw * scale / c) * kTcLog2e;
+}
+
+// 2^x by the hardware's approximate exponential (a few fp32 ulp; 2^-inf = 0). The P it
+// gives is rounded to bf16 terms.
+DEC_DEVINL float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+struct TcPrefArgs {
+    AttnPrefillArgs a;
+    int G, tok_per_cta;
+};
+
+__global__ void __launch_bounds__(192, 1)
+    attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, TcPrefArgs args) {
+    const AttnPrefillArgs& a = args.a;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* kv_full = q_full + 1;   // [2]
+    uint64_t* kv_empty = kv_full + 2; // [2]
+    uint64_t* s_full = kv_empty + 2;  // [2]
+    uint64_t* p_full = s_full + 2;    // the softmax warps are done with S[j & 1] and wrote P
+    uint64_t* pv_done = p_full + 1;   // O += P V of the last issued block completed
+    uint64_t* recvb = pv_done + 1;    // the other splits' rows of this CTA have landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recvb + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = args.G, TPC = args.tok_per_cta;
+    const int g = blockIdx.y;
+    const int t0 = blockIdx.x * TPC;                  // first token of this CTA
+    const int t_last = min(a.T - 1, t0 + TPC - 1);    // last valid token
+    const int hi_key = a.pos0 + t_last;               // the largest key any row sees
+    const int lo_key = a.window > 0 ? max(0, a.pos0 + t0 + 1 - a.window) : 0;  // the smallest
+    const int S = gridDim.z, z = blockIdx.z;           // key splits (a cluster), this split
+    const int RS = kTcRows / S;                        // rows each split finishes
+    const int kb_lo = lo_key / kTcKeys, nb_all = hi_key / kTcKeys - kb_lo + 1;
+    const int kb0 = kb_lo + (int)((long long)nb_all * z / S);  // this split's key blocks
+    const int nb = kb_lo + (int)((long long)nb_all * (z + 1) / S) - kb0;
+    const int np = (a.pos0 + a.T + kTcPage - 1) / kTcPage;  // pages holding keys of this chunk
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+            mbar_init(&s_full[i], 1);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(recvb, 1);
+        // armed before the first cluster barrier, so no byte can arrive before the count
+        if (S > 1) mbar_arrive_expect_tx(recvb, (uint32_t)(S - 1) * RS * kLdr * 4);
+        fence_mbar_init();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 2 * kTcKeys;  // S[0], S[1]: columns 0..255; O: 256..383
+    pdl_trigger();
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            pdl_wait();  // q and the chunk's own keys come from the previous kernels
+            mbar_arrive_expect_tx(q_full, 32768);
+            for (int h2 = 0; h2 < 2; ++h2)
+                tma_load_3d(smem + kOffQ + h2 * 16384, &tmQ, h2 * 64, g * G, t0, q_full);
+            for (int j = 0; j < nb; ++j) {
+                const int s = j & 1;
+                if (j >= 2 && !mbar_wait_bounded(&kv_empty[s], ((j >> 1) - 1) & 1, a.err)) break;
+                mbar_arrive_expect_tx(&kv_full[s], 65536);
+                uint8_t* kd = smem + kOffKV + s * kStageKV;
+                uint8_t* vd = kd + 32768;
+                for (int pi = 0; pi < kTcKeys / kTcPage; ++pi) {
+                    // pages past the chunk's last one hold only masked keys: any finite page
+                    // will do, so they reload the last page
+                    const int page = min((kb0 + j) * (kTcKeys / kTcPage) + pi, np - 1);
+                    const int row = (a.block_row[page] * a.nkv + g) * kTcPage;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        tma_load_2d(kd + h2 * 16384 + pi * 2048, &tmK, h2 * 64, row, &kv_full[s]);
+                        tma_load_2d(vd + h2 * 16384 + pi * 2048, &tmV, h2 * 64, row, &kv_full[s]);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        pdl_wait();
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t id_s = idesc_tc<128, 128, false>();
+            constexpr uint32_t id_o = idesc_tc<128, 64, true>();
+            const uint32_t sb = smem_u32(smem);
+            bool ok = mbar_wait_bounded(q_full, 0, a.err);
+            auto issue_s = [&](int j) {
+                const int s = j & 1;
+                const uint32_t kb = sb + kOffKV + s * kStageKV;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc_mma(tS + s * kTcKeys, sdesc_sw128(sb + kOffQ + (kk >> 2) * 16384 + (kk & 3) * 32),
+                           sdesc_sw128(kb + (kk >> 2) * 16384 + (kk & 3) * 32), id_s, kk > 0 ? 1u : 0u);
+                tc_commit(&s_full[s]);
+            };
+            if (ok && nb > 0) {
+                ok = mbar_wait_bounded(&kv_full[0], 0, a.err);
+                tc_fence_after();
+                if (ok) issue_s(0);
+            }
+            for (int j = 0; j < nb && ok; ++j) {
+                if (j + 1 < nb) {
+                    // S[(j + 1) & 1] was last read by the softmax of block j - 1 (waited below
+                    // in the previous iteration)
+                    if (!mbar_wait_bounded(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, a.err)) break;
+                    tc_fence_after();
+                    issue_s(j + 1);
+                }
+                if (!mbar_wait_bounded(p_full, j & 1, a.err)) break;
+                tc_fence_after();
+                const uint32_t vb = sb + kOffKV + (j & 1) * kStageKV + 32768;
+#pragma unroll
+                for (int dh = 0; dh < 2; ++dh)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t pa = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        const uint64_t vdesc = sdesc_sw128_mn(vb + dh * 16384 + kk * 2048);
+                        tc_mma(tO + dh * 64, sdesc_sw128(sb + kOffP + pa), vdesc, id_o, (j > 0 || kk > 0) ? 1u : 0u);
+                        tc_mma(tO + dh * 64, sdesc_sw128(sb + kOffPlo + pa), vdesc, id_o, 1u);
+                    }
+                tc_commit(pv_done);
+                tc_commit(&kv_empty[j & 1]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- softmax + epilogue (warps 0-3)
+        const int r = warp * 32 + lane;  // row = TMEM lane
+        const int tl = r / G;             // token within the CTA
+        const int t = t0 + tl;
+        const bool valid = tl < TPC && t < a.T;
+        const int pos = a.pos0 + t;       // the row's last visible key
+        const int lo = a.window > 0 ? pos + 1 - a.window : 0;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = a.scale * kTcLog2e;
+        const bool cap = a.softcap > 0.f;
+        float m = -INFINITY, l = 0.f;
+        pdl_wait();
+        uint8_t* prow = smem + kOffP + (uint32_t)r * 128;
+        bool ok = true;
+        for (int j = 0; j < nb; ++j) {
+            const int key0 = (kb0 + j) * kTcKeys;
+            if (ok && !mbar_wait_bounded(&s_full[j & 1], (j >> 1) & 1, a.err)) ok = false;
+            tc_fence_after();
+            const uint32_t sa = tS + (j & 1) * kTcKeys + lane_off;
+            // The row sees keys [lo, pos]: a block wholly inside needs no per-key test, one
+            // wholly outside contributes nothing.
+            const bool none = !valid || key0 > pos || key0 + kTcKeys - 1 < lo;
+            const bool whole = !none && key0 + kTcKeys - 1 <= pos && key0 >= lo;
+            // pass 1: the block's row maximum (log2 units), four independent partial maxima
+            float bm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            for (int c0 = 0; c0 < kTcKeys; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld16_issue(sa + c0, v);
+                tmem_ld16_issue(sa + c0 + 16, v + 16);
+                tmem_ld_wait32(v);
+                if (none) continue;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    float x = __uint_as_float(v[q]);
+                    x = cap ? capped_score(x, a.scale, a.softcap) : x * sl2;
+                    if (!whole) {
+                        const int key = key0 + c0 + q;
+                        if (key > pos || key < lo) x = -INFINITY;
+                    }
+                    bm4[q & 3] = fmaxf(bm4[q & 3], x);
+                }
+            }
+            const float bm = fmaxf(fmaxf(bm4[0], bm4[1]), fmaxf(bm4[2], bm4[3]));
+            // O and P of block j - 1 are done with before either is touched
+            if (j > 0 && ok && !mbar_wait_bounded(pv_done, (j - 1) & 1, a.err)) ok = false;
+            tc_fence_after();
+            const float mn = fmaxf(m, bm);
+            const bool grow = m != -INFINITY && mn > m + kTcRescale;
+            if (__any_sync(0xffffffffu, grow)) {
+                // move the reference maximum: O and l of the rows that grew scale by 2^(m - mn)
+                const float corr = grow ? ex2f(m - mn) : 1.f;
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld16_issue(tO + lane_off + c0, v);
+                    tmem_ld16_issue(tO + lane_off + c0 + 16, v + 16);
+                    tmem_ld_wait32(v);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * corr);
+                    tmem_st16(tO + lane_off + c0, v);
+                    tmem_st16(tO + lane_off + c0 + 16, v + 16);
+                }
+                tmem_st_wait();
+                l *= corr;
+            }
+            if (grow || m == -INFINITY) m = mn;
+            // pass 2: P = 2^(S' - m) as bf16 hi + lo in the swizzled A layout, and the row sum
+            // (four independent partial sums)
+            const bool zero = none || m == -INFINITY;
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c0 = 0; c0 < kTcKeys; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld16_issue(sa + c0, v);
+                tmem_ld16_issue(sa + c0 + 16, v + 16);
+                tmem_ld_wait32(v);
+                uint32_t ph[16], pl[16];
+                if (zero) {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) ph[q] = pl[q] = 0u;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 2) {
+                        float p2[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            float x = __uint_as_float(v[q + e]);
+                            x = cap ? capped_score(x, a.scale, a.softcap) : x * sl2;
+                            p2[e] = ex2f(x - m);
+                            if (!whole) {
+                                const int key = key0 + c0 + q + e;
+                                if (key > pos || key < lo) p2[e] = 0.f;
+                            }
+                            sum4[(q >> 1) & 3] += p2[e];
+                        }
+                        ph[q / 2] = pack_bf2(p2[0], p2[1]);
+                        pl[q / 2] = pack_bf2(p2[0] - bf_lo(ph[q / 2]), p2[1] - bf_hi(ph[q / 2]));
+                    }
+                }
+                // keys c0 .. c0 + 31 of this row: key-half c0 / 64, 16-byte chunks
+                // (c0 % 64) / 8 .. + 3, stored at chunk ^ (row % 8)
+                uint8_t* base = prow + (c0 >> 6) * 16384;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int chunk = ((c0 & 63) >> 3) + ch;
+                    const uint32_t off = (uint32_t)((chunk ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4*>(base + off) = make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]);
+                    *reinterpret_cast<uint4*>(base + (kOffPlo - kOffP) + off) =
+                        make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
+                }
+            }
+            const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            l += sum;
+            fence_proxy_async_smem();  // the MMA reads P through the async proxy
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        // ---- epilogue
+        if (nb > 0 && ok && !mbar_wait_bounded(pv_done, (nb - 1) & 1, a.err)) ok = false;
+        tc_fence_after();
+        if (S == 1) {
+            // O / l, bf16, to out[t][g G + (r % G)][:]
+            const float inv = l > 0.f ? 1.0f / l : 0.f;
+            uint16_t* dst = a.out + ((size_t)t * a.nq + (size_t)g * G + (r % G)) * 128;
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld16_issue(tO + lane_off + c0, v);
+                tmem_ld16_issue(tO + lane_off + c0 + 16, v + 16);
+                tmem_ld_wait32(v);
+                if (valid && ok) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 8) {
+                        uint4 o;
+                        o.x = pack_bf2(__uint_as_float(v[q]) * inv, __uint_as_float(v[q + 1]) * inv);
+                        o.y = pack_bf2(__uint_as_float(v[q + 2]) * inv, __uint_as_float(v[q + 3]) * inv);
+                        o.z = pack_bf2(__uint_as_float(v[q + 4]) * inv, __uint_as_float(v[q + 5]) * inv);
+                        o.w = pack_bf2(__uint_as_float(v[q + 6]) * inv, __uint_as_float(v[q + 7]) * inv);
+                        *reinterpret_cast<uint4*>(dst + c0 + q) = o;
+                    }
+                }
+            }
+        } else {
+            // this split's partial row (unnormalised O, m, l) into the drained ring
+            float* st = reinterpret_cast<float*>(smem + kOffStage) + (size_t)r * kLdr;
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t v[32];
+                if (nb > 0) {
+                    tmem_ld16_issue(tO + lane_off + c0, v);
+                    tmem_ld16_issue(tO + lane_off + c0 + 16, v + 16);
+                    tmem_ld_wait32(v);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q] = 0u;  // no key blocks: O = 0, m = -inf, l = 0
+                }
+#pragma unroll
+                for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<uint4*>(st + c0 + q) = make_uint4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+            }
+            *reinterpret_cast<float4*>(st + 128) = make_float4(m, l, 0.f, 0.f);
+            fence_proxy_async_smem();  // the copies read these writes through the async proxy
+        }
+    }
+    if (S > 1) {
+        // every split of the cluster is past its MMAs (its ring is free to receive) and has
+        // staged its partial
+        cluster_sync();
+        if (threadIdx.x == 0) {
+            for (int o = 0; o < S; ++o) {
+                if (o == z) continue;
+                const uint32_t dst = dsmem_map(smem_u32(smem + kOffRecv) + (uint32_t)z * RS * kLdr * 4, o);
+                bulk_s2cluster(dst, smem + kOffStage + (size_t)o * RS * kLdr * 4, (uint32_t)RS * kLdr * 4,
+                               dsmem_map(smem_u32(recvb), o));
+            }
+        }
+        if (warp < 4) {
+            // rows [z RS, z RS + RS): 128 / RS threads a row, 128 / (128 / RS) columns each
+            const int tpr = kTcRows / RS;
+            const int lr = threadIdx.x / tpr, part = threadIdx.x % tpr, cols = 128 / tpr;
+            const int rr = z * RS + lr;  // the row in the CTA's 128
+            const bool got = mbar_wait_bounded(recvb, 0, a.err);
+            const int tt = t0 + rr / G;
+            const float* mine = reinterpret_cast<const float*>(smem + kOffStage) + (size_t)rr * kLdr;
+            auto part_row = [&](int zz) {
+                return zz == z ? mine
+                               : reinterpret_cast<const float*>(smem + kOffRecv) + ((size_t)zz * RS + lr) * kLdr;
+            };
+            float M = -INFINITY;
+            for (int zz = 0; zz < S; ++zz) M = fmaxf(M, part_row(zz)[128]);
+            float L = 0.f;
+            float acc[128 / 2];  // at most 64 columns per thread (RS <= 64)
+#pragma unroll
+            for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+            for (int zz = 0; zz < S; ++zz) {
+                const float* pr = part_row(zz);
+                const float mz = pr[128];
+                if (mz == -INFINITY) continue;
+                const float wz = ex2f(mz - M);
+                L += wz * pr[129];
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    if (c < cols) {
+                        const float4 v = *reinterpret_cast<const float4*>(pr + part * cols + c);
+                        acc[c] += wz * v.x;
+                        acc[c + 1] += wz * v.y;
+                        acc[c + 2] += wz * v.z;
+                        acc[c + 3] += wz * v.w;
+                    }
+                }
+            }
+            if (got && tt < a.T && (rr / G) < TPC) {
+                const float inv = L > 0.f ? 1.0f / L : 0.f;
+                uint16_t* dst = a.out + ((size_t)tt * a.nq + (size_t)g * G + (rr % G)) * 128 + part * cols;
+#pragma unroll
+                for (int c = 0; c < 64; c += 8) {
+                    if (c < cols) {
+                        uint4 o;
+                        o.x = pack_bf2(acc[c] * inv, acc[c + 1] * inv);
+                        o.y = pack_bf2(acc[c + 2] * inv, acc[c + 3] * inv);
+                        o.z = pack_bf2(acc[c + 4] * inv, acc[c + 5] * inv);
+                        o.w = pack_bf2(acc[c + 6] * inv, acc[c + 7] * inv);
+                        *reinterpret_cast<uint4*>(dst + c) = o;
+                    }
+                }
+            }
+        }
+        // the copies out of this CTA's shared memory have landed at their owners
+        cluster_sync();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+    }
+}
+
+}  // namespace
+
+// The tensor-core kernel takes head dim 128, groups of 1, 2, 4, ..., 128 query heads, and
+// chunks of at least one CTA's tokens (the q box never exceeds the chunk).
+bool attn_prefill_tc_ok(const AttnPrefillArgs& a) {
+    const int G = a.nkv > 0 ? a.nq / a.nkv : 0;
+    return a.d == 128 && G >= 1 && G <= kTcRows && (G & (G - 1)) == 0 && a.nq % a.nkv == 0 && a.pool_rows > 0 &&
+           a.T >= kTcRows / G;
+}
+
+cudaError_t attn_prefill_tc_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl) {
+    if (a.T <= 0) return cudaSuccess;
+    if (!attn_prefill_tc_ok(a)) return cudaErrorInvalidValue;
+    const int G = a.nq / a.nkv;
+    TcPrefArgs args;
+    args.a = a;
+    args.G = G;
+    args.tok_per_cta = kTcRows / G;
+    // key splits: a power of two (rows split evenly between the owners), enough CTAs to
+    // cover the SMs, at most one per key block of the longest row, at most 8 (a portable
+    // cluster)
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    const int ctas = ((a.T + args.tok_per_cta - 1) / args.tok_per_cta) * a.nkv;
+    const int span_blocks = (attn_prefill_span(a.pos0, a.T, a.window) + kTcKeys - 1) / kTcKeys + 1;
+    int S = 1;
+    while (S < 8 && ctas * S * 2 <= sms && S * 2 <= span_blocks) S *= 2;
+    CUtensorMap tmQ, tmK, tmV;
+    {
+        const uint64_t dims[3] = {128, (uint64_t)a.nq, (uint64_t)a.T};
+        const uint64_t strides[2] = {128 * 2, (uint64_t)a.nq * 128 * 2};
+        const uint32_t box[3] = {64, (uint32_t)G, (uint32_t)(kTcRows / G)};
+        cudaError_t e = tmap_bf16_sw128(&tmQ, a.q, 3, dims, strides, box);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        const uint64_t dims[2] = {128, (uint64_t)a.pool_rows};
+        const uint64_t strides[1] = {128 * 2};
+        const uint32_t box[2] = {64, kTcPage};
+        cudaError_t e = tmap_bf16_sw128(&tmK, a.k_pool, 2, dims, strides, box);
+        if (e != cudaSuccess) return e;
+        e = tmap_bf16_sw128(&tmV, a.v_pool, 2, dims, strides, box);
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_prefill_tc_kernel), (int)kTcSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((a.T + args.tok_per_cta - 1) / args.tok_per_cta, a.nkv, S);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = kTcSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (S > 1) {  // the key splits of a row block: one cluster
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = S;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, attn_prefill_tc_kernel, tmQ, tmK, tmV, args);
+}
+
+}  // namespace dec

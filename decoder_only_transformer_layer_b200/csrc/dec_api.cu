@@ -432,6 +432,7 @@ dec_status forward_layers(dec_ctx* c, int n, bool decode, int seq, int pos0, cud
                                            c->num_sms);
             a.out = c->attn;
             a.err = c->d_err;
+            a.pool_rows = c->n_pages * k.n_kv_heads * 16;
             CUDA_TRY(attn_prefill_launch(a, st, true));
         }
         // o_proj + residual (sandwich: the output is RMS-normalised with its own gain first)

@@ -1003,6 +1003,24 @@ cudaError_t launch_splitk_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t 
 
 }  // namespace
 
+cudaError_t tmap_bf16_sw128(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides, const uint32_t* box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rank < 1 || rank > 5) return cudaErrorNotSupported;
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Row-major bf16 [rows][K] read in 128B-swizzled boxes of 64 columns x box_rows rows.
 cudaError_t tmap_bf16_rows(CUtensorMap* tm, const uint16_t* base, int rows, int K, int box_rows) {
     return encode_2d(tm, base, rows, K, box_rows);

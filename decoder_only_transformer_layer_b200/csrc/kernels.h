@@ -152,8 +152,15 @@ struct AttnPrefillArgs {
     int splits;         // key splits (1..8): the split CTAs of a row block form one cluster
     uint16_t* out;      // [T][nq*d]
     int* err;
+    int pool_rows;      // rows of the pools viewed as [pages * nkv * 16][d] (tensor-core path)
 };
 cudaError_t attn_prefill_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl);
+// The tensor-core prefill attention (tcgen05, TMEM): head dim 128, power-of-two groups.
+bool attn_prefill_tc_ok(const AttnPrefillArgs& a);
+cudaError_t attn_prefill_tc_launch(const AttnPrefillArgs& a, cudaStream_t st, bool pdl);
+// A bf16 tensor map with 128-byte swizzle: dims[0] contiguous; strides[i] (bytes) of dims[i + 1].
+cudaError_t tmap_bf16_sw128(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides, const uint32_t* box);
 int attn_prefill_splits(int T, int nq, int nkv, int ctx, int num_sms);
 // Keys a prefill chunk's rows may see: the whole causal prefix, or with a window the last
 // window + T - 1 positions (sizes the key splits).
