@@ -8,7 +8,7 @@
 //                      softcapped) score in log2 units; P written to shared memory as two
 //                      bf16 terms P_hi + P_lo (16 significant bits: a single bf16 P moved
 //                      the Llama-3-8B-shape logits by ~0.6%, past the parity bar)
-//   O += P V           tcgen05.mma M=128 N=64 K=16 (x 8 over keys, x 2 halves of d, x 2 terms)
+//   O += P V           tcgen05.mma M=128 N=128 K=16 (x 8 over keys, x 2 terms)
 // with S double-buffered in TMEM, so the scores of block j + 1 are computed while the
 // softmax warps work on block j. The running maximum m is moved, and O and l rescaled,
 // only when a row's maximum grows by more than 2^8 (P <= 2^8 never overflows, and O / l
@@ -55,13 +55,14 @@ constexpr uint32_t kOffStage = kOffKV;
 constexpr uint32_t kOffRecv = kOffKV + kTcRows * kLdr * 4;
 constexpr uint32_t kTcSmem = kOffBar + 256 + 1024;  // + alignment slack
 
-// Shared-memory descriptor of a 128-byte-swizzled operand whose 128-byte rows run along K
-// with the MN dimension contiguous inside a row (MN-major, one 64-element atom along MN):
-// both byte offsets are the stride between 8-row groups along K.
+// Shared-memory descriptor of a 128-byte-swizzled MN-major operand: each 128-byte row holds
+// 64 consecutive MN elements of one k, 8 rows (8 k) form a 1024-byte swizzle atom. The
+// leading byte offset is the stride between 64-element atoms along MN (the two d-halves of
+// V, 16 KB apart), the stride byte offset the stride between 8-row groups along K (1 KB).
 DEC_DEVINL uint64_t sdesc_sw128_mn(uint32_t saddr) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)(1024 >> 4) << 16;
+    d |= (uint64_t)(16384 >> 4) << 16;
     d |= (uint64_t)(1024 >> 4) << 32;
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)2 << 61;
@@ -85,6 +86,17 @@ DEC_DEVINL void tmem_st16(uint32_t taddr, const uint32_t* r) {
 }
 DEC_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// No instruction: tells the compiler the 32 registers change here, so no use of values
+// loaded before a tcgen05.wait::ld on another array can move above that wait.
+DEC_DEVINL void reg_fence32(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
 DEC_DEVINL void tma_load_3d(void* dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
@@ -105,6 +117,36 @@ DEC_DEVINL float ex2f(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// The row's 128 raw scores v -> scores in log2 units (times scale, or softcapped), keys
+// outside [lo, pos] -inf, in place; returns their maximum (four independent partial
+// maxima). CAP: `sc` is the attention scale and `c` the cap; otherwise `sc` is scale*log2e.
+template <bool CAP>
+DEC_DEVINL float scores_log2(uint32_t (&v)[4][32], float sc, float c, bool whole, int key0, int lo, int pos) {
+    float bm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    if (whole) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const float x = CAP ? capped_score(__uint_as_float(v[k][q]), sc, c) : __uint_as_float(v[k][q]) * sc;
+                v[k][q] = __float_as_uint(x);
+                bm4[q & 3] = fmaxf(bm4[q & 3], x);
+            }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int key = key0 + 32 * k + q;
+                float x = CAP ? capped_score(__uint_as_float(v[k][q]), sc, c) : __uint_as_float(v[k][q]) * sc;
+                x = key > pos || key < lo ? -INFINITY : x;
+                v[k][q] = __float_as_uint(x);
+                bm4[q & 3] = fmaxf(bm4[q & 3], x);
+            }
+    }
+    return fmaxf(fmaxf(bm4[0], bm4[1]), fmaxf(bm4[2], bm4[3]));
 }
 
 struct TcPrefArgs {
@@ -204,7 +246,7 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t id_s = idesc_tc<128, 128, false>();
-            constexpr uint32_t id_o = idesc_tc<128, 64, true>();
+            constexpr uint32_t id_o = idesc_tc<128, 128, true>();
             const uint32_t sb = smem_u32(smem);
             bool ok = mbar_wait_bounded(q_full, 0, a.err);
             auto issue_s = [&](int j) {
@@ -233,14 +275,12 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after();
                 const uint32_t vb = sb + kOffKV + (j & 1) * kStageKV + 32768;
 #pragma unroll
-                for (int dh = 0; dh < 2; ++dh)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t pa = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        const uint64_t vdesc = sdesc_sw128_mn(vb + dh * 16384 + kk * 2048);
-                        tc_mma(tO + dh * 64, sdesc_sw128(sb + kOffP + pa), vdesc, id_o, (j > 0 || kk > 0) ? 1u : 0u);
-                        tc_mma(tO + dh * 64, sdesc_sw128(sb + kOffPlo + pa), vdesc, id_o, 1u);
-                    }
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t pa = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint64_t vdesc = sdesc_sw128_mn(vb + kk * 2048);
+                    tc_mma(tO, sdesc_sw128(sb + kOffP + pa), vdesc, id_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma(tO, sdesc_sw128(sb + kOffPlo + pa), vdesc, id_o, 1u);
+                }
                 tc_commit(pv_done);
                 tc_commit(&kv_empty[j & 1]);
             }
@@ -270,26 +310,28 @@ __global__ void __launch_bounds__(192, 1)
             // wholly outside contributes nothing.
             const bool none = !valid || key0 > pos || key0 + kTcKeys - 1 < lo;
             const bool whole = !none && key0 + kTcKeys - 1 <= pos && key0 >= lo;
-            // pass 1: the block's row maximum (log2 units), four independent partial maxima
-            float bm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            for (int c0 = 0; c0 < kTcKeys; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld16_issue(sa + c0, v);
-                tmem_ld16_issue(sa + c0 + 16, v + 16);
-                tmem_ld_wait32(v);
-                if (none) continue;
+            // the row's 128 scores, in one TMEM round trip (all loads issued, one wait)
+            uint32_t v[4][32];
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    float x = __uint_as_float(v[q]);
-                    x = cap ? capped_score(x, a.scale, a.softcap) : x * sl2;
-                    if (!whole) {
-                        const int key = key0 + c0 + q;
-                        if (key > pos || key < lo) x = -INFINITY;
-                    }
-                    bm4[q & 3] = fmaxf(bm4[q & 3], x);
-                }
+            for (int c = 0; c < 4; ++c) {
+                tmem_ld16_issue(sa + 32 * c, v[c]);
+                tmem_ld16_issue(sa + 32 * c + 16, v[c] + 16);
             }
-            const float bm = fmaxf(fmaxf(bm4[0], bm4[1]), fmaxf(bm4[2], bm4[3]));
+            tmem_ld_wait32(v[3]);
+            reg_fence32(v[0]);
+            reg_fence32(v[1]);
+            reg_fence32(v[2]);
+            // pass 1: the scores in log2 units, masked, and the block's row maximum (four
+            // independent partial maxima)
+            // (the cap and mask tests sit outside the loops: a test, let alone a possible
+            // call, per element made this pass cost more than the rest of the block)
+            float bm = -INFINITY;
+            if (!none) {
+                if (cap)
+                    bm = scores_log2<true>(v, a.scale, a.softcap, whole, key0, lo, pos);
+                else
+                    bm = scores_log2<false>(v, sl2, 0.f, whole, key0, lo, pos);
+            }
             // O and P of block j - 1 are done with before either is touched
             if (j > 0 && ok && !mbar_wait_bounded(pv_done, (j - 1) & 1, a.err)) ok = false;
             tc_fence_after();
@@ -299,28 +341,25 @@ __global__ void __launch_bounds__(192, 1)
                 // move the reference maximum: O and l of the rows that grew scale by 2^(m - mn)
                 const float corr = grow ? ex2f(m - mn) : 1.f;
                 for (int c0 = 0; c0 < 128; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld16_issue(tO + lane_off + c0, v);
-                    tmem_ld16_issue(tO + lane_off + c0 + 16, v + 16);
-                    tmem_ld_wait32(v);
+                    uint32_t o[32];
+                    tmem_ld16_issue(tO + lane_off + c0, o);
+                    tmem_ld16_issue(tO + lane_off + c0 + 16, o + 16);
+                    tmem_ld_wait32(o);
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = __float_as_uint(__uint_as_float(v[q]) * corr);
-                    tmem_st16(tO + lane_off + c0, v);
-                    tmem_st16(tO + lane_off + c0 + 16, v + 16);
+                    for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * corr);
+                    tmem_st16(tO + lane_off + c0, o);
+                    tmem_st16(tO + lane_off + c0 + 16, o + 16);
                 }
                 tmem_st_wait();
                 l *= corr;
             }
             if (grow || m == -INFINITY) m = mn;
             // pass 2: P = 2^(S' - m) as bf16 hi + lo in the swizzled A layout, and the row sum
-            // (four independent partial sums)
+            // (four independent partial sums); masked scores are -inf and give 0
             const bool zero = none || m == -INFINITY;
             float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int c0 = 0; c0 < kTcKeys; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld16_issue(sa + c0, v);
-                tmem_ld16_issue(sa + c0 + 16, v + 16);
-                tmem_ld_wait32(v);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
                 uint32_t ph[16], pl[16];
                 if (zero) {
 #pragma unroll
@@ -328,28 +367,19 @@ __global__ void __launch_bounds__(192, 1)
                 } else {
 #pragma unroll
                     for (int q = 0; q < 32; q += 2) {
-                        float p2[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            float x = __uint_as_float(v[q + e]);
-                            x = cap ? capped_score(x, a.scale, a.softcap) : x * sl2;
-                            p2[e] = ex2f(x - m);
-                            if (!whole) {
-                                const int key = key0 + c0 + q + e;
-                                if (key > pos || key < lo) p2[e] = 0.f;
-                            }
-                            sum4[(q >> 1) & 3] += p2[e];
-                        }
-                        ph[q / 2] = pack_bf2(p2[0], p2[1]);
-                        pl[q / 2] = pack_bf2(p2[0] - bf_lo(ph[q / 2]), p2[1] - bf_hi(ph[q / 2]));
+                        const float p0 = ex2f(__uint_as_float(v[c][q]) - m);
+                        const float p1 = ex2f(__uint_as_float(v[c][q + 1]) - m);
+                        sum4[(q >> 1) & 3] += p0 + p1;
+                        ph[q / 2] = pack_bf2(p0, p1);
+                        pl[q / 2] = pack_bf2(p0 - bf_lo(ph[q / 2]), p1 - bf_hi(ph[q / 2]));
                     }
                 }
-                // keys c0 .. c0 + 31 of this row: key-half c0 / 64, 16-byte chunks
-                // (c0 % 64) / 8 .. + 3, stored at chunk ^ (row % 8)
-                uint8_t* base = prow + (c0 >> 6) * 16384;
+                // keys 32 c .. 32 c + 31 of this row: key-half c / 2, 16-byte chunks
+                // 4 (c % 2) .. + 3, stored at chunk ^ (row % 8)
+                uint8_t* base = prow + (c >> 1) * 16384;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
-                    const int chunk = ((c0 & 63) >> 3) + ch;
+                    const int chunk = 4 * (c & 1) + ch;
                     const uint32_t off = (uint32_t)((chunk ^ (r & 7)) << 4);
                     *reinterpret_cast<uint4*>(base + off) = make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]);
                     *reinterpret_cast<uint4*>(base + (kOffPlo - kOffP) + off) =
