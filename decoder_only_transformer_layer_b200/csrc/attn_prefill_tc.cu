@@ -4,13 +4,19 @@
 // (128 / G tokens x the G query heads that share the kv head), so every key and value it
 // loads serves all G heads. Per 128-key block of the paged cache:
 //   S = Q K^T          tcgen05.mma M=128 N=128 K=16 (x 8 over d = 128), fp32 in TMEM
-//   P = exp2(S' - m)   4 softmax warps, thread = row = TMEM lane; S' is the scaled (or
-//                      softcapped) score in log2 units; P written to shared memory as two
-//                      bf16 terms P_hi + P_lo (16 significant bits: a single bf16 P moved
+//   P = exp2(S' - m)   8 softmax warps, two per row quarter (TMEM lanes), each taking one
+//                      half of the keys and exchanging the row maximum through shared
+//                      memory; S' is the scaled (or softcapped) score in log2 units; P
+//                      written back over S in TMEM as
+//                      two bf16 terms P_hi + P_lo (P_hi the top 16 bits of the fp32 P, P_lo
+//                      those of the exact rest: 15 significant bits; a single bf16 P moved
 //                      the Llama-3-8B-shape logits by ~0.6%, past the parity bar)
-//   O += P V           tcgen05.mma M=128 N=128 K=16 (x 8 over keys, x 2 terms)
+//   O += P V           tcgen05.mma M=128 N=128 K=16, A (P) from TMEM, B (V) from shared
+//                      memory (x 8 over keys, x 2 terms)
 // with S double-buffered in TMEM, so the scores of block j + 1 are computed while the
-// softmax warps work on block j. The running maximum m is moved, and O and l rescaled,
+// softmax warps work on block j. K and V stream through separate 3-stage rings, each with
+// its own producer warp: a K stage is released as soon as its scores are computed, a V
+// stage when its PV product is, so the loads of later blocks overlap the softmax. The running maximum m is moved, and O and l rescaled,
 // only when a row's maximum grows by more than 2^8 (P <= 2^8 never overflows, and O / l
 // is unchanged by the choice of m), so O stays in TMEM untouched almost always.
 // Keys past a row's position (or before its window) are masked per element; blocks before
@@ -26,7 +32,8 @@
 //   Q  [2 d-halves][128 rows][64 d]   A of S, K-major      (TMA 3-D box {64, G, 128/G})
 //   K  [2 d-halves][128 keys][64 d]   B of S, K-major      (TMA box {64, 16} per page)
 //   V  [2 d-halves][128 keys][64 d]   B of O, MN-major (d contiguous)
-//   P  [2 key-halves][128 rows][64 keys]  A of O, K-major  (written by the softmax warps)
+// TMEM (512 columns): S/P of even blocks at 0, of odd blocks at 128 (P_hi in the first 64
+// columns, P_lo in the next 64, two keys per column), O at 256.
 #include <math.h>
 
 #include "common.cuh"
@@ -43,17 +50,20 @@ constexpr int kTcPage = 16;
 constexpr float kTcLog2e = 1.4426950408889634f;
 constexpr float kTcRescale = 8.0f;  // log2 units
 
+constexpr int kTcStages = 3;
+constexpr uint32_t kStage = 32768;  // one 128-key block of K or of V
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = 32768;         // 2 stages of [K 32 KB][V 32 KB]
-constexpr uint32_t kStageKV = 65536;
-constexpr uint32_t kOffP = kOffKV + 2 * kStageKV;  // P as two bf16 terms: hi, then lo
-constexpr uint32_t kOffPlo = kOffP + 32768;
-constexpr uint32_t kOffBar = kOffPlo + 32768;
+constexpr uint32_t kOffK = 32768;
+constexpr uint32_t kOffV = kOffK + kTcStages * kStage;
+constexpr uint32_t kOffBar = kOffV + kTcStages * kStage;
 // after the last block: [stage: 128 rows][LDR] this CTA's partial, then [recv: S][128 / S][LDR]
 constexpr int kLdr = 132;  // O[128], m, l, 2 pad: 16-byte rows, conflict-free
-constexpr uint32_t kOffStage = kOffKV;
-constexpr uint32_t kOffRecv = kOffKV + kTcRows * kLdr * 4;
-constexpr uint32_t kTcSmem = kOffBar + 256 + 1024;  // + alignment slack
+constexpr uint32_t kOffStage = kOffK;
+constexpr uint32_t kOffRecv = kOffK + kTcRows * kLdr * 4;
+static_assert(kOffRecv + kTcRows * kLdr * 4 <= kOffBar, "the merge areas fit in the drained rings");
+constexpr uint32_t kOffXch = kOffBar + 256;  // softmax warp pairs' row maxima and sums
+constexpr uint32_t kTcSmem = kOffXch + 2 * kTcRows * 4 + 1024;  // + alignment slack
+static_assert(kTcSmem <= 232448, "fits the 227 KB a CTA may use");
 
 // Shared-memory descriptor of a 128-byte-swizzled MN-major operand: each 128-byte row holds
 // 64 consecutive MN elements of one k, 8 rows (8 k) form a 1024-byte swizzle atom. The
@@ -84,6 +94,28 @@ DEC_DEVINL void tmem_st16(uint32_t taddr, const uint32_t* r) {
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+// D (+)= A B with A read from TMEM (lanes = rows, two 16-bit elements per column, the lower
+// k in the low half) and B from shared memory.
+DEC_DEVINL void tc_mma_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
+// Two fp32 values' top halves as the two bf16 of one word (a's in the low half): the
+// values truncated to bf16.
+DEC_DEVINL uint32_t hi_halves(float a, float b) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(__float_as_uint(a)), "r"(__float_as_uint(b)));
+    return d;
+}
+DEC_DEVINL float trunc_bf(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFF0000u); }
+
+// Barrier `id` (1..15) over `n` threads of the CTA (a multiple of 32).
+DEC_DEVINL void named_bar_sync(uint32_t id, uint32_t n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
 DEC_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // No instruction: tells the compiler the 32 registers change here, so no use of values
@@ -119,28 +151,29 @@ DEC_DEVINL float ex2f(float x) {
     return y;
 }
 
-// The row's 128 raw scores v -> scores in log2 units (times scale, or softcapped), keys
-// outside [lo, pos] -inf, in place; returns their maximum (four independent partial
-// maxima). CAP: `sc` is the attention scale and `c` the cap; otherwise `sc` is scale*log2e.
-template <bool CAP>
-DEC_DEVINL float scores_log2(uint32_t (&v)[4][32], float sc, float c, bool whole, int key0, int lo, int pos) {
+// Pass 1 over NC x 32 raw scores of a row (keys key0 ..), in place: keys outside [lo, pos]
+// become -inf; with CAP the others become the softcapped score in log2 units (`sc` the
+// attention scale, `c` the cap), without it they stay raw (the scale, positive, is applied
+// in pass 2). Returns their maximum (four independent partial maxima).
+template <bool CAP, int NC>
+DEC_DEVINL float scores_log2(uint32_t (&v)[NC][32], float sc, float c, bool whole, int key0, int lo, int pos) {
     float bm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     if (whole) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < NC; ++k)
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-                const float x = CAP ? capped_score(__uint_as_float(v[k][q]), sc, c) : __uint_as_float(v[k][q]) * sc;
-                v[k][q] = __float_as_uint(x);
+                const float x = CAP ? capped_score(__uint_as_float(v[k][q]), sc, c) : __uint_as_float(v[k][q]);
+                if (CAP) v[k][q] = __float_as_uint(x);
                 bm4[q & 3] = fmaxf(bm4[q & 3], x);
             }
     } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < NC; ++k)
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
                 const int key = key0 + 32 * k + q;
-                float x = CAP ? capped_score(__uint_as_float(v[k][q]), sc, c) : __uint_as_float(v[k][q]) * sc;
+                float x = CAP ? capped_score(__uint_as_float(v[k][q]), sc, c) : __uint_as_float(v[k][q]);
                 x = key > pos || key < lo ? -INFINITY : x;
                 v[k][q] = __float_as_uint(x);
                 bm4[q & 3] = fmaxf(bm4[q & 3], x);
@@ -154,19 +187,21 @@ struct TcPrefArgs {
     int G, tok_per_cta;
 };
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, TcPrefArgs args) {
     const AttnPrefillArgs& a = args.a;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* kv_full = q_full + 1;   // [2]
-    uint64_t* kv_empty = kv_full + 2; // [2]
-    uint64_t* s_full = kv_empty + 2;  // [2]
-    uint64_t* p_full = s_full + 2;    // the softmax warps are done with S[j & 1] and wrote P
-    uint64_t* pv_done = p_full + 1;   // O += P V of the last issued block completed
-    uint64_t* recvb = pv_done + 1;    // the other splits' rows of this CTA have landed
+    uint64_t* k_full = q_full + 1;               // [kTcStages]
+    uint64_t* k_empty = k_full + kTcStages;      // [kTcStages]
+    uint64_t* v_full = k_empty + kTcStages;      // [kTcStages]
+    uint64_t* v_empty = v_full + kTcStages;      // [kTcStages]
+    uint64_t* s_full = v_empty + kTcStages;      // [2]
+    uint64_t* p_full = s_full + 2;    // the softmax warps read S[j & 1] and wrote P over it
+    uint64_t* pv_done = p_full + 1;   // [2] O += P V of block j completed: pv_done[j & 1]
+    uint64_t* recvb = pv_done + 2;    // the other splits' rows of this CTA have landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recvb + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,19 +220,22 @@ __global__ void __launch_bounds__(192, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
-            mbar_init(&s_full[i], 1);
+        for (int i = 0; i < kTcStages; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
         }
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
+        for (int i = 0; i < 2; ++i) mbar_init(&s_full[i], 1);
+        mbar_init(p_full, 8);
+        mbar_init(&pv_done[0], 1);
+        mbar_init(&pv_done[1], 1);
         mbar_init(recvb, 1);
         // armed before the first cluster barrier, so no byte can arrive before the count
         if (S > 1) mbar_arrive_expect_tx(recvb, (uint32_t)(S - 1) * RS * kLdr * 4);
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
@@ -215,33 +253,37 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tS = tmem, tO = tmem + 2 * kTcKeys;  // S[0], S[1]: columns 0..255; O: 256..383
     pdl_trigger();
 
-    if (warp == 4) {
+    if (warp == 8 || warp == 10) {
         if (lane == 0) {
-            // ------------------------------------------------ TMA producer
+            // ------------------------------------------------ TMA producers: K (warp 8, with
+            // q first) and V (warp 10)
+            const bool isv = warp == 10;
+            uint64_t* full = isv ? v_full : k_full;
+            uint64_t* empty = isv ? v_empty : k_empty;
+            const CUtensorMap* tm = isv ? &tmV : &tmK;
+            uint8_t* ring = smem + (isv ? kOffV : kOffK);
             pdl_wait();  // q and the chunk's own keys come from the previous kernels
-            mbar_arrive_expect_tx(q_full, 32768);
-            for (int h2 = 0; h2 < 2; ++h2)
-                tma_load_3d(smem + kOffQ + h2 * 16384, &tmQ, h2 * 64, g * G, t0, q_full);
+            if (!isv) {
+                mbar_arrive_expect_tx(q_full, 32768);
+                for (int h2 = 0; h2 < 2; ++h2)
+                    tma_load_3d(smem + kOffQ + h2 * 16384, &tmQ, h2 * 64, g * G, t0, q_full);
+            }
             for (int j = 0; j < nb; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !mbar_wait_bounded(&kv_empty[s], ((j >> 1) - 1) & 1, a.err)) break;
-                mbar_arrive_expect_tx(&kv_full[s], 65536);
-                uint8_t* kd = smem + kOffKV + s * kStageKV;
-                uint8_t* vd = kd + 32768;
+                const int s = j % kTcStages;
+                if (j >= kTcStages && !mbar_wait_bounded(&empty[s], (j / kTcStages - 1) & 1, a.err)) break;
+                mbar_arrive_expect_tx(&full[s], kStage);
+                uint8_t* d = ring + s * kStage;
                 for (int pi = 0; pi < kTcKeys / kTcPage; ++pi) {
                     // pages past the chunk's last one hold only masked keys: any finite page
                     // will do, so they reload the last page
                     const int page = min((kb0 + j) * (kTcKeys / kTcPage) + pi, np - 1);
                     const int row = (a.block_row[page] * a.nkv + g) * kTcPage;
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        tma_load_2d(kd + h2 * 16384 + pi * 2048, &tmK, h2 * 64, row, &kv_full[s]);
-                        tma_load_2d(vd + h2 * 16384 + pi * 2048, &tmV, h2 * 64, row, &kv_full[s]);
-                    }
+                    for (int h2 = 0; h2 < 2; ++h2) tma_load_2d(d + h2 * 16384 + pi * 2048, tm, h2 * 64, row, &full[s]);
                 }
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         pdl_wait();
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
@@ -249,57 +291,66 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t id_o = idesc_tc<128, 128, true>();
             const uint32_t sb = smem_u32(smem);
             bool ok = mbar_wait_bounded(q_full, 0, a.err);
+            // S(j) into TMEM columns (j & 1) * 128; the K stage is free once these complete
             auto issue_s = [&](int j) {
-                const int s = j & 1;
-                const uint32_t kb = sb + kOffKV + s * kStageKV;
+                const int s = j % kTcStages;
+                const uint32_t kb = sb + kOffK + s * kStage;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc_mma(tS + s * kTcKeys, sdesc_sw128(sb + kOffQ + (kk >> 2) * 16384 + (kk & 3) * 32),
+                    tc_mma(tS + (j & 1) * kTcKeys, sdesc_sw128(sb + kOffQ + (kk >> 2) * 16384 + (kk & 3) * 32),
                            sdesc_sw128(kb + (kk >> 2) * 16384 + (kk & 3) * 32), id_s, kk > 0 ? 1u : 0u);
-                tc_commit(&s_full[s]);
+                tc_commit(&s_full[j & 1]);
+                tc_commit(&k_empty[s]);
             };
             if (ok && nb > 0) {
-                ok = mbar_wait_bounded(&kv_full[0], 0, a.err);
+                ok = mbar_wait_bounded(&k_full[0], 0, a.err);
                 tc_fence_after();
                 if (ok) issue_s(0);
             }
             for (int j = 0; j < nb && ok; ++j) {
                 if (j + 1 < nb) {
-                    // S[(j + 1) & 1] was last read by the softmax of block j - 1 (waited below
-                    // in the previous iteration)
-                    if (!mbar_wait_bounded(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, a.err)) break;
+                    // TMEM columns ((j + 1) & 1) * 128 held P(j - 1), whose PV product was
+                    // issued before this (tcgen05 MMAs of one thread run in order)
+                    const int s1 = (j + 1) % kTcStages;
+                    if (!mbar_wait_bounded(&k_full[s1], ((j + 1) / kTcStages) & 1, a.err)) break;
                     tc_fence_after();
                     issue_s(j + 1);
                 }
+                const int sv = j % kTcStages;
                 if (!mbar_wait_bounded(p_full, j & 1, a.err)) break;
+                if (!mbar_wait_bounded(&v_full[sv], (j / kTcStages) & 1, a.err)) break;
                 tc_fence_after();
-                const uint32_t vb = sb + kOffKV + (j & 1) * kStageKV + 32768;
+                const uint32_t vb = sb + kOffV + sv * kStage;
+                const uint32_t tp = tS + (j & 1) * kTcKeys;  // P_hi at tp, P_lo at tp + 64
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t pa = (kk >> 2) * 16384 + (kk & 3) * 32;
                     const uint64_t vdesc = sdesc_sw128_mn(vb + kk * 2048);
-                    tc_mma(tO, sdesc_sw128(sb + kOffP + pa), vdesc, id_o, (j > 0 || kk > 0) ? 1u : 0u);
-                    tc_mma(tO, sdesc_sw128(sb + kOffPlo + pa), vdesc, id_o, 1u);
+                    tc_mma_tmem_a(tO, tp + kk * 8, vdesc, id_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_tmem_a(tO, tp + 64 + kk * 8, vdesc, id_o, 1u);
                 }
-                tc_commit(pv_done);
-                tc_commit(&kv_empty[j & 1]);
+                tc_commit(&pv_done[j & 1]);
+                tc_commit(&v_empty[sv]);
             }
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------- softmax + epilogue (warps 0-3)
-        const int r = warp * 32 + lane;  // row = TMEM lane
+        // ------------------------------------ softmax + epilogue (warps 0-7): warps w and w + 4
+        // share the 32 rows (TMEM lanes) 32 (w % 4) ..; warp w takes keys 0-63 of each block,
+        // warp w + 4 keys 64-127
+        const int quad = warp & 3, half = warp >> 2;
+        const int r = quad * 32 + lane;  // row = TMEM lane
         const int tl = r / G;             // token within the CTA
         const int t = t0 + tl;
         const bool valid = tl < TPC && t < a.T;
         const int pos = a.pos0 + t;       // the row's last visible key
         const int lo = a.window > 0 ? pos + 1 - a.window : 0;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const float sl2 = a.scale * kTcLog2e;
         const bool cap = a.softcap > 0.f;
-        float m = -INFINITY, l = 0.f;
+        float* xch = reinterpret_cast<float*>(smem + kOffXch);  // [2 halves][128 rows]
+        const uint32_t pair_bar = 1 + quad;                     // named barrier of warps w, w + 4
+        float m = -INFINITY, l = 0.f;  // l: this half's keys only
         pdl_wait();
-        uint8_t* prow = smem + kOffP + (uint32_t)r * 128;
         bool ok = true;
         for (int j = 0; j < nb; ++j) {
             const int key0 = (kb0 + j) * kTcKeys;
@@ -310,37 +361,45 @@ __global__ void __launch_bounds__(192, 1)
             // wholly outside contributes nothing.
             const bool none = !valid || key0 > pos || key0 + kTcKeys - 1 < lo;
             const bool whole = !none && key0 + kTcKeys - 1 <= pos && key0 >= lo;
-            // the row's 128 scores, in one TMEM round trip (all loads issued, one wait)
-            uint32_t v[4][32];
+            // this half's 64 scores of the row, in one TMEM round trip
+            uint32_t v[2][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_ld16_issue(sa + 32 * c, v[c]);
-                tmem_ld16_issue(sa + 32 * c + 16, v[c] + 16);
+            for (int c = 0; c < 2; ++c) {
+                tmem_ld16_issue(sa + 64 * half + 32 * c, v[c]);
+                tmem_ld16_issue(sa + 64 * half + 32 * c + 16, v[c] + 16);
             }
-            tmem_ld_wait32(v[3]);
+            tmem_ld_wait32(v[1]);
             reg_fence32(v[0]);
-            reg_fence32(v[1]);
-            reg_fence32(v[2]);
-            // pass 1: the scores in log2 units, masked, and the block's row maximum (four
-            // independent partial maxima)
+            // pass 1: the scores in log2 units, masked, and their maximum
             // (the cap and mask tests sit outside the loops: a test, let alone a possible
             // call, per element made this pass cost more than the rest of the block)
             float bm = -INFINITY;
             if (!none) {
                 if (cap)
-                    bm = scores_log2<true>(v, a.scale, a.softcap, whole, key0, lo, pos);
+                    bm = scores_log2<true>(v, a.scale, a.softcap, whole, key0 + 64 * half, lo, pos);
                 else
-                    bm = scores_log2<false>(v, sl2, 0.f, whole, key0, lo, pos);
+                    bm = scores_log2<false>(v, 0.f, 0.f, whole, key0 + 64 * half, lo, pos) * sl2;
             }
-            // O and P of block j - 1 are done with before either is touched
-            if (j > 0 && ok && !mbar_wait_bounded(pv_done, (j - 1) & 1, a.err)) ok = false;
+            // the row maximum over both halves (the first barrier: the partner has read the
+            // last value; the second also orders both halves' score loads before either
+            // writes P over the scores)
+            if (j > 0) named_bar_sync(pair_bar, 64);
+            xch[half * 128 + r] = bm;
+            tc_fence_before();
+            named_bar_sync(pair_bar, 64);
             tc_fence_after();
+            bm = fmaxf(bm, xch[(half ^ 1) * 128 + r]);
             const float mn = fmaxf(m, bm);
             const bool grow = m != -INFINITY && mn > m + kTcRescale;
             if (__any_sync(0xffffffffu, grow)) {
                 // move the reference maximum: O and l of the rows that grew scale by 2^(m - mn)
+                // (each half rescales its 64 columns of O) once O += P V of block j - 1 is in.
+                // Nothing else waits for it: P of block j goes where P of block j - 2 was,
+                // whose product completed before the scores of block j did.
+                if (j > 0 && ok && !mbar_wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, a.err)) ok = false;
+                tc_fence_after();
                 const float corr = grow ? ex2f(m - mn) : 1.f;
-                for (int c0 = 0; c0 < 128; c0 += 32) {
+                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld16_issue(tO + lane_off + c0, o);
                     tmem_ld16_issue(tO + lane_off + c0 + 16, o + 16);
@@ -354,12 +413,18 @@ __global__ void __launch_bounds__(192, 1)
                 l *= corr;
             }
             if (grow || m == -INFINITY) m = mn;
-            // pass 2: P = 2^(S' - m) as bf16 hi + lo in the swizzled A layout, and the row sum
-            // (four independent partial sums); masked scores are -inf and give 0
+            // pass 2: P = 2^(S' - m) as bf16 hi + lo, written over the row's scores in TMEM
+            // (keys 2i, 2i + 1 in column i of each term), and the row sum (four independent
+            // partial sums); masked scores are -inf and give 0. P_hi is P truncated to bf16,
+            // P_lo the exact rest P - P_hi truncated: |P - P_hi - P_lo| < 2^-14 P.
+            // Pairs of keys go through the packed fp32x2 pipe: x = s mul - m, the sums, and
+            // P - P_hi.
             const bool zero = none || m == -INFINITY;
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float2 mul2 = cap ? make_float2(1.f, 1.f) : make_float2(sl2, sl2);
+            const float2 nm2 = make_float2(-m, -m), neg1 = make_float2(-1.f, -1.f);
+            float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t ph[16], pl[16];
                 if (zero) {
 #pragma unroll
@@ -367,40 +432,37 @@ __global__ void __launch_bounds__(192, 1)
                 } else {
 #pragma unroll
                     for (int q = 0; q < 32; q += 2) {
-                        const float p0 = ex2f(__uint_as_float(v[c][q]) - m);
-                        const float p1 = ex2f(__uint_as_float(v[c][q + 1]) - m);
-                        sum4[(q >> 1) & 3] += p0 + p1;
-                        ph[q / 2] = pack_bf2(p0, p1);
-                        pl[q / 2] = pack_bf2(p0 - bf_lo(ph[q / 2]), p1 - bf_hi(ph[q / 2]));
+                        const float2 x =
+                            ffma2(make_float2(__uint_as_float(v[c][q]), __uint_as_float(v[c][q + 1])), mul2, nm2);
+                        const float2 p = make_float2(ex2f(x.x), ex2f(x.y));
+                        sum2[(q >> 1) & 1] = fadd2(sum2[(q >> 1) & 1], p);
+                        ph[q / 2] = hi_halves(p.x, p.y);
+                        const float2 rest = ffma2(make_float2(trunc_bf(p.x), trunc_bf(p.y)), neg1, p);
+                        pl[q / 2] = hi_halves(rest.x, rest.y);
                     }
                 }
-                // keys 32 c .. 32 c + 31 of this row: key-half c / 2, 16-byte chunks
-                // 4 (c % 2) .. + 3, stored at chunk ^ (row % 8)
-                uint8_t* base = prow + (c >> 1) * 16384;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int chunk = 4 * (c & 1) + ch;
-                    const uint32_t off = (uint32_t)((chunk ^ (r & 7)) << 4);
-                    *reinterpret_cast<uint4*>(base + off) = make_uint4(ph[4 * ch], ph[4 * ch + 1], ph[4 * ch + 2], ph[4 * ch + 3]);
-                    *reinterpret_cast<uint4*>(base + (kOffPlo - kOffP) + off) =
-                        make_uint4(pl[4 * ch], pl[4 * ch + 1], pl[4 * ch + 2], pl[4 * ch + 3]);
-                }
+                const int cg = 2 * half + c;  // keys 32 cg .. 32 cg + 31 of the block
+                tmem_st16(sa + 16 * cg, ph);
+                tmem_st16(sa + 64 + 16 * cg, pl);
             }
-            const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-            l += sum;
-            fence_proxy_async_smem();  // the MMA reads P through the async proxy
+            l += (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);
+            tmem_st_wait();  // the MMA reads P from TMEM
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        // ---- epilogue
-        if (nb > 0 && ok && !mbar_wait_bounded(pv_done, (nb - 1) & 1, a.err)) ok = false;
+        // ---- epilogue: the row sum over both halves
+        named_bar_sync(pair_bar, 64);
+        xch[half * 128 + r] = l;
+        named_bar_sync(pair_bar, 64);
+        l += xch[(half ^ 1) * 128 + r];
+        if (nb > 0 && ok && !mbar_wait_bounded(&pv_done[(nb - 1) & 1], ((nb - 1) >> 1) & 1, a.err)) ok = false;
         tc_fence_after();
         if (S == 1) {
-            // O / l, bf16, to out[t][g G + (r % G)][:]
+            // O / l, bf16, to out[t][g G + (r % G)][:] (each half its 64 columns)
             const float inv = l > 0.f ? 1.0f / l : 0.f;
             uint16_t* dst = a.out + ((size_t)t * a.nq + (size_t)g * G + (r % G)) * 128;
-            for (int c0 = 0; c0 < 128; c0 += 32) {
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld16_issue(tO + lane_off + c0, v);
                 tmem_ld16_issue(tO + lane_off + c0 + 16, v + 16);
@@ -420,7 +482,7 @@ __global__ void __launch_bounds__(192, 1)
         } else {
             // this split's partial row (unnormalised O, m, l) into the drained ring
             float* st = reinterpret_cast<float*>(smem + kOffStage) + (size_t)r * kLdr;
-            for (int c0 = 0; c0 < 128; c0 += 32) {
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                 uint32_t v[32];
                 if (nb > 0) {
                     tmem_ld16_issue(tO + lane_off + c0, v);
@@ -434,7 +496,7 @@ __global__ void __launch_bounds__(192, 1)
                 for (int q = 0; q < 32; q += 4)
                     *reinterpret_cast<uint4*>(st + c0 + q) = make_uint4(v[q], v[q + 1], v[q + 2], v[q + 3]);
             }
-            *reinterpret_cast<float4*>(st + 128) = make_float4(m, l, 0.f, 0.f);
+            if (half == 0) *reinterpret_cast<float4*>(st + 128) = make_float4(m, l, 0.f, 0.f);
             fence_proxy_async_smem();  // the copies read these writes through the async proxy
         }
     }
@@ -565,7 +627,7 @@ cudaError_t attn_prefill_tc_launch(const AttnPrefillArgs& a, cudaStream_t st, bo
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((a.T + args.tok_per_cta - 1) / args.tok_per_cta, a.nkv, S);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(352);
     cfg.dynamicSmemBytes = kTcSmem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
