@@ -28,6 +28,10 @@
 //    64-key blocks of the cache among its 4 warps and skips fully masked pages.
 #include <math.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -36,7 +40,6 @@ namespace dec {
 namespace {
 
 constexpr int kPage = 16;
-constexpr int kRing = 3;  // pages in flight per warp in the decode kernel
 constexpr int kDecodeMaxSplits = 16;  // context splits of one (sequence, kv head): one cluster
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -174,8 +177,10 @@ DEC_DEVINL void softmax_page(float (&sc)[2][4], float (&m)[2], float (&l)[2], fl
 }
 
 // O += P V for one 16-key page: P (rows g, g+8) from sc, V page rows in shared memory
-// with row stride LD. P enters as bf16 hi + lo parts.
-template <int D, int LD>
+// with row stride LD, chunks swizzled as load_page_warp stores them. P enters as bf16 hi + lo parts. PACK (at most 8 query rows): row
+// g + 8 of the A tile carries P_lo of row g, so one MMA per tile takes both terms; the
+// accumulator's rows g and g + 8 then hold the two terms' products of row g.
+template <int D, int LD, bool PACK>
 DEC_DEVINL void pv_page(const float (&sc)[2][4], const uint16_t* vd, float (&o)[D / 8][4]) {
     const int lane = threadIdx.x & 31;
     uint32_t ph[4], pl[4];
@@ -190,19 +195,28 @@ DEC_DEVINL void pv_page(const float (&sc)[2][4], const uint16_t* vd, float (&o)[
         pl[i] = pack_bf2(a - ah, b - bh);
     }
     const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+    // A fragment: [0] row g keys 2t.., [1] row g + 8 keys 2t.., [2] row g keys 8 + 2t..,
+    // [3] row g + 8 keys 8 + 2t..
+    const uint32_t pk[4] = {ph[0], pl[0], ph[2], pl[2]};
 #pragma unroll
     for (int dt2 = 0; dt2 < D / 16; ++dt2) {
         uint32_t vb[4];
-        ldsm_x4_trans(vb, vd + key * LD + dt2 * 16 + (lane >> 4) * 8);
+        ldsm_x4_trans(vb, vd + key * LD + (((dt2 * 2 + (lane >> 4)) ^ (key & 7)) << 3));
         const uint32_t b0[2] = {vb[0], vb[1]}, b1[2] = {vb[2], vb[3]};
-        mma_bf16_16816(o[2 * dt2], ph, b0);
-        mma_bf16_16816(o[2 * dt2], pl, b0);
-        mma_bf16_16816(o[2 * dt2 + 1], ph, b1);
-        mma_bf16_16816(o[2 * dt2 + 1], pl, b1);
+        if constexpr (PACK) {
+            mma_bf16_16816(o[2 * dt2], pk, b0);
+            mma_bf16_16816(o[2 * dt2 + 1], pk, b1);
+        } else {
+            mma_bf16_16816(o[2 * dt2], ph, b0);
+            mma_bf16_16816(o[2 * dt2], pl, b0);
+            mma_bf16_16816(o[2 * dt2 + 1], ph, b1);
+            mma_bf16_16816(o[2 * dt2 + 1], pl, b1);
+        }
     }
 }
 
-// S = Q K^T for one 16-key page: Q fragments qf (rows 0..15), K page rows in shared memory.
+// S = Q K^T for one 16-key page: Q fragments qf (rows 0..15), K page rows in shared memory
+// (swizzled as load_page_warp stores them).
 template <int D, int LD>
 DEC_DEVINL void qk_page(const uint32_t (&qf)[D / 16][4], const uint16_t* kd, float (&sc)[2][4]) {
     const int lane = threadIdx.x & 31;
@@ -211,14 +225,21 @@ DEC_DEVINL void qk_page(const uint32_t (&qf)[D / 16][4], const uint16_t* kd, flo
 #pragma unroll
         for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
     const int key = (lane & 7) + (lane >> 4) * 8;
+    // even and odd k steps accumulate separately: two dependent chains of D / 32 MMAs per
+    // tile instead of one of D / 16
+    float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
         uint32_t kb[4];
-        ldsm_x4(kb, kd + key * LD + ks * 16 + ((lane >> 3) & 1) * 8);
+        ldsm_x4(kb, kd + key * LD + (((ks * 2 + ((lane >> 3) & 1)) ^ (key & 7)) << 3));
         const uint32_t b0[2] = {kb[0], kb[1]}, b1[2] = {kb[2], kb[3]};
-        mma_bf16_16816(sc[0], qf[ks], b0);
-        mma_bf16_16816(sc[1], qf[ks], b1);
+        mma_bf16_16816((ks & 1) ? s2[0] : sc[0], qf[ks], b0);
+        mma_bf16_16816((ks & 1) ? s2[1] : sc[1], qf[ks], b1);
     }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[nt][c] += s2[nt][c];
 }
 
 template <int D, int LD>
@@ -229,7 +250,9 @@ DEC_DEVINL void load_q_frags(const uint16_t* qs, uint32_t (&qf)[D / 16][4]) {
     for (int ks = 0; ks < D / 16; ++ks) ldsm_x4(qf[ks], qs + row * LD + ks * 16 + (lane >> 4) * 8);
 }
 
-// Copy one page (16 rows x D) of K and V of kv head g into padded shared rows (one warp).
+// Copy one page (16 rows x D) of K and V of kv head g into shared rows of stride LD (one
+// warp). Decode pages are unpadded (LD = D) with the 16-byte chunks of row r stored at
+// chunk ^ (r % 8): the 8 rows an ldmatrix phase reads then fall in distinct banks.
 template <int D, int LD>
 DEC_DEVINL void load_page_warp(const uint16_t* kpool, const uint16_t* vpool, int phys, int nkv, int g,
                                uint16_t* kd, uint16_t* vd) {
@@ -239,8 +262,9 @@ DEC_DEVINL void load_page_warp(const uint16_t* kpool, const uint16_t* vpool, int
 #pragma unroll
     for (int c = lane; c < CH; c += 32) {
         const int row = c / (D / 8), col = (c % (D / 8)) * 8;
-        cp_async16(kd + row * LD + col, kpool + base + row * D + col);
-        cp_async16(vd + row * LD + col, vpool + base + row * D + col);
+        const int sw = (((col >> 3) ^ (row & 7)) << 3);
+        cp_async16(kd + row * LD + sw, kpool + base + row * D + col);
+        cp_async16(vd + row * LD + sw, vpool + base + row * D + col);
     }
     cp_async_commit();
 }
@@ -249,23 +273,33 @@ DEC_DEVINL void load_page_warp(const uint16_t* kpool, const uint16_t* vpool, int
 
 // Page ring depth per warp: 8-warp CTAs (split contexts, few pages each) keep 2 pages in
 // flight per warp, 4-warp CTAs (one CTA per sequence and kv head, many pages) keep 3.
-template <int NW>
-constexpr int kDecRing = NW >= 8 ? 2 : kRing;
+// Shared memory of the decode kernel: the page rings (the warps' partials reuse them after
+// the page loop) and, for a cluster merge, the receive area of the rows a CTA finishes. At
+// ~110 KB two CTAs fit on an SM, so a 16-CTA cluster can be placed on 8 SMs of a GPC (at
+// 1 CTA per SM some 16-CTA clusters waited for a second wave).
+template <int D, int NW, int RING>
+__host__ __device__ constexpr size_t dec_rings_bytes() {
+    const size_t ring = (size_t)NW * RING * 2 * kPage * D * 2;
+    const size_t wo = (size_t)NW * 16 * D * 4;
+    return ring > wo ? ring : wo;
+}
 
-template <int D, int NW>
+template <int D, int NW, int RING>
 __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) {
-    constexpr int LD = D + 8;
-    constexpr int PAGE = kPage * LD;
+    constexpr int LD = D + 8;      // q tile rows
+    constexpr int PLD = D;         // page rows (chunk-swizzled)
+    constexpr int PAGE = kPage * PLD;
     constexpr int LDR = D + 4;  // receive rows: o[D], m, l, 2 pad (16-byte aligned)
-    constexpr int RING = kDecRing<NW>;
     constexpr int NT = NW * 32;
     __shared__ __align__(16) uint16_t qs[16 * LD];
     __shared__ __align__(16) uint16_t newkv[2][D];  // the appended k and v rows (bf16)
     __shared__ float wm[NW][16], wl[NW][16];
+    __shared__ __align__(8) uint64_t recv_bar;  // the partials of this CTA's rows have landed
     extern __shared__ __align__(16) uint8_t dyn[];
-    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [NW warps][RING][K,V][16][LD]
+    uint16_t* kvbuf = reinterpret_cast<uint16_t*>(dyn);  // [NW warps][RING][K,V][16][D]
     float* wo = reinterpret_cast<float*>(dyn);           // [NW][16][D] after the page loop
-    float* recv = wo + NW * 16 * D;                      // [rows owned][splits][LDR]
+    // [rows owned][splits][LDR]: every split's partial of the rows this CTA finishes
+    float* recv = reinterpret_cast<float*>(dyn + dec_rings_bytes<D, NW, RING>());
 
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z, S = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -276,6 +310,18 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
     // done, and nobody writes into another CTA's shared memory before every CTA has arrived.
     const bool cl = S > 1 && a.part == nullptr;
     __shared__ int ticket_s;
+    // At most 8 query heads per group: P_lo rides in the tile's spare rows 8-15 (pv_page).
+    const bool pack = G <= 8;
+    if (cl) {
+        // Each CTA will send its partial rows straight to the CTA finishing them (st.async,
+        // completing as transaction bytes on that CTA's recv_bar). The barrier is initialised
+        // before this CTA arrives on the cluster barrier; senders wait on it before sending.
+        if (tid == 0) {
+            mbar_init(&recv_bar, 1);
+            fence_mbar_init();
+        }
+        asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    }
 
     // ---- independent of the previous kernel: positions, block table and the cache pages
     // (the row being appended is patched in after it is written, below)
@@ -308,7 +354,7 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
     int issued = 0;
     for (; issued < cnt && issued < RING; ++issued) {
         uint16_t* slot = wbuf + (size_t)issued * 2 * PAGE;
-        load_page_warp<D, LD>(a.k_pool, a.v_pool, page_entry(issued), a.nkv, g, slot, slot + PAGE);
+        load_page_warp<D, PLD>(a.k_pool, a.v_pool, page_entry(issued), a.nkv, g, slot, slot + PAGE);
     }
     // the model path's angles and QK-norm gains do not depend on the previous kernel either
     const float2* tab = a.rope_tab ? a.rope_tab + (size_t)p * (D / 2) : nullptr;
@@ -391,13 +437,15 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
             uint16_t* kd = wbuf + (size_t)(i % RING) * 2 * PAGE;
             if (pg == np - 1 && has_last && have_new) {
                 // the page was fetched before row p existed: copy the staged row in
-                uint16_t* row = kd + (lane < 16 ? 0 : PAGE) + (p % kPage) * LD;
+                const int pr = p % kPage;
+                uint16_t* row = kd + (lane < 16 ? 0 : PAGE) + pr * PLD;
                 for (int c = (lane & 15) * 8; c < D; c += 128)
-                    *reinterpret_cast<uint4*>(row + c) = *reinterpret_cast<const uint4*>(&newkv[lane >> 4][c]);
+                    *reinterpret_cast<uint4*>(row + ((((c >> 3) ^ (pr & 7))) << 3)) =
+                        *reinterpret_cast<const uint4*>(&newkv[lane >> 4][c]);
                 __syncwarp();
             }
             float sc[2][4];
-            qk_page<D, LD>(qf, kd, sc);
+            qk_page<D, PLD>(qf, kd, sc);
             // the softcap test stays outside the loops: the plain path carries no tanh at all
             if (a.softcap > 0.f) {
 #pragma unroll
@@ -419,6 +467,7 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
                 }
             float corr[2];
             softmax_page(sc, m, l, corr);
+            if (pack) corr[1] = corr[0];  // rows g + 8 hold row g's P_lo products
 #pragma unroll
             for (int q = 0; q < D / 8; ++q) {
                 o[q][0] *= corr[0];
@@ -426,10 +475,13 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
                 o[q][2] *= corr[1];
                 o[q][3] *= corr[1];
             }
-            pv_page<D, LD>(sc, kd + PAGE, o);
+            if (pack)
+                pv_page<D, PLD, true>(sc, kd + PAGE, o);
+            else
+                pv_page<D, PLD, false>(sc, kd + PAGE, o);
             __syncwarp();
             if (issued < cnt) {
-                load_page_warp<D, LD>(a.k_pool, a.v_pool, page_entry(issued), a.nkv, g, kd, kd + PAGE);
+                load_page_warp<D, PLD>(a.k_pool, a.v_pool, page_entry(issued), a.nkv, g, kd, kd + PAGE);
                 ++issued;
             }
         }
@@ -439,13 +491,18 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
             l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
         }
     }
+    if (pack) {
+        // row g's two terms; rows 8-15 are past the group
+#pragma unroll
+        for (int q = 0; q < D / 8; ++q) {
+            o[q][0] += o[q][2];
+            o[q][1] += o[q][3];
+        }
+    }
 
     // ---- merge the 4 warps of the CTA through shared memory (a CTA without pages
     // contributes m = -inf, l = 0, o = 0)
     __syncthreads();  // page buffers are free
-    // this CTA no longer reads its page rings: the other CTAs of the cluster may write
-    // their partials into them once everyone has arrived (release: the reads come first)
-    if (cl) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     if (t4 == 0) {
         wm[warp][gr] = m[0];
         wm[warp][gr + 8] = m[1];
@@ -462,11 +519,13 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
         r1[1] = o[i][3];
     }
     __syncthreads();
-    // Split partial of row r: o (relative to M) and M, L. In a cluster, row r is finished
-    // by CTA r % S, which receives every split's partial of it in slot [r / S][s];
-    // otherwise the partials go to the scratch and the last CTA of (b, g) merges them.
-    // every CTA of the cluster is past its page loop (and still running)
-    if (cl) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // Split partial of row r: o (relative to M) and M, L. In a cluster row r is finished by
+    // CTA r % S, which receives every split's partial of it in slot [r / S][s]; otherwise the
+    // partials go to the scratch and the last CTA of (b, g) merges them.
+    uint32_t rbar = 0;
+    if (cl) {
+        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every recv_bar is initialised
+    }
     for (int idx = tid; idx < G * (D / 4); idx += NT) {
         const int r = idx / (D / 4), c = (idx % (D / 4)) * 4;
         float M = -INFINITY;
@@ -492,10 +551,11 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
             pk.y = pack_bf2(O.z * inv, O.w * inv);
             *reinterpret_cast<uint2*>(a.out + (size_t)b * a.nq * D + (size_t)(g * G + r) * D + c) = pk;
         } else if (cl) {
-            const uint32_t dst = smem_u32(recv + ((size_t)(r / S) * S + s) * LDR);
-            dsmem_st4(dst + c * 4, r % S, __float_as_uint(O.x), __float_as_uint(O.y), __float_as_uint(O.z),
-                      __float_as_uint(O.w));
-            if (c == 0) dsmem_st2f(dst + D * 4, r % S, M, L);
+            const int own = r % S;
+            const uint32_t dst = dsmem_map(smem_u32(recv + ((size_t)(r / S) * S + s) * LDR), own);
+            rbar = dsmem_map(smem_u32(&recv_bar), own);
+            st_async_4f(dst + c * 4, O.x, O.y, O.z, O.w, rbar);
+            if (c == 0) st_async_2f(dst + D * 4, M, L, rbar);
         } else {
             float* pp = a.part + (((size_t)b * a.nq + g * G + r) * S + s) * (D + 2);
             pp[c] = O.x;
@@ -511,12 +571,16 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
     if (S == 1) return;
 
     if (cl) {
-        cluster_sync();  // all partials have arrived
-        // rows r = s, s + S, ...: weighted sum over the splits in split order
-        // (unrolled to the cluster bound: the split weights are computed once per row, and
-        // the loads of every split are in flight together)
-        for (int r = s; r < G; r += S) {
-            const float* rv = recv + (size_t)(r / S) * S * LDR;
+        // ---- rows r = s, s + S, ...: weighted sum over the splits in split order
+        const int owned = s < G ? (G - 1 - s) / S + 1 : 0;
+        if (owned == 0) return;  // nothing reads this CTA's shared memory
+        if (tid == 0) mbar_arrive_expect_tx(&recv_bar, (uint32_t)(owned * S * (D * 4 + 8)));
+        const bool got = mbar_wait_cluster_bounded(&recv_bar, 0, a.err);
+        for (int j = 0; j < owned; ++j) {
+            const int r = s + j * S;
+            const float* rv = recv + (size_t)j * S * LDR;
+            // (unrolled to the cluster bound: the split weights are computed once per row,
+            // and the loads of every split are in flight together)
             float mz[kDecodeMaxSplits], wz[kDecodeMaxSplits];
             float M = -INFINITY;
 #pragma unroll
@@ -536,7 +600,7 @@ __global__ void __launch_bounds__(NW * 32) attn_decode_kernel(AttnDecodeArgs a) 
 #pragma unroll
                 for (int z = 0; z < kDecodeMaxSplits; ++z)
                     if (mz[z] != -INFINITY) O += wz[z] * rv[(size_t)z * LDR + c];
-                a.out[(size_t)b * a.nq * D + (size_t)(g * G + r) * D + c] = f2bf(O * invL);
+                if (got) a.out[(size_t)b * a.nq * D + (size_t)(g * G + r) * D + c] = f2bf(O * invL);
             }
         }
         return;
@@ -955,26 +1019,27 @@ int attn_decode_splits(int B, int nkv, int max_ctx, int num_sms, bool cluster) {
     return s;
 }
 
-template <int D, int NW>
-size_t decode_smem(int G, int splits) {
-    const size_t ring = (size_t)NW * kDecRing<NW> * 2 * kPage * (D + 8) * 2;  // page rings of NW warps
-    const size_t rows_owned = (size_t)(G + splits - 1) / splits;
-    const size_t merge = (size_t)NW * 16 * D * 4 + rows_owned * splits * (D + 4) * 4;  // warp partials + receive
-    return ring > merge ? ring : merge;
+template <int D, int NW, int RING>
+size_t decode_smem(int G, int splits, bool cl) {
+    size_t sm = dec_rings_bytes<D, NW, RING>();
+    if (cl) sm += (size_t)((G + splits - 1) / splits) * splits * (D + 4) * 4;  // receive area
+    return sm;
 }
 
-template <int D, int NW>
+template <int D, int NW, int RING>
 cudaError_t decode_launch_dw(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
     const int G = a.nq / a.nkv;
-    const size_t smem = decode_smem<D, NW>(G, a.splits);
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(attn_decode_kernel<D, NW>), (int)smem);
-    if (e != cudaSuccess) return e;
     const bool cl = a.splits > 1 && a.part == nullptr;
+    const size_t smem = decode_smem<D, NW, RING>(G, a.splits, cl);
+    auto kern = attn_decode_kernel<D, NW, RING>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), (int)smem);
+    if (e != cudaSuccess) return e;
     if (cl && a.splits > 8) {
         static std::once_flag once;
         static cudaError_t ce = cudaSuccess;
         std::call_once(once, [] {
-            ce = cudaFuncSetAttribute(attn_decode_kernel<D, NW>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            ce = cudaFuncSetAttribute(attn_decode_kernel<D, NW, RING>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                      1);
         });
         if (ce != cudaSuccess) return ce;
     }
@@ -999,20 +1064,73 @@ cudaError_t decode_launch_dw(const AttnDecodeArgs& a, cudaStream_t st, bool pdl)
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, attn_decode_kernel<D, NW>, a);
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// 4 warps with 3-page rings. (8 warps with 2-page rings, all of a split's pages in flight at
-// once, measured slower at batch 1: 20.8 against 11-13 us per launch of the Llama-3-8B shape.)
+// How many clusters of S CTAs of attn_decode_kernel<D, 4, 4> the device holds at once (GPCs
+// hold whole clusters, so at one CTA per SM this can be below SMs / S). Cached per device,
+// group size and S.
+template <int D>
+int decode_resident(int G, int S) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int>, int> known;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_tuple(dev, G, S);
+    auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    int n = 0;
+    auto kern = attn_decode_kernel<D, 4, 4>;
+    const size_t smem = decode_smem<D, 4, 4>(G, S, true);
+    bool ok = ensure_smem(reinterpret_cast<const void*>(kern), (int)smem) == cudaSuccess;
+    if (ok && S > 8) ok = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    if (ok) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(S, 8, 1);
+        cfg.blockDim = dim3(128);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();  // a refused query leaves no error behind
+    known[key] = n;
+    return n;
+}
+
+// 4 warps. Split contexts merged in a cluster get 4-page rings at one CTA per SM (every
+// page of a split of up to 16 pages is in flight before the wait on the previous kernel,
+// and no warp shares its scheduler with another CTA's), with the largest split count whose
+// clusters are all resident at once; otherwise 3-page rings, two CTAs per SM. (8 warps
+// with 2-page rings measured slower at batch 1: 20.8 against 11-13 us per launch of the
+// Llama-3-8B shape. 16-CTA clusters at one CTA per SM: one of the 8 waited for a second
+// wave.)
 template <int D>
 cudaError_t decode_launch_d(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
-    return decode_launch_dw<D, 4>(a, st, pdl);
+    if (a.splits > 1 && a.part == nullptr) {
+        const int G = a.nq / a.nkv, clusters = a.B * a.nkv;
+        for (int S = a.splits; S >= 2; --S) {
+            if (decode_resident<D>(G, S) >= clusters) {
+                AttnDecodeArgs b = a;
+                b.splits = S;
+                return decode_launch_dw<D, 4, 4>(b, st, pdl);
+            }
+        }
+    }
+    return decode_launch_dw<D, 4, 3>(a, st, pdl);
 }
 
 cudaError_t attn_decode_launch(const AttnDecodeArgs& a, cudaStream_t st, bool pdl) {
     if (a.splits < 1 || a.nkv <= 0 || a.nq % a.nkv != 0 || a.nq / a.nkv > 16) return cudaErrorInvalidValue;
     if (a.splits > 1 && a.part == nullptr && a.splits > kDecodeMaxSplits) return cudaErrorInvalidValue;
-    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > decode_smem<64, 4>(a.nq / a.nkv, a.splits)) return cudaErrorInvalidValue;
+    // the scratch merge keeps [G][splits] weights in the page rings
+    if ((size_t)(a.nq / a.nkv) * a.splits * 4 > dec_rings_bytes<64, 4, 3>()) return cudaErrorInvalidValue;
     if (a.d == 128) return decode_launch_d<128>(a, st, pdl);
     if (a.d == 64) return decode_launch_d<64>(a, st, pdl);
     return cudaErrorInvalidValue;

@@ -85,6 +85,31 @@ DEC_DEVINL bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err) {
     return true;
 }
 
+// The same wait with acquire at cluster scope: for a phase completed by other CTAs'
+// st.async transactions (their data is visible once the phase is seen complete).
+DEC_DEVINL bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+DEC_DEVINL bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, int* err) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (clock64() - t0 > (1ll << 32)) {
+            if (err) atomicExch(err, 1);
+            return false;
+        }
+    }
+    return true;
+}
+
 // ----------------------------------------------------------------- bulk copy global -> shared (TMA engine)
 
 // Contiguous copy of `bytes` (multiple of 16, both addresses 16-byte aligned),
@@ -177,6 +202,22 @@ DEC_DEVINL uint32_t dsmem_map(uint32_t saddr, int rank) {
 DEC_DEVINL void dsmem_st4(uint32_t saddr, int rank, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     const uint32_t remote = dsmem_map(saddr, rank);
     asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// Stores of two (four) floats to a cluster shared-memory address (dsmem_map) that complete
+// as 8 (16) transaction bytes on the destination CTA's mbarrier `bar` (also a cluster
+// address). The data comes from registers, so the sending CTA may exit right after.
+DEC_DEVINL void st_async_2f(uint32_t dst, float a, float b, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(dst),
+                 "f"(a), "f"(b), "r"(bar)
+                 : "memory");
+}
+
+DEC_DEVINL void st_async_4f(uint32_t dst, float a, float b, float c, float d, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     dst),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
                  : "memory");
 }
 
