@@ -11,9 +11,10 @@
 //  * persistent: one CTA per SM; the (128 x BN tile, 64-wide k block) units of the
 //    product (BN = 32/64/128 tokens) are cut into equal contiguous ranges, one per
 //    CTA (stream-K), so every SM streams the same share of the weights whatever the
-//    tile count; a tile shared by several CTAs is finished by the CTA whose piece
-//    arrives last, which sums the fp32 pieces in k order (deterministic, no atomics
-//    on data);
+//    tile count; a tile shared by several CTAs is finished by the CTA holding its
+//    last k blocks: the others publish their fp32 pieces first thing, and the
+//    finisher adds them, in k order, to its own accumulator (deterministic, no
+//    atomics on data, and no CTA waits for another's wait);
 //  * warp 4 / lane 0 drives TMA: 128B-swizzled 64-wide K slices of A and B into a
 //    6-8 stage shared-memory ring (mbarrier complete_tx); the weight slices of
 //    the first stages are issued before griddepcontrol.wait (they do not depend
@@ -220,10 +221,10 @@ struct Seg {
     int tile, kb0, kb1, slot;  // slot: 0 = first tile of the range, 1 = any later one
 };
 
-// The j-th segment in processing order: the stream-K pieces at the two ends of the range
-// come first (their tiles are finished by whichever CTA completes its piece last, so those
-// reductions overlap the whole tiles processed afterwards), then the middle tiles, then
-// the round-robin whole tiles.
+// The j-th segment in processing order: the head piece of the range's last tile first (a
+// piece some later CTA finishes, so it is published as early as possible), then the
+// first tile (this CTA holds its last k blocks and finishes it), then the middle tiles,
+// then the round-robin whole tiles.
 DEC_DEVINL Seg segment(const Work& w, const Range& r, int j) {
     Seg s;
     if (j >= r.nsk) {
@@ -277,10 +278,9 @@ DEC_DEVINL int ld_acquire_gpu(const int* p) {
     return v;
 }
 
-// Whether every piece of a shared tile has been published (tile counter >= P), waiting
-// for it (bounded: on time-out sets the error flag and returns false). It is only called
-// once the CTA's own operand loads and MMAs have all completed and before it issues any
-// reduction load, so a CTA that gives up here leaves nothing in flight.
+// Whether P pieces of a shared tile have been published (tile counter >= P), waiting for
+// them (bounded: on time-out sets the error flag and returns false). Only the CTA that
+// finishes the tile calls it, after its own piece's MMAs have completed.
 DEC_DEVINL bool tile_ready(const GemmArgs& a, int tile, int P, volatile int* flag_s) {
     if (threadIdx.x == 0) {
         int r = 1;
@@ -293,8 +293,6 @@ DEC_DEVINL bool tile_ready(const GemmArgs& a, int tile, int P, volatile int* fla
                 break;
             }
         }
-        // the pieces were written through the generic proxy; they are read by TMA below
-        asm volatile("fence.proxy.async.global;" ::: "memory");
         *flag_s = r;
     }
     epi_bar();
@@ -303,182 +301,10 @@ DEC_DEVINL bool tile_ready(const GemmArgs& a, int tile, int P, volatile int* fla
     return r != 0;
 }
 
-// Cooperative finish of a tile shared by CTAs c_lo..c_hi (k order), once all of them have
-// published their pieces: CTA c takes a slice of the tile's rows, fetches that slice of
-// every piece into shared memory with TMA (32-row boxes, [column][row] fp32), sums the
-// pieces in k order (deterministic) and applies the epilogue; lane = row and warp w
-// = 16-column chunks w, w + 4, as in the accumulator epilogue. The tile counter goes from
-// 0 to P (pieces published) and on to 2P (slices done); the CTA that completes it resets
-// it to 0. `buf` is the drained operand ring, room for `cap` boxes.
-template <int BN>
-DEC_DEVINL bool reduce_slice(const GemmArgs& a, const Work& w, int c, int tile, const CUtensorMap* tmW,
-                             uint8_t* buf, int cap, uint64_t* redb, uint32_t& red_phase) {
-    constexpr int BOX = 32 * BN * 4;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long t0 = (long long)tile * w.nkb;
-    const int c_lo = cta_of(w, t0), c_hi = cta_of(w, t0 + w.nkb - 1);
-    const int P = c_hi - c_lo + 1;
-    // every CTA after the first starts inside the tile (its slot 0); the first holds the
-    // tile in slot 0 only if its range starts exactly at the tile
-    const int slot_lo = piece_slot(w, c_lo, tile);
-    const int rs = (((BM + P - 1) / P) + 3) & ~3;  // multiple of 4 rows: 16-byte TMA x
-    const int r0 = min(BM, (c - c_lo) * rs), r1 = min(BM, r0 + rs);
-    const int m0 = tile / w.tiles_n * BM, n0 = tile % w.tiles_n * BN;
-    for (int rb = r0; rb < r1; rb += 32) {
-        float acc[kChunks<BN>][16];
-#pragma unroll
-        for (int h = 0; h < kChunks<BN>; ++h)
-#pragma unroll
-            for (int q = 0; q < 16; ++q) acc[h][q] = 0.f;
-        for (int cb = c_lo; cb <= c_hi; cb += cap) {
-            const int n = min(cap, c_hi - cb + 1);
-            if (threadIdx.x == 0) {
-                mbar_arrive_expect_tx(redb, (uint32_t)(n * BOX));
-                for (int u = 0; u < n; ++u) {
-                    const int cc = cb + u;
-                    tma_load_2d(buf + u * BOX, tmW, rb, (cc * 2 + (cc == c_lo ? slot_lo : 0)) * BN, redb);
-                }
-            }
-            if (!mbar_wait_bounded(redb, red_phase & 1u, a.err)) return false;
-            ++red_phase;
-            for (int u = 0; u < n; ++u) {
-                const float* bx = reinterpret_cast<const float*>(buf + u * BOX);
-#pragma unroll
-                for (int h = 0; h < kChunks<BN>; ++h) {
-                    const int ch = warp + 4 * h;
-                    if (ch * 16 < BN) {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) acc[h][q] += bx[(ch * 16 + q) * 32 + lane];
-                    }
-                }
-            }
-            epi_bar();  // every thread is done with the boxes before the next batch lands
-        }
-        const int rl = rb + lane;
-        const int row = rl < r1 ? m0 + rl : 0x3fffffff;  // rows outside the slice write nothing
-#pragma unroll
-        for (int h = 0; h < kChunks<BN>; ++h) {
-            const int ch = warp + 4 * h;
-            if (ch * 16 < BN) {
-                epilogue16(a, row, n0 + ch * 16, acc[h]);
-                if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + ch * 16, acc[h]);
-            }
-        }
-    }
-    epi_bar();
-    if (threadIdx.x == 0 && atomicAdd(&a.cnt[tile], 1) == 2 * P - 1) atomicExch(&a.cnt[tile], 0);
-    return true;
-}
-
-// The slice of a shared tile that CTA c finishes (see reduce_slice).
-struct RedPlan {
-    int tile, c_lo, c_hi, slot_lo, r0, r1;
-};
-
-DEC_DEVINL RedPlan red_plan(const Work& w, int c, int tile) {
-    RedPlan r;
-    const long long t0 = (long long)tile * w.nkb;
-    r.tile = tile;
-    r.c_lo = cta_of(w, t0);
-    r.c_hi = cta_of(w, t0 + w.nkb - 1);
-    const int P = r.c_hi - r.c_lo + 1;
-    r.slot_lo = piece_slot(w, r.c_lo, tile);
-    const int rs = (((BM + P - 1) / P) + 3) & ~3;
-    r.r0 = min(BM, (c - r.c_lo) * rs);
-    r.r1 = min(BM, r.r0 + rs);
-    return r;
-}
-
-DEC_DEVINL int red_boxes(const RedPlan& r) { return ((r.r1 - r.r0 + 31) / 32) * (r.c_hi - r.c_lo + 1); }
-
-// Thread 0 issues the boxes of every plan in one batch (plan, row box, piece order).
-template <int BN>
-DEC_DEVINL void red_issue(const RedPlan* rp, int n, int total, const CUtensorMap* tmW, uint8_t* buf,
-                          uint64_t* redb) {
-    constexpr int BOX = 32 * BN * 4;
-    if (threadIdx.x != 0) return;
-    mbar_arrive_expect_tx(redb, (uint32_t)(total * BOX));
-    int k = 0;
-    for (int i = 0; i < n; ++i)
-        for (int rb = rp[i].r0; rb < rp[i].r1; rb += 32)
-            for (int cc = rp[i].c_lo; cc <= rp[i].c_hi; ++cc, ++k)
-                tma_load_2d(buf + k * BOX, tmW, rb, (cc * 2 + (cc == rp[i].c_lo ? rp[i].slot_lo : 0)) * BN, redb);
-}
-
-// Sums the boxes issued by red_issue in k order, applies the epilogue and advances the
-// tile counters (see reduce_slice).
-template <int BN>
-DEC_DEVINL void red_finish(const GemmArgs& a, const Work& w, const RedPlan* rp, int n, const uint8_t* buf) {
-    constexpr int BOX = 32 * BN * 4;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int k = 0;
-    for (int i = 0; i < n; ++i) {
-        const RedPlan& r = rp[i];
-        const int m0 = r.tile / w.tiles_n * BM, n0 = r.tile % w.tiles_n * BN;
-        for (int rb = r.r0; rb < r.r1; rb += 32) {
-            float acc[kChunks<BN>][16];
-#pragma unroll
-            for (int h = 0; h < kChunks<BN>; ++h)
-#pragma unroll
-                for (int q = 0; q < 16; ++q) acc[h][q] = 0.f;
-            for (int cc = r.c_lo; cc <= r.c_hi; ++cc, ++k) {
-                const float* bx = reinterpret_cast<const float*>(buf + k * BOX);
-#pragma unroll
-                for (int h = 0; h < kChunks<BN>; ++h) {
-                    const int ch = warp + 4 * h;
-                    if (ch * 16 < BN) {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) acc[h][q] += bx[(ch * 16 + q) * 32 + lane];
-                    }
-                }
-            }
-            const int rl = rb + lane;
-            const int row = rl < r.r1 ? m0 + rl : 0x3fffffff;
-#pragma unroll
-            for (int h = 0; h < kChunks<BN>; ++h) {
-                const int ch = warp + 4 * h;
-                if (ch * 16 < BN) {
-                    epilogue16(a, row, n0 + ch * 16, acc[h]);
-                    if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + ch * 16, acc[h]);
-                }
-            }
-        }
-    }
-    epi_bar();
-    if (threadIdx.x == 0)
-        for (int i = 0; i < n; ++i) {
-            const int P = rp[i].c_hi - rp[i].c_lo + 1;
-            if (atomicAdd(&a.cnt[rp[i].tile], 1) == 2 * P - 1) atomicExch(&a.cnt[rp[i].tile], 0);
-        }
-}
-
-DEC_DEVINL int tile_pieces(const Work& w, int tile) {
-    const long long t0 = (long long)tile * w.nkb;
-    return cta_of(w, t0 + w.nkb - 1) - cta_of(w, t0) + 1;
-}
-
-// Waits until every pending shared tile has all its pieces, then (when their boxes fit
-// the ring) issues the fetch of all of them in one batch. `issued` = boxes in flight, or
-// 0 when they do not fit (reduce_slice then fetches tile by tile).
-template <int BN>
-DEC_DEVINL bool begin_reductions(const GemmArgs& a, const Work& w, int c, const int* pend, int npend,
-                                 RedPlan* plans, const CUtensorMap* tmW, uint8_t* buf, int cap, uint64_t* redb,
-                                 volatile int* flag_s, int& issued) {
-    int total = 0;
-    for (int i = 0; i < npend; ++i) {
-        if (!tile_ready(a, pend[i], tile_pieces(w, pend[i]), flag_s)) return false;
-        plans[i] = red_plan(w, c, pend[i]);
-        total += red_boxes(plans[i]);
-    }
-    issued = total <= cap ? total : 0;
-    if (issued > 0) red_issue<BN>(plans, npend, total, tmW, buf, redb);
-    return true;
-}
-
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmW, GemmArgs a) {
+                   GemmArgs a) {
     using C = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -486,15 +312,13 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* empty = full + C::STAGES;
     uint64_t* accf = empty + C::STAGES;  // [2] accumulator buffer ready for the epilogue
     uint64_t* acce = accf + 2;           // [2] accumulator buffer drained by the epilogue
-    uint64_t* redb = acce + 2;           // reduction boxes landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redb + 1);
-    int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);  // reduction wait timed out
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+    int* flag_s = reinterpret_cast<int*>(tmem_slot + 1);  // a wait for a tile's pieces timed out
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 4 && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        prefetch_tmap(&tmW);
     }
     const Work w = make_work(a, BN);
     const int c = blockIdx.x;
@@ -509,7 +333,6 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 128);
         }
-        mbar_init(redb, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -597,10 +420,6 @@ __global__ void __launch_bounds__(192, 1)
         pdl_wait();
         const int rloc = warp * 32 + lane;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        int pend_tile[2], npend = 0;
-        RedPlan plans[2];
-        int issued = -1;  // reduction boxes fetched in one batch (0: too many, per-tile batches)
-        const int cap = (C::STAGES * C::STAGE) / (32 * BN * 4);
         bool ok = true;
         for (int j = 0; j < rg.nseg && ok; ++j) {
             const Seg sg = segment(w, rg, j);
@@ -609,26 +428,47 @@ __global__ void __launch_bounds__(192, 1)
             tc_fence_after();
             const uint32_t acc = tmem + lane_off + (uint32_t)(buf * BN);
             const bool whole = sg.kb0 == 0 && sg.kb1 == w.nkb;
-            if (whole && j == rg.nseg - 1 && npend > 0) {
-                // every piece of this CTA is published and the operand ring is drained
-                // (the last MMA has completed): start fetching the shared tiles' pieces now,
-                // so the fetch overlaps this tile's epilogue
-                ok = begin_reductions<BN>(a, w, c, pend_tile, npend, plans, &tmW, smem, cap, redb, flag_s, issued);
-            }
-            if (whole) {
+            // A shared tile is finished by the CTA holding its last k blocks. The other pieces
+            // are the first segment their CTAs process (segment() order), so they are
+            // published early and nobody waits for the finisher.
+            const bool fin = !whole && sg.kb1 == w.nkb;
+            if (whole || fin) {
+                int c_lo = c, slot_lo = 0;
+                if (fin) {
+                    c_lo = cta_of(w, (long long)sg.tile * w.nkb);
+                    slot_lo = piece_slot(w, c_lo, sg.tile);
+                    if (!tile_ready(a, sg.tile, c - c_lo, flag_s)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 const int row = sg.tile / w.tiles_n * BM + rloc, n0 = sg.tile % w.tiles_n * BN;
                 for (int c0 = 0; c0 < BN; c0 += 32) {
                     uint32_t r[32];
                     tmem_ld16_issue(acc + (uint32_t)c0, r);
                     tmem_ld16_issue(acc + (uint32_t)c0 + 16, r + 16);
+                    // the published pieces ([column][row] fp32) in k order, then this CTA's
+                    float v[2][16];
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] = 0.f;
+                    for (int cc = c_lo; cc < c; ++cc) {
+                        const float* pc =
+                            a.ws + ((size_t)cc * 2 + (cc == c_lo ? slot_lo : 0)) * (BM * BN) + (size_t)c0 * BM + rloc;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] += __ldcg(pc + (size_t)q * BM);
+                    }
                     tmem_ld_wait32(r);
+                    if (fin) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {  // the two 16-column halves of r
-                        float v[16];
+                        for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] += __uint_as_float(r[q]);
+                    } else {
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[16 * h + q]);
-                        epilogue16(a, row, n0 + c0 + 16 * h, v);
-                        if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0 + 16 * h, v);
+                        for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] = __uint_as_float(r[q]);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {  // the two 16-column halves
+                        epilogue16(a, row, n0 + c0 + 16 * h, v[h]);
+                        if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0 + 16 * h, v[h]);
                     }
                 }
             } else {
@@ -642,28 +482,19 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int q = 0; q < 32; ++q) __stcg(mine + (size_t)(c0 + q) * BM + rloc, __uint_as_float(r[q]));
                 }
-                asm volatile("fence.proxy.async.global;" ::: "memory");  // read back by TMA
                 __threadfence();
-                pend_tile[npend++] = sg.tile;
             }
             tc_fence_before();
             mbar_arrive(&acce[buf]);
             if (!whole) {
                 epi_bar();
-                if (threadIdx.x == 0) atomicAdd(&a.cnt[sg.tile], 1);
+                if (threadIdx.x == 0) {
+                    if (fin)
+                        atomicExch(&a.cnt[sg.tile], 0);  // every piece is read: ready for the next launch
+                    else
+                        atomicAdd(&a.cnt[sg.tile], 1);
+                }
             }
-        }
-        // the shared tiles are finished once this CTA's own work is done: its pieces were
-        // published first, so no CTA ever waits on another CTA's wait, and the operand
-        // ring is free to receive the pieces
-        if (ok && npend > 0 && issued < 0)
-            ok = begin_reductions<BN>(a, w, c, pend_tile, npend, plans, &tmW, smem, cap, redb, flag_s, issued);
-        if (ok && issued > 0) {
-            if (mbar_wait_bounded(redb, 0, a.err)) red_finish<BN>(a, w, plans, npend, smem);
-        } else if (ok && issued == 0) {
-            uint32_t red_phase = 0;
-            for (int i = 0; i < npend && ok; ++i)
-                ok = reduce_slice<BN>(a, w, c, pend_tile[i], &tmW, smem, cap, redb, red_phase);
         }
     }
     tc_fence_before();
@@ -930,21 +761,6 @@ cudaError_t encode_2d(CUtensorMap* tm, const uint16_t* base, int rows, int K, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// The stream-K pieces: fp32 [slot * bn + column][BM rows], read back in boxes of 32 rows
-// x bn columns.
-cudaError_t encode_ws(CUtensorMap* tm, const float* ws, int slots, int bn) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return cudaErrorNotSupported;
-    cuuint64_t dims[2] = {(cuuint64_t)BM, (cuuint64_t)slots * bn};
-    cuuint64_t strides[1] = {(cuuint64_t)BM * 4};
-    cuuint32_t box[2] = {32, (cuuint32_t)bn};
-    cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ws), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 template <int BN>
 cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, bool pdl) {
     using C = Cfg<BN>;
@@ -960,7 +776,7 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, p.tmW, a);
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, p.tmA, p.tmB, a);
 }
 
 template <int BN, int EPI>
@@ -1119,9 +935,7 @@ cudaError_t gemm_plan(GemmPlan* p, const uint16_t* A, int M, int K, const uint16
     p->ws = ws;
     cudaError_t e = encode_2d(&p->tmA, A, M, K, BM);
     if (e != cudaSuccess) return e;
-    e = encode_2d(&p->tmB, B, N, K, p->bn);
-    if (e != cudaSuccess) return e;
-    return encode_ws(&p->tmW, ws, 2 * p->nc, p->bn);
+    return encode_2d(&p->tmB, B, N, K, p->bn);
 }
 
 namespace {

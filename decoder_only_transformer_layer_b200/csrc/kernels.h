@@ -47,7 +47,6 @@ enum GemmEpi { GEMM_STORE = 0, GEMM_RESID = 1, GEMM_SWIGLU = 2 };
 struct GemmPlan {
     CUtensorMap tmA;  // weights [M][K], box 64 x 128
     CUtensorMap tmB;  // activations [N][K], box 64 x BN
-    CUtensorMap tmW;  // stream-K pieces (fp32 workspace), box 32 rows x BN
     const float* ws;
     int M, N, K, bn, nc;  // nc: persistent CTAs (stream-K ranges)
     int splitk;           // >= 2: cluster split-K with this many CTAs per tile (N <= 128, few tiles)
