@@ -22,11 +22,12 @@
 // Keys past a row's position (or before its window) are masked per element; blocks before
 // every row's window are skipped.
 // With S > 1 key splits (short chunks would otherwise fill few SMs) the S CTAs of a row
-// block form a cluster, each taking a contiguous run of key blocks. Each stages its rows'
-// unnormalised O with their m and l in its own drained ring; after one cluster barrier the
-// DMA engine copies every owner's rows (128 / S of them) into the owner's receive slots
-// (cp.async.bulk shared::cta -> shared::cluster, completing on the owner's mbarrier), and
-// the owner merges the S partials in split order (deterministic).
+// block form a cluster, each taking a contiguous run of key blocks. After one cluster
+// barrier (every ring drained) each sends its rows' unnormalised O with their m and l
+// straight from TMEM-loaded registers to the owner of the rows (128 / S of them), with
+// st.async completing on the owner's mbarrier, and the owner merges the S partials in
+// split order (deterministic). No CTA reads another's shared memory, so there is no
+// second barrier before leaving.
 //
 // Operand layouts in shared memory (all 128-byte swizzled, 1024-byte aligned):
 //   Q  [2 d-halves][128 rows][64 d]   A of S, K-major      (TMA 3-D box {64, G, 128/G})
@@ -56,11 +57,10 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = 32768;
 constexpr uint32_t kOffV = kOffK + kTcStages * kStage;
 constexpr uint32_t kOffBar = kOffV + kTcStages * kStage;
-// after the last block: [stage: 128 rows][LDR] this CTA's partial, then [recv: S][128 / S][LDR]
+// after the last block: [recv: S][128 / S][LDR] every split's partial of this CTA's rows
 constexpr int kLdr = 132;  // O[128], m, l, 2 pad: 16-byte rows, conflict-free
-constexpr uint32_t kOffStage = kOffK;
-constexpr uint32_t kOffRecv = kOffK + kTcRows * kLdr * 4;
-static_assert(kOffRecv + kTcRows * kLdr * 4 <= kOffBar, "the merge areas fit in the drained rings");
+constexpr uint32_t kOffRecv = kOffK;
+static_assert(kOffRecv + kTcRows * kLdr * 4 <= kOffBar, "the merge area fits in the drained rings");
 constexpr uint32_t kOffXch = kOffBar + 256;  // softmax warp pairs' row maxima and sums
 constexpr uint32_t kTcSmem = kOffXch + 2 * kTcRows * 4 + 1024;  // + alignment slack
 static_assert(kTcSmem <= 232448, "fits the 227 KB a CTA may use");
@@ -480,8 +480,23 @@ __global__ void __launch_bounds__(352, 1)
                 }
             }
         } else {
-            // this split's partial row (unnormalised O, m, l) into the drained ring
-            float* st = reinterpret_cast<float*>(smem + kOffStage) + (size_t)r * kLdr;
+            // every split of the cluster is past its MMAs: every ring is drained, free to
+            // receive (the producer and MMA warps arrive below)
+            cluster_sync();
+            // this split's partial of row r (unnormalised O, m, l) into slot [z] of the row's
+            // owner: kept here for own rows, st.async from registers (transaction bytes on the
+            // owner's recvb) for the others, so no copy reads this CTA's shared memory
+            const int own = r / RS, lr = r - own * RS;
+            float* slot = reinterpret_cast<float*>(smem + kOffRecv) + ((size_t)z * RS + lr) * kLdr;
+            const uint32_t rdst = own == z ? 0u : dsmem_map(smem_u32(slot), own);
+            const uint32_t rbar = own == z ? 0u : dsmem_map(smem_u32(recvb), own);
+            auto put4 = [&](int c, uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+                if (own == z)
+                    *reinterpret_cast<uint4*>(slot + c) = make_uint4(x0, x1, x2, x3);
+                else
+                    st_async_4f(rdst + (uint32_t)c * 4, __uint_as_float(x0), __uint_as_float(x1), __uint_as_float(x2),
+                                __uint_as_float(x3), rbar);
+            };
             for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                 uint32_t v[32];
                 if (nb > 0) {
@@ -493,36 +508,23 @@ __global__ void __launch_bounds__(352, 1)
                     for (int q = 0; q < 32; ++q) v[q] = 0u;  // no key blocks: O = 0, m = -inf, l = 0
                 }
 #pragma unroll
-                for (int q = 0; q < 32; q += 4)
-                    *reinterpret_cast<uint4*>(st + c0 + q) = make_uint4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                for (int q = 0; q < 32; q += 4) put4(c0 + q, v[q], v[q + 1], v[q + 2], v[q + 3]);
             }
-            if (half == 0) *reinterpret_cast<float4*>(st + 128) = make_float4(m, l, 0.f, 0.f);
-            fence_proxy_async_smem();  // the copies read these writes through the async proxy
+            if (half == 0) put4(128, __float_as_uint(m), __float_as_uint(l), 0u, 0u);
+            named_bar_sync(5, 256);  // every own row is in place before the merge reads it
         }
     }
     if (S > 1) {
-        // every split of the cluster is past its MMAs (its ring is free to receive) and has
-        // staged its partial
-        cluster_sync();
-        if (threadIdx.x == 0) {
-            for (int o = 0; o < S; ++o) {
-                if (o == z) continue;
-                const uint32_t dst = dsmem_map(smem_u32(smem + kOffRecv) + (uint32_t)z * RS * kLdr * 4, o);
-                bulk_s2cluster(dst, smem + kOffStage + (size_t)o * RS * kLdr * 4, (uint32_t)RS * kLdr * 4,
-                               dsmem_map(smem_u32(recvb), o));
-            }
-        }
+        if (warp >= 8) cluster_sync();  // the producer and MMA warps' arrivals
         if (warp < 4) {
             // rows [z RS, z RS + RS): 128 / RS threads a row, 128 / (128 / RS) columns each
             const int tpr = kTcRows / RS;
             const int lr = threadIdx.x / tpr, part = threadIdx.x % tpr, cols = 128 / tpr;
             const int rr = z * RS + lr;  // the row in the CTA's 128
-            const bool got = mbar_wait_bounded(recvb, 0, a.err);
+            const bool got = mbar_wait_cluster_bounded(recvb, 0, a.err);
             const int tt = t0 + rr / G;
-            const float* mine = reinterpret_cast<const float*>(smem + kOffStage) + (size_t)rr * kLdr;
             auto part_row = [&](int zz) {
-                return zz == z ? mine
-                               : reinterpret_cast<const float*>(smem + kOffRecv) + ((size_t)zz * RS + lr) * kLdr;
+                return reinterpret_cast<const float*>(smem + kOffRecv) + ((size_t)zz * RS + lr) * kLdr;
             };
             float M = -INFINITY;
             for (int zz = 0; zz < S; ++zz) M = fmaxf(M, part_row(zz)[128]);
@@ -563,8 +565,8 @@ __global__ void __launch_bounds__(352, 1)
                 }
             }
         }
-        // the copies out of this CTA's shared memory have landed at their owners
-        cluster_sync();
+        // nothing reads another CTA's shared memory, and this CTA's incoming bytes completed
+        // before its merge: no cluster barrier before leaving
     }
     tc_fence_before();
     __syncthreads();

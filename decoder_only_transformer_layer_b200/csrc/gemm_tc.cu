@@ -511,17 +511,19 @@ __global__ void __launch_bounds__(192, 1)
 // Products with one column tile (N <= 128: prefill chunks, decode batches) and few 128-row
 // tiles (the QKV, o_proj and down projections) split each tile's k blocks over the S <= 8
 // CTAs of one thread-block cluster. Every CTA streams 1/S of the tile's weights into its
-// own TMEM accumulator. The partial tiles are then summed inside the cluster: each CTA
-// writes its partial into its own shared memory, and once every CTA of the cluster is past
-// its MMAs (one cluster barrier) the DMA engine copies each 32-row-aligned slice to the CTA
-// that owns it (cp.async.bulk shared::cta -> shared::cluster, completing on the owner's
-// mbarrier). The owner sums the S partials of its rows in rank order (deterministic) and
-// applies the epilogue. There is no global round trip and no wait on CTAs outside the
-// cluster; a last cluster barrier keeps every CTA (the copies' sources) alive until the
-// owners have their bytes.
+// own TMEM accumulator. The partial tiles are then summed inside the cluster: once every CTA
+// of the cluster is past its MMAs (one cluster barrier: every operand ring is drained), each
+// CTA reads its accumulator rows and sends every 32-row-aligned slice to the CTA that owns
+// it, straight from registers (st.async, completing as transaction bytes on the owner's
+// mbarrier; its own slice it keeps). The owner sums the S partials of its rows in rank
+// order (deterministic) and applies the epilogue. There is no global round trip, no wait
+// on CTAs outside the cluster, and no second cluster barrier: no CTA reads another's
+// shared memory. (Staging every partial and copying slices with the DMA engine, which
+// reads the sender's shared memory and so needs a last barrier before anyone leaves, took
+// 0.2-0.4 us longer a launch.)
 //
 // Shared memory after the main loop (it overlays the drained operand ring):
-// [recv: S slots x rows per owner x LDR floats][stage: BM x LDR floats], LDR = BN + 4.
+// [recv: S slots x rows per owner x LDR floats], LDR = BN + 4.
 
 constexpr int kMaxSplitK = 8;
 
@@ -533,12 +535,13 @@ __host__ __device__ constexpr size_t splitk_recv_bytes(int S) {
     return (size_t)S * splitk_rows(S) * (BN + 4) * 4;
 }
 
-// The largest receive area over every S <= kMaxSplitK, then this CTA's own partial.
+// The largest receive area over every S <= kMaxSplitK (every split's partial of the rows a
+// CTA finishes, its own included).
 template <int BN>
 __host__ __device__ constexpr size_t splitk_exchange_bytes() {
     size_t m = 0;
     for (int S = 2; S <= kMaxSplitK; ++S) m = splitk_recv_bytes<BN>(S) > m ? splitk_recv_bytes<BN>(S) : m;
-    return m + (size_t)BM * (BN + 4) * 4;
+    return m;
 }
 
 template <int BN>
@@ -567,7 +570,6 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* recvb = accf + 1;          // the other CTAs' slices of this CTA's rows have landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recvb + 1);
     float* recv = reinterpret_cast<float*>(smem);  // [S][rows per owner][LDR], over the drained ring
-    float* stage = recv + splitk_recv_bytes<BN>(S) / 4;  // [BM][LDR]: this CTA's partial
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)cluster_rank();
@@ -583,7 +585,6 @@ __global__ void __launch_bounds__(192, 1)
 
     const int RS = splitk_rows(S);
     const int my0 = rank * RS, my1 = min(BM, my0 + RS);  // the rows this CTA finishes
-    const uint32_t slice_bytes = (uint32_t)RS * LDR * 4;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -591,9 +592,9 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(accf, 1);
         mbar_init(recvb, 1);
-        // the S - 1 other CTAs each send (my1 - my0) rows; armed before the first cluster
-        // barrier, so no byte can arrive before the count
-        if (my1 > my0) mbar_arrive_expect_tx(recvb, (uint32_t)(S - 1) * (my1 - my0) * LDR * 4);
+        // the S - 1 other CTAs each send (my1 - my0) rows of BN floats; armed before the
+        // cluster barrier, so no byte can arrive before the count
+        if (my1 > my0) mbar_arrive_expect_tx(recvb, (uint32_t)(S - 1) * (my1 - my0) * BN * 4);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -656,11 +657,18 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait_bounded(accf, 0, a.err);  // on a time-out the partial is garbage, the flag is set
         tc_fence_after();
     }
+    // every CTA of the cluster is past its MMAs: every ring is drained, free to receive
+    cluster_sync();
     if (warp < 4) {
-        // this CTA's partial into its own (drained) ring: lane = TMEM lane = row
-        const int row = warp * 32 + lane;
+        // my partial of each row into slot [rank] of the row's owner: kept here for my own
+        // rows, st.async from registers (transaction bytes on the owner's recvb) for the
+        // others, so no copy reads this CTA's shared memory once it moves on
+        const int row = warp * 32 + lane;  // = TMEM lane
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        float* dst = stage + (size_t)row * LDR;
+        const int o = row / RS, lr = row - o * RS;  // owner and row within its slice
+        float* slot = recv + ((size_t)rank * RS + lr) * LDR;
+        const uint32_t rdst = o == rank ? 0u : dsmem_map(smem_u32(slot), o);
+        const uint32_t rbar = o == rank ? 0u : dsmem_map(smem_u32(recvb), o);
         for (int c0 = 0; c0 < BN; c0 += 32) {
             uint32_t r[32];
             if (iters > 0) {
@@ -671,30 +679,24 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                 for (int q = 0; q < 32; ++q) r[q] = 0u;
             }
+            if (o == rank) {
 #pragma unroll
-            for (int q = 0; q < 32; q += 4)
-                *reinterpret_cast<uint4*>(dst + c0 + q) = make_uint4(r[q], r[q + 1], r[q + 2], r[q + 3]);
+                for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<uint4*>(slot + c0 + q) = make_uint4(r[q], r[q + 1], r[q + 2], r[q + 3]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 32; q += 4)
+                    st_async_4f(rdst + (uint32_t)(c0 + q) * 4, __uint_as_float(r[q]), __uint_as_float(r[q + 1]),
+                                __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]), rbar);
+            }
         }
-        fence_proxy_async_smem();  // the copies below read these writes through the async proxy
-    }
-    // every CTA of the cluster has its accumulator (its ring is free to receive) and its
-    // partial staged
-    cluster_sync();
-
-    if (threadIdx.x == 0) {
-        // one DMA copy per other owner: my partial of its rows into its slot [rank]
-        for (int o = 0; o < S; ++o) {
-            const int o0 = o * RS, o1 = min(BM, o0 + RS);
-            if (o == rank || o1 <= o0) continue;
-            const uint32_t dst = dsmem_map(smem_u32(recv) + (uint32_t)rank * slice_bytes, o);
-            bulk_s2cluster(dst, stage + (size_t)o0 * LDR, (uint32_t)(o1 - o0) * LDR * 4, dsmem_map(smem_u32(recvb), o));
-        }
+        epi_bar();  // my own slot is written
     }
 
     if (warp < 4 && my1 > my0) {
         // the owner sums its rows' partials in rank order and applies the epilogue:
         // units of (32 rows, 16 columns), lane = row
-        const bool got = mbar_wait_bounded(recvb, 0, a.err);
+        const bool got = mbar_wait_cluster_bounded(recvb, 0, a.err);
         const int groups = (my1 - my0) / 32;
         for (int u = warp; got && u < groups * (BN / 16); u += 4) {
             const int gi = u / (BN / 16), c0 = (u % (BN / 16)) * 16;
@@ -703,8 +705,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int q = 0; q < 16; ++q) acc[q] = 0.f;
             for (int z = 0; z < S; ++z) {
-                const float* zrow = z == rank ? stage + (size_t)(my0 + lr) * LDR : recv + ((size_t)z * RS + lr) * LDR;
-                const float4* src = reinterpret_cast<const float4*>(zrow + c0);
+                const float4* src = reinterpret_cast<const float4*>(recv + ((size_t)z * RS + lr) * LDR + c0);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float4 v = src[q];
@@ -721,9 +722,8 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     }
-    // the copies out of this CTA's shared memory have landed at their owners (each owner
-    // arrives here only after its barrier completed): only now may any CTA exit
-    cluster_sync();
+    // nothing reads another CTA's shared memory, and every CTA's incoming bytes completed
+    // before it got here: no cluster barrier before leaving
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
