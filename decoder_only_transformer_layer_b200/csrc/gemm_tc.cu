@@ -23,8 +23,9 @@
 //    K=16 per instruction, fp32 accumulator in TMEM) and frees each stage with
 //    tcgen05.commit; the accumulator is double-buffered in TMEM (2 x BN columns),
 //    so one tile's epilogue overlaps the next tile's main loop;
-//  * warps 0-3 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
-//    32w..32w+31 = weight rows) and apply the epilogue: store (+bias, + greedy
+//  * warps 0-3 and 6-9 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
+//    32 (w % 4).. = weight rows; warps 0-3 one half of the columns, 6-9 the other;
+//    the cluster split-K kernel has warps 0-3 only) and apply the epilogue: store (+bias, + greedy
 //    argmax; the destination may be read from device memory, and a null one stores
 //    nothing), residual add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
 #include <cuda.h>
@@ -271,6 +272,8 @@ struct SegIter {
 
 // Barrier of the four epilogue warps only.
 DEC_DEVINL void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier of the persistent kernel's eight epilogue warps only.
+DEC_DEVINL void epi_bar8() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 DEC_DEVINL int ld_acquire_gpu(const int* p) {
     int v;
@@ -295,14 +298,14 @@ DEC_DEVINL bool tile_ready(const GemmArgs& a, int tile, int P, volatile int* fla
         }
         *flag_s = r;
     }
-    epi_bar();
+    epi_bar8();
     const int r = *flag_s;
-    epi_bar();
+    epi_bar8();
     return r != 0;
 }
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    GemmArgs a) {
     using C = Cfg<BN>;
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accf[b], 1);
-            mbar_init(&acce[b], 128);
+            mbar_init(&acce[b], 256);
         }
         fence_mbar_init();
     }
@@ -416,10 +419,15 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------- epilogue (warps 0-3: TMEM lanes 32w..)
+        // ------------------------------------------ epilogue (warps 0-3 and 6-9): warp w reads
+        // TMEM lanes 32 (w % 4) .. (rows), warps 0-3 the first half of the columns, 6-9 the
+        // second (one warp a scheduler left the last tile's SwiGLU epilogue latency-bound)
         pdl_wait();
-        const int rloc = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int q4 = warp & 3;
+        constexpr int HC = BN / 2;  // columns of each half
+        const int cb = warp >= 6 ? HC : 0;
+        const int rloc = q4 * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
         bool ok = true;
         for (int j = 0; j < rg.nseg && ok; ++j) {
             const Seg sg = segment(w, rg, j);
@@ -443,51 +451,46 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
                 const int row = sg.tile / w.tiles_n * BM + rloc, n0 = sg.tile % w.tiles_n * BN;
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t r[32];
+                for (int c0 = cb; c0 < cb + HC; c0 += 16) {
+                    uint32_t r[16];
                     tmem_ld16_issue(acc + (uint32_t)c0, r);
-                    tmem_ld16_issue(acc + (uint32_t)c0 + 16, r + 16);
                     // the published pieces ([column][row] fp32) in k order, then this CTA's
-                    float v[2][16];
+                    float v[16];
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] = 0.f;
+                    for (int q = 0; q < 16; ++q) v[q] = 0.f;
                     for (int cc = c_lo; cc < c; ++cc) {
                         const float* pc =
                             a.ws + ((size_t)cc * 2 + (cc == c_lo ? slot_lo : 0)) * (BM * BN) + (size_t)c0 * BM + rloc;
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] += __ldcg(pc + (size_t)q * BM);
+                        for (int q = 0; q < 16; ++q) v[q] += __ldcg(pc + (size_t)q * BM);
                     }
-                    tmem_ld_wait32(r);
+                    tmem_ld_wait16(r);
                     if (fin) {
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] += __uint_as_float(r[q]);
+                        for (int q = 0; q < 16; ++q) v[q] += __uint_as_float(r[q]);
                     } else {
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) v[q >> 4][q & 15] = __uint_as_float(r[q]);
+                        for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[q]);
                     }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {  // the two 16-column halves
-                        epilogue16(a, row, n0 + c0 + 16 * h, v[h]);
-                        if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0 + 16 * h, v[h]);
-                    }
+                    epilogue16(a, row, n0 + c0, v);
+                    if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0, v);
                 }
             } else {
                 // publish this piece ([column][row] fp32, coalesced) and free the accumulator
                 float* mine = a.ws + ((size_t)c * 2 + sg.slot) * (BM * BN);
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t r[32];
+                for (int c0 = cb; c0 < cb + HC; c0 += 16) {
+                    uint32_t r[16];
                     tmem_ld16_issue(acc + (uint32_t)c0, r);
-                    tmem_ld16_issue(acc + (uint32_t)c0 + 16, r + 16);
-                    tmem_ld_wait32(r);
+                    tmem_ld_wait16(r);
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) __stcg(mine + (size_t)(c0 + q) * BM + rloc, __uint_as_float(r[q]));
+                    for (int q = 0; q < 16; ++q) __stcg(mine + (size_t)(c0 + q) * BM + rloc, __uint_as_float(r[q]));
                 }
                 __threadfence();
             }
             tc_fence_before();
             mbar_arrive(&acce[buf]);
             if (!whole) {
-                epi_bar();
+                epi_bar8();
                 if (threadIdx.x == 0) {
                     if (fin)
                         atomicExch(&a.cnt[sg.tile], 0);  // every piece is read: ready for the next launch
@@ -768,7 +771,7 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmArgs& a, cudaStream_t st, boo
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.nc);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(320);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
