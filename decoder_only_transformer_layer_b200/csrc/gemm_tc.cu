@@ -25,7 +25,7 @@
 //    so one tile's epilogue overlaps the next tile's main loop;
 //  * warps 0-3 and 6-9 read the accumulator with tcgen05.ld (warp w owns TMEM lanes
 //    32 (w % 4).. = weight rows; warps 0-3 one half of the columns, 6-9 the other;
-//    the cluster split-K kernel has warps 0-3 only) and apply the epilogue: store (+bias, + greedy
+//    the cluster split-K kernel likewise) and apply the epilogue: store (+bias, + greedy
 //    argmax; the destination may be read from device memory, and a null one stores
 //    nothing), residual add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
 #include <cuda.h>
@@ -40,10 +40,6 @@ namespace {
 
 constexpr int BM = 128, BK = 64;
 
-// 16-column chunks of a BN-wide tile that each of the 4 epilogue warps handles in the
-// reductions (warp w takes chunks w, w + 4, ...; BN < 128 leaves some warps idle).
-template <int BN>
-constexpr int kChunks = BN >= 128 ? BN / 64 : 2;
 
 template <int BN>
 struct Cfg {
@@ -270,9 +266,7 @@ struct SegIter {
     }
 };
 
-// Barrier of the four epilogue warps only.
-DEC_DEVINL void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Barrier of the persistent kernel's eight epilogue warps only.
+// Barrier of the eight epilogue warps only.
 DEC_DEVINL void epi_bar8() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 DEC_DEVINL int ld_acquire_gpu(const int* p) {
@@ -560,7 +554,7 @@ __host__ __device__ constexpr int splitk_smem() {
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_splitk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs a,
                        int S) {
     using C = Cfg<BN>;
@@ -662,46 +656,51 @@ __global__ void __launch_bounds__(192, 1)
     }
     // every CTA of the cluster is past its MMAs: every ring is drained, free to receive
     cluster_sync();
-    if (warp < 4) {
+    // epilogue warps 0-3 and 6-9: warp w reads TMEM lanes 32 (w % 4).. (rows), warps 0-3
+    // one half of the columns, 6-9 the other
+    const bool epi = warp < 4 || warp >= 6;
+    const int ew = warp < 4 ? warp : warp - 2;  // 0..7
+    if (epi) {
         // my partial of each row into slot [rank] of the row's owner: kept here for my own
         // rows, st.async from registers (transaction bytes on the owner's recvb) for the
         // others, so no copy reads this CTA's shared memory once it moves on
-        const int row = warp * 32 + lane;  // = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;  // = TMEM lane
+        const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        const int cb = warp >= 6 ? BN / 2 : 0;
         const int o = row / RS, lr = row - o * RS;  // owner and row within its slice
         float* slot = recv + ((size_t)rank * RS + lr) * LDR;
         const uint32_t rdst = o == rank ? 0u : dsmem_map(smem_u32(slot), o);
         const uint32_t rbar = o == rank ? 0u : dsmem_map(smem_u32(recvb), o);
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t r[32];
+        for (int c0 = cb; c0 < cb + BN / 2; c0 += 16) {
+            uint32_t r[16];
             if (iters > 0) {
                 tmem_ld16_issue(tmem + lane_off + (uint32_t)c0, r);
-                tmem_ld16_issue(tmem + lane_off + (uint32_t)c0 + 16, r + 16);
-                tmem_ld_wait32(r);
+                tmem_ld_wait16(r);
             } else {
 #pragma unroll
-                for (int q = 0; q < 32; ++q) r[q] = 0u;
+                for (int q = 0; q < 16; ++q) r[q] = 0u;
             }
             if (o == rank) {
 #pragma unroll
-                for (int q = 0; q < 32; q += 4)
+                for (int q = 0; q < 16; q += 4)
                     *reinterpret_cast<uint4*>(slot + c0 + q) = make_uint4(r[q], r[q + 1], r[q + 2], r[q + 3]);
             } else {
 #pragma unroll
-                for (int q = 0; q < 32; q += 4)
+                for (int q = 0; q < 16; q += 4)
                     st_async_4f(rdst + (uint32_t)(c0 + q) * 4, __uint_as_float(r[q]), __uint_as_float(r[q + 1]),
                                 __uint_as_float(r[q + 2]), __uint_as_float(r[q + 3]), rbar);
             }
         }
-        epi_bar();  // my own slot is written
+        epi_bar8();  // my own slot is written
     }
 
-    if (warp < 4 && my1 > my0) {
+    if (epi && my1 > my0) {
         // the owner sums its rows' partials in rank order and applies the epilogue:
         // units of (32 rows, 16 columns), lane = row
         const bool got = mbar_wait_cluster_bounded(recvb, 0, a.err);
         const int groups = (my1 - my0) / 32;
-        for (int u = warp; got && u < groups * (BN / 16); u += 4) {
+        for (int u = ew; got && u < groups * (BN / 16); u += 8) {
             const int gi = u / (BN / 16), c0 = (u % (BN / 16)) * 16;
             const int lr = gi * 32 + lane;
             float acc[16];
@@ -790,7 +789,7 @@ cudaError_t launch_splitk(const GemmPlan& p, const GemmArgs& a, cudaStream_t st,
     const int tiles = (p.M + BM - 1) / BM;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles * p.splitk);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(320);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -866,7 +865,7 @@ int splitk_resident(int S) {
         cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(S * 8);
-        cfg.blockDim = dim3(192);
+        cfg.blockDim = dim3(320);
         cfg.dynamicSmemBytes = splitk_smem<BN>();
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
