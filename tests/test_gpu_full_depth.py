@@ -9,10 +9,12 @@ shape, 32 layers). fp32 accumulation lands a fraction of the bf16 roundings of e
 one ulp away from the fp64 oracle's, so no fp32 implementation can stay closer than that
 floor. Each test therefore also runs the oracle with every embedding value moved by one bf16
 ulp, a change of the same order as that rounding noise. Logits must pass the fixed bar or
-stay within twice the measured floor. Greedy tokens must match exactly wherever the
-perturbed oracle made the same decision (a decision that noise of this size moves is not
-determined by the arithmetic); MoE routing must match where, in addition, the decision's
-margin is at least twice the perturbation's movement of the router logits.
+stay within twice the measured floor. The greedy token follows from the logits: it must be
+the argmax of the GPU's own logits (exactly), and it must be the oracle's token wherever
+the oracle's top-2 gap exceeds twice the logit bar; below that gap the decision is not
+determined by the arithmetic, and the token's oracle logit must lie within twice the bar
+of the top. MoE routing must match where the perturbed oracle made the same decision and
+the decision's margin is at least twice the perturbation's movement of the router logits.
 
 These take minutes of host work (the oracle is fp64 on the CPU and reads every weight for
 every token), so they are marked slow as well as gpu."""
@@ -23,7 +25,7 @@ import oracle
 import synth
 from synth import configs
 import decoder_only_transformer_layer_b200 as dec
-from _util import assert_parity, assert_within_conditioning, perturb_inputs
+from _util import ABS_TOL, assert_parity, assert_within_conditioning, perturb_inputs
 from test_gpu_model import gated_run
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -33,6 +35,22 @@ MARGIN = 1e-3
 def top_gap(v):
     s = np.sort(np.asarray(v, np.float64))
     return s[-1] - s[-2]
+
+
+def check_greedy(tok, got, ref, pert, what):
+    """The greedy token `tok` against the logits it came from (`got`, the GPU's) and the
+    oracle's (`ref`, and `pert` for the one-ulp-perturbed input); see the module docstring."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    bar = max(ABS_TOL, 2.0 * float(np.max(np.abs(ref - np.asarray(pert, np.float64)))))
+    err = float(np.max(np.abs(got - ref)))
+    assert got[tok] == got.max(), f"{what}: greedy {tok} is not the argmax of its own logits"
+    top, gap = oracle.argmax(ref), top_gap(ref)
+    if gap > 2.0 * bar:
+        assert tok == top, f"{what}: greedy {tok} vs {top} (gap {gap:.2e}, bar {bar:.2e}, err {err:.2e})"
+    else:
+        assert ref[tok] >= ref[top] - 2.0 * bar, (
+            f"{what}: greedy {tok} is {ref[top] - ref[tok]:.2e} below the oracle's top {top} (bar {bar:.2e})")
 
 
 def _perturbed_run(cfg, w, toks, greedy):
@@ -54,8 +72,7 @@ def _dense_full(cfg, n_prompt, n_steps, seed):
         got = d.prefill_logits(0, toks, 0) if s == 0 else d.step_logits([greedy[s - 1]], [n_prompt + s - 1])[0]
         what = f"{cfg['name']} " + ("prefill" if s == 0 else f"step {s - 1}")
         assert_within_conditioning(got, ref[s], pert[s], what=what)
-        if oracle.argmax(pert[s]) == oracle.argmax(ref[s]):
-            assert d.last_argmax(1)[0] == oracle.argmax(ref[s]), what
+        check_greedy(int(d.last_argmax(1)[0]), got, ref[s], pert[s], what)
     return d, m, ref, pert
 
 
@@ -91,8 +108,7 @@ def test_llama8b_shape_prefill_one_4096_token_chunk():
     d = dec.Decoder(cfg, w)
     got = d.prefill_logits(0, toks, 0)
     assert_within_conditioning(got, ref, pert, what="llama3-8b 4096-token chunk")
-    if oracle.argmax(pert) == oracle.argmax(ref):
-        assert d.last_argmax(1)[0] == oracle.argmax(ref)
+    check_greedy(int(d.last_argmax(1)[0]), got, ref, pert, "llama3-8b 4096-token chunk")
     # all 4096 cache rows of both layers; rows reach |v| ~ 8, where one bf16 ulp is 0.03 and the
     # second layer's rows carry the first layer's drift: a few ulps at the largest values
     for li in range(cfg["layers"]):
@@ -174,8 +190,7 @@ def test_qwen_moe_shape_full_depth_batch1_decode4(qwen_weights):
         got = d.step_logits([toks[s]], [ctx + s])[0]
         assert_within_conditioning(got, lgs[s], pl[s], what=f"qwen-moe full depth B=1 step {s}")
         n_checked += _check_routes(d.last_routes(1)[:, 0, :], rts[s], pr[s], f"step {s}")
-        if oracle.argmax(pl[s]) == oracle.argmax(lgs[s]):
-            assert d.last_argmax(1)[0] == oracle.argmax(lgs[s])
+        check_greedy(int(d.last_argmax(1)[0]), got, lgs[s], pl[s], f"qwen-moe full depth B=1 step {s}")
     print(f"routing checked at {n_checked} of {4 * cfg['layers']} (step, layer) decisions")
     d.close()
 
@@ -234,6 +249,5 @@ def test_qwen_moe_shape_full_depth_batch64_decode2_sampled(qwen_weights):
             lg, rt, pl, pr = ref[b][s]
             assert_within_conditioning(got[b], lg, pl, what=f"qwen-moe B=64 step {s} seq {b}")
             _check_routes(routes[:, b, :], rt, pr, f"B=64 step {s} seq {b}")
-            if oracle.argmax(pl) == oracle.argmax(lg):
-                assert am[b] == oracle.argmax(lg)
+            check_greedy(int(am[b]), got[b], lg, pl, f"qwen-moe B=64 step {s} seq {b}")
     d.close()
