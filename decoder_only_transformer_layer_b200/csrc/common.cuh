@@ -46,7 +46,6 @@ DEC_DEVINL void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 DEC_DEVINL void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-DEC_DEVINL void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 DEC_DEVINL void mbar_arrive(uint64_t* bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
@@ -197,14 +196,6 @@ DEC_DEVINL uint32_t dsmem_map(uint32_t saddr, int rank) {
     return remote;
 }
 
-// 16-byte store into the shared memory of CTA `rank` of this cluster, at the same offset as
-// the local shared address `saddr` (fire-and-forget; ordered by the next cluster barrier).
-DEC_DEVINL void dsmem_st4(uint32_t saddr, int rank, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    const uint32_t remote = dsmem_map(saddr, rank);
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-
 // Stores of two (four) floats to a cluster shared-memory address (dsmem_map) that complete
 // as 8 (16) transaction bytes on the destination CTA's mbarrier `bar` (also a cluster
 // address). The data comes from registers, so the sending CTA may exit right after.
@@ -221,27 +212,13 @@ DEC_DEVINL void st_async_4f(uint32_t dst, float a, float b, float c, float d, ui
                  : "memory");
 }
 
-// 8-byte store of two floats into CTA `rank`'s shared memory (see dsmem_st4).
+// 8-byte store of two floats into the shared memory of CTA `rank` of this cluster, at the
+// same offset as the local shared address `saddr` (fire-and-forget; ordered by the next
+// cluster barrier).
 DEC_DEVINL void dsmem_st2f(uint32_t saddr, int rank, float a, float b) {
     const uint32_t remote = dsmem_map(saddr, rank);
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(remote), "f"(a), "f"(b) : "memory");
 }
-
-// Bulk copy (DMA engine) of `bytes` from this CTA's shared memory to shared memory of
-// another CTA of the cluster: `dst` and `bar` are cluster addresses (dsmem_map), the bytes
-// complete as transactions on the destination's mbarrier. 16-byte aligned, size a multiple
-// of 16. The source must stay untouched (and its CTA alive) until the destination has
-// seen the bytes arrive.
-DEC_DEVINL void bulk_s2cluster(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     dst),
-                 "r"(smem_u32(src)), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-// Make this thread's generic-proxy shared-memory writes visible to the async proxy (bulk
-// copies, TMA stores) issued after the next barrier.
-DEC_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Packed fp32x2 arithmetic (sm_100): d = a * b + c and d = a + b on both halves.
 DEC_DEVINL float2 ffma2(float2 a, float2 b, float2 c) {
