@@ -422,8 +422,11 @@ __global__ void __launch_bounds__(320, 1)
         const int cb = warp >= 6 ? HC : 0;
         const int rloc = q4 * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+        // ok turns false when a wait for a shared tile's pieces runs out: the remaining
+        // accumulators are still drained (every MMA completes and every TMA load is consumed
+        // before TMEM is freed), only their outputs are skipped
         bool ok = true;
-        for (int j = 0; j < rg.nseg && ok; ++j) {
+        for (int j = 0; j < rg.nseg; ++j) {
             const Seg sg = segment(w, rg, j);
             const int buf = j & 1;
             if (!mbar_wait_bounded(&accf[buf], (uint32_t)((j >> 1) & 1), a.err)) break;
@@ -434,15 +437,12 @@ __global__ void __launch_bounds__(320, 1)
             // are the first segment their CTAs process (segment() order), so they are
             // published early and nobody waits for the finisher.
             const bool fin = !whole && sg.kb1 == w.nkb;
-            if (whole || fin) {
+            if (fin && ok) ok = tile_ready(a, sg.tile, c - cta_of(w, (long long)sg.tile * w.nkb), flag_s);
+            if ((whole || fin) && ok) {
                 int c_lo = c, slot_lo = 0;
                 if (fin) {
                     c_lo = cta_of(w, (long long)sg.tile * w.nkb);
                     slot_lo = piece_slot(w, c_lo, sg.tile);
-                    if (!tile_ready(a, sg.tile, c - c_lo, flag_s)) {
-                        ok = false;
-                        break;
-                    }
                 }
                 const int row = sg.tile / w.tiles_n * BM + rloc, n0 = sg.tile % w.tiles_n * BN;
                 for (int c0 = cb; c0 < cb + HC; c0 += 16) {
@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(320, 1)
                     epilogue16(a, row, n0 + c0, v);
                     if (a.amax && a.epi == GEMM_STORE) argmax16(a, row, n0 + c0, v);
                 }
-            } else {
+            } else if (!whole && !fin) {
                 // publish this piece ([column][row] fp32, coalesced) and free the accumulator
                 float* mine = a.ws + ((size_t)c * 2 + sg.slot) * (BM * BN);
                 for (int c0 = cb; c0 < cb + HC; c0 += 16) {
@@ -486,10 +486,11 @@ __global__ void __launch_bounds__(320, 1)
             if (!whole) {
                 epi_bar8();
                 if (threadIdx.x == 0) {
-                    if (fin)
-                        atomicExch(&a.cnt[sg.tile], 0);  // every piece is read: ready for the next launch
-                    else
+                    if (!fin)
                         atomicAdd(&a.cnt[sg.tile], 1);
+                    else if (ok)
+                        atomicExch(&a.cnt[sg.tile], 0);  // every piece is read: ready for the next launch
+                    // (after a wait that ran out the host zeroes the counters)
                 }
             }
         }
