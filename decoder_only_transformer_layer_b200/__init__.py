@@ -92,6 +92,8 @@ def lib():
         L.dec_check_standalone.argtypes = [_P]
         L.dec_test_fail_alloc.argtypes = [_I]
         L.dec_test_gemm_wait.argtypes = [_I, C.c_int64]
+        L.dec_test_streamk_check.argtypes = [_I, _I, _I, _I]
+        L.dec_test_streamk_check.restype = C.c_int
         for f in ("dec_init", "dec_free", "dec_reset", "dec_prefill", "dec_step", "dec_last_argmax", "dec_kv_read",
                   "dec_kv_write", "dec_last_routes", "dec_last_hidden", "dec_seq_len", "gqa_decode_attn",
                   "gqa_decode_attn_noalloc", "moe_route_topk", "moe_experts", "weight_gemv", "dec_check",
@@ -341,6 +343,12 @@ def check_standalone(stream=None):
 def test_fail_alloc(n: int):
     """Test hook: the n-th device allocation of the library from now on fails (0 = off)."""
     _check(lib().dec_test_fail_alloc(int(n)))
+
+
+def test_streamk_check(M: int, N: int, K: int, ctas: int) -> int:
+    """Test hook: violations of the persistent GEMM's work-split invariants for an
+    M x N x K product over `ctas` CTAs, checked on the host (0 = sound)."""
+    return int(lib().dec_test_streamk_check(int(M), int(N), int(K), int(ctas)))
 
 
 def test_gemm_wait(extra_pieces: int, limit_cycles: int):

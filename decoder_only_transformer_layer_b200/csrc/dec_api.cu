@@ -1566,4 +1566,8 @@ dec_status dec_test_gemm_wait(int32_t extra_pieces, int64_t limit_cycles) {
     return DEC_OK;
 }
 
+int32_t dec_test_streamk_check(int32_t M, int32_t N, int32_t K, int32_t ctas) {
+    return gemm_streamk_check(M, N, K, ctas);
+}
+
 }  // extern "C"

@@ -30,6 +30,8 @@
 //    nothing), residual add, or SwiGLU on interleaved gate/up rows (bf16 silu(g)*u).
 #include <cuda.h>
 
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
@@ -180,12 +182,12 @@ struct Work {
 // in L2; the rest (at least one tile per CTA, so no piece is shorter than a tile's worth of
 // k blocks on average) is split by stream-K and processed first. With one column tile
 // every tile is split by stream-K.
-DEC_DEVINL Work make_work(const GemmArgs& a, int bn) {
+__host__ __device__ inline Work make_work(const GemmArgs& a, int bn, int nc) {
     Work w;
     w.nkb = (a.K + BK - 1) / BK;
     w.tiles_n = (a.N + bn - 1) / bn;
     w.bn = bn;
-    w.nc = gridDim.x;
+    w.nc = nc;
     const int T = ((a.M + BM - 1) / BM) * w.tiles_n;
     w.dp = (w.tiles_n > 1 && T >= 2 * w.nc) ? T / w.nc - 1 : 0;
     w.tsk = T - w.dp * w.nc;
@@ -193,16 +195,16 @@ DEC_DEVINL Work make_work(const GemmArgs& a, int bn) {
     return w;
 }
 
-DEC_DEVINL long long unit0(const Work& w, int c) { return w.U * c / w.nc; }
+__host__ __device__ inline long long unit0(const Work& w, int c) { return w.U * c / w.nc; }
 // CTA whose range holds stream-K unit u (w.U > 0).
-DEC_DEVINL int cta_of(const Work& w, long long u) { return (int)(((u + 1) * w.nc - 1) / w.U); }
+__host__ __device__ inline int cta_of(const Work& w, long long u) { return (int)(((u + 1) * w.nc - 1) / w.U); }
 
 struct Range {
     long long u0, u1;
     int c, tf, nsk, nseg, iters;  // nsk: stream-K segments, then w.dp whole tiles
 };
 
-DEC_DEVINL Range cta_range(const Work& w, int c) {
+__host__ __device__ inline Range cta_range(const Work& w, int c) {
     Range r;
     r.c = c;
     r.u0 = unit0(w, c);
@@ -222,7 +224,7 @@ struct Seg {
 // piece some later CTA finishes, so it is published as early as possible), then the
 // first tile (this CTA holds its last k blocks and finishes it), then the middle tiles,
 // then the round-robin whole tiles.
-DEC_DEVINL Seg segment(const Work& w, const Range& r, int j) {
+__host__ __device__ inline Seg segment(const Work& w, const Range& r, int j) {
     Seg s;
     if (j >= r.nsk) {
         s.tile = w.tsk + r.c + (j - r.nsk) * w.nc;
@@ -242,7 +244,7 @@ DEC_DEVINL Seg segment(const Work& w, const Range& r, int j) {
 }
 
 // Workspace slot of CTA cc's piece of (stream-K) `tile`.
-DEC_DEVINL int piece_slot(const Work& w, int cc, int tile) { return (int)(unit0(w, cc) / w.nkb) == tile ? 0 : 1; }
+__host__ __device__ inline int piece_slot(const Work& w, int cc, int tile) { return (int)(unit0(w, cc) / w.nkb) == tile ? 0 : 1; }
 
 // Walks the k blocks of a range in processing order (the producer's view).
 struct SegIter {
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(320, 1)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
     }
-    const Work w = make_work(a, BN);
+    const Work w = make_work(a, BN, gridDim.x);
     const int c = blockIdx.x;
     const Range rg = cta_range(w, c);
 
@@ -920,6 +922,60 @@ int gemm_ctas(int M, int N, int K, int num_sms) {
     if (nc > num_sms) nc = num_sms;
     if (nc < 1) nc = 1;
     return (int)nc;
+}
+
+// Host-side check of the persistent kernel's work split for an M x N x K product over
+// `nc` CTAs (the plan the kernel derives from its grid): every (tile, k block) unit is
+// covered exactly once; every piece that another CTA finishes is the first segment its
+// CTA processes (so it is published before that CTA waits on anything, which is what
+// keeps the finishers' waits free of cycles); every tile split between CTAs has exactly
+// one finisher, the CTA holding its last k blocks, whose expected pieces are the other
+// CTAs' segments of the tile in the slots it reads. Returns the number of violations.
+int gemm_streamk_check(int M, int N, int K, int nc) {
+    if (M <= 0 || N <= 0 || K <= 0 || nc <= 0) return -1;
+    GemmArgs a{};
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    const Work w = make_work(a, gemm_bn(N), nc);
+    const int T = ((M + BM - 1) / BM) * w.tiles_n;
+    std::vector<int> cover((size_t)T * w.nkb, 0), fins(T, 0), pieces(T, 0);
+    int bad = 0;
+    for (int c = 0; c < nc; ++c) {
+        const Range r = cta_range(w, c);
+        for (int j = 0; j < r.nseg; ++j) {
+            const Seg sg = segment(w, r, j);
+            if (sg.tile < 0 || sg.tile >= T || sg.kb0 < 0 || sg.kb1 > w.nkb || sg.kb0 >= sg.kb1) {
+                ++bad;
+                continue;
+            }
+            for (int kb = sg.kb0; kb < sg.kb1; ++kb) ++cover[(size_t)sg.tile * w.nkb + kb];
+            const bool whole = sg.kb0 == 0 && sg.kb1 == w.nkb, fin = !whole && sg.kb1 == w.nkb;
+            if (!whole && !fin) {
+                ++pieces[sg.tile];
+                if (j != 0) ++bad;                                // published late
+                if (sg.slot != piece_slot(w, c, sg.tile)) ++bad;  // not where the finisher reads
+            }
+            if (fin) {
+                ++fins[sg.tile];
+                if (c - cta_of(w, (long long)sg.tile * w.nkb) < 1) ++bad;  // nothing to wait for
+            }
+        }
+    }
+    for (size_t u = 0; u < cover.size(); ++u) bad += cover[u] != 1;
+    for (int t = 0; t < T; ++t) {
+        if (t >= w.tsk) {  // round-robin whole tiles
+            bad += fins[t] != 0 || pieces[t] != 0;
+            continue;
+        }
+        const long long t0 = (long long)t * w.nkb;
+        const int P = cta_of(w, t0 + w.nkb - 1) - cta_of(w, t0) + 1;
+        if (P == 1)
+            bad += fins[t] != 0 || pieces[t] != 0;
+        else
+            bad += fins[t] != 1 || pieces[t] != P - 1;
+    }
+    return bad;
 }
 
 size_t gemm_ws_floats(int num_sms) { return (size_t)2 * num_sms * BM * 256; }

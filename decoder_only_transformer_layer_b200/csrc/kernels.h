@@ -78,6 +78,8 @@ struct GemmArgs {
 // own completed and no reduction load issued, so it exits cleanly; the tile counters it
 // leaves behind must be zeroed by the host before the next launch.
 void gemm_set_test_wait(int extra_pieces, long long limit_cycles);
+// Host-side check of the persistent GEMM's work split (see gemm_tc.cu); violations or -1.
+int gemm_streamk_check(int M, int N, int K, int nc);
 
 // Build the tensor maps for one GEMM shape (host; encodes the A, B and workspace
 // addresses). ws holds gemm_ws_floats(num_sms) floats.

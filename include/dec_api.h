@@ -335,8 +335,18 @@ dec_status dec_test_fail_alloc(int32_t n);
  * for `extra_pieces` more partial tiles than exist, giving up after `limit_cycles` SM
  * clock cycles (0 = the normal limit of about 1 s). (0, 0) restores normal operation.
  * Process-wide; a dec_step graph keeps the setting it was captured with. For testing the
- * DEC_ERR_TIMEOUT path: a CTA leaves that wait with all its loads and MMAs complete. */
+ * DEC_ERR_TIMEOUT path: a CTA whose wait runs out skips its remaining outputs but still
+ * drains its accumulators, so it leaves with all its loads and MMAs complete. */
 dec_status dec_test_gemm_wait(int32_t extra_pieces, int64_t limit_cycles);
+
+/* Host-side check (no GPU needed) of the work split the persistent tensor-core GEMM uses
+ * for an M x N x K product over `ctas` CTAs (it launches min(SMs, units / 8) of them, a
+ * unit being one 128-row tile x one 64-wide k block): every unit is covered once, every
+ * partial tile another CTA finishes is the first segment its CTA processes, and every tile
+ * split between CTAs has exactly one finisher, the CTA holding its last k blocks, whose
+ * expected pieces all exist. Returns the number of violations (0 = sound), or -1 for a
+ * non-positive argument. */
+int32_t dec_test_streamk_check(int32_t M, int32_t N, int32_t K, int32_t ctas);
 
 /* Copy cache rows [pos0, pos0+n) of layer `layer` of sequence `seq` to / from host
  * buffers bf16 [n][nkv*d] (k and v). dec_kv_write also extends the sequence's length
